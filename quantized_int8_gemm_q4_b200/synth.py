@@ -1,0 +1,119 @@
+"""Seeded synthetic inputs and workload shapes.
+
+This module holds no arithmetic of the method: it only draws random bytes and
+numbers with the distributions the workloads call for, and lays the bytes out
+in the GGUF block order.  Both the oracle-side tests and the CUDA-side tests
+and benchmark take their inputs from here.
+
+Distributions (the synthetic stand-ins for real GGUF weights, which are not used):
+  * Q4_K: the 12 scale bytes and 128 quant bytes are uniform random bytes, so
+    every 4-bit quant is uniform on 0..15 and every 6-bit scale and min is
+    uniform on 0..63; d and dmin are uniform on [1e-3, 1e-2] rounded to f16.
+  * Q6_K: the 128 low-bit bytes and 64 high-bit bytes are uniform random bytes,
+    so every 6-bit quant is uniform on 0..63; the 16 int8 scales are uniform on
+    -32..31 (configurable); d as above.
+  * Activations: f32 standard normal.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+Q4_K = 12
+Q6_K = 14
+QK_K = 256
+BLOCK_BYTES = {Q4_K: 144, Q6_K: 210}
+
+
+def _rng(seed, *sub):
+    return np.random.default_rng([int(seed), *[int(s) for s in sub]])
+
+
+def _f16_bytes(rng, n, lo=1e-3, hi=1e-2):
+    v = rng.uniform(lo, hi, size=n).astype(np.float16)
+    return v.view(np.uint8).reshape(n, 2)
+
+
+def q4k_weights(N: int, K: int, seed, *sub) -> np.ndarray:
+    """uint8 [N, K/256, 144] GGUF Q4_K blocks: d | dmin | 12 scale bytes | 128 quant bytes."""
+    assert K % QK_K == 0
+    nb = N * (K // QK_K)
+    rng = _rng(seed, 4, *sub)
+    blk = np.empty((nb, 144), np.uint8)
+    blk[:, 0:2] = _f16_bytes(rng, nb)
+    blk[:, 2:4] = _f16_bytes(rng, nb)
+    blk[:, 4:144] = rng.integers(0, 256, size=(nb, 140), dtype=np.uint8)
+    return blk.reshape(N, K // QK_K, 144)
+
+
+def q6k_weights(N: int, K: int, seed, *sub, sc_lo: int = -32, sc_hi: int = 31) -> np.ndarray:
+    """uint8 [N, K/256, 210] GGUF Q6_K blocks: 128 low | 64 high | 16 int8 scales | d."""
+    assert K % QK_K == 0
+    nb = N * (K // QK_K)
+    rng = _rng(seed, 6, *sub)
+    blk = np.empty((nb, 210), np.uint8)
+    blk[:, 0:192] = rng.integers(0, 256, size=(nb, 192), dtype=np.uint8)
+    blk[:, 192:208] = rng.integers(sc_lo, sc_hi + 1, size=(nb, 16)).astype(np.int8).view(np.uint8)
+    blk[:, 208:210] = _f16_bytes(rng, nb)
+    return blk.reshape(N, K // QK_K, 210)
+
+
+def weights(qtype: int, N: int, K: int, seed, *sub) -> np.ndarray:
+    return q4k_weights(N, K, seed, *sub) if qtype == Q4_K else q6k_weights(N, K, seed, *sub)
+
+
+def activations(M: int, K: int, seed, *sub) -> np.ndarray:
+    """f32 [M, K] standard normal."""
+    return _rng(seed, 8, *sub).standard_normal((M, K), dtype=np.float32)
+
+
+def block_rows(M: int, n_rows: int, seed, *sub, block: int | None = None) -> np.ndarray:
+    """n_rows distinct canvas rows in random order, drawn from one 32-row window
+    [32 + 32b, 64 + 32b) of an M-row canvas whose first 32 rows are the prompt."""
+    rng = _rng(seed, 9, *sub)
+    nblk = max(1, (M - 32) // 32)
+    b = int(rng.integers(0, nblk)) if block is None else block
+    lo = min(32 + 32 * b, M - 32)
+    return (lo + rng.permutation(32)[:n_rows]).astype(np.int32)
+
+
+@dataclass(frozen=True)
+class Proj:
+    """One projection GEMM of a layer: N output features, K inputs, weight type."""
+    name: str
+    qtype: int
+    N: int
+    K: int
+
+
+@dataclass(frozen=True)
+class Model:
+    name: str
+    hidden: int
+    ffn: int
+    n_layers: int
+    q_out: int
+    kv_out: int
+    vocab: int
+    out_rows: int = 32
+    layer: tuple = field(default=())
+
+
+def llada_8b() -> Model:
+    h, f = 4096, 12288
+    return Model("llada-8b", h, f, 32, h, h, 126464, 32,
+                 (Proj("q", Q4_K, h, h), Proj("k", Q4_K, h, h), Proj("v", Q4_K, h, h),
+                  Proj("o", Q4_K, h, h), Proj("gate", Q4_K, f, h), Proj("up", Q4_K, f, h),
+                  Proj("down", Q6_K, h, f)))
+
+
+def dream_7b() -> Model:
+    h, f = 3584, 18944
+    return Model("dream-7b", h, f, 28, h, 512, 152064, 32,
+                 (Proj("q", Q4_K, h, h), Proj("k", Q4_K, 512, h), Proj("v", Q4_K, 512, h),
+                  Proj("o", Q4_K, h, h), Proj("gate", Q4_K, f, h), Proj("up", Q4_K, f, h),
+                  Proj("down", Q6_K, h, f)))
+
+
+MODELS = {"llada-8b": llada_8b, "dream-7b": dream_7b}

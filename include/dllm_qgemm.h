@@ -1,0 +1,166 @@
+/*
+ * dllm_qgemm — quantized projection GEMM of a diffusion-LLM denoising step, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (mojo-dllm Architecture page, "A forward pass", steps 2 and 4, and
+ * "Source map", kernels/packed.mojo, kernels/qgemm.mojo and gpu/kernels.mojo rows):
+ * every projection of every layer multiplies GGUF Q4_K or Q6_K super-block weights
+ * by activations quantized to int8 with one f32 scale per 256 elements; the
+ * activation is quantized once and reused by the Q, K and V projections (and once
+ * for gate and up); the output projection runs only on the canvas rows whose logits
+ * the sampler needs.
+ *
+ *   out[i][n] = sum_k w[n][k] * a[row(i)][k]
+ *   w = d*sc_j*q - dmin*m_j   (Q4_K, 8 sub-blocks of 32, q in 0..15, 6-bit sc, m)
+ *   w = d*sc_j*(q - 32)       (Q6_K, 16 sub-blocks of 16, q in 0..63, int8 sc)
+ *   a = scale[m][k/256] * qa  (qa int8 in [-127, 127])
+ *
+ * Integer parts are exact (int32 tensor-core accumulation per super-block); the
+ * per-super-block combine with d, dmin and the activation scale is f32.
+ *
+ * Conventions for every call:
+ *   - Device pointers unless stated otherwise; the caller allocates and owns every
+ *     buffer.  Calls are asynchronous on `stream` and allocate nothing.
+ *   - Returns DLLM_OK (0) or a negative DLLM_ERR_* code.  Argument errors are found
+ *     on the host before anything is launched.  Errors found on the device (a row
+ *     index out of range, a bounded wait that ran out) set a per-device error word
+ *     that dllm_get_device_status() reports and clears; the kernel never traps.
+ *   - N must be a multiple of 128 and K a multiple of 256.  Device pointers must be
+ *     16-byte aligned.
+ *   - Inputs must be finite.
+ */
+#ifndef DLLM_QGEMM_H
+#define DLLM_QGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dllm_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+/* GGML type ids of the two weight formats. */
+typedef enum { DLLM_Q4_K = 12, DLLM_Q6_K = 14 } dllm_qtype;
+
+enum {
+    DLLM_OK = 0,
+    DLLM_ERR_ARG = -1,         /* null pointer, bad size, K % 256, N % 128, ld too small, ... */
+    DLLM_ERR_ALIGN = -2,       /* a pointer or leading dimension is not 16-byte aligned       */
+    DLLM_ERR_UNSUPPORTED = -3, /* the current device is not sm_100                           */
+    DLLM_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed                         */
+    DLLM_ERR_ROW_RANGE = -5,   /* device-detected: a rows[] entry outside [0, M)               */
+    DLLM_ERR_TIMEOUT = -6,     /* device-detected: a bounded wait inside a kernel ran out      */
+    DLLM_ERR_WORKSPACE = -7    /* workspace smaller than dllm_qgemm_workspace_bytes() asks     */
+};
+
+/* ------------------------------------------------------------------------------
+ * Weights: load-time repack of GGUF blocks into the device tile layout.
+ *
+ * Input: row-major [N][K/256] GGUF blocks (144 bytes each for Q4_K, 210 for Q6_K),
+ * on the device.  Output: the same bytes regrouped into tiles of 128 rows x 1
+ * super-block, tile (t, s) at byte offset (t*(K/256) + s) * 128 * block_bytes, so
+ * that one bulk copy brings a tile into shared memory.  Inside a tile:
+ *   Q4_K (18432 B): quants [8][128 rows][16 B] | scale bytes [128][12] | d,dmin [128][2 x f16]
+ *   Q6_K (26880 B): low bits [8][128][16 B] | high bits [4][128][16 B] |
+ *                   int8 scales [128][16] | d [128][f16]
+ * The repacked size equals the GGUF size (4.5 / 6.5625 bits per weight): nothing is
+ * expanded (Architecture page, "Memory": the model stays resident once).
+ * `gguf` and `dst` must not overlap.
+ * ---------------------------------------------------------------------------- */
+int dllm_repacked_bytes(dllm_qtype t, int64_t N, int64_t K, size_t* out_bytes); /* host pointer */
+int dllm_repack_q4k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
+int dllm_repack_q6k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Activations: int8 with one f32 scale per 256 elements, plus per-32 sums
+ * (Architecture page, "Source map", kernels/qgemm.mojo row; "A forward pass",
+ * step 2: quantized once, reused by Q/K/V and by gate/up).
+ *
+ * Rounding (the page leaves it open; this is the reading the library implements):
+ * amax over the 256-block; iscale = 127/amax and scale = amax/127, each one IEEE
+ * f32 division; qa = round-half-even(x * iscale) (one f32 multiply), clamped to
+ * [-127, 127]; a block with amax = 0 has scale 0 and qa 0.
+ *
+ * x: f32 [M][ldx] row-major (ldx >= K, ldx % 4 == 0).  Outputs, with Mp = M rounded
+ * up to a multiple of 16 (rows M..Mp-1 are written as zeros):
+ *   q     int8  [K/256][Mp/8][16][8][16]: super-block s, 8-row group g, 16-byte chunk c
+ *                (k = 256 s + 16 c + j), row r of the group, byte j.  Each group of 8
+ *                rows x 16 bytes is one 128-byte core matrix of the tensor-core B operand.
+ *   scale f32   [K/256][Mp]
+ *   sums  uint8 [K/256][Mp][16]: for the 8 sub-blocks of 32 of super-block s, the sum
+ *                t_j of the 32 qa values split as t_j = lo_j + 256*hi_j with lo_j =
+ *                t_j & 255 in byte j (unsigned) and hi_j = t_j >> 8 in byte 8 + j (signed).
+ * dllm_act_bytes() gives the three sizes for (M, K).
+ * ---------------------------------------------------------------------------- */
+int dllm_act_bytes(int64_t M, int64_t K, size_t* q_bytes, size_t* scale_bytes, size_t* sums_bytes);
+int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* scale,
+                      uint8_t* sums, dllm_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * GEMM: out[i][n] for n in [0, N) of one repacked weight matrix `w` (from
+ * dllm_repack_*), activations (q, scale, sums) of an M-row canvas from
+ * dllm_quantize_act.
+ *   rows == NULL : i = m over all M rows; out is [M][ldo].
+ *   rows != NULL : device int32 list of n_rows canvas rows (1 <= n_rows <= 32,
+ *                  duplicates allowed, any order); out row i is canvas row rows[i];
+ *                  out is [n_rows][ldo].  An entry outside [0, M) zero-fills its
+ *                  output row and sets DLLM_ERR_ROW_RANGE in the device error word.
+ *                  (Architecture page, "A forward pass", step 4: the output projection
+ *                  runs only on the requested rows.)
+ * ldo >= N, ldo % 4 == 0.  Results are deterministic and do not depend on M or on the
+ * row set: a gathered row equals the same row of the full-canvas result bit for bit.
+ * workspace: optional device scratch (may be NULL with workspace_bytes 0); reserved
+ * for split-K scheduling, see dllm_qgemm_workspace_bytes().
+ * ---------------------------------------------------------------------------- */
+int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, size_t* bytes);
+int dllm_qgemm(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
+               const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows, float* out, int64_t ldo,
+               void* workspace, size_t workspace_bytes, dllm_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Several projections of one quantized activation in one launch (Architecture page,
+ * "A forward pass", step 2: quantize once, reuse for Q, K and V; the same holds for
+ * the FFN's gate and up).  wq has Nq rows, wk and wv Nkv rows; wv == NULL runs two
+ * projections (e.g. gate and up).  oq is [M][ldo_q], ok and ov are [M][ldo_kv].
+ * ---------------------------------------------------------------------------- */
+int dllm_qkv_qgemm(const void* wq, const void* wk, const void* wv, dllm_qtype t, int64_t Nq, int64_t Nkv,
+                   int64_t K, const int8_t* q, const float* scale, const uint8_t* sums, int64_t M, float* oq,
+                   int64_t ldo_q, float* ok, float* ov, int64_t ldo_kv, void* workspace, size_t workspace_bytes,
+                   dllm_stream_t stream);
+
+/* Synchronizes `stream`, then returns and clears the device error word
+ * (DLLM_OK, DLLM_ERR_ROW_RANGE or DLLM_ERR_TIMEOUT). */
+int dllm_get_device_status(dllm_stream_t stream);
+const char* dllm_status_string(int code);
+
+/* ------------------------------------------------------------------------------
+ * Test and measurement entry points (not on the hot path).
+ * ---------------------------------------------------------------------------- */
+
+/* Per-sub-block integer dot products on CUDA cores, for bit-exact checking:
+ * dots[m][n][j] (int32, [M][N][K/32] for Q4_K with q in 0..15, [M][N][K/16] for
+ * Q6_K with q - 32), from the repacked weights and the quantized activations. */
+int dllm_debug_subblock_dots(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, int64_t M,
+                             int32_t* dots, dllm_stream_t stream);
+
+/* The per-super-block integers the tensor-core path forms, read back from tensor
+ * memory instead of being combined: S[m][n][s] = sum_j sc_j * dot_j and (Q4_K)
+ * Smin[m][n][s] = sum_j m_j * sum32_j, int32 [M][N][K/256] each (Smin untouched for
+ * Q6_K).  Same kernel and schedule as dllm_qgemm with the f32 epilogue replaced. */
+int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
+                       const uint8_t* sums, int64_t M, int32_t* S, int32_t* Smin, dllm_stream_t stream);
+
+/* int8 tensor-core throughput probe: `iters` back-to-back tcgen05 kind::i8 MMAs of
+ * 128 x n x 32 per CTA on `ctas` CTAs, rotating over n_acc independent accumulators,
+ * with A in tensor memory (a_from_tmem != 0) or in shared memory.  Writes elapsed
+ * device nanoseconds per CTA to ns_out (device, [ctas] uint64).
+ * 16 <= n <= 256, n % 16 == 0, n * n_acc <= 448. */
+int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int iters, int ctas, unsigned long long* ns_out,
+                      dllm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DLLM_QGEMM_H */

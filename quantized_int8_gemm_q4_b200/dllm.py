@@ -1,0 +1,194 @@
+"""Python binding of the dllm_qgemm C-ABI (include/dllm_qgemm.h).
+
+Argument marshalling only: every step runs in the CUDA library.  torch supplies
+device memory and streams.  There is no CPU fallback: if the compiled library is
+missing, importing a function raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+LIB_PATH = Path(__file__).resolve().parent / "_build" / "libdllm_qgemm.so"
+
+DLLM_Q4_K = 12
+DLLM_Q6_K = 14
+QK_K = 256
+BLOCK_BYTES = {DLLM_Q4_K: 144, DLLM_Q6_K: 210}
+
+DLLM_OK = 0
+DLLM_ERR_ARG = -1
+DLLM_ERR_ALIGN = -2
+DLLM_ERR_UNSUPPORTED = -3
+DLLM_ERR_CUDA = -4
+DLLM_ERR_ROW_RANGE = -5
+DLLM_ERR_TIMEOUT = -6
+DLLM_ERR_WORKSPACE = -7
+
+EXPORTS = (
+    "dllm_repacked_bytes", "dllm_repack_q4k", "dllm_repack_q6k", "dllm_act_bytes", "dllm_quantize_act",
+    "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qkv_qgemm", "dllm_get_device_status",
+    "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_bench_mma_i8",
+)
+
+
+class DllmError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the compiled library; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise ImportError(f"dllm_qgemm CUDA library not built: {LIB_PATH} is missing "
+                          "(run __graft_entry__.build() or python -m quantized_int8_gemm_q4_b200.build)")
+    L = ctypes.CDLL(str(LIB_PATH))
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    SZ = ctypes.c_size_t
+    PSZ = ctypes.POINTER(ctypes.c_size_t)
+    sig = {
+        "dllm_repacked_bytes": [I, I64, I64, PSZ],
+        "dllm_repack_q4k": [P, I64, I64, P, P],
+        "dllm_repack_q6k": [P, I64, I64, P, P],
+        "dllm_act_bytes": [I64, I64, PSZ, PSZ, PSZ],
+        "dllm_quantize_act": [P, I64, I64, I64, P, P, P, P],
+        "dllm_qgemm_workspace_bytes": [I, I64, I64, I64, PSZ],
+        "dllm_qgemm": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P, SZ, P],
+        "dllm_qkv_qgemm": [P, P, P, I, I64, I64, I64, P, P, P, I64, P, I64, P, P, I64, P, SZ, P],
+        "dllm_get_device_status": [P],
+        "dllm_status_string": [I],
+        "dllm_debug_subblock_dots": [P, I, I64, I64, P, I64, P, P],
+        "dllm_debug_sb_ints": [P, I, I64, I64, P, P, P, I64, P, P, P],
+        "dllm_bench_mma_i8": [I, I, I, I, I, P, P],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = ctypes.c_char_p if name == "dllm_status_string" else ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    try:
+        return load().dllm_status_string(code).decode()
+    except ImportError:
+        return "library not loaded"
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != DLLM_OK:
+        raise DllmError(rc, where)
+
+
+# ------------------------------------------------------------------ C-ABI, same names
+
+def dllm_repacked_bytes(qtype: int, N: int, K: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load().dllm_repacked_bytes(qtype, N, K, ctypes.byref(out)), "dllm_repacked_bytes")
+    return out.value
+
+
+def dllm_repack_q4k(gguf_blocks, N: int, K: int, dst, stream=None):
+    _check(load().dllm_repack_q4k(_ptr(gguf_blocks), N, K, _ptr(dst), _stream(stream)), "dllm_repack_q4k")
+
+
+def dllm_repack_q6k(gguf_blocks, N: int, K: int, dst, stream=None):
+    _check(load().dllm_repack_q6k(_ptr(gguf_blocks), N, K, _ptr(dst), _stream(stream)), "dllm_repack_q6k")
+
+
+def dllm_act_bytes(M: int, K: int):
+    a, b, c = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(load().dllm_act_bytes(M, K, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)), "dllm_act_bytes")
+    return a.value, b.value, c.value
+
+
+def dllm_quantize_act(x, M: int, K: int, ldx: int, q, scale, sums, stream=None):
+    _check(load().dllm_quantize_act(_ptr(x), M, K, ldx, _ptr(q), _ptr(scale), _ptr(sums), _stream(stream)),
+           "dllm_quantize_act")
+
+
+def dllm_qgemm_workspace_bytes(qtype: int, N: int, K: int, M: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load().dllm_qgemm_workspace_bytes(qtype, N, K, M, ctypes.byref(out)), "dllm_qgemm_workspace_bytes")
+    return out.value
+
+
+def dllm_qgemm(w, qtype: int, N: int, K: int, q, scale, sums, M: int, rows, n_rows: int, out, ldo: int,
+               workspace=None, workspace_bytes: int = 0, stream=None):
+    _check(load().dllm_qgemm(_ptr(w), qtype, N, K, _ptr(q), _ptr(scale), _ptr(sums), M, _ptr(rows), n_rows,
+                             _ptr(out), ldo, _ptr(workspace), workspace_bytes, _stream(stream)), "dllm_qgemm")
+
+
+def dllm_qkv_qgemm(wq, wk, wv, qtype: int, Nq: int, Nkv: int, K: int, q, scale, sums, M: int, oq, ldo_q: int,
+                   ok, ov, ldo_kv: int, workspace=None, workspace_bytes: int = 0, stream=None):
+    _check(load().dllm_qkv_qgemm(_ptr(wq), _ptr(wk), _ptr(wv), qtype, Nq, Nkv, K, _ptr(q), _ptr(scale), _ptr(sums),
+                                 M, _ptr(oq), ldo_q, _ptr(ok), _ptr(ov), ldo_kv, _ptr(workspace), workspace_bytes,
+                                 _stream(stream)), "dllm_qkv_qgemm")
+
+
+def dllm_get_device_status(stream=None) -> int:
+    return load().dllm_get_device_status(_stream(stream))
+
+
+def dllm_status_string(code: int) -> str:
+    return status_string(code)
+
+
+def dllm_debug_subblock_dots(w, qtype: int, N: int, K: int, q, M: int, dots, stream=None):
+    _check(load().dllm_debug_subblock_dots(_ptr(w), qtype, N, K, _ptr(q), M, _ptr(dots), _stream(stream)),
+           "dllm_debug_subblock_dots")
+
+
+def dllm_debug_sb_ints(w, qtype: int, N: int, K: int, q, scale, sums, M: int, S, Smin, stream=None):
+    _check(load().dllm_debug_sb_ints(_ptr(w), qtype, N, K, _ptr(q), _ptr(scale), _ptr(sums), M, _ptr(S),
+                                     _ptr(Smin), _stream(stream)), "dllm_debug_sb_ints")
+
+
+def dllm_bench_mma_i8(n: int, n_acc: int, a_from_tmem: int, iters: int, ctas: int, ns_out, stream=None):
+    _check(load().dllm_bench_mma_i8(n, n_acc, a_from_tmem, iters, ctas, _ptr(ns_out), _stream(stream)),
+           "dllm_bench_mma_i8")
+
+
+# ------------------------------------------------------------------ small conveniences (allocation via torch)
+
+def repack(qtype: int, blocks, N: int, K: int, device="cuda", stream=None):
+    """GGUF blocks (numpy uint8 [N, K/256, bytes] or a device tensor) -> repacked device tensor."""
+    import torch
+    if not isinstance(blocks, torch.Tensor):
+        blocks = torch.from_numpy(blocks.reshape(-1).copy())
+    src = blocks.reshape(-1).to(device)
+    dst = torch.empty(dllm_repacked_bytes(qtype, N, K), dtype=torch.uint8, device=device)
+    (dllm_repack_q4k if qtype == DLLM_Q4_K else dllm_repack_q6k)(src, N, K, dst, stream)
+    return dst
+
+
+def alloc_act(M: int, K: int, device="cuda"):
+    """Device buffers (q, scale, sums) for M x K quantized activations."""
+    import torch
+    qb, sb, ub = dllm_act_bytes(M, K)
+    return (torch.empty(qb, dtype=torch.int8, device=device),
+            torch.empty(sb // 4, dtype=torch.float32, device=device),
+            torch.empty(ub, dtype=torch.uint8, device=device))

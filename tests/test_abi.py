@@ -1,0 +1,117 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every entry
+point include/*.h declares, and rejects bad arguments on the host before any launch.
+No compute call is made here."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from quantized_int8_gemm_q4_b200 import build as nbuild
+from quantized_int8_gemm_q4_b200 import dllm
+
+ROOT = Path(__file__).resolve().parent.parent
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nbuild.build()
+    return dllm.load()
+
+
+def declared_symbols():
+    names = set()
+    for h in (ROOT / "include").glob("*.h"):
+        text = re.sub(r"/\*.*?\*/", "", h.read_text(), flags=re.S)
+        names |= set(re.findall(r"\b(dllm_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for must in ("dllm_repack_q4k", "dllm_repack_q6k", "dllm_quantize_act", "dllm_qgemm", "dllm_qkv_qgemm",
+                 "dllm_get_device_status", "dllm_status_string", "dllm_debug_subblock_dots"):
+        assert must in syms
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(declared_symbols()) <= set(dllm.EXPORTS) | {"dllm_repacked_bytes"}
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+        assert dllm.status_string(code) not in ("", "unknown status")
+    assert dllm.status_string(-99) == "unknown status"
+
+
+def test_sizes_on_host(lib):
+    assert dllm.dllm_repacked_bytes(dllm.DLLM_Q4_K, 256, 512) == 256 * 2 * 144
+    assert dllm.dllm_repacked_bytes(dllm.DLLM_Q6_K, 128, 4096) == 128 * 16 * 210
+    q, s, u = dllm.dllm_act_bytes(17, 512)
+    assert (q, s, u) == (32 * 512, 32 * 2 * 4, 32 * 2 * 16)
+    assert dllm.dllm_qgemm_workspace_bytes(dllm.DLLM_Q4_K, 4096, 4096, 160) >= 0
+
+
+@pytest.mark.parametrize("N,K", [(100, 512), (128, 300), (0, 256), (128, 0), (-128, 256)])
+def test_bad_shapes_rejected(lib, N, K):
+    with pytest.raises(dllm.DllmError) as e:
+        dllm.dllm_repacked_bytes(dllm.DLLM_Q4_K, N, K)
+    assert e.value.code == dllm.DLLM_ERR_ARG
+
+
+def test_bad_qtype_rejected(lib):
+    out = ctypes.c_size_t(0)
+    assert lib.dllm_repacked_bytes(13, 128, 256, ctypes.byref(out)) == dllm.DLLM_ERR_ARG
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_gemm_argument_checks_before_launch(lib):
+    A = 0x10000  # never dereferenced: validation fails first
+    args = dict(w=_fake(A), t=dllm.DLLM_Q4_K, N=256, K=512, q=_fake(A), s=_fake(A), u=_fake(A), M=64,
+                rows=None, n_rows=0, out=_fake(A), ldo=256)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return lib.dllm_qgemm(a["w"], a["t"], a["N"], a["K"], a["q"], a["s"], a["u"], a["M"], a["rows"],
+                              a["n_rows"], a["out"], a["ldo"], None, 0, None)
+
+    assert call(K=300) == dllm.DLLM_ERR_ARG
+    assert call(N=200) == dllm.DLLM_ERR_ARG
+    assert call(M=0) == dllm.DLLM_ERR_ARG
+    assert call(ldo=128) == dllm.DLLM_ERR_ARG
+    assert call(w=None) == dllm.DLLM_ERR_ARG
+    assert call(q=None) == dllm.DLLM_ERR_ARG
+    assert call(q=_fake(A + 4)) == dllm.DLLM_ERR_ALIGN
+    assert call(out=_fake(A + 8)) == dllm.DLLM_ERR_ALIGN
+    assert call(ldo=258) == dllm.DLLM_ERR_ALIGN
+    assert call(rows=_fake(A), n_rows=0) == dllm.DLLM_ERR_ARG
+    assert call(rows=_fake(A), n_rows=33) == dllm.DLLM_ERR_ARG
+    assert call(t=13) == dllm.DLLM_ERR_ARG
+
+
+def test_quantize_argument_checks(lib):
+    A = 0x10000
+    f = lib.dllm_quantize_act
+    assert f(None, 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert f(_fake(A), 4, 300, 300, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert f(_fake(A), 4, 256, 128, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert f(_fake(A + 4), 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ALIGN
+    assert f(_fake(A), 4, 256, 258, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ALIGN
+
+
+def test_repack_rejects_overlap(lib):
+    A = 0x10000
+    assert lib.dllm_repack_q4k(_fake(A), 128, 256, _fake(A + 16), None) == dllm.DLLM_ERR_ARG
+
+
+def test_qkv_argument_checks(lib):
+    A = 0x10000
+    f = lib.dllm_qkv_qgemm
+    ok = f(_fake(A), _fake(A), None, dllm.DLLM_Q4_K, 256, 100, 512, _fake(A), _fake(A), _fake(A), 16,
+           _fake(A), 256, _fake(A), None, 128, None, 0, None)
+    assert ok == dllm.DLLM_ERR_ARG

@@ -1,0 +1,289 @@
+"""CUDA path vs the CPU oracle, element by element, through the C-ABI.
+
+Bit-exact: activation quantization (int8, scales, per-32 sums), the weight repack,
+the per-sub-block int32 dots, and the per-super-block integers the tensor-core path
+forms.  Floating point: |gpu - oracle| <= max(1e-5 |oracle|, 1e-6 T), T the sum of
+absolute terms (the tolerance the method's target states).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_int8_gemm_q4_b200 import dllm, synth
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+Q4, Q6 = dllm.DLLM_Q4_K, dllm.DLLM_Q6_K
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test run without a CUDA device")
+    from quantized_int8_gemm_q4_b200 import build
+    build.build()
+    dllm.load()
+    yield
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+
+# ------------------------------------------------------------------ quantize
+
+def _special_rows(M, K):
+    x = synth.activations(M, K, 21, M, K)
+    rng = np.random.default_rng(M * 7 + K)
+    x *= rng.uniform(1e-4, 1e4, (M, 1)).astype(np.float32)
+    if M > 3:
+        x[1] = 0.0                                   # all-zero row
+        x[2, :256] = -2.5                            # constant block
+        x[3, :8] = [127, 0.5, 1.5, 2.5, -0.5, -1.5, 63.5, -127]  # ties with iscale = 1
+        x[3, 8:256] = 0
+    return x
+
+
+@pytest.mark.parametrize("M,K", [(1, 256), (15, 512), (16, 256), (17, 768), (64, 4096), (160, 4096), (257, 1024)])
+def test_quantize_bitexact(M, K):
+    x = _special_rows(M, K)
+    act = gu.Act(x)
+    q, s, a = act.host()
+    oq, os_, oa = oracle.quantize_act(x)
+    assert np.array_equal(q, oq)
+    assert np.array_equal(s.view(np.uint32), os_.view(np.uint32))
+    assert np.array_equal(a, oa)
+    Mp = (M + 15) // 16 * 16
+    if Mp > M:  # padded rows are zero
+        full = act.q.cpu().numpy().reshape(K // 256, Mp // 8, 16, 8, 16).transpose(1, 3, 0, 2, 4).reshape(Mp, K)
+        assert not full[M:].any()
+
+
+def test_quantize_strided_input():
+    M, K, ldx = 20, 512, 1024
+    xb = synth.activations(M, ldx, 22)
+    x = torch.from_numpy(xb).cuda()
+    q, s, u = dllm.alloc_act(M, K)
+    dllm.dllm_quantize_act(x, M, K, ldx, q, s, u)
+    oq, os_, _ = oracle.quantize_act(np.ascontiguousarray(xb[:, :K]))
+    assert np.array_equal(gu.untile_q(q, M, K), oq)
+    assert np.array_equal(gu.untile_scale(s, M, K), os_)
+
+
+# ------------------------------------------------------------------ repack and integer paths
+
+@pytest.mark.parametrize("qtype", [Q4, Q6])
+def test_repack_bitexact(qtype):
+    N, K = 256, 768
+    w = synth.weights(qtype, N, K, 31)
+    dev = dllm.repack(qtype, w, N, K)
+    assert np.array_equal(dev.cpu().numpy(), gu.repack_reference(qtype, w))
+
+
+@pytest.mark.parametrize("qtype", [Q4, Q6])
+@pytest.mark.parametrize("M,N,K", [(3, 128, 256), (17, 256, 512)])
+def test_subblock_dots_bitexact(qtype, M, N, K):
+    w, x = gu.make_case(qtype, M, N, K, 32)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    nsub = K // 32 if qtype == Q4 else K // 16
+    dots = torch.zeros((M, N, nsub), dtype=torch.int32, device="cuda")
+    dllm.dllm_debug_subblock_dots(wd, qtype, N, K, act.q, M, dots)
+    oq, _, _ = oracle.quantize_act(x)
+    od, _, _ = oracle.sb_ints(qtype, w, N, K, oq)
+    assert np.array_equal(dots.cpu().numpy(), od)
+
+
+@pytest.mark.parametrize("qtype", [Q4, Q6])
+@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (17, 256, 768), (64, 128, 512), (160, 384, 256)])
+def test_tensor_core_integers_bitexact(qtype, M, N, K):
+    w, x = gu.make_case(qtype, M, N, K, 33)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    S = torch.zeros((M, N, K // 256), dtype=torch.int32, device="cuda")
+    Sm = torch.zeros_like(S)
+    dllm.dllm_debug_sb_ints(wd, qtype, N, K, act.q, act.scale, act.sums, M, S, Sm)
+    oq, _, _ = oracle.quantize_act(x)
+    _, oS, oSm = oracle.sb_ints(qtype, w, N, K, oq)
+    assert np.array_equal(S.cpu().numpy().astype(np.int64), oS)
+    if qtype == Q4:
+        assert np.array_equal(Sm.cpu().numpy().astype(np.int64), oSm)
+
+
+def test_tensor_core_integers_extreme_values():
+    # largest magnitudes the planes and sums can take: every quant at its maximum,
+    # every 6-bit scale and min 63, every activation +-127
+    M, N, K = 16, 128, 512
+    w = synth.q4k_weights(N, K, 34).copy()
+    w[..., 4:144] = 0xFF
+    x = np.full((M, K), 3.0, np.float32)
+    x[::2] *= -1
+    wd = dllm.repack(Q4, w, N, K)
+    act = gu.Act(x)
+    S = torch.zeros((M, N, K // 256), dtype=torch.int32, device="cuda")
+    Sm = torch.zeros_like(S)
+    dllm.dllm_debug_sb_ints(wd, Q4, N, K, act.q, act.scale, act.sums, M, S, Sm)
+    oq, _, _ = oracle.quantize_act(x)
+    _, oS, oSm = oracle.sb_ints(Q4, w, N, K, oq)
+    assert np.abs(oS).max() == 945 * 127 * 256
+    assert np.array_equal(S.cpu().numpy().astype(np.int64), oS)
+    assert np.array_equal(Sm.cpu().numpy().astype(np.int64), oSm)
+    # Q6_K: q = 0 with scale -128 gives (q-32)*sc = 4096, the largest product
+    w6 = synth.q6k_weights(N, K, 34).copy()
+    w6[..., 0:192] = 0
+    w6[..., 192:208] = np.uint8(0x80)
+    wd6 = dllm.repack(Q6, w6, N, K)
+    S6 = torch.zeros((M, N, K // 256), dtype=torch.int32, device="cuda")
+    dllm.dllm_debug_sb_ints(wd6, Q6, N, K, act.q, act.scale, act.sums, M, S6, S6)
+    _, oS6, _ = oracle.sb_ints(Q6, w6, N, K, oq)
+    assert np.array_equal(S6.cpu().numpy().astype(np.int64), oS6)
+
+
+# ------------------------------------------------------------------ f32 GEMM
+
+SHAPES = [(1, 128, 256), (15, 128, 512), (16, 256, 256), (17, 384, 768), (64, 256, 512), (160, 128, 512),
+          (257, 256, 256)]
+
+
+@pytest.mark.parametrize("qtype", [Q4, Q6])
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_qgemm_parity(qtype, M, N, K):
+    w, x = gu.make_case(qtype, M, N, K, 40)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, qtype, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    _, ref, T = oracle.qgemm(qtype, w, N, K, oq, os_)
+    ok, worst = gu.tol_ok(out, ref, T)
+    assert ok, worst
+
+
+def test_config0_exact_case():
+    """Q4_K, M=64, K=512, N=256, seed 0 (the smallest named workload)."""
+    M, N, K = 64, 256, 512
+    w = synth.q4k_weights(N, K, 0)
+    x = synth.activations(M, K, 0)
+    wd = dllm.repack(Q4, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, Q4, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    _, ref, T = oracle.qgemm(Q4, w, N, K, oq, os_)
+    ok, worst = gu.tol_ok(out, ref, T)
+    assert ok, worst
+    dots = torch.zeros((M, N, K // 32), dtype=torch.int32, device="cuda")
+    dllm.dllm_debug_subblock_dots(wd, Q4, N, K, act.q, M, dots)
+    od, _, _ = oracle.sb_ints(Q4, w, N, K, oq)
+    assert np.array_equal(dots.cpu().numpy(), od)
+
+
+@pytest.mark.parametrize("qtype", [Q4, Q6])
+def test_qgemm_ldo_and_determinism(qtype):
+    M, N, K, ldo = 40, 256, 512, 300
+    w, x = gu.make_case(qtype, M, N, K, 41)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    a = gu.gemm(wd, qtype, N, K, act, ldo=ldo)
+    b = gu.gemm(wd, qtype, N, K, act, ldo=ldo)
+    assert torch.equal(a[:, :N], b[:, :N])
+    assert torch.isnan(a[:, N:]).all()
+    oq, os_, _ = oracle.quantize_act(x)
+    _, ref, T = oracle.qgemm(qtype, w, N, K, oq, os_)
+    assert gu.tol_ok(a[:, :N].cpu().numpy(), ref, T)[0]
+
+
+# ------------------------------------------------------------------ rows (logits only on requested rows)
+
+@pytest.mark.parametrize("qtype", [Q6, Q4])
+@pytest.mark.parametrize("n_rows", [1, 2, 4, 8, 16, 32])
+def test_rows_equal_full_slice(qtype, n_rows):
+    M, N, K = 160, 256, 512
+    w, x = gu.make_case(qtype, M, N, K, 50)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    full = gu.gemm(wd, qtype, N, K, act)
+    rows = synth.block_rows(M, n_rows, 50, n_rows)
+    got = gu.gemm(wd, qtype, N, K, act, rows=rows)
+    assert torch.equal(got, full[torch.from_numpy(rows).long().cuda()])
+    oq, os_, _ = oracle.quantize_act(x)
+    _, ref, T = oracle.qgemm(qtype, w, N, K, oq, os_, rows=rows)
+    assert gu.tol_ok(got.cpu().numpy(), ref, T)[0]
+
+
+def test_rows_duplicates_and_order():
+    M, N, K = 64, 128, 256
+    w, x = gu.make_case(Q6, M, N, K, 51)
+    wd = dllm.repack(Q6, w, N, K)
+    act = gu.Act(x)
+    full = gu.gemm(wd, Q6, N, K, act)
+    rows = np.array([63, 0, 0, 17, 63], np.int32)
+    got = gu.gemm(wd, Q6, N, K, act, rows=rows)
+    assert torch.equal(got, full[torch.from_numpy(rows).long().cuda()])
+
+
+def test_rows_out_of_range_sets_status():
+    M, N, K = 48, 128, 256
+    w, x = gu.make_case(Q4, M, N, K, 52)
+    wd = dllm.repack(Q4, w, N, K)
+    act = gu.Act(x)
+    full = gu.gemm(wd, Q4, N, K, act)
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    rows = np.array([5, 48, -1, 7], np.int32)
+    got = gu.gemm(wd, Q4, N, K, act, rows=rows)
+    assert dllm.dllm_get_device_status() == dllm.DLLM_ERR_ROW_RANGE
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK  # cleared
+    assert torch.equal(got[0], full[5]) and torch.equal(got[3], full[7])
+    assert (got[1] == 0).all() and (got[2] == 0).all()
+
+
+# ------------------------------------------------------------------ Q/K/V in one launch
+
+@pytest.mark.parametrize("qtype", [Q4, Q6])
+@pytest.mark.parametrize("with_v", [True, False])
+def test_qkv_matches_separate(qtype, with_v):
+    M, Nq, Nkv, K = 40, 256, 128, 512
+    x = synth.activations(M, K, 60)
+    ws = [synth.weights(qtype, n, K, 60, i) for i, n in enumerate((Nq, Nkv, Nkv))]
+    wd = [dllm.repack(qtype, w, w.shape[0], K) for w in ws]
+    act = gu.Act(x)
+    oq = torch.empty((M, Nq), device="cuda")
+    ok = torch.empty((M, Nkv), device="cuda")
+    ov = torch.empty((M, Nkv), device="cuda") if with_v else None
+    dllm.dllm_qkv_qgemm(wd[0], wd[1], wd[2] if with_v else None, qtype, Nq, Nkv, K, act.q, act.scale, act.sums,
+                        M, oq, Nq, ok, ov, Nkv)
+    outs = [oq, ok] + ([ov] if with_v else [])
+    for i, o in enumerate(outs):
+        sep = gu.gemm(wd[i], qtype, ws[i].shape[0], K, act)
+        assert torch.equal(o, sep)
+
+
+# ------------------------------------------------------------------ full-size shapes, sampled outputs
+
+def _sampled_parity(qtype, M, N, K, seed, rows=None, n_samples=3, width=64):
+    w = synth.weights(qtype, N, K, seed)
+    x = synth.activations(M, K, seed)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, qtype, N, K, act, rows=rows).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    rng = np.random.default_rng(seed)
+    starts = sorted(set([0, N - width] + list(rng.integers(0, N - width, n_samples))))
+    for n0 in starts:
+        _, ref, T = oracle.qgemm(qtype, w, N, K, oq, os_, rows=rows, n0=int(n0), n1=int(n0) + width)
+        ok, worst = gu.tol_ok(out[:, n0:n0 + width], ref, T)
+        assert ok, (n0, worst)
+    return out
+
+
+def test_full_qkv_shape_sampled():
+    # LLaDA-8B-shaped attention projections on a 160-token canvas: Q|K|V as one N = 12288 launch
+    _sampled_parity(Q4, 160, 12288, 4096, 1)
+
+
+def test_full_ffn_shapes_sampled():
+    _sampled_parity(Q4, 256, 12288, 4096, 2, width=32)
+    _sampled_parity(Q6, 160, 4096, 12288, 2, width=32)
+
+
+def test_full_output_projection_rows_sampled():
+    M = 160
+    rows = synth.block_rows(M, 32, 3)
+    _sampled_parity(Q6, M, 126464, 4096, 3, rows=rows, n_samples=4, width=128)

@@ -1,0 +1,508 @@
+#!/usr/bin/env python3
+"""Benchmark: the projection GEMMs of one LLaDA-8B-shaped denoising step on B200.
+
+A step is one pass of the whole hot path over one synthetic canvas: for each of the
+32 layers, quantize the attention input once and run Q, K and V in one launch,
+quantize and run O, quantize once and run gate and up in one launch, quantize and
+run down (Q6_K); then quantize the final hidden state and run the 126464-wide output
+projection (Q6_K) on the 32 rows of the current block only.  Weights are random
+(the GGUF Q4_K / Q6_K distributions of the synthetic workloads), drawn on the device,
+repacked once and kept resident (4.77 GB, far above the 126 MB L2, so every step
+streams them from HBM).
+
+One JSON line on rank 0.  `value` is algorithmic int8 TOPS (2*M*N*K summed over the
+step's GEMMs) over the device-timed step; `ms_per_step` is the step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--model llada-8b|dream-7b] [--canvas L] [--layers n]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "int8 TOPS & weight GB/s of dllm_qgemm (% roofline); ms/LLaDA-8B-shaped step"
+UNIT = "int8 TOPS"
+PEAKS_FILE = ROOT / "MEASURED_PEAKS.json"
+TRAFFIC_FILE = ROOT / "profiles" / "qgemm_dram_traffic.json"
+FALLBACK_HBM_GBS = 6650.0
+Q4, Q6 = 12, 14
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=500)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--model", default="llada-8b")
+    p.add_argument("--canvas", type=int, default=128)
+    p.add_argument("--layers", type=int, default=None, help="override the layer count (small profiling cases)")
+    p.add_argument("--cpu-layers", type=int, default=4, help="layers in the oracle's timed sample")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------- workload
+
+class Gemm:
+    def __init__(self, name, qtype, N, K, M_out, M_act, nseg=1):
+        self.name, self.qtype, self.N, self.K, self.M_out, self.M_act = name, qtype, N, K, M_out, M_act
+
+    @property
+    def ops(self):
+        return 2 * self.M_out * self.N * self.K
+
+    @property
+    def weight_bytes(self):
+        return self.N * (self.K // 256) * (144 if self.qtype == Q4 else 210)
+
+    @property
+    def bytes(self):
+        per = 1 + 4 / 256 + (16 / 256 if self.qtype == Q4 else 0)
+        return self.weight_bytes + self.M_act * self.K * per + self.M_out * self.N * 4
+
+
+def step_gemms(model, L, n_layers):
+    """The GEMM launches of one step, in order (QKV and gate/up are single launches)."""
+    h, f = model.hidden, model.ffn
+    per_layer = [Gemm("qkv", Q4, model.q_out + 2 * model.kv_out, h, L, L),
+                 Gemm("o", Q4, h, h, L, L),
+                 Gemm("gate_up", Q4, 2 * f, h, L, L),
+                 Gemm("down", Q6, h, f, L, L)]
+    return per_layer * n_layers + [Gemm("output", Q6, model.vocab, h, model.out_rows, model.out_rows)]
+
+
+def roofline_time(gemms, hbm_gbs, p_int8):
+    return sum(max(g.bytes / (hbm_gbs * 1e9), g.ops / p_int8) for g in gemms)
+
+
+def load_peaks():
+    if PEAKS_FILE.exists():
+        d = json.loads(PEAKS_FILE.read_text())
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for p in sorted((ROOT / "quantized_int8_gemm_q4_b200" / "csrc").glob("*.cu*")):
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload_key):
+    """Per-launch DRAM bytes of the GEMM kernel from a stored ncu capture, if it was
+    taken on the current kernel source; otherwise None."""
+    if not TRAFFIC_FILE.exists():
+        return None
+    d = json.loads(TRAFFIC_FILE.read_text())
+    if d.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    return d.get("per_launch_bytes", {}).get(workload_key)
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in Path(self.path).read_text().splitlines():
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world):
+    import torch
+    from quantized_int8_gemm_q4_b200 import build, dllm, synth
+
+    build.build()
+    dllm.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    model = synth.MODELS[args.model]()
+    n_layers = args.layers or model.n_layers
+    L = args.canvas
+    h, f = model.hidden, model.ffn
+    seed = 4  # the full-step workload's seed
+
+    # ---- weights: draw GGUF blocks on the device, repack once, keep resident
+    cpu_sample = {}
+    layers = []
+    for l in range(n_layers):
+        mats = {}
+        for pi, p in enumerate(model.layer):
+            g = synth.device_weights(p.qtype, p.N, p.K, seed, l, pi, device=dev)
+            if l < args.cpu_layers and rank == 0 and not args.no_cpu:
+                cpu_sample.setdefault(l, {})[p.name] = (p, g.cpu().numpy())
+            w = torch.empty(dllm.dllm_repacked_bytes(p.qtype, p.N, p.K), dtype=torch.uint8, device=dev)
+            (dllm.dllm_repack_q4k if p.qtype == Q4 else dllm.dllm_repack_q6k)(g, p.N, p.K, w)
+            del g
+            mats[p.name] = w
+        layers.append(mats)
+    g = synth.device_weights(Q6, model.vocab, h, seed, 999, 0, device=dev)
+    if rank == 0 and not args.no_cpu:
+        cpu_sample["output"] = g.cpu().numpy()
+    w_out = torch.empty(dllm.dllm_repacked_bytes(Q6, model.vocab, h), dtype=torch.uint8, device=dev)
+    dllm.dllm_repack_q6k(g, model.vocab, h, w_out)
+    del g
+    torch.cuda.synchronize()
+
+    # ---- activations (the f32 inputs of each projection), one contiguous buffer
+    sizes = [L * h, L * h, L * h, L * f, L * h]
+    xin = torch.empty(sum(sizes), dtype=torch.float32, device=dev)
+    views, off = [], 0
+    for i, sz in enumerate(sizes):
+        v = xin[off:off + sz].view(L, -1)
+        v.copy_(synth.device_activations(L, sz // L, seed, 100 + i, device=dev))
+        views.append(v)
+        off += sz
+    x_attn, x_o, x_ffn, x_down, x_fin = views
+    act_h = dllm.alloc_act(L, h, dev)
+    act_f = dllm.alloc_act(L, f, dev)
+    o_q = torch.empty((L, model.q_out), device=dev)
+    o_k = torch.empty((L, model.kv_out), device=dev)
+    o_v = torch.empty((L, model.kv_out), device=dev)
+    o_o = torch.empty((L, h), device=dev)
+    o_g = torch.empty((L, f), device=dev)
+    o_u = torch.empty((L, f), device=dev)
+    o_d = torch.empty((L, h), device=dev)
+    rows_np = synth.block_rows(L, model.out_rows, seed) if L >= 64 else np.arange(min(L, model.out_rows),
+                                                                                     dtype=np.int32)
+    rows = torch.from_numpy(rows_np).to(dev)
+    logits = torch.empty((len(rows_np), model.vocab), device=dev)
+    # one zero-filled workspace, large enough for every GEMM of the step (stream-ordered)
+    wsb = max(dllm.dllm_qgemm_workspace_bytes(Q4, model.q_out + 2 * model.kv_out, h, L),
+              dllm.dllm_qgemm_workspace_bytes(Q4, h, h, L),
+              dllm.dllm_qgemm_workspace_bytes(Q4, 2 * f, h, L),
+              dllm.dllm_qgemm_workspace_bytes(Q6, h, f, L),
+              dllm.dllm_qgemm_workspace_bytes(Q6, model.vocab, h, L, len(rows_np)))
+    ws = dllm.alloc_workspace(max(wsb, 256), dev)
+
+    def step(ev=None):
+        k = 0
+
+        def mark():
+            nonlocal k
+            if ev is not None:
+                ev[k].record()
+                k += 1
+
+        for l in range(n_layers):
+            W = layers[l]
+            dllm.dllm_quantize_act(x_attn, L, h, h, *act_h)
+            mark()
+            dllm.dllm_qkv_qgemm(W["q"], W["k"], W["v"], Q4, model.q_out, model.kv_out, h, *act_h, L,
+                                o_q, model.q_out, o_k, o_v, model.kv_out, ws, wsb)
+            mark()
+            dllm.dllm_quantize_act(x_o, L, h, h, *act_h)
+            mark()
+            dllm.dllm_qgemm(W["o"], Q4, h, h, *act_h, L, None, 0, o_o, h, ws, wsb)
+            mark()
+            dllm.dllm_quantize_act(x_ffn, L, h, h, *act_h)
+            mark()
+            dllm.dllm_qkv_qgemm(W["gate"], W["up"], None, Q4, f, f, h, *act_h, L, o_g, f, o_u, None, f, ws, wsb)
+            mark()
+            dllm.dllm_quantize_act(x_down, L, f, f, *act_f)
+            mark()
+            dllm.dllm_qgemm(W["down"], Q6, h, f, *act_f, L, None, 0, o_d, h, ws, wsb)
+            mark()
+        dllm.dllm_quantize_act(x_fin, L, h, h, *act_h)
+        mark()
+        dllm.dllm_qgemm(w_out, Q6, model.vocab, h, *act_h, L, rows, len(rows_np), logits, model.vocab, ws, wsb)
+        mark()
+
+    launches_per_step = n_layers * 8 + 3  # + the row gather of the output projection
+    gemms = step_gemms(model, L, n_layers)
+
+    # eager warm-up of every kernel (attribute setup happens outside capture)
+    step()
+    torch.cuda.synchronize()
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+    S = max(1, min(args.steps, 10))
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=s):
+        step()
+    n_marks = 2 * len(gemms)
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks)] for _ in range(S)]
+    gS = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gS, stream=s):
+        for i in range(S):
+            step(evs[i])
+    torch.cuda.synchronize()
+
+    # ---- warm-up: W steps
+    with torch.cuda.stream(s):
+        for _ in range(args.warmup):
+            g1.replay()
+        gS.replay()  # first replay of the timed graph also uploads it (untimed)
+    torch.cuda.synchronize()
+
+    sampler = None
+    if rank == 0:
+        sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+        sampler.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        t0.record(s)
+        for _ in range(args.steps // S):
+            gS.replay()
+        for _ in range(args.steps % S):
+            g1.replay()
+        t1.record(s)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+    # per-launch GEMM durations from the last S timed steps (events inside the graph)
+    gemm_ms = 0.0
+    quant_ms = 0.0
+    if args.steps >= S:
+        for i in range(S):
+            e = evs[i]
+            # marks: after quantize (even index), after gemm (odd index)
+            prev = None
+            for j in range(0, n_marks, 2):
+                if j > 0:
+                    quant_ms += e[j - 1].elapsed_time(e[j])
+                gemm_ms += e[j].elapsed_time(e[j + 1])
+        gemm_ms /= S
+        quant_ms /= S
+
+    ms_step = elapsed_ms / args.steps
+    ops_step = sum(g.ops for g in gemms)
+    wbytes_step = sum(g.weight_bytes for g in gemms)
+    abytes_step = sum(g.bytes for g in gemms)
+    hbm_gbs, peak_kind = load_peaks()
+    p_int8 = 4.5e15
+    tstar = roofline_time(gemms, hbm_gbs, p_int8)
+    value = ops_step * world / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e and rank == 0:
+        x_host = torch.empty(xin.numel(), dtype=torch.float32, pin_memory=True)
+        x_host.copy_(xin.cpu())
+        out_host = torch.empty(logits.shape, dtype=torch.float32, pin_memory=True)
+        ke = max(1, min(args.steps, 100))
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            for it in range(ke + 1):
+                if it == 1:
+                    a0.record(s)
+                xin.copy_(x_host, non_blocking=True)
+                g1.replay()
+                out_host.copy_(logits, non_blocking=True)
+            a1.record(s)
+        torch.cuda.synchronize()
+        ms_e2e = a0.elapsed_time(a1) / ke
+        e2e = {"value": ops_step / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": int(xin.numel() * 4), "d2h_bytes_per_step": int(logits.numel() * 4)}
+
+    traffic = stored_traffic(f"{args.model}_L{L}")
+    roof = None
+    if gemm_ms > 0:
+        achieved = abytes_step / (gemm_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
+                "frac": round(achieved / hbm_gbs, 4), "traffic": traffic,
+                "kernel": "qgemm_kernel", "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                "launches_per_step": len(gemms), "gemm_ms_per_step": round(gemm_ms, 4),
+                "algorithmic_bytes_per_step": int(abytes_step)}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu and cpu_sample:
+        cpu = cpu_baseline(model, L, cpu_sample, rows_np, seed)
+
+    del gS, g1
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": f"{model.name}-shaped denoising step: {n_layers} layers (QKV, O, gate/up Q4_K; "
+                               f"down Q6_K) + output projection (Q6_K, {model.vocab} wide) on "
+                               f"{len(rows_np)} requested rows",
+                   "canvas_tokens": L, "layers": n_layers, "weight_bytes_per_step": int(wbytes_step),
+                   "l2": "inputs larger than L2: every step streams all weights from HBM",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "graph": "one CUDA graph per step, replayed"},
+        "weight_gbs": round(wbytes_step / (ms_step * 1e-3) / 1e9, 1),
+        "step_roofline": {"t_star_ms": round(tstar * 1e3, 4), "frac": round(tstar * 1e3 / ms_step, 4),
+                          "p_int8_tops": p_int8 / 1e12, "hbm_gbs": hbm_gbs},
+        "gemm_ms_per_step": round(gemm_ms, 4), "quantize_ms_per_step": round(quant_ms, 4),
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    return result
+
+
+def cpu_baseline(model, L, sample, rows_np, seed, max_threads=None):
+    """The oracle, as it stands, on a bounded sample of the same step: the projection
+    sets of the first few layers and the output projection on the requested rows."""
+    import oracle
+    from quantized_int8_gemm_q4_b200 import synth
+    nt = max_threads or oracle.max_threads()
+    h, f = model.hidden, model.ffn
+    x = {"attn": synth.activations(L, h, seed, 100), "o": synth.activations(L, h, seed, 101),
+         "ffn": synth.activations(L, h, seed, 102), "down": synth.activations(L, f, seed, 103),
+         "fin": synth.activations(L, h, seed, 104)}
+    src = {"q": "attn", "k": "attn", "v": "attn", "o": "o", "gate": "ffn", "up": "ffn", "down": "down"}
+    ops = 0
+    t0 = time.perf_counter()
+    qa = {k: oracle.quantize_act(v)[:2] for k, v in x.items()}
+    nl = 0
+    for l, mats in sample.items():
+        if l == "output":
+            continue
+        nl += 1
+        for name, (p, blocks) in mats.items():
+            q, s = qa[src[name]]
+            oracle.qgemm(p.qtype, blocks, p.N, p.K, q, s, nthreads=nt)
+            ops += 2 * L * p.N * p.K
+    if "output" in sample:
+        q, s = qa["fin"]
+        oracle.qgemm(Q6, sample["output"], model.vocab, h, q, s, rows=rows_np, nthreads=nt)
+        ops += 2 * len(rows_np) * model.vocab * h
+    dt = time.perf_counter() - t0
+    return {"value": round(ops / dt / 1e12, 6), "unit": UNIT, "cores": nt, "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"{nl} of {model.n_layers} layers' projection sets + output projection on "
+                      f"{len(rows_np)} rows, canvas {L} (quantize included)"}
+
+
+# ---------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The oracle on the host cores: same metric on bounded samples of the workload."""
+    import oracle
+    from quantized_int8_gemm_q4_b200 import synth
+    model = synth.MODELS[args.model]()
+    L, h, seed = args.canvas, model.hidden, 4
+    nt = oracle.max_threads()
+    p = model.layer[0]  # the Q projection of layer 0
+    w = synth.weights(p.qtype, p.N, p.K, seed, 0)
+    q, s, _ = oracle.quantize_act(synth.activations(L, h, seed, 100))
+    # size one step so that warm-up + steps take about two minutes
+    t0 = time.perf_counter()
+    oracle.qgemm(p.qtype, w, p.N, p.K, q, s, n0=0, n1=256, nthreads=nt)
+    per_col = (time.perf_counter() - t0) / 256
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    ncols = int(max(128, min(p.N, budget / max(per_col, 1e-9))) // 128 * 128)
+    for i in range(args.warmup):
+        oracle.qgemm(p.qtype, w, p.N, p.K, q, s, n0=0, n1=ncols, nthreads=nt)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        n0 = (i * ncols) % p.N
+        n1 = min(p.N, n0 + ncols)
+        oracle.qgemm(p.qtype, w, p.N, p.K, q, s, n0=n0, n1=n1, nthreads=nt)
+    dt = time.perf_counter() - t0
+    ops = 2 * L * ncols * p.K * args.steps
+    v = ops / dt / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": f"{model.name}-shaped denoising step (oracle sample)", "canvas_tokens": L},
+        "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": nt, "kind": "oracle",
+                         "sample": f"per step: {ncols} of {p.N} output columns of the layer-0 Q projection, "
+                                   f"M={L}, K={p.K}"},
+        "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_ours(args, rank, world)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -111,10 +111,17 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  *                  runs only on the requested rows.)
  * ldo >= N, ldo % 4 == 0.  Results are deterministic and do not depend on M or on the
  * row set: a gathered row equals the same row of the full-canvas result bit for bit.
- * workspace: optional device scratch (may be NULL with workspace_bytes 0); reserved
- * for split-K scheduling, see dllm_qgemm_workspace_bytes().
+ *
+ * workspace: device scratch owned by the caller, at least dllm_qgemm_workspace_bytes()
+ * bytes (that size may be 0, and then workspace may be NULL); otherwise the call
+ * returns DLLM_ERR_WORKSPACE.  It holds the gathered rows and, when a tile's K range
+ * is split over several CTAs, their partial sums and one arrival counter per tile.
+ * It must be zero-filled before its first use; every call that completes leaves the
+ * counters as it found them (a call that ends in DLLM_ERR_TIMEOUT may not, so zero
+ * it again after one).  Calls that share a workspace must be ordered on one stream.
+ * For dllm_qkv_qgemm pass N = Nq + 2*Nkv (Nq + Nkv without wv) and n_rows = 0.
  * ---------------------------------------------------------------------------- */
-int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, size_t* bytes);
+int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, int64_t n_rows, size_t* bytes);
 int dllm_qgemm(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
                const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows, float* out, int64_t ldo,
                void* workspace, size_t workspace_bytes, dllm_stream_t stream);
@@ -152,13 +159,13 @@ int dllm_debug_subblock_dots(const void* w, dllm_qtype t, int64_t N, int64_t K, 
 int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
                        const uint8_t* sums, int64_t M, int32_t* S, int32_t* Smin, dllm_stream_t stream);
 
-/* int8 tensor-core throughput probe: `iters` back-to-back tcgen05 kind::i8 MMAs of
- * 128 x n x 32 per CTA on `ctas` CTAs, rotating over n_acc independent accumulators,
- * with A in tensor memory (a_from_tmem != 0) or in shared memory.  Writes elapsed
- * device nanoseconds per CTA to ns_out (device, [ctas] uint64).
- * 16 <= n <= 256, n % 16 == 0, n * n_acc <= 448. */
-int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int iters, int ctas, unsigned long long* ns_out,
-                      dllm_stream_t stream);
+/* int8 tensor-core throughput probe: on each of `ctas` CTAs, `issuers` warps (1..4)
+ * each issue `iters` back-to-back tcgen05 kind::i8 MMAs of 128 x n x 32 into their own
+ * n_acc accumulators, with A in tensor memory (a_from_tmem != 0) or shared memory.
+ * Writes elapsed device nanoseconds per CTA to ns_out (device, [ctas] uint64).
+ * 16 <= n <= 256, n % 16 == 0, n * n_acc * issuers <= 448, iters % 8 == 0. */
+int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int issuers, int iters, int ctas,
+                      unsigned long long* ns_out, dllm_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -39,6 +39,60 @@ int grid_for(int64_t work, int64_t per_block) {
     return (int)(g < 1 ? 1 : g);
 }
 
+// K-chunks per tile.  A function of the tile count, the super-block count and the
+// SM count only (never of M or of a row list), so that every call on the same
+// weight shape sums the same partials in the same order.  Cost model in units of one
+// super-block of one tile: the busiest SM's share, plus one unit per chunk for
+// writing and re-reading its partial; chunks are at least 4 super-blocks long.
+int choose_kc(int64_t n_tiles, int64_t nsb, int sms) {
+    int best = 1;
+    int64_t best_cost = -1;
+    for (int kc = 1; kc <= MAX_KC && kc <= nsb; kc++) {
+        const int64_t len = (nsb + kc - 1) / kc;
+        if (kc > 1 && len < 4) break;
+        const int64_t waves = (n_tiles * kc + sms - 1) / sms;
+        const int64_t cost = waves * (len + (kc > 1 ? 1 : 0));
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = kc;
+        }
+    }
+    return best;
+}
+
+struct Plan {
+    int kc, n_st, mu;
+    int64_t Mp;        // activation rows seen by the GEMM
+    size_t ctr_off, part_off, gq_off, gs_off, gu_off, bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
+    Plan p;
+    const int64_t nsb = K / QK;
+    p.Mp = round_up(n_rows > 0 ? n_rows : M, 16);
+    p.kc = choose_kc(n_tiles, nsb, sms);
+    p.n_st = (int)((p.Mp + UNIT_TOKENS - 1) / UNIT_TOKENS);
+    p.mu = (int)round_up((p.Mp + p.n_st - 1) / p.n_st, 16);
+    size_t off = 0;
+    p.ctr_off = off;
+    off += align256((size_t)n_tiles * p.n_st * 4);
+    p.part_off = off;
+    if (p.kc > 1) off += align256((size_t)n_tiles * p.n_st * p.kc * p.mu * TROWS * 4);
+    p.gq_off = p.gs_off = p.gu_off = off;
+    if (n_rows > 0) {
+        p.gq_off = off;
+        off += align256((size_t)p.Mp * K);
+        p.gs_off = off;
+        off += align256((size_t)nsb * p.Mp * 4);
+        p.gu_off = off;
+        off += align256((size_t)nsb * p.Mp * 16);
+    }
+    p.bytes = (p.kc > 1 || n_rows > 0) ? off : 0;
+    return p;
+}
+
 template <int QT, bool DBG>
 int run_gemm(GemmArgs& a, cudaStream_t s) {
     int dev;
@@ -52,10 +106,7 @@ int run_gemm(GemmArgs& a, cudaStream_t s) {
             return DLLM_ERR_CUDA;
         g_attr_done[dev][slot] = true;
     }
-    const int64_t rows_total = a.rows ? round_up(a.n_rows, 16) : a.Mp;
-    a.n_st = (int32_t)((rows_total + UNIT_TOKENS - 1) / UNIT_TOKENS);
-    a.mu = (int32_t)round_up((rows_total + a.n_st - 1) / a.n_st, 16);
-    const int64_t units = (int64_t)a.n_tiles * a.n_st;
+    const int64_t units = (int64_t)a.n_tiles * a.n_st * a.kc;
     const int grid = (int)(units < g_num_sms[dev] ? units : g_num_sms[dev]);
     qgemm_kernel<QT, DBG><<<grid, GEMM_THREADS, smem, s>>>(a);
     return launch_status();
@@ -137,36 +188,68 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     return launch_status();
 }
 
-int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, size_t* bytes) {
+int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, int64_t n_rows, size_t* bytes) {
     int rc = check_shape(t, N, K);
     if (rc) return rc;
-    if (M <= 0 || !bytes) return DLLM_ERR_ARG;
-    *bytes = 0;  // the current schedule needs no scratch
+    if (M <= 0 || n_rows < 0 || n_rows > 32 || !bytes) return DLLM_ERR_ARG;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    *bytes = make_plan(N / TROWS, K, M, n_rows, g_num_sms[dev]).bytes;
     return DLLM_OK;
 }
 
-static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
-                       const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows) {
-    int rc = check_shape(t, N, K);
+// Validates the activation arguments and fills the parts of the launch that do not
+// depend on the weights; gathers requested rows into the workspace first.
+static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, const int8_t* q, const float* scale,
+                       const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows, void* workspace,
+                       size_t workspace_bytes, bool dbg, cudaStream_t s) {
+    int rc = check_shape(t, N_total, K);
     if (rc) return rc;
     if ((rc = check_act(q, scale, sums, M))) return rc;
     if (rows && (n_rows < 1 || n_rows > 32)) return DLLM_ERR_ARG;
+    if (rows && !aligned16(rows)) return DLLM_ERR_ALIGN;
     if (M > (1LL << 31)) return DLLM_ERR_ARG;
+    if (workspace && !aligned16(workspace)) return DLLM_ERR_ALIGN;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    Plan p = make_plan(N_total / TROWS, K, M, rows ? n_rows : 0, g_num_sms[dev]);
+    if (dbg) {  // integers per super-block: no chunk partials to combine
+        p.kc = 1;
+        if (!rows) p.bytes = 0;
+    }
+    if (p.bytes > 0 && (!workspace || workspace_bytes < p.bytes)) return DLLM_ERR_WORKSPACE;
     memset(&a, 0, sizeof(a));
-    a.nsb = (int32_t)(K / QK);
+    const int64_t nsb = K / QK;
+    a.nsb = (int32_t)nsb;
+    a.kc = p.kc;
+    a.n_st = p.n_st;
+    a.mu = p.mu;
+    a.Mp = p.Mp;
+    a.m_out = rows ? n_rows : M;
     a.q = q;
     a.scale = scale;
     a.sums = sums;
-    a.M = M;
-    a.Mp = round_up(M, 16);
-    a.rows = rows;
-    a.n_rows = rows ? (int32_t)n_rows : 0;
-    a.m_out = rows ? n_rows : M;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (p.kc > 1) {
+        a.counters = reinterpret_cast<uint32_t*>(ws + p.ctr_off);
+        a.partials = reinterpret_cast<float*>(ws + p.part_off);
+    }
+    if (rows) {
+        int8_t* gq = reinterpret_cast<int8_t*>(ws + p.gq_off);
+        float* gs = reinterpret_cast<float*>(ws + p.gs_off);
+        uint8_t* gu = ws + p.gu_off;
+        const int64_t work = nsb * p.Mp * 18;
+        gather_rows_kernel<<<grid_for(work, 256), 256, 0, s>>>(q, scale, sums, M, round_up(M, 16), rows,
+                                                                (int32_t)n_rows, p.Mp, (int32_t)nsb, gq, gs, gu);
+        if ((rc = launch_status())) return rc;
+        a.q = gq;
+        a.scale = gs;
+        a.sums = gu;
+    }
     return DLLM_OK;
 }
 
-static int dispatch(GemmArgs& a, dllm_qtype t, bool dbg, dllm_stream_t stream) {
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+static int dispatch(GemmArgs& a, dllm_qtype t, bool dbg, cudaStream_t s) {
     if (t == DLLM_Q4_K) return dbg ? run_gemm<12, true>(a, s) : run_gemm<12, false>(a, s);
     return dbg ? run_gemm<14, true>(a, s) : run_gemm<14, false>(a, s);
 }
@@ -174,34 +257,34 @@ static int dispatch(GemmArgs& a, dllm_qtype t, bool dbg, dllm_stream_t stream) {
 int dllm_qgemm(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
                const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows, float* out, int64_t ldo,
                void* workspace, size_t workspace_bytes, dllm_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
-    GemmArgs a;
-    int rc = gemm_common(a, t, N, K, q, scale, sums, M, rows, n_rows);
-    if (rc) return rc;
     if (!w || !out || ldo < N) return DLLM_ERR_ARG;
     if (!aligned16(w) || !aligned16(out) || ldo % 4) return DLLM_ERR_ALIGN;
-    if (rows && !aligned16(rows)) return DLLM_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    GemmArgs a;
+    int rc = gemm_common(a, t, N, K, q, scale, sums, M, rows, n_rows, workspace, workspace_bytes, false, s);
+    if (rc) return rc;
     a.seg[0] = Segment{static_cast<const uint8_t*>(w), out, ldo, 0};
     a.nseg = 1;
     a.n_tiles = (int32_t)(N / TROWS);
-    return dispatch(a, t, false, stream);
+    return dispatch(a, t, false, s);
 }
 
 int dllm_qkv_qgemm(const void* wq, const void* wk, const void* wv, dllm_qtype t, int64_t Nq, int64_t Nkv, int64_t K,
                    const int8_t* q, const float* scale, const uint8_t* sums, int64_t M, float* oq, int64_t ldo_q,
                    float* ok, float* ov, int64_t ldo_kv, void* workspace, size_t workspace_bytes,
                    dllm_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
-    GemmArgs a;
-    int rc = gemm_common(a, t, Nq, K, q, scale, sums, M, nullptr, 0);
+    int rc = check_shape(t, Nq, K);
     if (rc) return rc;
     if ((rc = check_shape(t, Nkv, K))) return rc;
     if (!wq || !wk || !oq || !ok || (wv && !ov) || ldo_q < Nq || ldo_kv < Nkv) return DLLM_ERR_ARG;
     if (!aligned16(wq) || !aligned16(wk) || (wv && !aligned16(wv)) || !aligned16(oq) || !aligned16(ok) ||
         (wv && !aligned16(ov)) || ldo_q % 4 || ldo_kv % 4)
         return DLLM_ERR_ALIGN;
+    const int64_t N_total = Nq + (wv ? 2 : 1) * Nkv;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    GemmArgs a;
+    rc = gemm_common(a, t, N_total, K, q, scale, sums, M, nullptr, 0, workspace, workspace_bytes, false, s);
+    if (rc) return rc;
     const int32_t tq = (int32_t)(Nq / TROWS), tkv = (int32_t)(Nkv / TROWS);
     a.seg[0] = Segment{static_cast<const uint8_t*>(wq), oq, ldo_q, 0};
     a.seg[1] = Segment{static_cast<const uint8_t*>(wk), ok, ldo_kv, tq};
@@ -212,7 +295,7 @@ int dllm_qkv_qgemm(const void* wq, const void* wk, const void* wv, dllm_qtype t,
         a.nseg = 3;
         a.n_tiles += tkv;
     }
-    return dispatch(a, t, false, stream);
+    return dispatch(a, t, false, s);
 }
 
 int dllm_get_device_status(dllm_stream_t stream) {
@@ -290,17 +373,18 @@ __global__ void subblock_dots_kernel(const uint8_t* __restrict__ w, int qt, int6
 }
 
 // Back-to-back 128 x n x 32 int8 MMAs, B in shared memory, A in tensor memory
-// (a_tmem != 0) or shared memory, rotating over n_acc independent accumulators.
-__global__ void __launch_bounds__(128, 1) bench_mma_kernel(int n, int n_acc, int a_tmem, int iters,
+// (a_tmem != 0) or shared memory.  `issuers` warps each issue `iters` MMAs (eight
+// per loop trip, addresses precomputed) into their own n_acc accumulators.
+__global__ void __launch_bounds__(128, 1) bench_mma_kernel(int n, int n_acc, int a_tmem, int iters, int issuers,
                                                            unsigned long long* ns_out) {
     extern __shared__ __align__(1024) uint8_t bsm[];
     __shared__ uint32_t tbase;
-    __shared__ __align__(8) uint64_t bar;
-    const int warp = threadIdx.x >> 5;
+    __shared__ __align__(8) uint64_t bar[4];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < (256 * 32 + 128 * 32) / 4; i += blockDim.x)
         reinterpret_cast<uint32_t*>(bsm)[i] = 0x01010101u;
     if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
+        for (int i = 0; i < 4; i++) mbar_init(&bar[i], 1);
         fence_mbar_init();
     }
     fence_proxy_async_smem();
@@ -312,25 +396,36 @@ __global__ void __launch_bounds__(128, 1) bench_mma_kernel(int n, int n_acc, int
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tbase;
-    if (threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    if (lane == 0 && warp < issuers) {
         const uint32_t id = idesc_i8(128, n, 0, 1);
         const uint64_t bd = sdesc_kmajor_noswz(smem_u32(bsm), 128, 256);
         const uint64_t ad = sdesc_kmajor_noswz(smem_u32(bsm + 256 * 32), 128, 256);
-        const uint64_t t0 = globaltimer_ns();
-        for (int i = 0; i < iters; i++) {
-            const uint32_t d = tm + (uint32_t)((i % n_acc) * n);
-            if (a_tmem)
-                mma_i8_ts(d, tm + 448 + 8 * (i & 7), bd, id, i >= n_acc);
-            else
-                mma_i8_ss(d, ad, bd, id, i >= n_acc);
+        uint32_t dk[8], ak[8];
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            dk[k] = tm + (uint32_t)(warp * n * n_acc + (k % n_acc) * n);
+            ak[k] = tm + 448 + 8 * k;
         }
-        tc_commit(&bar);
+        if (a_tmem) {
+            for (int i = 0; i < iters; i += 8) {
+#pragma unroll
+                for (int k = 0; k < 8; k++) mma_i8_ts(dk[k], ak[k], bd, id, 1);
+            }
+        } else {
+            for (int i = 0; i < iters; i += 8) {
+#pragma unroll
+                for (int k = 0; k < 8; k++) mma_i8_ss(dk[k], ad, bd, id, 1);
+            }
+        }
+        tc_commit(&bar[warp]);
         uint64_t tw = globaltimer_ns();
-        while (!mbar_try_wait(&bar, 0)) {
+        while (!mbar_try_wait(&bar[warp], 0)) {
             if (globaltimer_ns() - tw > WAIT_LIMIT_NS) { set_err(ERR_TIMEOUT); break; }
         }
-        ns_out[blockIdx.x] = globaltimer_ns() - t0;
     }
+    __syncthreads();
+    if (threadIdx.x == 0) ns_out[blockIdx.x] = globaltimer_ns() - t0;
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -358,23 +453,24 @@ int dllm_debug_subblock_dots(const void* w, dllm_qtype t, int64_t N, int64_t K, 
 
 int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
                        const uint8_t* sums, int64_t M, int32_t* S, int32_t* Smin, dllm_stream_t stream) {
-    GemmArgs a;
-    int rc = gemm_common(a, t, N, K, q, scale, sums, M, nullptr, 0);
-    if (rc) return rc;
     if (!w || !S || (t == DLLM_Q4_K && !Smin)) return DLLM_ERR_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    GemmArgs a;
+    int rc = gemm_common(a, t, N, K, q, scale, sums, M, nullptr, 0, nullptr, 0, true, s);
+    if (rc) return rc;
     a.seg[0] = Segment{static_cast<const uint8_t*>(w), nullptr, N, 0};
     a.nseg = 1;
     a.n_tiles = (int32_t)(N / TROWS);
     a.dbg_S = S;
     a.dbg_Smin = Smin;
     a.dbg_N = N;
-    return dispatch(a, t, true, stream);
+    return dispatch(a, t, true, s);
 }
 
-int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int iters, int ctas, unsigned long long* ns_out,
-                      dllm_stream_t stream) {
-    if (n < 16 || n > 256 || n % 16 || n_acc < 1 || n * n_acc > 448 || iters < 1 || ctas < 1 || ctas > 4096 ||
-        !ns_out)
+int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int issuers, int iters, int ctas,
+                      unsigned long long* ns_out, dllm_stream_t stream) {
+    if (n < 16 || n > 256 || n % 16 || n_acc < 1 || n_acc > 8 || issuers < 1 || issuers > 4 ||
+        n * n_acc * issuers > 448 || iters < 8 || iters % 8 || ctas < 1 || ctas > 4096 || !ns_out)
         return DLLM_ERR_ARG;
     int dev;
     int rc = current_device(&dev);
@@ -383,7 +479,7 @@ int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int iters, int ctas, un
     if (cudaFuncSetAttribute(bench_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return DLLM_ERR_CUDA;
     bench_mma_kernel<<<ctas, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(n, n_acc, a_from_tmem, iters,
-                                                                                  ns_out);
+                                                                                  issuers, ns_out);
     return launch_status();
 }
 

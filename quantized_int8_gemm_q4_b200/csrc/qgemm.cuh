@@ -19,23 +19,33 @@
 // and the per-32 activation sums, split into an unsigned low byte and a signed high
 // byte, as B: Smin = Ml + 256*Mh.
 //
-// Every integer accumulator stays within 2^22 in magnitude.  Tensor memory is
-// preset to the bit pattern of 1.5*2^23 before each super-block, so the int32 the
-// MMAs leave there, read as an f32, is exactly 1.5*2^23 + value; the epilogue turns
-// it into floats with one FFMA and one FADD per pair of accumulators, with no
-// integer-to-float conversion instruction.
+// Every integer accumulator stays within 2^22 in magnitude.  Tensor memory is preset
+// to the bit pattern of 1.5*2^23 before each super-block, so the int32 the MMAs
+// leave there, read as an f32, is exactly 1.5*2^23 + value; the epilogue turns it
+// into floats with one FFMA and one FADD per pair of accumulators (no
+// integer-to-float conversion instruction), in packed f32x2 arithmetic.
 //
 // Roles (16 warps, one CTA per SM, persistent over work units):
 //   warp 0      producer: bulk copies of weight tiles and activation tiles into
-//               shared-memory rings (or a gather of requested rows)
-//   warp 1      tensor-memory allocation, and one thread issuing every tcgen05.mma
+//               shared-memory rings
+//   warps 1-3   tensor-memory allocation (warp 1) and MMA issue.  One thread can
+//               issue a tcgen05.mma only every ~28 ns, longer than a 48-token MMA
+//               takes, so three warps share the work: for each token tile the roles
+//               plane 0, plane 1 and min term rotate over them, each role owning its
+//               own accumulators, and a role's MMAs go out back to back with
+//               precomputed descriptors
 //   warps 4-7   unpack: thread = weight row; decode the super-block, build the two
-//               weight planes for each K-step of 32 and store them into tensor
-//               memory (the A operand), plus the mins and the f32 d/dmin
+//               weight planes per K-step of 32 into tensor memory (the A operand),
+//               the mins into shared memory, and the f32 d/dmin
 //   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each on half of
-//               the token columns; per super-block, read the integer accumulators,
-//               preset them again, and accumulate the f32 result in registers
-// A work unit is (128 weight rows, up to 128 canvas rows, all of K).
+//               the token columns; per super-block, read the integer accumulators in
+//               a few wide loads, preset them again, and accumulate the f32 result in
+//               registers
+//
+// A work unit is (128 weight rows, up to 128 canvas rows, one K-chunk).  The number
+// of K-chunks per tile depends only on N, K and the SM count, never on M or on the
+// rows requested, and chunk partials are summed in chunk order by whichever CTA
+// finishes a tile last; so results are deterministic and the same for every M.
 #pragma once
 #include "layout.cuh"
 
@@ -45,6 +55,7 @@ constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float MAGIC = 12582912.0f;
 constexpr int GEMM_THREADS = 512;
 constexpr int UNIT_TOKENS = 128;
+constexpr int MAX_KC = 16;                         // K-chunks per tile, at most
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 
 template <int QT>
@@ -52,13 +63,14 @@ struct GemmCfg;
 template <>
 struct GemmCfg<12> {  // Q4_K
     static constexpr int TILE = Q4K_TILE;
-    static constexpr int NTOK = 32;  // token columns per MMA and per accumulator
+    static constexpr int NTOK = 48;  // token columns per MMA and per accumulator
     static constexpr int NACC = 4;   // P0, P1, Ml, Mh
     static constexpr int W_STAGES = 4;
-    static constexpr int B_STAGES = 8;
+    static constexpr int B_STAGES = 6;
     static constexpr int B_Q = NTOK * 256;
     static constexpr int B_SUMS = NTOK * 16 + 128;
-    static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
+    static constexpr int B_STAGE = (B_Q + B_SUMS + NTOK * 4 + 127) / 128 * 128;
+    static constexpr int MINA = 2 * 4096;  // [Ml-A | Mh-A], canonical K-major 128 rows x 32 B
 };
 template <>
 struct GemmCfg<14> {  // Q6_K
@@ -69,40 +81,41 @@ struct GemmCfg<14> {  // Q6_K
     static constexpr int B_STAGES = 4;
     static constexpr int B_Q = NTOK * 256;
     static constexpr int B_SUMS = 0;
-    static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
+    static constexpr int B_STAGE = (B_Q + B_SUMS + NTOK * 4 + 127) / 128 * 128;
+    static constexpr int MINA = 0;
 };
 
 constexpr int S_SLOTS = 4;  // d/dmin ring (unpack -> epilogue)
+constexpr int ISSUERS = 3;  // MMA-issuing warps
 constexpr int ACC_SETS = 2;
 // tensor-memory columns
-constexpr uint32_t TM_A = 0;       // 8 K-step slots x 16 columns (plane 0 | plane 1)
-constexpr uint32_t TM_AMIN = 128;  // 2 buffers x 16 columns (Ml-A | Mh-A)
-constexpr uint32_t TM_ACC = 160;   // ACC_SETS x NACC x NTOK columns
+constexpr uint32_t TM_A = 0;      // 8 K-step slots x 16 columns (plane 0 | plane 1)
+constexpr uint32_t TM_ACC = 128;  // ACC_SETS x NACC x NTOK columns
 constexpr uint32_t TM_COLS = 512;
 
 struct Segment {
-    const uint8_t* w;   // repacked weights
+    const uint8_t* w;  // repacked weights
     float* out;
     int64_t ldo;
-    int32_t tile0;      // first global n-tile of this segment
+    int32_t tile0;     // first global n-tile of this segment
 };
 
 struct GemmArgs {
     Segment seg[3];
     int nseg;
-    int32_t n_tiles;    // total 128-row tiles over all segments
-    int32_t nsb;        // K / 256
-    const int8_t* q;    // tiled activations of the source canvas
+    int32_t n_tiles;   // total 128-row tiles over all segments
+    int32_t nsb;       // K / 256
+    int32_t kc;        // K-chunks per tile
+    const int8_t* q;   // tiled activations
     const float* scale;
     const uint8_t* sums;
-    int64_t M;          // source canvas rows
-    int64_t Mp;         // M rounded up to 16 (the layout's row count)
-    const int32_t* rows;  // nullable
-    int32_t n_rows;
-    int32_t n_st;       // token super-tiles per n-tile
-    int32_t mu;         // tokens per super-tile (multiple of 16)
-    int64_t m_out;      // output rows (M or n_rows)
-    int32_t* dbg_S;     // debug: integer outputs instead of f32 (nullable)
+    int64_t Mp;        // rows of the activation layout (multiple of 16)
+    int64_t m_out;     // output rows
+    int32_t n_st;      // token super-tiles
+    int32_t mu;        // tokens per super-tile (multiple of 16)
+    uint32_t* counters;  // [n_tiles * n_st], when kc > 1
+    float* partials;     // [units][mu][128], when kc > 1
+    int32_t* dbg_S;    // debug: integer outputs instead of f32 (nullable)
     int32_t* dbg_Smin;
     int64_t dbg_N;
 };
@@ -110,23 +123,26 @@ struct GemmArgs {
 struct GemmShared {
     uint64_t w_full[8], w_empty[8];
     uint64_t b_full[8], b_empty[8];
-    uint64_t a_full[8], a_empty[8];
-    uint64_t amin_full[2], amin_empty[2];
+    uint64_t a_full[2], a_empty[2];  // A ring halves: K-steps 0-3, and 4-7 (+ the min-term A)
     uint64_t s_full[S_SLOTS], s_empty[S_SLOTS];
     uint64_t acc_full[ACC_SETS], acc_empty[ACC_SETS];
-    uint64_t final_bar;
+    uint64_t final_bar[4];
+    uint64_t epi_bar;
     uint32_t tmem_base;
     volatile int abort_flag;
+    int last_flag;
     float2 dd[S_SLOTS][TROWS];
 };
 
-// Bounded wait on an mbarrier phase; false if this CTA is aborting.  Raises the
-// abort flag and the device error word when the limit runs out.
+// Bounded wait on an mbarrier phase; false if this CTA is aborting.  Waiting threads
+// sleep inside try_wait instead of spinning, so the warps sharing their scheduler keep
+// its issue slots.  Raises the abort flag and the device error word when the limit
+// runs out.
 __device__ __forceinline__ bool wait_bar(GemmShared& sh, uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
         if (sh.abort_flag) return false;
         if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
             sh.abort_flag = 1;
@@ -135,30 +151,67 @@ __device__ __forceinline__ bool wait_bar(GemmShared& sh, uint64_t* bar, uint32_t
         }
     }
 }
-// Warp-uniform variant: every lane waits, and the warp agrees on the outcome.
 __device__ __forceinline__ bool wait_bar_warp(GemmShared& sh, uint64_t* bar, uint32_t parity) {
     const bool ok = wait_bar(sh, bar, parity);
     return __all_sync(0xffffffffu, ok);
 }
 
+// Bounded barrier among the 256 epilogue threads.
+__device__ __forceinline__ bool epi_sync(GemmShared& sh, uint32_t& phase) {
+    mbar_arrive(&sh.epi_bar);
+    const bool ok = wait_bar_warp(sh, &sh.epi_bar, phase);
+    phase ^= 1;
+    return ok;
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Load / preset this warp's HC (16 + 8 or 16 + 16) consecutive accumulator columns.
+template <int HC>
+__device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&x)[HC]) {
+    static_assert(HC == 24 || HC == 32, "column split");
+    tmem_ld16(taddr, x);
+    if constexpr (HC == 24) tmem_ld8p(taddr + 16, x + 16);
+    else tmem_ld16(taddr + 16, x + 16);
+}
+template <int HC>
+__device__ __forceinline__ void fill_cols(uint32_t taddr, uint32_t v) {
+    tmem_fill16(taddr, v);
+    if constexpr (HC == 24) tmem_fill8(taddr + 16, v);
+    else tmem_fill16(taddr + 16, v);
+}
+
 struct Unit {
     int seg;
     int64_t tile;   // tile index inside the segment
-    int64_t m0;     // first token of the super-tile (in the gathered numbering when rows)
+    int32_t gtile;  // global tile index
+    int32_t st;     // token super-tile
+    int32_t chunk;  // K-chunk
+    int64_t m0;     // first token of the super-tile
     int32_t len;    // tokens in the super-tile (multiple of 16)
+    int32_t sb0, sb1;
 };
 
 __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int64_t u) {
     Unit r;
-    const int64_t nt = u / a.n_st;
-    const int32_t st = (int32_t)(u % a.n_st);
+    r.chunk = (int32_t)(u % a.kc);
+    const int64_t ts = u / a.kc;
+    r.st = (int32_t)(ts % a.n_st);
+    r.gtile = (int32_t)(ts / a.n_st);
     r.seg = 0;
-    if (a.nseg > 1 && nt >= a.seg[1].tile0) r.seg = 1;
-    if (a.nseg > 2 && nt >= a.seg[2].tile0) r.seg = 2;
-    r.tile = nt - a.seg[r.seg].tile0;
-    r.m0 = (int64_t)st * a.mu;
-    const int64_t rows_total = a.rows ? round_up(a.n_rows, 16) : a.Mp;
-    r.len = (int32_t)min((int64_t)a.mu, rows_total - r.m0);
+    if (a.nseg > 1 && r.gtile >= a.seg[1].tile0) r.seg = 1;
+    if (a.nseg > 2 && r.gtile >= a.seg[2].tile0) r.seg = 2;
+    r.tile = r.gtile - a.seg[r.seg].tile0;
+    r.m0 = (int64_t)r.st * a.mu;
+    r.len = (int32_t)min((int64_t)a.mu, a.Mp - r.m0);
+    r.sb0 = (int32_t)((int64_t)r.chunk * a.nsb / a.kc);
+    r.sb1 = (int32_t)((int64_t)(r.chunk + 1) * a.nsb / a.kc);
     return r;
 }
 
@@ -166,26 +219,38 @@ template <int QT, bool DBG>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<QT>;
     constexpr int NTOK = C::NTOK;
-    constexpr int TMAX = UNIT_TOKENS / NTOK;
+    constexpr int TMAX = (UNIT_TOKENS + NTOK - 1) / NTOK;
+    constexpr int HC = NTOK / 2;  // token columns per epilogue warp
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* w_stage = smem_raw;
     uint8_t* b_stage = w_stage + C::W_STAGES * C::TILE;
-    GemmShared& sh = *reinterpret_cast<GemmShared*>(b_stage + C::B_STAGES * C::B_STAGE);
+    uint8_t* mina = b_stage + C::B_STAGES * C::B_STAGE;
+    GemmShared& sh = *reinterpret_cast<GemmShared*>(mina + C::MINA);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n_units = (int64_t)args.n_tiles * args.n_st;
-    const int nsb = args.nsb;
+    const int64_t n_units = (int64_t)args.n_tiles * args.n_st * args.kc;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 128); }
-        for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 1 + 256); }
-        for (int i = 0; i < 8; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], 1); }
-        for (int i = 0; i < 2; i++) { mbar_init(&sh.amin_full[i], 128); mbar_init(&sh.amin_empty[i], 1); }
+        for (int i = 0; i < C::B_STAGES; i++) {
+            mbar_init(&sh.b_full[i], 1);
+            mbar_init(&sh.b_empty[i], 256);
+        }
+        for (int i = 0; i < 2; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], ISSUERS); }
         for (int i = 0; i < S_SLOTS; i++) { mbar_init(&sh.s_full[i], 128); mbar_init(&sh.s_empty[i], 256); }
-        for (int i = 0; i < ACC_SETS; i++) { mbar_init(&sh.acc_full[i], 1); mbar_init(&sh.acc_empty[i], 256); }
-        mbar_init(&sh.final_bar, 1);
+        for (int i = 0; i < ACC_SETS; i++) {
+            mbar_init(&sh.acc_full[i], ISSUERS);
+            mbar_init(&sh.acc_empty[i], 256);
+        }
+        for (int i = 0; i < 4; i++) mbar_init(&sh.final_bar[i], 1);
+        mbar_init(&sh.epi_bar, 256);
         sh.abort_flag = 0;
         fence_mbar_init();
+    }
+    if constexpr (C::MINA > 0) {  // the second 16-byte K chunk of the min-term A operands is zero
+        for (int i = threadIdx.x; i < C::MINA / 16; i += GEMM_THREADS)
+            reinterpret_cast<uint4*>(mina)[i] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
     }
     if (warp == 1) {
         tmem_alloc(&sh.tmem_base, TM_COLS);
@@ -196,159 +261,140 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
 
-    if (warp == 0) {
-        // ============================================================ producer
-        uint32_t ws = 0, wph = 0, bs = 0, bph = 0;
-        uint32_t w_issued_ph[C::W_STAGES], b_issued_ph[C::B_STAGES];
-        bool w_issued[C::W_STAGES], b_issued[C::B_STAGES];
-        for (int i = 0; i < C::W_STAGES; i++) w_issued[i] = false;
-        for (int i = 0; i < C::B_STAGES; i++) b_issued[i] = false;
-        const uint64_t pol_w = policy_evict_first();
-        const uint64_t pol_a = policy_evict_last();
-        for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const Unit un = unit_of(args, u);
-            const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * nsb * C::TILE;
-            const int T = (un.len + NTOK - 1) / NTOK;
-            for (int s = 0; s < nsb; s++) {
-                if (!wait_bar_warp(sh, &sh.w_empty[ws], wph ^ 1)) goto done;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&sh.w_full[ws], C::TILE);
-                    bulk_g2s_hint(w_stage + ws * C::TILE, wt + (size_t)s * C::TILE, C::TILE, &sh.w_full[ws], pol_w);
-                }
-                w_issued[ws] = true;
-                w_issued_ph[ws] = wph;
-                if (++ws == C::W_STAGES) { ws = 0; wph ^= 1; }
-                for (int tt = 0; tt < T; tt++) {
-                    const int64_t t0 = un.m0 + (int64_t)tt * NTOK;
-                    const int ntok = min(NTOK, un.len - tt * NTOK);
-                    if (!wait_bar_warp(sh, &sh.b_empty[bs], bph ^ 1)) goto done;
-                    uint8_t* st = b_stage + bs * C::B_STAGE;
-                    if (args.rows == nullptr) {
+    if (warp < 4) {
+        setmaxnreg_dec<56>();
+        if (warp == 0) {
+            // ======================================================== producer
+            uint32_t ws = 0, wph = 0, bs = 0, bph = 0;
+            uint32_t w_ph_issued[C::W_STAGES], b_ph_issued[C::B_STAGES];
+            bool w_iss[C::W_STAGES], b_iss[C::B_STAGES];
+            for (int i = 0; i < C::W_STAGES; i++) w_iss[i] = false;
+            for (int i = 0; i < C::B_STAGES; i++) b_iss[i] = false;
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_a = policy_evict_last();
+            for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+                const Unit un = unit_of(args, u);
+                const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
+                const int T = (un.len + NTOK - 1) / NTOK;
+                for (int s = un.sb0; s < un.sb1; s++) {
+                    if (!wait_bar_warp(sh, &sh.w_empty[ws], wph ^ 1)) goto prod_done;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sh.w_full[ws], C::TILE);
+                        bulk_g2s_hint(w_stage + ws * C::TILE, wt + (size_t)s * C::TILE, C::TILE, &sh.w_full[ws],
+                                      pol_w);
+                    }
+                    w_iss[ws] = true;
+                    w_ph_issued[ws] = wph;
+                    if (++ws == C::W_STAGES) { ws = 0; wph ^= 1; }
+                    for (int tt = 0; tt < T; tt++) {
+                        const int64_t t0 = un.m0 + (int64_t)tt * NTOK;
+                        const int ntok = min(NTOK, un.len - tt * NTOK);
+                        if (!wait_bar_warp(sh, &sh.b_empty[bs], bph ^ 1)) goto prod_done;
                         if (lane == 0) {
+                            uint8_t* st = b_stage + bs * C::B_STAGE;
                             const uint32_t bytes = ntok * 256 + (C::B_SUMS ? ntok * 16 : 0) + ntok * 4;
                             mbar_arrive_expect_tx(&sh.b_full[bs], bytes);
-                            bulk_g2s_hint(st, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256,
-                                          &sh.b_full[bs], pol_a);
+                            bulk_g2s_hint(st, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256, &sh.b_full[bs],
+                                          pol_a);
                             if (C::B_SUMS)
                                 bulk_g2s_hint(st + C::B_Q, args.sums + ((size_t)s * args.Mp + t0) * 16, ntok * 16,
                                               &sh.b_full[bs], pol_a);
                             bulk_g2s_hint(st + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
                                           &sh.b_full[bs], pol_a);
                         }
-                    } else {
-                        // gather requested rows: 16-byte chunks, canvas row rows[i]
-                        for (int idx = lane; idx < ntok * 18; idx += 32) {
-                            const int i = idx / 18, c = idx % 18;  // c < 16: q chunk; 16: sums; 17: scale
-                            const int64_t gi = t0 + i;
-                            int64_t m = -1;
-                            if (gi < args.n_rows) {
-                                m = args.rows[gi];
-                                if (m < 0 || m >= args.M) {
-                                    if (c == 0) set_err(ERR_ROW_RANGE);
-                                    m = -1;
-                                }
-                            }
-                            if (c < 16) {
-                                uint4 v = make_uint4(0, 0, 0, 0);
-                                if (m >= 0)
-                                    v = *reinterpret_cast<const uint4*>(
-                                        args.q + (((size_t)s * (args.Mp / 8) + m / 8) * 16 + c) * 128 + (m % 8) * 16);
-                                *reinterpret_cast<uint4*>(st + ((i / 8) * 16 + c) * 128 + (i % 8) * 16) = v;
-                            } else if (c == 16) {
-                                if (C::B_SUMS) {
-                                    uint4 v = make_uint4(0, 0, 0, 0);
-                                    if (m >= 0)
-                                        v = *reinterpret_cast<const uint4*>(args.sums + ((size_t)s * args.Mp + m) * 16);
-                                    *reinterpret_cast<uint4*>(st + C::B_Q + i * 16) = v;
-                                }
-                            } else {
-                                float v = 0.0f;
-                                if (m >= 0) v = args.scale[(size_t)s * args.Mp + m];
-                                reinterpret_cast<float*>(st + C::B_Q + C::B_SUMS)[i] = v;
-                            }
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sh.b_full[bs]);
+                        b_iss[bs] = true;
+                        b_ph_issued[bs] = bph;
+                        if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
                     }
-                    b_issued[bs] = args.rows == nullptr;
-                    b_issued_ph[bs] = bph;
-                    if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
                 }
             }
-        }
-    done:
-        // never leave with bulk copies in flight into this CTA's shared memory
-        if (sh.abort_flag) {
-            for (int i = 0; i < C::W_STAGES; i++)
-                if (w_issued[i]) (void)wait_bar(sh, &sh.w_full[i], w_issued_ph[i]);
-            for (int i = 0; i < C::B_STAGES; i++)
-                if (b_issued[i]) (void)wait_bar(sh, &sh.b_full[i], b_issued_ph[i]);
-        }
-    } else if (warp == 1) {
-        // ============================================================ MMA issuer
-        if (lane == 0) {
-            uint32_t bs = 0, bph = 0, r = 0, rph = 0, ab = 0, sbc = 0;
-            uint32_t amin_ph[2] = {0, 0};
+        prod_done:
+            if (sh.abort_flag) {  // never leave with bulk copies in flight into this CTA's shared memory
+                for (int i = 0; i < C::W_STAGES; i++)
+                    if (w_iss[i]) (void)wait_bar(sh, &sh.w_full[i], w_ph_issued[i]);
+                for (int i = 0; i < C::B_STAGES; i++)
+                    if (b_iss[i]) (void)wait_bar(sh, &sh.b_full[i], b_ph_issued[i]);
+            }
+        } else if (warp - 1 < ISSUERS) {
+            // ======================================================== MMA issuers
+            // All lanes walk the schedule and wait together; lane 0 issues.  Tile g of
+            // this CTA gives plane 0 to issuer (2g) % 3, plane 1 to (2g+1) % 3 and the
+            // min term (Q4_K) to (2g+2) % 3.  Every issuer commits once per tile to
+            // the accumulator set and once per super-block to each half of the A ring.
+            const int who = warp - 1;
+            const bool leader = lane == 0;
+            uint32_t bs = 0, bph = 0, r = 0, rph = 0, sbc = 0, g = 0;
             for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
                 const Unit un = unit_of(args, u);
                 const int T = (un.len + NTOK - 1) / NTOK;
-                for (int s = 0; s < nsb; s++, sbc++) {
-                    for (int tt = 0; tt < T; tt++) {
+                for (int s = un.sb0; s < un.sb1; s++, sbc++) {
+                    for (int tt = 0; tt < T; tt++, g++) {
                         const int ntok = min(NTOK, un.len - tt * NTOK);
-                        if (!wait_bar(sh, &sh.b_full[bs], bph)) goto mma_done;
-                        if (!wait_bar(sh, &sh.acc_empty[r], rph)) goto mma_done;
+                        const bool last = tt == T - 1;
+                        if (!wait_bar_warp(sh, &sh.b_full[bs], bph)) goto mma_done;
+                        if (!wait_bar_warp(sh, &sh.acc_empty[r], rph)) goto mma_done;
+                        if (tt == 0) {
+                            if (!wait_bar_warp(sh, &sh.a_full[0], sbc & 1)) goto mma_done;
+                            if (!wait_bar_warp(sh, &sh.a_full[1], sbc & 1)) goto mma_done;
+                        }
                         tc_fence_after();
-                        const uint32_t st = smem_u32(b_stage + bs * C::B_STAGE);
-                        const uint32_t acc = tmem + TM_ACC + r * C::NACC * NTOK;
-                        const uint32_t id_p = QT == 12 ? idesc_i8(128, ntok, 0, 1) : idesc_i8(128, ntok, 1, 1);
-                        for (int ks = 0; ks < 8; ks++) {
-                            if (tt == 0) {
-                                if (!wait_bar(sh, &sh.a_full[ks], sbc & 1)) goto mma_done;
-                                tc_fence_after();
+                        const int role = (int)((who + 3 - (2 * g) % 3) % 3);  // 0: plane 0, 1: plane 1, 2: min
+                        if (leader) {
+                            const uint32_t acc = tmem + TM_ACC + r * C::NACC * NTOK;
+                            const uint32_t st = smem_u32(b_stage + bs * C::B_STAGE);
+                            if (role < 2) {
+                                const uint32_t id = QT == 12 ? idesc_i8(128, ntok, 0, 1) : idesc_i8(128, ntok, 1, 1);
+                                const uint32_t d = acc + role * NTOK;
+                                const uint32_t a0 = tmem + TM_A + 8 * role;
+                                const uint64_t b0 = sdesc_kmajor_noswz(st, 128, 2048);
+#pragma unroll
+                                for (int ks = 0; ks < 4; ks++) mma_i8_ts(d, a0 + 16 * ks, b0 + 16 * ks, id, 1);
+                                if (last) tc_commit(&sh.a_empty[0]);
+#pragma unroll
+                                for (int ks = 4; ks < 8; ks++) mma_i8_ts(d, a0 + 16 * ks, b0 + 16 * ks, id, 1);
+                                if (last) tc_commit(&sh.a_empty[1]);
+                            } else {
+                                if (last) tc_commit(&sh.a_empty[0]);
+                                if constexpr (QT == 12) {
+                                    const uint32_t ma = smem_u32(mina);
+                                    const uint64_t bd = sdesc_kmajor_noswz(st + C::B_Q, 128, 128);
+                                    mma_i8_ss(acc + 2 * NTOK, sdesc_kmajor_noswz(ma, 128, 256), bd,
+                                              idesc_i8(128, ntok, 0, 0), 1);
+                                    mma_i8_ss(acc + 3 * NTOK, sdesc_kmajor_noswz(ma + 4096, 128, 256), bd,
+                                              idesc_i8(128, ntok, 0, 1), 1);
+                                }
+                                if (last) tc_commit(&sh.a_empty[1]);
                             }
-                            const uint64_t bd = sdesc_kmajor_noswz(st + 256 * ks, 128, 2048);
-                            mma_i8_ts(acc + 0 * NTOK, tmem + TM_A + 16 * ks, bd, id_p, 1);
-                            mma_i8_ts(acc + 1 * NTOK, tmem + TM_A + 16 * ks + 8, bd, id_p, 1);
-                            if (tt == T - 1) tc_commit(&sh.a_empty[ks]);
+                            tc_commit(&sh.acc_full[r]);
                         }
-                        if constexpr (QT == 12) {
-                            if (tt == 0) {
-                                if (!wait_bar(sh, &sh.amin_full[ab], amin_ph[ab])) goto mma_done;
-                                tc_fence_after();
-                            }
-                            const uint64_t bd = sdesc_kmajor_noswz(st + C::B_Q, 128, 128);
-                            mma_i8_ts(acc + 2 * NTOK, tmem + TM_AMIN + 16 * ab, bd, idesc_i8(128, ntok, 0, 0), 1);
-                            mma_i8_ts(acc + 3 * NTOK, tmem + TM_AMIN + 16 * ab + 8, bd, idesc_i8(128, ntok, 0, 1), 1);
-                            if (tt == T - 1) tc_commit(&sh.amin_empty[ab]);
-                        }
-                        tc_commit(&sh.acc_full[r]);
-                        tc_commit(&sh.b_empty[bs]);
+                        __syncwarp();
                         if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
                         if (++r == ACC_SETS) { r = 0; rph ^= 1; }
                     }
-                    if (QT == 12) { amin_ph[ab] ^= 1; ab ^= 1; }
                 }
             }
         mma_done:
-            // every MMA this thread issued has completed before tensor memory is freed
-            tc_commit(&sh.final_bar);
-            (void)wait_bar(sh, &sh.final_bar, 0);
+            // every MMA this warp issued has completed before tensor memory is freed
+            if (leader) tc_commit(&sh.final_bar[who]);
+            __syncwarp();
+            (void)wait_bar_warp(sh, &sh.final_bar[who], 0);
         }
-        __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp < 8) {
+        setmaxnreg_dec<88>();
         // ============================================================ unpack
+        // Per super-block: decode this row, then build the planes of K-steps 0-3,
+        // publish them together, then K-steps 4-7 (and the min-term A), so the MMAs
+        // of a super-block can start while the second half is still being built.
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        uint32_t ws = 0, wph = 0, ss = 0, sph = 0, ab = 0, sbc = 0;
-        uint32_t amin_ph[2] = {0, 0};
+        uint32_t ws = 0, wph = 0, ss = 0, sph = 0, sbc = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-            for (int s = 0; s < nsb; s++, sbc++) {
+            const Unit un = unit_of(args, u);
+            for (int s = un.sb0; s < un.sb1; s++, sbc++) {
                 if (!wait_bar_warp(sh, &sh.w_full[ws], wph)) goto unpack_done;
                 const uint8_t* tl = w_stage + ws * C::TILE;
                 if constexpr (QT == 12) {
-                    // ---- Q4_K: scales, mins, d, dmin of this row
                     const uint32_t b0 = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_SC + 12 * row);
                     const uint32_t b1 = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_SC + 12 * row + 4);
                     const uint32_t b2 = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_SC + 12 * row + 8);
@@ -367,49 +413,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     sh.dd[ss][row] = make_float2(d, -dmin);
                     mbar_arrive(&sh.s_full[ss]);
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
-                    // mins as the A operand of the two min-term MMAs
-                    if (!wait_bar_warp(sh, &sh.amin_empty[ab], amin_ph[ab] ^ 1)) goto unpack_done;
-                    {
-                        uint32_t v[16];
 #pragma unroll
-                        for (int i = 0; i < 16; i++) v[i] = 0;
-                        v[0] = mn[0] | (mn[1] << 8) | (mn[2] << 16) | (mn[3] << 24);
-                        v[1] = mn[4] | (mn[5] << 8) | (mn[6] << 16) | (mn[7] << 24);
-                        v[10] = v[0];
-                        v[11] = v[1];
-                        tmem_st16(tmem + lane_off + TM_AMIN + 16 * ab, v);
+                    for (int half = 0; half < 2; half++) {
+                        if (!wait_bar_warp(sh, &sh.a_empty[half], (sbc & 1) ^ 1)) goto unpack_done;
+                        if (half == 1) {
+                            // mins: the A operands of the two min-term MMAs, row `row` of
+                            // the canonical K-major layout (8-row groups of 256 bytes)
+                            const uint32_t m03 = mn[0] | (mn[1] << 8) | (mn[2] << 16) | (mn[3] << 24);
+                            const uint32_t m47 = mn[4] | (mn[5] << 8) | (mn[6] << 16) | (mn[7] << 24);
+                            uint8_t* base = mina + (row >> 3) * 256 + (row & 7) * 16;
+                            *reinterpret_cast<uint4*>(base) = make_uint4(m03, m47, 0, 0);
+                            *reinterpret_cast<uint4*>(base + 4096) = make_uint4(0, 0, m03, m47);
+                            fence_proxy_async_smem();
+                        }
+#pragma unroll
+                        for (int cc = 0; cc < 2; cc++) {
+                            const int c = 2 * half + cc;  // 32-byte quant chunk: sub-blocks 2c, 2c+1
+                            const uint4 p0 = *reinterpret_cast<const uint4*>(tl + ((2 * c) * TROWS + row) * 16);
+                            const uint4 p1 = *reinterpret_cast<const uint4*>(tl + ((2 * c + 1) * TROWS + row) * 16);
+                            const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                            for (int h = 0; h < 2; h++) {
+                                const int ks = 2 * c + h;
+                                const uint32_t lo3 = sc[ks] & 7, hi3 = sc[ks] >> 3;
+                                uint32_t v[16];
+#pragma unroll
+                                for (int i = 0; i < 8; i++) {
+                                    const uint32_t nib = (wv[i] >> (4 * h)) & 0x0F0F0F0Fu;
+                                    v[i] = nib * lo3;
+                                    v[8 + i] = nib * hi3;
+                                }
+                                tmem_st16(tmem + lane_off + TM_A + 16 * ks, v);
+                            }
+                        }
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(&sh.amin_full[ab]);
-                    }
-                    amin_ph[ab] ^= 1;
-                    ab ^= 1;
-                    // weight planes, one K-step (= one sub-block of 32) at a time
-#pragma unroll 1
-                    for (int c = 0; c < 4; c++) {
-                        const uint4 p0 = *reinterpret_cast<const uint4*>(tl + ((2 * c) * TROWS + row) * 16);
-                        const uint4 p1 = *reinterpret_cast<const uint4*>(tl + ((2 * c + 1) * TROWS + row) * 16);
-                        const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-                        for (int h = 0; h < 2; h++) {
-                            const int ks = 2 * c + h;
-                            if (!wait_bar_warp(sh, &sh.a_empty[ks], (sbc & 1) ^ 1)) goto unpack_done;
-                            const uint32_t lo3 = sc[ks] & 7, hi3 = sc[ks] >> 3;
-                            uint32_t v[16];
-#pragma unroll
-                            for (int i = 0; i < 8; i++) {
-                                const uint32_t nib = (wv[i] >> (4 * h)) & 0x0F0F0F0Fu;
-                                v[i] = nib * lo3;
-                                v[8 + i] = nib * hi3;
-                            }
-                            tmem_st16(tmem + lane_off + TM_A + 16 * ks, v);
-                            tmem_wait_st();
-                            tc_fence_before();
-                            mbar_arrive(&sh.a_full[ks]);
-                        }
+                        mbar_arrive(&sh.a_full[half]);
                     }
                 } else {
-                    // ---- Q6_K
                     const uint4 scv = *reinterpret_cast<const uint4*>(tl + Q6K_OFF_SC + 16 * row);
                     const uint32_t scw[4] = {scv.x, scv.y, scv.z, scv.w};
                     const float d = __half2float(
@@ -418,39 +459,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     sh.dd[ss][row] = make_float2(d, 0.0f);
                     mbar_arrive(&sh.s_full[ss]);
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
-#pragma unroll 1
-                    for (int ks = 0; ks < 8; ks++) {
-                        const int h = ks >> 2, g = ks & 3;
-                        const int lp = 2 * (2 * h + (g & 1));  // low-bit piece index
-                        const uint4 l0 = *reinterpret_cast<const uint4*>(tl + (lp * TROWS + row) * 16);
-                        const uint4 l1 = *reinterpret_cast<const uint4*>(tl + ((lp + 1) * TROWS + row) * 16);
-                        const uint4 h0 =
-                            *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h) * TROWS + row) * 16);
-                        const uint4 h1 =
-                            *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h + 1) * TROWS + row) * 16);
-                        const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-                        const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-                        const int sh_lo = 4 * (g >> 1), sh_hi = 2 * g;
-                        const int32_t sca = (int32_t)(int8_t)((scw[ks >> 1] >> (16 * (ks & 1))) & 0xFF);
-                        const int32_t scb = (int32_t)(int8_t)((scw[ks >> 1] >> (16 * (ks & 1) + 8)) & 0xFF);
-                        const uint32_t adda = (uint32_t)(32896 - 32 * sca) * 0x10001u;
-                        const uint32_t addb = (uint32_t)(32896 - 32 * scb) * 0x10001u;
-                        if (!wait_bar_warp(sh, &sh.a_empty[ks], (sbc & 1) ^ 1)) goto unpack_done;
-                        uint32_t v[16];
 #pragma unroll
-                        for (int i = 0; i < 8; i++) {
-                            const uint32_t qv = ((lw[i] >> sh_lo) & 0x0F0F0F0Fu) | (((hw[i] >> sh_hi) & 0x03030303u) << 4);
-                            const int32_t sc = i < 4 ? sca : scb;
-                            const uint32_t add = i < 4 ? adda : addb;
-                            const uint32_t pa = __byte_perm(qv, 0, 0x4140) * (uint32_t)sc + add;
-                            const uint32_t pb = __byte_perm(qv, 0, 0x4342) * (uint32_t)sc + add;
-                            v[i] = __byte_perm(pa, pb, 0x6420) ^ 0x80808080u;
-                            v[8 + i] = __byte_perm(pa, pb, 0x7531) ^ 0x80808080u;
+                    for (int half = 0; half < 2; half++) {
+                        if (!wait_bar_warp(sh, &sh.a_empty[half], (sbc & 1) ^ 1)) goto unpack_done;
+#pragma unroll 1
+                        for (int kq = 0; kq < 4; kq++) {
+                            const int ks = 4 * half + kq;
+                            const int h = ks >> 2, g = ks & 3;
+                            const int lp = 2 * (2 * h + (g & 1));  // low-bit piece index
+                            const uint4 l0 = *reinterpret_cast<const uint4*>(tl + (lp * TROWS + row) * 16);
+                            const uint4 l1 = *reinterpret_cast<const uint4*>(tl + ((lp + 1) * TROWS + row) * 16);
+                            const uint4 h0 =
+                                *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h) * TROWS + row) * 16);
+                            const uint4 h1 =
+                                *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h + 1) * TROWS + row) * 16);
+                            const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+                            const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+                            const int sh_lo = 4 * (g >> 1), sh_hi = 2 * g;
+                            const int32_t sca = (int32_t)(int8_t)((scw[ks >> 1] >> (16 * (ks & 1))) & 0xFF);
+                            const int32_t scb = (int32_t)(int8_t)((scw[ks >> 1] >> (16 * (ks & 1) + 8)) & 0xFF);
+                            const uint32_t adda = (uint32_t)(32896 - 32 * sca) * 0x10001u;
+                            const uint32_t addb = (uint32_t)(32896 - 32 * scb) * 0x10001u;
+                            uint32_t v[16];
+#pragma unroll
+                            for (int i = 0; i < 8; i++) {
+                                const uint32_t qv =
+                                    ((lw[i] >> sh_lo) & 0x0F0F0F0Fu) | (((hw[i] >> sh_hi) & 0x03030303u) << 4);
+                                const int32_t scs = i < 4 ? sca : scb;
+                                const uint32_t add = i < 4 ? adda : addb;
+                                const uint32_t pa = __byte_perm(qv, 0, 0x4140) * (uint32_t)scs + add;
+                                const uint32_t pb = __byte_perm(qv, 0, 0x4342) * (uint32_t)scs + add;
+                                v[i] = __byte_perm(pa, pb, 0x6420) ^ 0x80808080u;
+                                v[8 + i] = __byte_perm(pa, pb, 0x7531) ^ 0x80808080u;
+                            }
+                            tmem_st16(tmem + lane_off + TM_A + 16 * ks, v);
                         }
-                        tmem_st16(tmem + lane_off + TM_A + 16 * ks, v);
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(&sh.a_full[ks]);
+                        mbar_arrive(&sh.a_full[half]);
                     }
                 }
                 mbar_arrive(&sh.w_empty[ws]);
@@ -458,41 +504,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             }
         }
     unpack_done:;
-    } else if (warp >= 8) {
+    } else {
+        setmaxnreg_inc<184>();
         // ============================================================ epilogue
         const int quad = warp & 3;
         const int half = (warp - 8) >> 2;
         const int row = quad * 32 + lane;
+        const int etid = threadIdx.x - 256;  // 0..255
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        constexpr int HC = NTOK / 2;  // columns per epilogue warp
-        // preset every accumulator column this warp owns
         {
-            uint32_t cv[8];
-#pragma unroll
-            for (int i = 0; i < 8; i++) cv[i] = MAGIC_BITS;
             for (int r = 0; r < ACC_SETS; r++)
                 for (int a = 0; a < C::NACC; a++)
-                    for (int c = 0; c < HC; c += 8)
-                        tmem_st8(tmem + lane_off + TM_ACC + (r * C::NACC + a) * NTOK + half * HC + c, cv);
+                    fill_cols<HC>(tmem + lane_off + TM_ACC + (r * C::NACC + a) * NTOK + half * HC, MAGIC_BITS);
             tmem_wait_st();
             tc_fence_before();
             for (int r = 0; r < ACC_SETS; r++) mbar_arrive(&sh.acc_empty[r]);
         }
-        uint32_t bs = 0, bph = 0, r = 0, rph = 0, ss = 0, sph = 0;
+        const float2 k8 = make_float2(8.0f, 8.0f), k256 = make_float2(256.0f, 256.0f);
+        const float2 m9 = make_float2(-9.0f * MAGIC, -9.0f * MAGIC);
+        const float2 m257 = make_float2(-257.0f * MAGIC, -257.0f * MAGIC);
+        uint32_t bs = 0, bph = 0, r = 0, rph = 0, ss = 0, sph = 0, epi_ph = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
             const Unit un = unit_of(args, u);
             const int T = (un.len + NTOK - 1) / NTOK;
             const Segment& sg = args.seg[un.seg];
-            float acc[TMAX][HC];
+            float2 acc[TMAX][HC / 2];
 #pragma unroll
             for (int t = 0; t < TMAX; t++)
 #pragma unroll
-                for (int j = 0; j < HC; j++) acc[t][j] = 0.0f;
-            for (int s = 0; s < nsb; s++) {
+                for (int j = 0; j < HC / 2; j++) acc[t][j] = make_float2(0.0f, 0.0f);
+            for (int s = un.sb0; s < un.sb1; s++) {
                 if (!wait_bar_warp(sh, &sh.s_full[ss], sph)) goto epi_done;
                 const float2 dd = sh.dd[ss][row];
                 mbar_arrive(&sh.s_empty[ss]);
                 if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
+                const float2 d2 = make_float2(dd.x, dd.x), nm2 = make_float2(dd.y, dd.y);
 #pragma unroll
                 for (int tt = 0; tt < TMAX; tt++) {
                     if (tt < T) {
@@ -502,57 +548,68 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         tc_fence_after();
                         const uint32_t acc_t = tmem + lane_off + TM_ACC + r * C::NACC * NTOK + half * HC;
                         const float* da = reinterpret_cast<const float*>(b_stage + bs * C::B_STAGE + C::B_Q + C::B_SUMS);
+                        if (half * HC < ntok) {
+                            // plane accumulators: S = P0 + 8 P1 (Q4_K) or P0 + 256 P1 (Q6_K)
+                            uint32_t x0[HC], x1[HC];
+                            load_cols<HC>(acc_t, x0);
+                            load_cols<HC>(acc_t + NTOK, x1);
+                            tmem_wait_ld();
+                            fill_cols<HC>(acc_t, MAGIC_BITS);
+                            fill_cols<HC>(acc_t + NTOK, MAGIC_BITS);
+                            float2 S[HC / 2];
 #pragma unroll
-                        for (int c = 0; c < HC; c += 8) {
-                            if (half * HC + c < ntok) {
-                                uint32_t x0[8], x1[8], x2[8], x3[8];
-                                tmem_ld8(acc_t + c, x0);
-                                tmem_ld8(acc_t + NTOK + c, x1);
+                            for (int i = 0; i < HC / 2; i++) {
+                                const float2 X0 = make_float2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
+                                const float2 X1 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+                                S[i] = QT == 12 ? __fadd2_rn(__ffma2_rn(X1, k8, m9), X0)
+                                                : __fadd2_rn(__ffma2_rn(X1, k256, m257), X0);
+                            }
+                            if constexpr (DBG) {
+                                uint32_t y0[HC], y1[HC];
                                 if constexpr (QT == 12) {
-                                    tmem_ld8(acc_t + 2 * NTOK + c, x2);
-                                    tmem_ld8(acc_t + 3 * NTOK + c, x3);
+                                    load_cols<HC>(acc_t + 2 * NTOK, y0);
+                                    load_cols<HC>(acc_t + 3 * NTOK, y1);
+                                    tmem_wait_ld();
+                                    fill_cols<HC>(acc_t + 2 * NTOK, MAGIC_BITS);
+                                    fill_cols<HC>(acc_t + 3 * NTOK, MAGIC_BITS);
                                 }
-                                tmem_wait_ld();
-                                uint32_t cv[8];
 #pragma unroll
-                                for (int i = 0; i < 8; i++) cv[i] = MAGIC_BITS;
-                                tmem_st8(acc_t + c, cv);
-                                tmem_st8(acc_t + NTOK + c, cv);
-                                if constexpr (QT == 12) {
-                                    tmem_st8(acc_t + 2 * NTOK + c, cv);
-                                    tmem_st8(acc_t + 3 * NTOK + c, cv);
-                                }
-                                if constexpr (DBG) {
-#pragma unroll
-                                    for (int i = 0; i < 8; i++) {
-                                        const int64_t m = un.m0 + tt * NTOK + half * HC + c + i;
-                                        if (m < args.m_out) {
-                                            const int n = (int)(un.tile * TROWS + row);
-                                            const int64_t o = (m * args.dbg_N + n) * nsb + s;
-                                            if (QT == 12) {
-                                                args.dbg_S[o] = (int32_t)(x0[i] - MAGIC_BITS) + 8 * (int32_t)(x1[i] - MAGIC_BITS);
-                                                args.dbg_Smin[o] = (int32_t)(x2[i] - MAGIC_BITS) + 256 * (int32_t)(x3[i] - MAGIC_BITS);
-                                            } else {
-                                                args.dbg_S[o] = (int32_t)(x0[i] - MAGIC_BITS) + 256 * (int32_t)(x1[i] - MAGIC_BITS);
-                                            }
+                                for (int i = 0; i < HC; i++) {
+                                    const int64_t m = un.m0 + tt * NTOK + half * HC + i;
+                                    if (half * HC + i < ntok && m < args.m_out) {
+                                        const int64_t n = un.tile * TROWS + row;
+                                        const int64_t o = (m * args.dbg_N + n) * args.nsb + s;
+                                        if constexpr (QT == 12) {
+                                            args.dbg_S[o] = (int32_t)(x0[i] - MAGIC_BITS) + 8 * (int32_t)(x1[i] - MAGIC_BITS);
+                                            args.dbg_Smin[o] = (int32_t)(y0[i] - MAGIC_BITS) + 256 * (int32_t)(y1[i] - MAGIC_BITS);
+                                        } else {
+                                            args.dbg_S[o] = (int32_t)(x0[i] - MAGIC_BITS) + 256 * (int32_t)(x1[i] - MAGIC_BITS);
                                         }
                                     }
-                                } else {
-                                    const float4 da0 = *reinterpret_cast<const float4*>(da + half * HC + c);
-                                    const float4 da1 = *reinterpret_cast<const float4*>(da + half * HC + c + 4);
-                                    const float dav[8] = {da0.x, da0.y, da0.z, da0.w, da1.x, da1.y, da1.z, da1.w};
+                                }
+                            } else {
+                                if constexpr (QT == 12) {
+                                    // min accumulators: Smin = Ml + 256 Mh
+                                    load_cols<HC>(acc_t + 2 * NTOK, x0);
+                                    load_cols<HC>(acc_t + 3 * NTOK, x1);
+                                    tmem_wait_ld();
+                                    fill_cols<HC>(acc_t + 2 * NTOK, MAGIC_BITS);
+                                    fill_cols<HC>(acc_t + 3 * NTOK, MAGIC_BITS);
 #pragma unroll
-                                    for (int i = 0; i < 8; i++) {
-                                        float t;
-                                        if constexpr (QT == 12) {
-                                            const float S = fmaf(__uint_as_float(x1[i]), 8.0f, -9.0f * MAGIC) + __uint_as_float(x0[i]);
-                                            const float Sm = fmaf(__uint_as_float(x3[i]), 256.0f, -257.0f * MAGIC) + __uint_as_float(x2[i]);
-                                            t = fmaf(Sm, dd.y, S * dd.x);
-                                        } else {
-                                            const float S = fmaf(__uint_as_float(x1[i]), 256.0f, -257.0f * MAGIC) + __uint_as_float(x0[i]);
-                                            t = S * dd.x;
-                                        }
-                                        acc[tt][c + i] = fmaf(t, dav[i], acc[tt][c + i]);
+                                    for (int i = 0; i < HC / 2; i++) {
+                                        const float2 X2 = make_float2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
+                                        const float2 X3 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+                                        const float2 Sm = __fadd2_rn(__ffma2_rn(X3, k256, m257), X2);
+                                        const float2 t = __ffma2_rn(Sm, nm2, __fmul2_rn(S[i], d2));
+                                        const float2 dav = *reinterpret_cast<const float2*>(da + half * HC + 2 * i);
+                                        acc[tt][i] = __ffma2_rn(t, dav, acc[tt][i]);
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int i = 0; i < HC / 2; i++) {
+                                        const float2 t = __fmul2_rn(S[i], d2);
+                                        const float2 dav = *reinterpret_cast<const float2*>(da + half * HC + 2 * i);
+                                        acc[tt][i] = __ffma2_rn(t, dav, acc[tt][i]);
                                     }
                                 }
                             }
@@ -567,15 +624,93 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                 }
             }
             if constexpr (!DBG) {
-                float* out = sg.out;
                 const int64_t n = un.tile * TROWS + row;
+                if (args.kc == 1) {
+                    float* out = sg.out;
 #pragma unroll
-                for (int tt = 0; tt < TMAX; tt++) {
-                    if (tt < T) {
+                    for (int tt = 0; tt < TMAX; tt++) {
+                        if (tt < T) {
 #pragma unroll
-                        for (int j = 0; j < HC; j++) {
-                            const int64_t m = un.m0 + tt * NTOK + half * HC + j;
-                            if (m < args.m_out && m < un.m0 + un.len) out[m * sg.ldo + n] = acc[tt][j];
+                            for (int j = 0; j < HC; j++) {
+                                const int64_t m = un.m0 + tt * NTOK + half * HC + j;
+                                if (m < args.m_out && m < un.m0 + un.len)
+                                    out[m * sg.ldo + n] = j & 1 ? acc[tt][j / 2].y : acc[tt][j / 2].x;
+                            }
+                        }
+                    }
+                } else {
+                    // this K-chunk's partial: [unit][128 rows][mu tokens]; a thread's
+                    // columns of one token tile are contiguous
+                    float* part = args.partials + ((size_t)u * TROWS + row) * args.mu;
+#pragma unroll
+                    for (int tt = 0; tt < TMAX; tt++) {
+                        if (tt < T) {
+                            const int ml0 = tt * NTOK + half * HC;
+                            if (ml0 + HC <= un.len) {
+#pragma unroll
+                                for (int j = 0; j < HC / 2; j += 2)
+                                    *reinterpret_cast<float4*>(part + ml0 + 2 * j) =
+                                        make_float4(acc[tt][j].x, acc[tt][j].y, acc[tt][j + 1].x, acc[tt][j + 1].y);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < HC / 2; j++) {
+                                    if (ml0 + 2 * j < un.len) *reinterpret_cast<float2*>(part + ml0 + 2 * j) = acc[tt][j];
+                                }
+                            }
+                        }
+                    }
+                    __threadfence();
+                    if (!epi_sync(sh, epi_ph)) goto epi_done;
+                    if (etid == 0) {
+                        uint32_t* ctr = args.counters + (size_t)un.gtile * args.n_st + un.st;
+                        const uint32_t old = atomicAdd(ctr, 1u);
+                        // counters advance by 16 per call and tile: the last of the kc
+                        // arrivals tops the counter up to the next multiple of 16
+                        const int last = (int)(old & 15u) == args.kc - 1;
+                        if (last) atomicAdd(ctr, (uint32_t)(16 - args.kc));
+                        __threadfence();
+                        sh.last_flag = last;
+                    }
+                    if (!epi_sync(sh, epi_ph)) goto epi_done;
+                    if (sh.last_flag) {
+                        // sum the chunk partials in chunk order; every load of a chunk is
+                        // issued before any is used
+                        const int64_t u0 = u - un.chunk;
+#pragma unroll
+                        for (int tt = 0; tt < TMAX; tt++)
+#pragma unroll
+                            for (int j = 0; j < HC / 2; j++) acc[tt][j] = make_float2(0.0f, 0.0f);
+                        for (int c2 = 0; c2 < args.kc; c2++) {
+                            const float* part = args.partials + ((size_t)(u0 + c2) * TROWS + row) * args.mu;
+                            float2 pv[TMAX][HC / 2];
+#pragma unroll
+                            for (int tt = 0; tt < TMAX; tt++) {
+#pragma unroll
+                                for (int j = 0; j < HC / 2; j++) {
+                                    const int ml = tt * NTOK + half * HC + 2 * j;
+                                    pv[tt][j] = (tt < T && ml < un.len)
+                                                    ? __ldcg(reinterpret_cast<const float2*>(part + ml))
+                                                    : make_float2(0.0f, 0.0f);
+                                }
+                            }
+#pragma unroll
+                            for (int tt = 0; tt < TMAX; tt++)
+#pragma unroll
+                                for (int j = 0; j < HC / 2; j++)
+                                    acc[tt][j] = c2 == 0 ? pv[tt][j] : __fadd2_rn(acc[tt][j], pv[tt][j]);
+                        }
+                        float* out = sg.out;
+#pragma unroll
+                        for (int tt = 0; tt < TMAX; tt++) {
+                            if (tt < T) {
+#pragma unroll
+                                for (int j = 0; j < HC; j++) {
+                                    const int ml = tt * NTOK + half * HC + j;
+                                    const int64_t m = un.m0 + ml;
+                                    if (ml < un.len && m < args.m_out)
+                                        out[m * sg.ldo + n] = j & 1 ? acc[tt][j / 2].y : acc[tt][j / 2].x;
+                                }
+                            }
                         }
                     }
                 }
@@ -594,7 +729,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
 template <int QT>
 constexpr size_t gemm_smem_bytes() {
     using C = GemmCfg<QT>;
-    return (size_t)C::W_STAGES * C::TILE + (size_t)C::B_STAGES * C::B_STAGE + sizeof(GemmShared);
+    return (size_t)C::W_STAGES * C::TILE + (size_t)C::B_STAGES * C::B_STAGE + C::MINA + sizeof(GemmShared);
+}
+
+// Gather the requested canvas rows of a tiled activation into a compact tiled
+// activation of Mp_r rows (rows past n_rows are zero).  One thread per 16-byte
+// chunk: 16 quant chunks, one sums chunk and one scale per (super-block, row).
+__global__ void gather_rows_kernel(const int8_t* __restrict__ q, const float* __restrict__ scale,
+                                   const uint8_t* __restrict__ sums, int64_t M, int64_t Mp,
+                                   const int32_t* __restrict__ rows, int32_t n_rows, int64_t Mp_r, int32_t nsb,
+                                   int8_t* __restrict__ gq, float* __restrict__ gscale, uint8_t* __restrict__ gsums) {
+    const int64_t total = (int64_t)nsb * Mp_r * 18;
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total; g += (int64_t)gridDim.x * blockDim.x) {
+        const int c = (int)(g % 18);
+        const int64_t i = (g / 18) % Mp_r;
+        const int64_t s = g / 18 / Mp_r;
+        int64_t m = -1;
+        if (i < n_rows) {
+            m = rows[i];
+            if (m < 0 || m >= M) {
+                if (c == 0) set_err(ERR_ROW_RANGE);
+                m = -1;
+            }
+        }
+        if (c < 16) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (m >= 0)
+                v = *reinterpret_cast<const uint4*>(q + ((s * (Mp / 8) + m / 8) * 16 + c) * 128 + (m % 8) * 16);
+            *reinterpret_cast<uint4*>(gq + ((s * (Mp_r / 8) + i / 8) * 16 + c) * 128 + (i % 8) * 16) = v;
+        } else if (c == 16) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (m >= 0) v = *reinterpret_cast<const uint4*>(sums + (s * Mp + m) * 16);
+            *reinterpret_cast<uint4*>(gsums + (s * Mp_r + i) * 16) = v;
+        } else {
+            gscale[s * Mp_r + i] = m >= 0 ? scale[s * Mp + m] : 0.0f;
+        }
+    }
 }
 
 }  // namespace dllm

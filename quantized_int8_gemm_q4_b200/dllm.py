@@ -59,14 +59,14 @@ def load() -> ctypes.CDLL:
         "dllm_repack_q6k": [P, I64, I64, P, P],
         "dllm_act_bytes": [I64, I64, PSZ, PSZ, PSZ],
         "dllm_quantize_act": [P, I64, I64, I64, P, P, P, P],
-        "dllm_qgemm_workspace_bytes": [I, I64, I64, I64, PSZ],
+        "dllm_qgemm_workspace_bytes": [I, I64, I64, I64, I64, PSZ],
         "dllm_qgemm": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P, SZ, P],
         "dllm_qkv_qgemm": [P, P, P, I, I64, I64, I64, P, P, P, I64, P, I64, P, P, I64, P, SZ, P],
         "dllm_get_device_status": [P],
         "dllm_status_string": [I],
         "dllm_debug_subblock_dots": [P, I, I64, I64, P, I64, P, P],
         "dllm_debug_sb_ints": [P, I, I64, I64, P, P, P, I64, P, P, P],
-        "dllm_bench_mma_i8": [I, I, I, I, I, P, P],
+        "dllm_bench_mma_i8": [I, I, I, I, I, I, P, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -130,9 +130,10 @@ def dllm_quantize_act(x, M: int, K: int, ldx: int, q, scale, sums, stream=None):
            "dllm_quantize_act")
 
 
-def dllm_qgemm_workspace_bytes(qtype: int, N: int, K: int, M: int) -> int:
+def dllm_qgemm_workspace_bytes(qtype: int, N: int, K: int, M: int, n_rows: int = 0) -> int:
     out = ctypes.c_size_t(0)
-    _check(load().dllm_qgemm_workspace_bytes(qtype, N, K, M, ctypes.byref(out)), "dllm_qgemm_workspace_bytes")
+    _check(load().dllm_qgemm_workspace_bytes(qtype, N, K, M, n_rows, ctypes.byref(out)),
+           "dllm_qgemm_workspace_bytes")
     return out.value
 
 
@@ -167,8 +168,9 @@ def dllm_debug_sb_ints(w, qtype: int, N: int, K: int, q, scale, sums, M: int, S,
                                      _ptr(Smin), _stream(stream)), "dllm_debug_sb_ints")
 
 
-def dllm_bench_mma_i8(n: int, n_acc: int, a_from_tmem: int, iters: int, ctas: int, ns_out, stream=None):
-    _check(load().dllm_bench_mma_i8(n, n_acc, a_from_tmem, iters, ctas, _ptr(ns_out), _stream(stream)),
+def dllm_bench_mma_i8(n: int, n_acc: int, a_from_tmem: int, issuers: int, iters: int, ctas: int, ns_out,
+                      stream=None):
+    _check(load().dllm_bench_mma_i8(n, n_acc, a_from_tmem, issuers, iters, ctas, _ptr(ns_out), _stream(stream)),
            "dllm_bench_mma_i8")
 
 
@@ -183,6 +185,14 @@ def repack(qtype: int, blocks, N: int, K: int, device="cuda", stream=None):
     dst = torch.empty(dllm_repacked_bytes(qtype, N, K), dtype=torch.uint8, device=device)
     (dllm_repack_q4k if qtype == DLLM_Q4_K else dllm_repack_q6k)(src, N, K, dst, stream)
     return dst
+
+
+def alloc_workspace(nbytes: int, device="cuda"):
+    """A zero-filled device workspace of at least nbytes (None when nbytes is 0)."""
+    import torch
+    if nbytes == 0:
+        return None
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
 def alloc_act(M: int, K: int, device="cuda"):

@@ -117,3 +117,44 @@ def dream_7b() -> Model:
 
 
 MODELS = {"llada-8b": llada_8b, "dream-7b": dream_7b}
+
+
+# ---------------------------------------------------------------------------
+# Device-side draws with the same distributions (for the multi-GB benchmark
+# models, which would take minutes to draw and copy from the host).
+
+def _torch_gen(device, seed, *sub):
+    import torch
+    g = torch.Generator(device=device)
+    h = int(seed) & 0xFFFFFFFF
+    for s in sub:
+        h = (h * 1000003 + (int(s) & 0xFFFFFFFF)) & 0x7FFFFFFFFFFFFFFF
+    g.manual_seed(h)
+    return g
+
+
+def device_weights(qtype: int, N: int, K: int, seed, *sub, device="cuda"):
+    """GGUF blocks as a flat uint8 device tensor, drawn on the device (torch generator)."""
+    import torch
+    assert K % QK_K == 0
+    nb = N * (K // QK_K)
+    g = _torch_gen(device, seed, qtype, *sub)
+    bb = BLOCK_BYTES[qtype]
+    blk = torch.empty((nb, bb), dtype=torch.uint8, device=device)
+    d = (torch.rand((nb, 2 if qtype == Q4_K else 1), generator=g, device=device) * (1e-2 - 1e-3) + 1e-3)
+    d16 = d.to(torch.float16).contiguous().view(torch.uint8).reshape(nb, -1)
+    if qtype == Q4_K:
+        blk[:, 0:4] = d16
+        blk[:, 4:] = torch.randint(0, 256, (nb, 140), generator=g, device=device, dtype=torch.uint8)
+    else:
+        blk[:, 0:192] = torch.randint(0, 256, (nb, 192), generator=g, device=device, dtype=torch.uint8)
+        blk[:, 192:208] = torch.randint(-32, 32, (nb, 16), generator=g, device=device,
+                                        dtype=torch.int8).view(torch.uint8)
+        blk[:, 208:210] = d16
+    return blk.reshape(-1)
+
+
+def device_activations(M: int, K: int, seed, *sub, device="cuda"):
+    import torch
+    g = _torch_gen(device, seed, 8, *sub)
+    return torch.randn((M, K), generator=g, device=device, dtype=torch.float32)

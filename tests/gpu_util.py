@@ -68,8 +68,10 @@ def gemm(w_dev, qtype, N, K, act: Act, rows=None, ldo=None, stream=None):
     n_out = act.M if rows is None else len(rows)
     out = torch.full((n_out, ldo), float("nan"), dtype=torch.float32, device="cuda")
     r = None if rows is None else torch.tensor(np.asarray(rows, np.int32), device="cuda")
-    dllm.dllm_qgemm(w_dev, qtype, N, K, act.q, act.scale, act.sums, act.M, r, 0 if rows is None else len(rows),
-                    out, ldo, None, 0, stream)
+    nr = 0 if rows is None else len(rows)
+    wsb = dllm.dllm_qgemm_workspace_bytes(qtype, N, K, act.M, nr)
+    ws = dllm.alloc_workspace(wsb)
+    dllm.dllm_qgemm(w_dev, qtype, N, K, act.q, act.scale, act.sums, act.M, r, nr, out, ldo, ws, wsb, stream)
     return out
 
 

@@ -141,7 +141,9 @@ def test_tensor_core_integers_extreme_values():
 # ------------------------------------------------------------------ f32 GEMM
 
 SHAPES = [(1, 128, 256), (15, 128, 512), (16, 256, 256), (17, 384, 768), (64, 256, 512), (160, 128, 512),
-          (257, 256, 256)]
+          (257, 256, 256),
+          # K long enough that tiles are split over several CTAs (chunk partials + fix-up)
+          (17, 256, 2048), (160, 128, 4096), (1, 384, 4096), (300, 256, 3072)]
 
 
 @pytest.mark.parametrize("qtype", [Q4, Q6])
@@ -238,21 +240,35 @@ def test_rows_out_of_range_sets_status():
 
 @pytest.mark.parametrize("qtype", [Q4, Q6])
 @pytest.mark.parametrize("with_v", [True, False])
-def test_qkv_matches_separate(qtype, with_v):
+def test_qkv_matches_oracle_and_separate(qtype, with_v):
+    """One launch over two or three weight matrices sharing one quantized activation.
+    The fused launch may split K differently from separate launches (the split
+    depends on the launch's total N), so it is compared with the oracle and with the
+    separate launches within the tolerance, and with itself bit for bit."""
     M, Nq, Nkv, K = 40, 256, 128, 512
     x = synth.activations(M, K, 60)
-    ws = [synth.weights(qtype, n, K, 60, i) for i, n in enumerate((Nq, Nkv, Nkv))]
-    wd = [dllm.repack(qtype, w, w.shape[0], K) for w in ws]
+    wts = [synth.weights(qtype, n, K, 60, i) for i, n in enumerate((Nq, Nkv, Nkv))]
+    wd = [dllm.repack(qtype, w, w.shape[0], K) for w in wts]
     act = gu.Act(x)
-    oq = torch.empty((M, Nq), device="cuda")
-    ok = torch.empty((M, Nkv), device="cuda")
-    ov = torch.empty((M, Nkv), device="cuda") if with_v else None
-    dllm.dllm_qkv_qgemm(wd[0], wd[1], wd[2] if with_v else None, qtype, Nq, Nkv, K, act.q, act.scale, act.sums,
-                        M, oq, Nq, ok, ov, Nkv)
-    outs = [oq, ok] + ([ov] if with_v else [])
+    oq_, os_, _ = oracle.quantize_act(x)
+
+    def fused():
+        oq = torch.empty((M, Nq), device="cuda")
+        ok = torch.empty((M, Nkv), device="cuda")
+        ov = torch.empty((M, Nkv), device="cuda") if with_v else None
+        wsb = dllm.dllm_qgemm_workspace_bytes(qtype, Nq + (2 if with_v else 1) * Nkv, K, M)
+        work = dllm.alloc_workspace(wsb)
+        dllm.dllm_qkv_qgemm(wd[0], wd[1], wd[2] if with_v else None, qtype, Nq, Nkv, K, act.q, act.scale,
+                            act.sums, M, oq, Nq, ok, ov, Nkv, work, wsb)
+        return [oq, ok] + ([ov] if with_v else [])
+
+    outs, again = fused(), fused()
     for i, o in enumerate(outs):
-        sep = gu.gemm(wd[i], qtype, ws[i].shape[0], K, act)
-        assert torch.equal(o, sep)
+        assert torch.equal(o, again[i])
+        _, ref, T = oracle.qgemm(qtype, wts[i], wts[i].shape[0], K, oq_, os_)
+        assert gu.tol_ok(o.cpu().numpy(), ref, T)[0]
+        sep = gu.gemm(wd[i], qtype, wts[i].shape[0], K, act).cpu().numpy()
+        assert gu.tol_ok(sep, ref, T)[0]
 
 
 # ------------------------------------------------------------------ full-size shapes, sampled outputs
@@ -287,3 +303,52 @@ def test_full_output_projection_rows_sampled():
     M = 160
     rows = synth.block_rows(M, 32, 3)
     _sampled_parity(Q6, M, 126464, 4096, 3, rows=rows, n_samples=4, width=128)
+
+
+# ------------------------------------------------------------------ split-K workspace contract
+
+def test_workspace_shared_across_calls_and_shapes():
+    """One zero-filled workspace reused by GEMMs whose tiles split K differently: every
+    call stays correct and leaves each arrival counter at a multiple of 16."""
+    M, K = 48, 4096
+    x = synth.activations(M, K, 70)
+    act = gu.Act(x)
+    oq, os_, _ = oracle.quantize_act(x)
+    cases = []
+    # few tiles split K four ways; 128 tiles fill the SMs without splitting
+    for i, (qtype, N) in enumerate([(Q4, 128), (Q6, 384), (Q4, 16384), (Q6, 128)]):
+        w = synth.weights(qtype, N, K, 70, i)
+        _, ref, T = oracle.qgemm(qtype, w, N, K, oq, os_)
+        cases.append((qtype, N, dllm.repack(qtype, w, N, K), ref, T))
+    wsb = max(dllm.dllm_qgemm_workspace_bytes(qt, N, K, M) for qt, N, *_ in cases)
+    ws = dllm.alloc_workspace(wsb)
+    first = {}
+    for rep in range(3):
+        for qtype, N, wd, ref, T in cases:
+            out = torch.empty((M, N), device="cuda")
+            dllm.dllm_qgemm(wd, qtype, N, K, act.q, act.scale, act.sums, M, None, 0, out, N, ws, wsb)
+            got = out.cpu().numpy()
+            assert gu.tol_ok(got, ref, T)[0]
+            if rep == 0:
+                first[N, qtype] = got
+            else:
+                assert np.array_equal(first[N, qtype], got)
+    torch.cuda.synchronize()
+    ctr = ws[:4 * 3].cpu().numpy().view(np.uint32)  # tiles of the split calls: one counter each
+    assert np.all(ctr % 16 == 0) and np.all(ctr > 0)
+
+
+def test_workspace_too_small_is_rejected():
+    M, N, K = 32, 256, 2048
+    w, x = gu.make_case(Q4, M, N, K, 71)
+    wd = dllm.repack(Q4, w, N, K)
+    act = gu.Act(x)
+    wsb = dllm.dllm_qgemm_workspace_bytes(Q4, N, K, M)
+    assert wsb > 0  # two tiles on many SMs: K is split
+    out = torch.empty((M, N), device="cuda")
+    with pytest.raises(dllm.DllmError) as e:
+        dllm.dllm_qgemm(wd, Q4, N, K, act.q, act.scale, act.sums, M, None, 0, out, N, None, 0)
+    assert e.value.code == dllm.DLLM_ERR_WORKSPACE
+    small = dllm.alloc_workspace(wsb - 256)
+    with pytest.raises(dllm.DllmError):
+        dllm.dllm_qgemm(wd, Q4, N, K, act.q, act.scale, act.sums, M, None, 0, out, N, small, wsb - 256)

@@ -74,7 +74,7 @@ int dllm_repack_q4k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dl
 int dllm_repack_q6k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
 
 /* ------------------------------------------------------------------------------
- * Activations: int8 with one f32 scale per 256 elements, plus per-32 sums
+ * Activations: int8 with one f32 scale per 256 elements, plus scaled per-32 sums
  * (Architecture page, "Source map", kernels/qgemm.mojo row; "A forward pass",
  * step 2: quantized once, reused by Q/K/V and by gate/up).
  *
@@ -89,9 +89,12 @@ int dllm_repack_q6k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dl
  *                (k = 256 s + 16 c + j), row r of the group, byte j.  Each group of 8
  *                rows x 16 bytes is one 128-byte core matrix of the tensor-core B operand.
  *   scale f32   [K/256][Mp]
- *   sums  uint8 [K/256][Mp][16]: for the 8 sub-blocks of 32 of super-block s, the sum
- *                t_j of the 32 qa values split as t_j = lo_j + 256*hi_j with lo_j =
- *                t_j & 255 in byte j (unsigned) and hi_j = t_j >> 8 in byte 8 + j (signed).
+ *   sums  f32   [K/256][Mp/8][4][8][4]: for the 8 sub-blocks of 32 of super-block s,
+ *                v_j = scale * t_j (t_j the sum of the sub-block's 32 qa values, one f32
+ *                multiply), stored as v_j = hi_j + lo_j where hi_j is v_j with its low 13
+ *                mantissa bits cleared and lo_j = v_j - hi_j (exact).  Per super-block and
+ *                8-row group, 512 bytes: [hi j0-3 | hi j4-7 | lo j0-3 | lo j4-7], each a
+ *                [8 rows][4 floats] block (the tensor-core operand order of the min term).
  * dllm_act_bytes() gives the three sizes for (M, K).
  * ---------------------------------------------------------------------------- */
 int dllm_act_bytes(int64_t M, int64_t K, size_t* q_bytes, size_t* scale_bytes, size_t* sums_bytes);
@@ -152,12 +155,12 @@ const char* dllm_status_string(int code);
 int dllm_debug_subblock_dots(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, int64_t M,
                              int32_t* dots, dllm_stream_t stream);
 
-/* The per-super-block integers the tensor-core path forms, read back from tensor
- * memory instead of being combined: S[m][n][s] = sum_j sc_j * dot_j and (Q4_K)
- * Smin[m][n][s] = sum_j m_j * sum32_j, int32 [M][N][K/256] each (Smin untouched for
- * Q6_K).  Same kernel and schedule as dllm_qgemm with the f32 epilogue replaced. */
+/* The per-super-block integers the int8 tensor-core path forms, read back from
+ * tensor memory instead of being combined: S[m][n][s] = sum_j sc_j * dot_j (Q4_K) or
+ * sum_j sc_j * dot_j with q - 32 (Q6_K), int32 [M][N][K/256].  Same kernel and
+ * schedule as dllm_qgemm with the f32 epilogue replaced. */
 int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
-                       const uint8_t* sums, int64_t M, int32_t* S, int32_t* Smin, dllm_stream_t stream);
+                       const uint8_t* sums, int64_t M, int32_t* S, dllm_stream_t stream);
 
 /* int8 tensor-core throughput probe: on each of `ctas` CTAs, `issuers` warps (1..4)
  * each issue `iters` back-to-back tcgen05 kind::i8 MMAs of 128 x n x 32 into their own

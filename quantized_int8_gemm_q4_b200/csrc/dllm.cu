@@ -87,7 +87,7 @@ Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
         p.gs_off = off;
         off += align256((size_t)nsb * p.Mp * 4);
         p.gu_off = off;
-        off += align256((size_t)nsb * p.Mp * 16);
+        off += align256((size_t)nsb * p.Mp * 64);
     }
     p.bytes = (p.kc > 1 || n_rows > 0) ? off : 0;
     return p;
@@ -169,7 +169,7 @@ int dllm_act_bytes(int64_t M, int64_t K, size_t* q_bytes, size_t* scale_bytes, s
     const int64_t Mp = round_up(M, 16);
     *q_bytes = (size_t)Mp * K;
     *scale_bytes = (size_t)Mp * (K / QK) * 4;
-    *sums_bytes = (size_t)Mp * (K / QK) * 16;
+    *sums_bytes = (size_t)Mp * (K / QK) * 64;
     return DLLM_OK;
 }
 
@@ -238,7 +238,7 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
         int8_t* gq = reinterpret_cast<int8_t*>(ws + p.gq_off);
         float* gs = reinterpret_cast<float*>(ws + p.gs_off);
         uint8_t* gu = ws + p.gu_off;
-        const int64_t work = nsb * p.Mp * 18;
+        const int64_t work = nsb * p.Mp * 21;
         gather_rows_kernel<<<grid_for(work, 256), 256, 0, s>>>(q, scale, sums, M, round_up(M, 16), rows,
                                                                 (int32_t)n_rows, p.Mp, (int32_t)nsb, gq, gs, gu);
         if ((rc = launch_status())) return rc;
@@ -452,8 +452,8 @@ int dllm_debug_subblock_dots(const void* w, dllm_qtype t, int64_t N, int64_t K, 
 }
 
 int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
-                       const uint8_t* sums, int64_t M, int32_t* S, int32_t* Smin, dllm_stream_t stream) {
-    if (!w || !S || (t == DLLM_Q4_K && !Smin)) return DLLM_ERR_ARG;
+                       const uint8_t* sums, int64_t M, int32_t* S, dllm_stream_t stream) {
+    if (!w || !S) return DLLM_ERR_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     GemmArgs a;
     int rc = gemm_common(a, t, N, K, q, scale, sums, M, nullptr, 0, nullptr, 0, true, s);
@@ -462,7 +462,6 @@ int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
     a.nseg = 1;
     a.n_tiles = (int32_t)(N / TROWS);
     a.dbg_S = S;
-    a.dbg_Smin = Smin;
     a.dbg_N = N;
     return dispatch(a, t, true, s);
 }

@@ -113,14 +113,17 @@ __global__ void repack_q6k_kernel(const uint8_t* __restrict__ src, int64_t N, in
 // One CTA of 8 warps per (8-row group g, super-block s); warp w owns row 8g + w.
 // Lane l holds elements 8l..8l+7 of the 256-block: amax by warp reduction, then
 // iscale = 127/amax and scale = amax/127 as IEEE f32 divisions, qa =
-// round-half-even(x * iscale) clamped to [-127, 127].  The 8 x 256 bytes are
-// staged in shared memory in the core-matrix order and written with 16-byte stores.
+// round-half-even(x * iscale) clamped to [-127, 127].  For each sub-block of 32 the
+// sum t_j of its qa values is also emitted multiplied by the block scale, as two
+// floats v_hi + v_lo = scale * t_j (v_hi exact as a tf32 operand): the B operand of
+// the min-term MMA of Q4_K weights.  Outputs are staged in shared memory in the
+// tensor-core operand order and written with 16-byte stores.
 __global__ void __launch_bounds__(256) quantize_act_kernel(const float* __restrict__ x, int64_t M, int64_t ldx,
                                                            int64_t Mp, int8_t* __restrict__ q,
                                                            float* __restrict__ scale,
                                                            uint8_t* __restrict__ sums) {
     __shared__ __align__(16) uint8_t tile[16 * 8 * 16];  // [chunk][row][16 B]
-    __shared__ __align__(16) uint8_t tsum[8 * 16];       // [row][16 B]
+    __shared__ __align__(16) float tsum[4 * 8 * 4];      // [hi j0-3, hi j4-7, lo j0-3, lo j4-7][row][4]
     __shared__ float tscale[8];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t g = blockIdx.x, s = blockIdx.y;
@@ -141,6 +144,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const float* __restri
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float iscale = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    const float sc = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
     uint32_t packed[2] = {0u, 0u};
     int part = 0;
 #pragma unroll
@@ -157,20 +161,22 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const float* __restri
     part += __shfl_xor_sync(0xffffffffu, part, 2);
     if ((lane & 3) == 0) {
         const int j = lane >> 2;
-        tsum[w * 16 + j] = (uint8_t)(part & 255);
-        tsum[w * 16 + 8 + j] = (uint8_t)(int8_t)(part >> 8);
+        float hi, lo;
+        split_tf32(__fmul_rn(sc, (float)part), hi, lo);
+        tsum[((j >> 2) * 8 + w) * 4 + (j & 3)] = hi;
+        tsum[((2 + (j >> 2)) * 8 + w) * 4 + (j & 3)] = lo;
     }
-    if (lane == 0) tscale[w] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    if (lane == 0) tscale[w] = sc;
     __syncthreads();
     const int tid = threadIdx.x;
     if (tid < 128) {
         uint4* dq = reinterpret_cast<uint4*>(q + ((s * (Mp / 8) + g) * 16) * 128);
         dq[tid] = reinterpret_cast<const uint4*>(tile)[tid];
-    } else if (tid < 136) {
-        uint4* ds = reinterpret_cast<uint4*>(sums + (s * Mp + 8 * g) * 16);
+    } else if (tid < 160) {
+        uint4* ds = reinterpret_cast<uint4*>(sums + (s * (Mp / 8) + g) * 512);
         ds[tid - 128] = reinterpret_cast<const uint4*>(tsum)[tid - 128];
-    } else if (tid < 144) {
-        scale[s * Mp + 8 * g + (tid - 136)] = tscale[tid - 136];
+    } else if (tid < 168) {
+        scale[s * Mp + 8 * g + (tid - 160)] = tscale[tid - 160];
     }
 }
 

@@ -8,39 +8,42 @@
 //   S    = sum_k (q_k * sc_j(k)) * a_k      (Q6_K: (q_k - 32) * sc_j(k))
 //   Smin = sum_j m_j * sum32_j(a)
 //
-// How it is computed.  The tensor core multiplies 8-bit operands, and q*sc needs
-// 10 bits (Q4_K) or 13 bits (Q6_K), so the weight operand is split into two 8-bit
-// planes whose integer results are recombined exactly:
+// The d-term, on the int8 tensor pipe, exactly.  The tensor core multiplies 8-bit
+// operands, and q*sc needs 10 bits (Q4_K) or 13 bits (Q6_K), so the weight operand
+// is split into two 8-bit planes whose integer results are recombined exactly:
 //   Q4_K: sc = lo3 + 8*hi3 (3 bits each); plane 0 = q*lo3, plane 1 = q*hi3, both in
 //         0..105 (u8).  S = P0 + 8*P1.
 //   Q6_K: v = (q-32)*sc + 32896 lies in [28800, 36992]; plane 0 = (v & 255) - 128,
 //         plane 1 = (v >> 8) - 128 (both s8), and plane0 + 256*plane1 = (q-32)*sc.
-// The min term of Q4_K is two more MMAs per super-block with the mins m_j (u8) as A
-// and the per-32 activation sums, split into an unsigned low byte and a signed high
-// byte, as B: Smin = Ml + 256*Mh.
+// Each plane accumulator stays within 2^22 in magnitude.  Tensor memory is preset to
+// the bit pattern of 1.5*2^23 before each super-block, so the int32 the MMAs leave
+// there, read as an f32, is exactly 1.5*2^23 + value, and the epilogue recovers S
+// with one FFMA and one FADD (packed f32x2), with no integer-to-float instruction.
+// The epilogue then accumulates da * d * S in f32 registers.
 //
-// Every integer accumulator stays within 2^22 in magnitude.  Tensor memory is preset
-// to the bit pattern of 1.5*2^23 before each super-block, so the int32 the MMAs
-// leave there, read as an f32, is exactly 1.5*2^23 + value; the epilogue turns it
-// into floats with one FFMA and one FADD per pair of accumulators (no
-// integer-to-float conversion instruction), in packed f32x2 arithmetic.
+// The min term (Q4_K), on the tf32 tensor pipe.  Its per-super-block factor
+// dmin[n] * da[m] is a product of a row term and a column term, so
+//   -sum_sb da dmin Smin = sum over (sb, j) of (-dmin m_j)[n] * (da sum32_j)[m],
+// a GEMM with one K step per sub-block.  Both operands are split as hi + lo with hi
+// exact in tf32 (-dmin m_j is exact in hi + lo; da*sum32_j loses at most 2^-22 of
+// itself), and hi*hi + hi*lo + lo*hi accumulate in an f32 tensor-memory accumulator
+// over the whole K range, read once per work unit.  Its error is below 2^-21 of the
+// min term's magnitude, inside the 1e-6 * sum|terms| tolerance.
 //
 // Roles (16 warps, one CTA per SM, persistent over work units):
 //   warp 0      producer: bulk copies of weight tiles and activation tiles into
 //               shared-memory rings
 //   warps 1-3   tensor-memory allocation (warp 1) and MMA issue.  One thread can
-//               issue a tcgen05.mma only every ~28 ns, longer than a 48-token MMA
+//               issue a tcgen05.mma only every ~28 ns, longer than a 64-token MMA
 //               takes, so three warps share the work: for each token tile the roles
 //               plane 0, plane 1 and min term rotate over them, each role owning its
-//               own accumulators, and a role's MMAs go out back to back with
-//               precomputed descriptors
+//               own accumulator, and a role's MMAs go out back to back
 //   warps 4-7   unpack: thread = weight row; decode the super-block, build the two
 //               weight planes per K-step of 32 into tensor memory (the A operand),
-//               the mins into shared memory, and the f32 d/dmin
+//               the min-term A operand into shared memory, and the f32 d
 //   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each on half of
-//               the token columns; per super-block, read the integer accumulators in
-//               a few wide loads, preset them again, and accumulate the f32 result in
-//               registers
+//               the token columns; per super-block, read the two plane accumulators,
+//               preset them again, and accumulate the f32 result in registers
 //
 // A work unit is (128 weight rows, up to 128 canvas rows, one K-chunk).  The number
 // of K-chunks per tile depends only on N, K and the SM count, never on M or on the
@@ -55,43 +58,49 @@ constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float MAGIC = 12582912.0f;
 constexpr int GEMM_THREADS = 512;
 constexpr int UNIT_TOKENS = 128;
+constexpr int NTOK = 64;                           // token columns per MMA and per accumulator
+constexpr int TMAX = UNIT_TOKENS / NTOK;           // token tiles per unit
+constexpr int HC = NTOK / 2;                       // token columns per epilogue warp
 constexpr int MAX_KC = 16;                         // K-chunks per tile, at most
+constexpr int ISSUERS = 3;                         // MMA-issuing warps
+constexpr int S_SLOTS = 4;                         // d ring (unpack -> epilogue)
+constexpr int ACC_SETS = 2;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
+
+// tensor-memory columns
+constexpr uint32_t TM_A = 0;      // 8 K-step slots x 16 columns (plane 0 | plane 1)
+constexpr uint32_t TM_ACC = 128;  // ACC_SETS x 2 planes x NTOK columns
+constexpr uint32_t TM_MIN = 384;  // TMAX x NTOK columns: f32 min-term accumulators (Q4_K)
+constexpr uint32_t TM_COLS = 512;
+
+// Activation "sums" operand of one super-block: per 8-row group 512 bytes =
+// [hi j0-3 | hi j4-7 | lo j0-3 | lo j4-7] x [8 rows x 16 bytes].
+constexpr int SUMS_GROUP = 512;
 
 template <int QT>
 struct GemmCfg;
 template <>
 struct GemmCfg<12> {  // Q4_K
     static constexpr int TILE = Q4K_TILE;
-    static constexpr int NTOK = 48;  // token columns per MMA and per accumulator
-    static constexpr int NACC = 4;   // P0, P1, Ml, Mh
+    static constexpr bool MIN = true;
     static constexpr int W_STAGES = 4;
-    static constexpr int B_STAGES = 6;
+    static constexpr int B_STAGES = 4;
     static constexpr int B_Q = NTOK * 256;
-    static constexpr int B_SUMS = NTOK * 16 + 128;
-    static constexpr int B_STAGE = (B_Q + B_SUMS + NTOK * 4 + 127) / 128 * 128;
-    static constexpr int MINA = 2 * 4096;  // [Ml-A | Mh-A], canonical K-major 128 rows x 32 B
+    static constexpr int B_SUMS = NTOK / 8 * SUMS_GROUP;
+    static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
+    static constexpr int MINA = 2 * 4096;  // -dmin*m_j as [hi | lo], canonical K-major 128 rows x 32 B
 };
 template <>
 struct GemmCfg<14> {  // Q6_K
     static constexpr int TILE = Q6K_TILE;
-    static constexpr int NTOK = 64;
-    static constexpr int NACC = 2;  // P0, P1
+    static constexpr bool MIN = false;
     static constexpr int W_STAGES = 3;
     static constexpr int B_STAGES = 4;
     static constexpr int B_Q = NTOK * 256;
     static constexpr int B_SUMS = 0;
-    static constexpr int B_STAGE = (B_Q + B_SUMS + NTOK * 4 + 127) / 128 * 128;
+    static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
     static constexpr int MINA = 0;
 };
-
-constexpr int S_SLOTS = 4;  // d/dmin ring (unpack -> epilogue)
-constexpr int ISSUERS = 3;  // MMA-issuing warps
-constexpr int ACC_SETS = 2;
-// tensor-memory columns
-constexpr uint32_t TM_A = 0;      // 8 K-step slots x 16 columns (plane 0 | plane 1)
-constexpr uint32_t TM_ACC = 128;  // ACC_SETS x NACC x NTOK columns
-constexpr uint32_t TM_COLS = 512;
 
 struct Segment {
     const uint8_t* w;  // repacked weights
@@ -114,9 +123,8 @@ struct GemmArgs {
     int32_t n_st;      // token super-tiles
     int32_t mu;        // tokens per super-tile (multiple of 16)
     uint32_t* counters;  // [n_tiles * n_st], when kc > 1
-    float* partials;     // [units][mu][128], when kc > 1
-    int32_t* dbg_S;    // debug: integer outputs instead of f32 (nullable)
-    int32_t* dbg_Smin;
+    float* partials;     // [units][128 rows][mu], when kc > 1
+    int32_t* dbg_S;    // debug: per-super-block integer S instead of f32 (nullable)
     int64_t dbg_N;
 };
 
@@ -126,18 +134,18 @@ struct GemmShared {
     uint64_t a_full[2], a_empty[2];  // A ring halves: K-steps 0-3, and 4-7 (+ the min-term A)
     uint64_t s_full[S_SLOTS], s_empty[S_SLOTS];
     uint64_t acc_full[ACC_SETS], acc_empty[ACC_SETS];
+    uint64_t min_empty;
     uint64_t final_bar[4];
     uint64_t epi_bar;
     uint32_t tmem_base;
     volatile int abort_flag;
     int last_flag;
-    float2 dd[S_SLOTS][TROWS];
+    float dd[S_SLOTS][TROWS];
 };
 
 // Bounded wait on an mbarrier phase; false if this CTA is aborting.  Waiting threads
-// sleep inside try_wait instead of spinning, so the warps sharing their scheduler keep
-// its issue slots.  Raises the abort flag and the device error word when the limit
-// runs out.
+// sleep inside try_wait.  Raises the abort flag and the device error word when the
+// limit runs out.
 __device__ __forceinline__ bool wait_bar(GemmShared& sh, uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -151,11 +159,11 @@ __device__ __forceinline__ bool wait_bar(GemmShared& sh, uint64_t* bar, uint32_t
         }
     }
 }
+// Warp-uniform variant: every lane waits, and the warp agrees on the outcome.
 __device__ __forceinline__ bool wait_bar_warp(GemmShared& sh, uint64_t* bar, uint32_t parity) {
     const bool ok = wait_bar(sh, bar, parity);
     return __all_sync(0xffffffffu, ok);
 }
-
 // Bounded barrier among the 256 epilogue threads.
 __device__ __forceinline__ bool epi_sync(GemmShared& sh, uint32_t& phase) {
     mbar_arrive(&sh.epi_bar);
@@ -171,20 +179,14 @@ template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
-
-// Load / preset this warp's HC (16 + 8 or 16 + 16) consecutive accumulator columns.
-template <int HC>
+// This warp's HC = 32 consecutive accumulator columns.
 __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&x)[HC]) {
-    static_assert(HC == 24 || HC == 32, "column split");
     tmem_ld16(taddr, x);
-    if constexpr (HC == 24) tmem_ld8p(taddr + 16, x + 16);
-    else tmem_ld16(taddr + 16, x + 16);
+    tmem_ld16(taddr + 16, x + 16);
 }
-template <int HC>
 __device__ __forceinline__ void fill_cols(uint32_t taddr, uint32_t v) {
     tmem_fill16(taddr, v);
-    if constexpr (HC == 24) tmem_fill8(taddr + 16, v);
-    else tmem_fill16(taddr + 16, v);
+    tmem_fill16(taddr + 16, v);
 }
 
 struct Unit {
@@ -218,9 +220,6 @@ __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int64_t u) {
 template <int QT, bool DBG>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<QT>;
-    constexpr int NTOK = C::NTOK;
-    constexpr int TMAX = (UNIT_TOKENS + NTOK - 1) / NTOK;
-    constexpr int HC = NTOK / 2;  // token columns per epilogue warp
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* w_stage = smem_raw;
     uint8_t* b_stage = w_stage + C::W_STAGES * C::TILE;
@@ -232,25 +231,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 128); }
-        for (int i = 0; i < C::B_STAGES; i++) {
-            mbar_init(&sh.b_full[i], 1);
-            mbar_init(&sh.b_empty[i], 256);
-        }
+        for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 256); }
         for (int i = 0; i < 2; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], ISSUERS); }
         for (int i = 0; i < S_SLOTS; i++) { mbar_init(&sh.s_full[i], 128); mbar_init(&sh.s_empty[i], 256); }
-        for (int i = 0; i < ACC_SETS; i++) {
-            mbar_init(&sh.acc_full[i], ISSUERS);
-            mbar_init(&sh.acc_empty[i], 256);
-        }
+        for (int i = 0; i < ACC_SETS; i++) { mbar_init(&sh.acc_full[i], ISSUERS); mbar_init(&sh.acc_empty[i], 256); }
+        mbar_init(&sh.min_empty, 256);
         for (int i = 0; i < 4; i++) mbar_init(&sh.final_bar[i], 1);
         mbar_init(&sh.epi_bar, 256);
         sh.abort_flag = 0;
         fence_mbar_init();
-    }
-    if constexpr (C::MINA > 0) {  // the second 16-byte K chunk of the min-term A operands is zero
-        for (int i = threadIdx.x; i < C::MINA / 16; i += GEMM_THREADS)
-            reinterpret_cast<uint4*>(mina)[i] = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
     }
     if (warp == 1) {
         tmem_alloc(&sh.tmem_base, TM_COLS);
@@ -292,13 +281,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         if (!wait_bar_warp(sh, &sh.b_empty[bs], bph ^ 1)) goto prod_done;
                         if (lane == 0) {
                             uint8_t* st = b_stage + bs * C::B_STAGE;
-                            const uint32_t bytes = ntok * 256 + (C::B_SUMS ? ntok * 16 : 0) + ntok * 4;
-                            mbar_arrive_expect_tx(&sh.b_full[bs], bytes);
+                            const uint32_t sums_bytes = C::B_SUMS ? ntok / 8 * SUMS_GROUP : 0;
+                            mbar_arrive_expect_tx(&sh.b_full[bs], ntok * 256 + sums_bytes + ntok * 4);
                             bulk_g2s_hint(st, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256, &sh.b_full[bs],
                                           pol_a);
                             if (C::B_SUMS)
-                                bulk_g2s_hint(st + C::B_Q, args.sums + ((size_t)s * args.Mp + t0) * 16, ntok * 16,
-                                              &sh.b_full[bs], pol_a);
+                                bulk_g2s_hint(st + C::B_Q, args.sums + ((size_t)s * args.Mp + t0) / 8 * SUMS_GROUP,
+                                              sums_bytes, &sh.b_full[bs], pol_a);
                             bulk_g2s_hint(st + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
                                           &sh.b_full[bs], pol_a);
                         }
@@ -315,36 +304,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                 for (int i = 0; i < C::B_STAGES; i++)
                     if (b_iss[i]) (void)wait_bar(sh, &sh.b_full[i], b_ph_issued[i]);
             }
-        } else if (warp - 1 < ISSUERS) {
+        } else {
             // ======================================================== MMA issuers
             // All lanes walk the schedule and wait together; lane 0 issues.  Tile g of
             // this CTA gives plane 0 to issuer (2g) % 3, plane 1 to (2g+1) % 3 and the
-            // min term (Q4_K) to (2g+2) % 3.  Every issuer commits once per tile to
-            // the accumulator set and once per super-block to each half of the A ring.
+            // min term (Q4_K) to (2g+2) % 3.  Every issuer commits once per tile to the
+            // accumulator set and once per super-block to each half of the A ring.
             const int who = warp - 1;
             const bool leader = lane == 0;
-            uint32_t bs = 0, bph = 0, r = 0, rph = 0, sbc = 0, g = 0;
-            for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+            uint32_t bs = 0, bph = 0, r = 0, rph = 0, sbc = 0, g = 0, uc = 0;
+            for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
                 const Unit un = unit_of(args, u);
                 const int T = (un.len + NTOK - 1) / NTOK;
                 for (int s = un.sb0; s < un.sb1; s++, sbc++) {
                     for (int tt = 0; tt < T; tt++, g++) {
                         const int ntok = min(NTOK, un.len - tt * NTOK);
                         const bool last = tt == T - 1;
+                        const int role = (int)((who + 3 - (2 * g) % 3) % 3);  // 0: plane 0, 1: plane 1, 2: min
                         if (!wait_bar_warp(sh, &sh.b_full[bs], bph)) goto mma_done;
                         if (!wait_bar_warp(sh, &sh.acc_empty[r], rph)) goto mma_done;
                         if (tt == 0) {
                             if (!wait_bar_warp(sh, &sh.a_full[0], sbc & 1)) goto mma_done;
                             if (!wait_bar_warp(sh, &sh.a_full[1], sbc & 1)) goto mma_done;
                         }
+                        // a unit's first min-term MMAs overwrite the min accumulators: the
+                        // previous unit's epilogue must have read them out
+                        if (C::MIN && role == 2 && s == un.sb0)
+                            if (!wait_bar_warp(sh, &sh.min_empty, (uc & 1) ^ 1)) goto mma_done;
                         tc_fence_after();
-                        const int role = (int)((who + 3 - (2 * g) % 3) % 3);  // 0: plane 0, 1: plane 1, 2: min
                         if (leader) {
-                            const uint32_t acc = tmem + TM_ACC + r * C::NACC * NTOK;
                             const uint32_t st = smem_u32(b_stage + bs * C::B_STAGE);
                             if (role < 2) {
                                 const uint32_t id = QT == 12 ? idesc_i8(128, ntok, 0, 1) : idesc_i8(128, ntok, 1, 1);
-                                const uint32_t d = acc + role * NTOK;
+                                const uint32_t d = tmem + TM_ACC + (r * 2 + role) * NTOK;
                                 const uint32_t a0 = tmem + TM_A + 8 * role;
                                 const uint64_t b0 = sdesc_kmajor_noswz(st, 128, 2048);
 #pragma unroll
@@ -355,13 +347,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 if (last) tc_commit(&sh.a_empty[1]);
                             } else {
                                 if (last) tc_commit(&sh.a_empty[0]);
-                                if constexpr (QT == 12) {
+                                if constexpr (C::MIN) {
+                                    const uint32_t d = tmem + TM_MIN + tt * NTOK;
+                                    const uint32_t id = idesc_tf32(128, ntok);
                                     const uint32_t ma = smem_u32(mina);
-                                    const uint64_t bd = sdesc_kmajor_noswz(st + C::B_Q, 128, 128);
-                                    mma_i8_ss(acc + 2 * NTOK, sdesc_kmajor_noswz(ma, 128, 256), bd,
-                                              idesc_i8(128, ntok, 0, 0), 1);
-                                    mma_i8_ss(acc + 3 * NTOK, sdesc_kmajor_noswz(ma + 4096, 128, 256), bd,
-                                              idesc_i8(128, ntok, 0, 1), 1);
+                                    const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
+                                    const uint64_t a_lo = sdesc_kmajor_noswz(ma + 4096, 128, 256);
+                                    const uint64_t b_hi = sdesc_kmajor_noswz(st + C::B_Q, 128, SUMS_GROUP);
+                                    const uint64_t b_lo = sdesc_kmajor_noswz(st + C::B_Q + 256, 128, SUMS_GROUP);
+                                    mma_tf32_ss(d, a_hi, b_hi, id, s > un.sb0 ? 1u : 0u);
+                                    mma_tf32_ss(d, a_hi, b_lo, id, 1);
+                                    mma_tf32_ss(d, a_lo, b_hi, id, 1);
                                 }
                                 if (last) tc_commit(&sh.a_empty[1]);
                             }
@@ -382,9 +378,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     } else if (warp < 8) {
         setmaxnreg_dec<88>();
         // ============================================================ unpack
-        // Per super-block: decode this row, then build the planes of K-steps 0-3,
-        // publish them together, then K-steps 4-7 (and the min-term A), so the MMAs
-        // of a super-block can start while the second half is still being built.
+        // Per super-block: decode this row, then build the planes of K-steps 0-3 and
+        // publish them together, then K-steps 4-7 (and the min-term A), so the MMAs of
+        // a super-block can start while the second half is still being built.
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -399,31 +395,37 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     const uint32_t b1 = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_SC + 12 * row + 4);
                     const uint32_t b2 = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_SC + 12 * row + 8);
                     const uint32_t dm = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_D + 4 * row);
-                    uint32_t sc[8], mn[8];
+                    uint32_t sc[8];
+                    float nmin[8];  // -dmin * m_j, exact in f32
+                    const float d = __half2float(__ushort_as_half((unsigned short)(dm & 0xFFFF)));
+                    const float dmin = __half2float(__ushort_as_half((unsigned short)(dm >> 16)));
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
                         sc[j] = (b0 >> (8 * j)) & 63;
-                        mn[j] = (b1 >> (8 * j)) & 63;
                         sc[j + 4] = ((b2 >> (8 * j)) & 15) | (((b0 >> (8 * j + 6)) & 3) << 4);
-                        mn[j + 4] = ((b2 >> (8 * j + 4)) & 15) | (((b1 >> (8 * j + 6)) & 3) << 4);
+                        const uint32_t m_lo = (b1 >> (8 * j)) & 63;
+                        const uint32_t m_hi = ((b2 >> (8 * j + 4)) & 15) | (((b1 >> (8 * j + 6)) & 3) << 4);
+                        nmin[j] = -dmin * (float)m_lo;
+                        nmin[j + 4] = -dmin * (float)m_hi;
                     }
-                    const float d = __half2float(__ushort_as_half((unsigned short)(dm & 0xFFFF)));
-                    const float dmin = __half2float(__ushort_as_half((unsigned short)(dm >> 16)));
                     if (!wait_bar_warp(sh, &sh.s_empty[ss], sph ^ 1)) goto unpack_done;
-                    sh.dd[ss][row] = make_float2(d, -dmin);
+                    sh.dd[ss][row] = d;
                     mbar_arrive(&sh.s_full[ss]);
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
 #pragma unroll
                     for (int half = 0; half < 2; half++) {
                         if (!wait_bar_warp(sh, &sh.a_empty[half], (sbc & 1) ^ 1)) goto unpack_done;
                         if (half == 1) {
-                            // mins: the A operands of the two min-term MMAs, row `row` of
-                            // the canonical K-major layout (8-row groups of 256 bytes)
-                            const uint32_t m03 = mn[0] | (mn[1] << 8) | (mn[2] << 16) | (mn[3] << 24);
-                            const uint32_t m47 = mn[4] | (mn[5] << 8) | (mn[6] << 16) | (mn[7] << 24);
+                            // -dmin*m_j as tf32 hi + lo: row `row` of the canonical K-major
+                            // layout (8-row groups of 256 bytes, two 16-byte K chunks)
+                            float hi[8], lo[8];
+#pragma unroll
+                            for (int j = 0; j < 8; j++) split_tf32(nmin[j], hi[j], lo[j]);
                             uint8_t* base = mina + (row >> 3) * 256 + (row & 7) * 16;
-                            *reinterpret_cast<uint4*>(base) = make_uint4(m03, m47, 0, 0);
-                            *reinterpret_cast<uint4*>(base + 4096) = make_uint4(0, 0, m03, m47);
+                            *reinterpret_cast<float4*>(base) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+                            *reinterpret_cast<float4*>(base + 128) = make_float4(hi[4], hi[5], hi[6], hi[7]);
+                            *reinterpret_cast<float4*>(base + 4096) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+                            *reinterpret_cast<float4*>(base + 4096 + 128) = make_float4(lo[4], lo[5], lo[6], lo[7]);
                             fence_proxy_async_smem();
                         }
 #pragma unroll
@@ -456,7 +458,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     const float d = __half2float(
                         __ushort_as_half(*reinterpret_cast<const unsigned short*>(tl + Q6K_OFF_D + 2 * row)));
                     if (!wait_bar_warp(sh, &sh.s_empty[ss], sph ^ 1)) goto unpack_done;
-                    sh.dd[ss][row] = make_float2(d, 0.0f);
+                    sh.dd[ss][row] = d;
                     mbar_arrive(&sh.s_full[ss]);
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
 #pragma unroll
@@ -512,14 +514,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         const int row = quad * 32 + lane;
         const int etid = threadIdx.x - 256;  // 0..255
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        {
-            for (int r = 0; r < ACC_SETS; r++)
-                for (int a = 0; a < C::NACC; a++)
-                    fill_cols<HC>(tmem + lane_off + TM_ACC + (r * C::NACC + a) * NTOK + half * HC, MAGIC_BITS);
-            tmem_wait_st();
-            tc_fence_before();
-            for (int r = 0; r < ACC_SETS; r++) mbar_arrive(&sh.acc_empty[r]);
-        }
+        for (int r = 0; r < ACC_SETS; r++)
+            for (int a = 0; a < 2; a++) fill_cols(tmem + lane_off + TM_ACC + (r * 2 + a) * NTOK + half * HC, MAGIC_BITS);
+        tmem_wait_st();
+        tc_fence_before();
+        for (int r = 0; r < ACC_SETS; r++) mbar_arrive(&sh.acc_empty[r]);
         const float2 k8 = make_float2(8.0f, 8.0f), k256 = make_float2(256.0f, 256.0f);
         const float2 m9 = make_float2(-9.0f * MAGIC, -9.0f * MAGIC);
         const float2 m257 = make_float2(-257.0f * MAGIC, -257.0f * MAGIC);
@@ -535,10 +534,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                 for (int j = 0; j < HC / 2; j++) acc[t][j] = make_float2(0.0f, 0.0f);
             for (int s = un.sb0; s < un.sb1; s++) {
                 if (!wait_bar_warp(sh, &sh.s_full[ss], sph)) goto epi_done;
-                const float2 dd = sh.dd[ss][row];
+                const float dv = sh.dd[ss][row];
                 mbar_arrive(&sh.s_empty[ss]);
                 if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
-                const float2 d2 = make_float2(dd.x, dd.x), nm2 = make_float2(dd.y, dd.y);
+                const float2 d2 = make_float2(dv, dv);
 #pragma unroll
                 for (int tt = 0; tt < TMAX; tt++) {
                     if (tt < T) {
@@ -546,71 +545,34 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         if (!wait_bar_warp(sh, &sh.acc_full[r], rph)) goto epi_done;
                         if (!wait_bar_warp(sh, &sh.b_full[bs], bph)) goto epi_done;
                         tc_fence_after();
-                        const uint32_t acc_t = tmem + lane_off + TM_ACC + r * C::NACC * NTOK + half * HC;
+                        const uint32_t acc_t = tmem + lane_off + TM_ACC + r * 2 * NTOK + half * HC;
                         const float* da = reinterpret_cast<const float*>(b_stage + bs * C::B_STAGE + C::B_Q + C::B_SUMS);
                         if (half * HC < ntok) {
-                            // plane accumulators: S = P0 + 8 P1 (Q4_K) or P0 + 256 P1 (Q6_K)
                             uint32_t x0[HC], x1[HC];
-                            load_cols<HC>(acc_t, x0);
-                            load_cols<HC>(acc_t + NTOK, x1);
+                            load_cols(acc_t, x0);
+                            load_cols(acc_t + NTOK, x1);
                             tmem_wait_ld();
-                            fill_cols<HC>(acc_t, MAGIC_BITS);
-                            fill_cols<HC>(acc_t + NTOK, MAGIC_BITS);
-                            float2 S[HC / 2];
-#pragma unroll
-                            for (int i = 0; i < HC / 2; i++) {
-                                const float2 X0 = make_float2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
-                                const float2 X1 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
-                                S[i] = QT == 12 ? __fadd2_rn(__ffma2_rn(X1, k8, m9), X0)
-                                                : __fadd2_rn(__ffma2_rn(X1, k256, m257), X0);
-                            }
+                            fill_cols(acc_t, MAGIC_BITS);
+                            fill_cols(acc_t + NTOK, MAGIC_BITS);
                             if constexpr (DBG) {
-                                uint32_t y0[HC], y1[HC];
-                                if constexpr (QT == 12) {
-                                    load_cols<HC>(acc_t + 2 * NTOK, y0);
-                                    load_cols<HC>(acc_t + 3 * NTOK, y1);
-                                    tmem_wait_ld();
-                                    fill_cols<HC>(acc_t + 2 * NTOK, MAGIC_BITS);
-                                    fill_cols<HC>(acc_t + 3 * NTOK, MAGIC_BITS);
-                                }
 #pragma unroll
                                 for (int i = 0; i < HC; i++) {
                                     const int64_t m = un.m0 + tt * NTOK + half * HC + i;
                                     if (half * HC + i < ntok && m < args.m_out) {
                                         const int64_t n = un.tile * TROWS + row;
-                                        const int64_t o = (m * args.dbg_N + n) * args.nsb + s;
-                                        if constexpr (QT == 12) {
-                                            args.dbg_S[o] = (int32_t)(x0[i] - MAGIC_BITS) + 8 * (int32_t)(x1[i] - MAGIC_BITS);
-                                            args.dbg_Smin[o] = (int32_t)(y0[i] - MAGIC_BITS) + 256 * (int32_t)(y1[i] - MAGIC_BITS);
-                                        } else {
-                                            args.dbg_S[o] = (int32_t)(x0[i] - MAGIC_BITS) + 256 * (int32_t)(x1[i] - MAGIC_BITS);
-                                        }
+                                        const int32_t P0 = (int32_t)(x0[i] - MAGIC_BITS), P1 = (int32_t)(x1[i] - MAGIC_BITS);
+                                        args.dbg_S[(m * args.dbg_N + n) * args.nsb + s] = P0 + (QT == 12 ? 8 : 256) * P1;
                                     }
                                 }
                             } else {
-                                if constexpr (QT == 12) {
-                                    // min accumulators: Smin = Ml + 256 Mh
-                                    load_cols<HC>(acc_t + 2 * NTOK, x0);
-                                    load_cols<HC>(acc_t + 3 * NTOK, x1);
-                                    tmem_wait_ld();
-                                    fill_cols<HC>(acc_t + 2 * NTOK, MAGIC_BITS);
-                                    fill_cols<HC>(acc_t + 3 * NTOK, MAGIC_BITS);
 #pragma unroll
-                                    for (int i = 0; i < HC / 2; i++) {
-                                        const float2 X2 = make_float2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
-                                        const float2 X3 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
-                                        const float2 Sm = __fadd2_rn(__ffma2_rn(X3, k256, m257), X2);
-                                        const float2 t = __ffma2_rn(Sm, nm2, __fmul2_rn(S[i], d2));
-                                        const float2 dav = *reinterpret_cast<const float2*>(da + half * HC + 2 * i);
-                                        acc[tt][i] = __ffma2_rn(t, dav, acc[tt][i]);
-                                    }
-                                } else {
-#pragma unroll
-                                    for (int i = 0; i < HC / 2; i++) {
-                                        const float2 t = __fmul2_rn(S[i], d2);
-                                        const float2 dav = *reinterpret_cast<const float2*>(da + half * HC + 2 * i);
-                                        acc[tt][i] = __ffma2_rn(t, dav, acc[tt][i]);
-                                    }
+                                for (int i = 0; i < HC / 2; i++) {
+                                    const float2 X0 = make_float2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
+                                    const float2 X1 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+                                    const float2 S = QT == 12 ? __fadd2_rn(__ffma2_rn(X1, k8, m9), X0)
+                                                              : __fadd2_rn(__ffma2_rn(X1, k256, m257), X0);
+                                    const float2 dav = *reinterpret_cast<const float2*>(da + half * HC + 2 * i);
+                                    acc[tt][i] = __ffma2_rn(__fmul2_rn(S, d2), dav, acc[tt][i]);
                                 }
                             }
                         }
@@ -622,6 +584,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         if (++r == ACC_SETS) { r = 0; rph ^= 1; }
                     }
                 }
+            }
+            if constexpr (C::MIN) {
+                // the min-term accumulators: complete, since every tile's last MMAs were
+                // covered by the accumulator barriers waited on above
+#pragma unroll
+                for (int tt = 0; tt < TMAX; tt++) {
+                    if (tt < T && half * HC < un.len - tt * NTOK) {
+                        uint32_t y[HC];
+                        load_cols(tmem + lane_off + TM_MIN + tt * NTOK + half * HC, y);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < HC / 2; i++)
+                            acc[tt][i] = __fadd2_rn(acc[tt][i], make_float2(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1])));
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sh.min_empty);
             }
             if constexpr (!DBG) {
                 const int64_t n = un.tile * TROWS + row;
@@ -644,8 +623,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     float* part = args.partials + ((size_t)u * TROWS + row) * args.mu;
 #pragma unroll
                     for (int tt = 0; tt < TMAX; tt++) {
-                        if (tt < T) {
-                            const int ml0 = tt * NTOK + half * HC;
+                        const int ml0 = tt * NTOK + half * HC;
+                        if (tt < T && ml0 < un.len) {
                             if (ml0 + HC <= un.len) {
 #pragma unroll
                                 for (int j = 0; j < HC / 2; j += 2)
@@ -653,9 +632,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                         make_float4(acc[tt][j].x, acc[tt][j].y, acc[tt][j + 1].x, acc[tt][j + 1].y);
                             } else {
 #pragma unroll
-                                for (int j = 0; j < HC / 2; j++) {
+                                for (int j = 0; j < HC / 2; j++)
                                     if (ml0 + 2 * j < un.len) *reinterpret_cast<float2*>(part + ml0 + 2 * j) = acc[tt][j];
-                                }
                             }
                         }
                     }
@@ -676,23 +654,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         // sum the chunk partials in chunk order; every load of a chunk is
                         // issued before any is used
                         const int64_t u0 = u - un.chunk;
-#pragma unroll
-                        for (int tt = 0; tt < TMAX; tt++)
-#pragma unroll
-                            for (int j = 0; j < HC / 2; j++) acc[tt][j] = make_float2(0.0f, 0.0f);
                         for (int c2 = 0; c2 < args.kc; c2++) {
                             const float* part = args.partials + ((size_t)(u0 + c2) * TROWS + row) * args.mu;
                             float2 pv[TMAX][HC / 2];
 #pragma unroll
-                            for (int tt = 0; tt < TMAX; tt++) {
+                            for (int tt = 0; tt < TMAX; tt++)
 #pragma unroll
                                 for (int j = 0; j < HC / 2; j++) {
                                     const int ml = tt * NTOK + half * HC + 2 * j;
-                                    pv[tt][j] = (tt < T && ml < un.len)
-                                                    ? __ldcg(reinterpret_cast<const float2*>(part + ml))
-                                                    : make_float2(0.0f, 0.0f);
+                                    pv[tt][j] = (tt < T && ml < un.len) ? __ldcg(reinterpret_cast<const float2*>(part + ml))
+                                                                        : make_float2(0.0f, 0.0f);
                                 }
-                            }
 #pragma unroll
                             for (int tt = 0; tt < TMAX; tt++)
 #pragma unroll
@@ -734,16 +706,16 @@ constexpr size_t gemm_smem_bytes() {
 
 // Gather the requested canvas rows of a tiled activation into a compact tiled
 // activation of Mp_r rows (rows past n_rows are zero).  One thread per 16-byte
-// chunk: 16 quant chunks, one sums chunk and one scale per (super-block, row).
+// chunk: 16 quant chunks, 4 sums chunks and one scale per (super-block, row).
 __global__ void gather_rows_kernel(const int8_t* __restrict__ q, const float* __restrict__ scale,
                                    const uint8_t* __restrict__ sums, int64_t M, int64_t Mp,
                                    const int32_t* __restrict__ rows, int32_t n_rows, int64_t Mp_r, int32_t nsb,
                                    int8_t* __restrict__ gq, float* __restrict__ gscale, uint8_t* __restrict__ gsums) {
-    const int64_t total = (int64_t)nsb * Mp_r * 18;
+    const int64_t total = (int64_t)nsb * Mp_r * 21;
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total; g += (int64_t)gridDim.x * blockDim.x) {
-        const int c = (int)(g % 18);
-        const int64_t i = (g / 18) % Mp_r;
-        const int64_t s = g / 18 / Mp_r;
+        const int c = (int)(g % 21);
+        const int64_t i = (g / 21) % Mp_r;
+        const int64_t s = g / 21 / Mp_r;
         int64_t m = -1;
         if (i < n_rows) {
             m = rows[i];
@@ -757,10 +729,12 @@ __global__ void gather_rows_kernel(const int8_t* __restrict__ q, const float* __
             if (m >= 0)
                 v = *reinterpret_cast<const uint4*>(q + ((s * (Mp / 8) + m / 8) * 16 + c) * 128 + (m % 8) * 16);
             *reinterpret_cast<uint4*>(gq + ((s * (Mp_r / 8) + i / 8) * 16 + c) * 128 + (i % 8) * 16) = v;
-        } else if (c == 16) {
+        } else if (c < 20) {
+            const int cs = c - 16;
             uint4 v = make_uint4(0, 0, 0, 0);
-            if (m >= 0) v = *reinterpret_cast<const uint4*>(sums + (s * Mp + m) * 16);
-            *reinterpret_cast<uint4*>(gsums + (s * Mp_r + i) * 16) = v;
+            if (m >= 0)
+                v = *reinterpret_cast<const uint4*>(sums + (s * (Mp / 8) + m / 8) * SUMS_GROUP + cs * 128 + (m % 8) * 16);
+            *reinterpret_cast<uint4*>(gsums + (s * (Mp_r / 8) + i / 8) * SUMS_GROUP + cs * 128 + (i % 8) * 16) = v;
         } else {
             gscale[s * Mp_r + i] = m >= 0 ? scale[s * Mp + m] : 0.0f;
         }

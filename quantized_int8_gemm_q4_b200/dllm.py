@@ -65,7 +65,7 @@ def load() -> ctypes.CDLL:
         "dllm_get_device_status": [P],
         "dllm_status_string": [I],
         "dllm_debug_subblock_dots": [P, I, I64, I64, P, I64, P, P],
-        "dllm_debug_sb_ints": [P, I, I64, I64, P, P, P, I64, P, P, P],
+        "dllm_debug_sb_ints": [P, I, I64, I64, P, P, P, I64, P, P],
         "dllm_bench_mma_i8": [I, I, I, I, I, I, P, P],
     }
     for name, args in sig.items():
@@ -163,9 +163,9 @@ def dllm_debug_subblock_dots(w, qtype: int, N: int, K: int, q, M: int, dots, str
            "dllm_debug_subblock_dots")
 
 
-def dllm_debug_sb_ints(w, qtype: int, N: int, K: int, q, scale, sums, M: int, S, Smin, stream=None):
+def dllm_debug_sb_ints(w, qtype: int, N: int, K: int, q, scale, sums, M: int, S, stream=None):
     _check(load().dllm_debug_sb_ints(_ptr(w), qtype, N, K, _ptr(q), _ptr(scale), _ptr(sums), M, _ptr(S),
-                                     _ptr(Smin), _stream(stream)), "dllm_debug_sb_ints")
+                                     _stream(stream)), "dllm_debug_sb_ints")
 
 
 def dllm_bench_mma_i8(n: int, n_acc: int, a_from_tmem: int, issuers: int, iters: int, ctas: int, ns_out,
@@ -201,4 +201,4 @@ def alloc_act(M: int, K: int, device="cuda"):
     qb, sb, ub = dllm_act_bytes(M, K)
     return (torch.empty(qb, dtype=torch.int8, device=device),
             torch.empty(sb // 4, dtype=torch.float32, device=device),
-            torch.empty(ub, dtype=torch.uint8, device=device))
+            torch.empty(ub // 4, dtype=torch.float32, device=device))

@@ -23,14 +23,12 @@ def untile_scale(s_t: torch.Tensor, M: int, K: int) -> np.ndarray:
     return s_t.cpu().numpy().reshape(K // QK, Mp).T[:M]
 
 
-def untile_sums(u_t: torch.Tensor, M: int, K: int) -> np.ndarray:
-    """-> per-32 sums [M][K/32] int32 (low byte unsigned + 256 * high byte signed)."""
+def untile_sums(u_t: torch.Tensor, M: int, K: int):
+    """-> (hi, lo) float32 [M][K/32]: the scaled per-32 sums split as hi + lo."""
     Mp = (M + 15) // 16 * 16
-    u = u_t.cpu().numpy().reshape(K // QK, Mp, 16)
-    lo = u[..., :8].astype(np.int32)
-    hi = u[..., 8:].view(np.int8).astype(np.int32)
-    t = lo + 256 * hi                        # [nsb][Mp][8]
-    return t.transpose(1, 0, 2).reshape(Mp, K // 32)[:M]
+    u = u_t.cpu().numpy().view(np.float32).reshape(K // QK, Mp // 8, 2, 2, 8, 4)  # s, g, hi/lo, j-chunk, row, j
+    a = u.transpose(1, 4, 0, 2, 3, 5).reshape(Mp, K // QK, 2, 8)                  # row, s, hi/lo, j
+    return a[:M, :, 0, :].reshape(M, K // 32), a[:M, :, 1, :].reshape(M, K // 32)
 
 
 def repack_reference(qtype: int, blocks: np.ndarray) -> np.ndarray:

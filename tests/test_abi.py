@@ -50,7 +50,7 @@ def test_sizes_on_host(lib):
     assert dllm.dllm_repacked_bytes(dllm.DLLM_Q4_K, 256, 512) == 256 * 2 * 144
     assert dllm.dllm_repacked_bytes(dllm.DLLM_Q6_K, 128, 4096) == 128 * 16 * 210
     q, s, u = dllm.dllm_act_bytes(17, 512)
-    assert (q, s, u) == (32 * 512, 32 * 2 * 4, 32 * 2 * 16)
+    assert (q, s, u) == (32 * 512, 32 * 2 * 4, 32 * 2 * 64)
 
 
 @pytest.mark.parametrize("N,K", [(100, 512), (128, 300), (0, 256), (128, 0), (-128, 256)])

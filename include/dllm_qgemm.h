@@ -52,7 +52,9 @@ enum {
     DLLM_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed                         */
     DLLM_ERR_ROW_RANGE = -5,   /* device-detected: a rows[] entry outside [0, M)               */
     DLLM_ERR_TIMEOUT = -6,     /* device-detected: a bounded wait inside a kernel ran out      */
-    DLLM_ERR_WORKSPACE = -7    /* workspace smaller than dllm_qgemm_workspace_bytes() asks     */
+    DLLM_ERR_WORKSPACE = -7,   /* workspace smaller than dllm_qgemm_workspace_bytes() asks     */
+    DLLM_ERR_SCRATCH_LIMIT = -8 /* dllm_qgemm_noalloc: the call needs more scratch than the
+                                   library's fixed array holds                               */
 };
 
 /* ------------------------------------------------------------------------------
@@ -128,6 +130,44 @@ int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, in
 int dllm_qgemm(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
                const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows, float* out, int64_t ldo,
                void* workspace, size_t workspace_bytes, dllm_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * dllm_qgemm with no caller workspace.  The paper has no counterpart of this entry
+ * point; it is a convenience of this library.
+ *
+ * Same operation, arguments, results and device-detected errors as dllm_qgemm, but
+ * the scratch (gathered rows, split-K partial sums, arrival counters) is a fixed
+ * array of DLLM_NOALLOC_SCRATCH_BYTES bytes in the library's own device memory, one
+ * per device, reserved when the library's device code is loaded on that device.  It
+ * serves callers that cannot obtain device memory where they call: a host runtime
+ * that passes this library only buffers it already owns and has no allocator to
+ * lend it; a step where a cudaMalloc, which may synchronize the whole device, would
+ * stall work on other streams; plain C code that would rather not size, own and
+ * zero a workspace.
+ *
+ *   - Limit: a call whose scratch need (dllm_qgemm_workspace_bytes() for the same
+ *     arguments) exceeds DLLM_NOALLOC_SCRATCH_BYTES returns DLLM_ERR_SCRATCH_LIMIT
+ *     and launches nothing.  32 MiB holds every single projection of LLaDA-8B and
+ *     Dream-7B on canvases of up to 128 rows (the largest, LLaDA-8B gate or up at
+ *     128 rows, needs 18 MiB) and the output projection on up to 32 rows.
+ *   - Zero state: only the arrival counters must start at zero.  The call clears
+ *     the counters it uses on `stream` (an asynchronous memset of at most a few KB)
+ *     before its kernel runs, so nothing carries over between calls, including from
+ *     a call that ended in DLLM_ERR_TIMEOUT.  The partial sums and gathered rows are
+ *     written in full before they are read.
+ *   - Set-up: the first call on a device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress, which also loads the library's
+ *     device code there) and sets the kernel's shared-memory limit; later calls on
+ *     that device reuse both.  Make that first call before any stream capture begins.
+ *   - Races: all calls on a device share its one array.  Calls that overlap in time
+ *     (issued to different streams, or from host threads without ordering between
+ *     their streams) race on it and give wrong results; issue every call of this
+ *     entry point on a device to one stream.
+ * ---------------------------------------------------------------------------- */
+#define DLLM_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int dllm_qgemm_noalloc(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
+                       const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows, float* out,
+                       int64_t ldo, dllm_stream_t stream);
 
 /* ------------------------------------------------------------------------------
  * Several projections of one quantized activation in one launch (Architecture page,

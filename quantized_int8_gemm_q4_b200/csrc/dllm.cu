@@ -298,6 +298,61 @@ int dllm_qkv_qgemm(const void* wq, const void* wk, const void* wv, dllm_qtype t,
     return dispatch(a, t, false, s);
 }
 
+// ---------------------------------------------------------------- no-workspace GEMM
+}  // extern "C"
+
+namespace {
+
+// The fixed scratch of dllm_qgemm_noalloc, in the library's own device memory.  A
+// zero-initialized __device__ array is reserved (and zeroed) by the CUDA runtime
+// when this module's device code is loaded on a device, so the library never calls
+// an allocator for it.
+__device__ __align__(256) uint8_t g_noalloc_scratch[DLLM_NOALLOC_SCRATCH_BYTES];
+
+uint8_t* g_noalloc_addr[MAX_DEV];  // device address of the array, per device, once known
+
+int noalloc_scratch(int dev, uint8_t** ptr) {
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DLLM_ERR_CUDA;
+        g_noalloc_addr[dev] = static_cast<uint8_t*>(p);
+    }
+    *ptr = g_noalloc_addr[dev];
+    return DLLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dllm_qgemm_noalloc(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
+                       const uint8_t* sums, int64_t M, const int32_t* rows, int64_t n_rows, float* out,
+                       int64_t ldo, dllm_stream_t stream) {
+    // Every argument check dllm_qgemm makes, before anything is queued on the stream.
+    if (!w || !out || ldo < N) return DLLM_ERR_ARG;
+    if (!aligned16(w) || !aligned16(out) || ldo % 4) return DLLM_ERR_ALIGN;
+    int rc = check_shape(t, N, K);
+    if (rc) return rc;
+    if ((rc = check_act(q, scale, sums, M))) return rc;
+    if (rows && (n_rows < 1 || n_rows > 32)) return DLLM_ERR_ARG;
+    if (rows && !aligned16(rows)) return DLLM_ERR_ALIGN;
+    if (M > (1LL << 31)) return DLLM_ERR_ARG;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    const Plan p = make_plan(N / TROWS, K, M, rows ? n_rows : 0, g_num_sms[dev]);
+    if (p.bytes > DLLM_NOALLOC_SCRATCH_BYTES) return DLLM_ERR_SCRATCH_LIMIT;
+    uint8_t* scratch;
+    if ((rc = noalloc_scratch(dev, &scratch))) return rc;
+    if (p.kc > 1) {
+        const size_t ctr_bytes = (size_t)(N / TROWS) * p.n_st * 4;
+        if (cudaMemsetAsync(scratch + p.ctr_off, 0, ctr_bytes, reinterpret_cast<cudaStream_t>(stream)) !=
+            cudaSuccess)
+            return DLLM_ERR_CUDA;
+    }
+    return dllm_qgemm(w, t, N, K, q, scale, sums, M, rows, n_rows, out, ldo, scratch, DLLM_NOALLOC_SCRATCH_BYTES,
+                      stream);
+}
+
 int dllm_get_device_status(dllm_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return DLLM_ERR_CUDA;
     int v = 0, zero = 0;
@@ -316,6 +371,7 @@ const char* dllm_status_string(int code) {
         case DLLM_ERR_ROW_RANGE: return "row index out of range";
         case DLLM_ERR_TIMEOUT: return "bounded device wait ran out";
         case DLLM_ERR_WORKSPACE: return "workspace too small";
+        case DLLM_ERR_SCRATCH_LIMIT: return "call needs more scratch than the fixed no-allocation array holds";
         default: return "unknown status";
     }
 }

@@ -24,10 +24,12 @@ DLLM_ERR_CUDA = -4
 DLLM_ERR_ROW_RANGE = -5
 DLLM_ERR_TIMEOUT = -6
 DLLM_ERR_WORKSPACE = -7
+DLLM_ERR_SCRATCH_LIMIT = -8
+DLLM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 EXPORTS = (
     "dllm_repacked_bytes", "dllm_repack_q4k", "dllm_repack_q6k", "dllm_act_bytes", "dllm_quantize_act",
-    "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qkv_qgemm", "dllm_get_device_status",
+    "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_get_device_status",
     "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_bench_mma_i8",
 )
 
@@ -61,6 +63,7 @@ def load() -> ctypes.CDLL:
         "dllm_quantize_act": [P, I64, I64, I64, P, P, P, P],
         "dllm_qgemm_workspace_bytes": [I, I64, I64, I64, I64, PSZ],
         "dllm_qgemm": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P, SZ, P],
+        "dllm_qgemm_noalloc": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P],
         "dllm_qkv_qgemm": [P, P, P, I, I64, I64, I64, P, P, P, I64, P, I64, P, P, I64, P, SZ, P],
         "dllm_get_device_status": [P],
         "dllm_status_string": [I],
@@ -141,6 +144,12 @@ def dllm_qgemm(w, qtype: int, N: int, K: int, q, scale, sums, M: int, rows, n_ro
                workspace=None, workspace_bytes: int = 0, stream=None):
     _check(load().dllm_qgemm(_ptr(w), qtype, N, K, _ptr(q), _ptr(scale), _ptr(sums), M, _ptr(rows), n_rows,
                              _ptr(out), ldo, _ptr(workspace), workspace_bytes, _stream(stream)), "dllm_qgemm")
+
+
+def dllm_qgemm_noalloc(w, qtype: int, N: int, K: int, q, scale, sums, M: int, rows, n_rows: int, out, ldo: int,
+                       stream=None):
+    _check(load().dllm_qgemm_noalloc(_ptr(w), qtype, N, K, _ptr(q), _ptr(scale), _ptr(sums), M, _ptr(rows),
+                                     n_rows, _ptr(out), ldo, _stream(stream)), "dllm_qgemm_noalloc")
 
 
 def dllm_qkv_qgemm(wq, wk, wv, qtype: int, Nq: int, Nkv: int, K: int, q, scale, sums, M: int, oq, ldo_q: int,

@@ -51,7 +51,7 @@ def parse():
     p.add_argument("--model", default="llada-8b")
     p.add_argument("--canvas", type=int, default=128)
     p.add_argument("--layers", type=int, default=None, help="override the layer count (small profiling cases)")
-    p.add_argument("--cpu-layers", type=int, default=4, help="layers in the oracle's timed sample")
+    p.add_argument("--cpu-layers", type=int, default=16, help="layers in the oracle's timed sample")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     return p.parse_args()
@@ -164,6 +164,25 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ---------------------------------------------------------------------------- ranks
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of every rank's value (each rank's device-timed region); every rank
+    gets it.  Uses the default process group (NCCL on GPUs, gloo in CPU tests)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units processed by all ranks together per second, over the slowest rank's time."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world):
@@ -274,25 +293,34 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     assert dllm.dllm_get_device_status() == dllm.DLLM_OK
 
+    # graphs: g1 = one step, gS = S steps (the timed region replays these; no events
+    # inside), gE = S steps with an event after every quantize and every GEMM launch
+    # (a second pass, right after the timed region, for per-launch durations)
     S = max(1, min(args.steps, 10))
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
     g1 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g1, stream=s):
         step()
-    n_marks = 2 * len(gemms)
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks)] for _ in range(S)]
     gS = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gS, stream=s):
+        for i in range(S):
+            step()
+    n_marks = 2 * len(gemms)
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks)] for _ in range(S)]
+    gE = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gE, stream=s):
         for i in range(S):
             step(evs[i])
     torch.cuda.synchronize()
 
-    # ---- warm-up: W steps
+    # ---- warm-up: W steps (plus one untimed replay of each multi-step graph, which
+    # uploads it)
     with torch.cuda.stream(s):
         for _ in range(args.warmup):
             g1.replay()
-        gS.replay()  # first replay of the timed graph also uploads it (untimed)
+        gS.replay()
+        gE.replay()
     torch.cuda.synchronize()
 
     sampler = None
@@ -316,27 +344,25 @@ def run_ours(args, rank, world):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
-    elapsed_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     assert dllm.dllm_get_device_status() == dllm.DLLM_OK
 
-    # per-launch GEMM durations from the last S timed steps (events inside the graph)
+    # ---- per-launch durations: S more steps with events on the launching stream
+    with torch.cuda.stream(s):
+        gE.replay()
+    torch.cuda.synchronize()
     gemm_ms = 0.0
     quant_ms = 0.0
-    if args.steps >= S:
-        for i in range(S):
-            e = evs[i]
-            # marks: after quantize (even index), after gemm (odd index)
-            prev = None
-            for j in range(0, n_marks, 2):
-                if j > 0:
-                    quant_ms += e[j - 1].elapsed_time(e[j])
-                gemm_ms += e[j].elapsed_time(e[j + 1])
-        gemm_ms /= S
-        quant_ms /= S
+    for i in range(S):
+        e = evs[i]
+        # marks: after each quantize (even index), after each GEMM (odd index)
+        for j in range(0, n_marks, 2):
+            if j > 0:
+                quant_ms += e[j - 1].elapsed_time(e[j])
+            gemm_ms += e[j].elapsed_time(e[j + 1])
+    gemm_ms /= S
+    quant_ms /= S
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
 
     ms_step = elapsed_ms / args.steps
     ops_step = sum(g.ops for g in gemms)
@@ -345,7 +371,7 @@ def run_ours(args, rank, world):
     hbm_gbs, peak_kind = load_peaks()
     p_int8 = 4.5e15
     tstar = roofline_time(gemms, hbm_gbs, p_int8)
-    value = ops_step * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_rate(ops_step, world, ms_step) / 1e12
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -378,13 +404,18 @@ def run_ours(args, rank, world):
                 "frac": round(achieved / hbm_gbs, 4), "traffic": traffic,
                 "kernel": "qgemm_kernel", "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
                 "launches_per_step": len(gemms), "gemm_ms_per_step": round(gemm_ms, 4),
-                "algorithmic_bytes_per_step": int(abytes_step)}
+                "algorithmic_bytes_per_step": int(abytes_step),
+                "algorithmic_bytes_per_launch": int(abytes_step / len(gemms)),
+                "mean_launch_us": round(gemm_ms * 1e3 / len(gemms), 3),
+                "traffic_per": "launch, mean over the step's launch mix (DRAM read + write, ncu)",
+                "durations": f"CUDA events on the launching stream around every GEMM launch, over {S} "
+                             "graph-replayed steps right after the timed region"}
 
     cpu = None
     if rank == 0 and not args.no_cpu and cpu_sample:
         cpu = cpu_baseline(model, L, cpu_sample, rows_np, seed)
 
-    del gS, g1
+    del gE, gS, g1
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -395,7 +426,7 @@ def run_ours(args, rank, world):
                    "canvas_tokens": L, "layers": n_layers, "weight_bytes_per_step": int(wbytes_step),
                    "l2": "inputs larger than L2: every step streams all weights from HBM",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                   "graph": "one CUDA graph per step, replayed"},
+                   "graph": f"CUDA graphs of {S} steps, replayed; no events inside the timed region"},
         "weight_gbs": round(wbytes_step / (ms_step * 1e-3) / 1e9, 1),
         "step_roofline": {"t_star_ms": round(tstar * 1e3, 4), "frac": round(tstar * 1e3 / ms_step, 4),
                           "p_int8_tops": p_int8 / 1e12, "hbm_gbs": hbm_gbs},

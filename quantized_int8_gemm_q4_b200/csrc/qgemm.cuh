@@ -33,11 +33,11 @@
 // Roles (16 warps, one CTA per SM, persistent over work units):
 //   warp 0      producer: bulk copies of weight tiles and activation tiles into
 //               shared-memory rings
-//   warps 1-3   tensor-memory allocation (warp 1) and MMA issue.  One thread can
+//   warps 1-2   MMA issue (warp 1 also allocates tensor memory).  One thread can
 //               issue a tcgen05.mma only every ~28 ns, longer than a 64-token MMA
-//               takes, so three warps share the work: for each token tile the roles
-//               plane 0, plane 1 and min term rotate over them, each role owning its
-//               own accumulator, and a role's MMAs go out back to back
+//               takes, so the two token tiles of a super-block go to two warps, each
+//               with its own accumulator set and a short wait/issue/commit loop
+//   warp 3      idle
 //   warps 4-7   unpack: thread = weight row; decode the super-block, build the two
 //               weight planes per K-step of 32 into tensor memory (the A operand),
 //               the min-term A operand into shared memory, and the f32 d
@@ -62,7 +62,7 @@ constexpr int NTOK = 64;                           // token columns per MMA and 
 constexpr int TMAX = UNIT_TOKENS / NTOK;           // token tiles per unit
 constexpr int HC = NTOK / 2;                       // token columns per epilogue warp
 constexpr int MAX_KC = 16;                         // K-chunks per tile, at most
-constexpr int ISSUERS = 3;                         // MMA-issuing warps
+constexpr int ISSUERS = 2;                         // MMA-issuing warps
 constexpr int S_SLOTS = 4;                         // d ring (unpack -> epilogue)
 constexpr int ACC_SETS = 2;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
@@ -123,7 +123,7 @@ struct GemmArgs {
     int32_t n_st;      // token super-tiles
     int32_t mu;        // tokens per super-tile (multiple of 16)
     uint32_t* counters;  // [n_tiles * n_st], when kc > 1
-    float* partials;     // [units][128 rows][mu], when kc > 1
+    float* partials;     // [units][mu/4][128 rows][4 tokens], when kc > 1
     int32_t* dbg_S;    // debug: per-super-block integer S instead of f32 (nullable)
     int64_t dbg_N;
 };
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 256); }
         for (int i = 0; i < 2; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], ISSUERS); }
         for (int i = 0; i < S_SLOTS; i++) { mbar_init(&sh.s_full[i], 128); mbar_init(&sh.s_empty[i], 256); }
-        for (int i = 0; i < ACC_SETS; i++) { mbar_init(&sh.acc_full[i], ISSUERS); mbar_init(&sh.acc_empty[i], 256); }
+        for (int i = 0; i < ACC_SETS; i++) { mbar_init(&sh.acc_full[i], 1); mbar_init(&sh.acc_empty[i], 256); }
         mbar_init(&sh.min_empty, 256);
         for (int i = 0; i < 4; i++) mbar_init(&sh.final_bar[i], 1);
         mbar_init(&sh.epi_bar, 256);
@@ -251,14 +251,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     const uint32_t tmem = sh.tmem_base;
 
     if (warp < 4) {
-        setmaxnreg_dec<56>();
+        setmaxnreg_dec<48>();
         if (warp == 0) {
             // ======================================================== producer
             uint32_t ws = 0, wph = 0, bs = 0, bph = 0;
-            uint32_t w_ph_issued[C::W_STAGES], b_ph_issued[C::B_STAGES];
-            bool w_iss[C::W_STAGES], b_iss[C::B_STAGES];
-            for (int i = 0; i < C::W_STAGES; i++) w_iss[i] = false;
-            for (int i = 0; i < C::B_STAGES; i++) b_iss[i] = false;
+            // stages with a copy issued (bit i) and the phase it completes (bit i)
+            uint32_t w_iss = 0, w_php = 0, b_iss = 0, b_php = 0;
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
             for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
@@ -272,8 +270,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         bulk_g2s_hint(w_stage + ws * C::TILE, wt + (size_t)s * C::TILE, C::TILE, &sh.w_full[ws],
                                       pol_w);
                     }
-                    w_iss[ws] = true;
-                    w_ph_issued[ws] = wph;
+                    w_iss |= 1u << ws;
+                    w_php = (w_php & ~(1u << ws)) | (wph << ws);
                     if (++ws == C::W_STAGES) { ws = 0; wph ^= 1; }
                     for (int tt = 0; tt < T; tt++) {
                         const int64_t t0 = un.m0 + (int64_t)tt * NTOK;
@@ -291,8 +289,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                             bulk_g2s_hint(st + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
                                           &sh.b_full[bs], pol_a);
                         }
-                        b_iss[bs] = true;
-                        b_ph_issued[bs] = bph;
+                        b_iss |= 1u << bs;
+                        b_php = (b_php & ~(1u << bs)) | (bph << bs);
                         if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
                     }
                 }
@@ -300,72 +298,74 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         prod_done:
             if (sh.abort_flag) {  // never leave with bulk copies in flight into this CTA's shared memory
                 for (int i = 0; i < C::W_STAGES; i++)
-                    if (w_iss[i]) (void)wait_bar(sh, &sh.w_full[i], w_ph_issued[i]);
+                    if ((w_iss >> i) & 1u) (void)wait_bar(sh, &sh.w_full[i], (w_php >> i) & 1u);
                 for (int i = 0; i < C::B_STAGES; i++)
-                    if (b_iss[i]) (void)wait_bar(sh, &sh.b_full[i], b_ph_issued[i]);
+                    if ((b_iss >> i) & 1u) (void)wait_bar(sh, &sh.b_full[i], (b_php >> i) & 1u);
             }
         } else {
             // ======================================================== MMA issuers
-            // All lanes walk the schedule and wait together; lane 0 issues.  Tile g of
-            // this CTA gives plane 0 to issuer (2g) % 3, plane 1 to (2g+1) % 3 and the
-            // min term (Q4_K) to (2g+2) % 3.  Every issuer commits once per tile to the
-            // accumulator set and once per super-block to each half of the A ring.
+            // The (super-block, token tile) items of this CTA alternate between warps 1
+            // and 2, and item i owns accumulator set i % 2; with two token tiles each
+            // issuer owns one tile.  Per super-block an issuer waits for each half of
+            // the A ring, issues its item's MMAs on that half (both planes; the min
+            // term with the second half), and commits once to the half's release
+            // barrier, so every release takes one arrival from each issuer.  Warp 3
+            // issues nothing.
             const int who = warp - 1;
             const bool leader = lane == 0;
-            uint32_t bs = 0, bph = 0, r = 0, rph = 0, sbc = 0, g = 0, uc = 0;
-            for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
-                const Unit un = unit_of(args, u);
-                const int T = (un.len + NTOK - 1) / NTOK;
-                for (int s = un.sb0; s < un.sb1; s++, sbc++) {
-                    for (int tt = 0; tt < T; tt++, g++) {
-                        const int ntok = min(NTOK, un.len - tt * NTOK);
-                        const bool last = tt == T - 1;
-                        const int role = (int)((who + 3 - (2 * g) % 3) % 3);  // 0: plane 0, 1: plane 1, 2: min
-                        if (!wait_bar_warp(sh, &sh.b_full[bs], bph)) goto mma_done;
-                        if (!wait_bar_warp(sh, &sh.acc_empty[r], rph)) goto mma_done;
-                        if (tt == 0) {
-                            if (!wait_bar_warp(sh, &sh.a_full[0], sbc & 1)) goto mma_done;
-                            if (!wait_bar_warp(sh, &sh.a_full[1], sbc & 1)) goto mma_done;
-                        }
-                        // a unit's first min-term MMAs overwrite the min accumulators: the
-                        // previous unit's epilogue must have read them out
-                        if (C::MIN && role == 2 && s == un.sb0)
-                            if (!wait_bar_warp(sh, &sh.min_empty, (uc & 1) ^ 1)) goto mma_done;
-                        tc_fence_after();
-                        if (leader) {
-                            const uint32_t st = smem_u32(b_stage + bs * C::B_STAGE);
-                            if (role < 2) {
-                                const uint32_t id = QT == 12 ? idesc_i8(128, ntok, 0, 1) : idesc_i8(128, ntok, 1, 1);
-                                const uint32_t d = tmem + TM_ACC + (r * 2 + role) * NTOK;
-                                const uint32_t a0 = tmem + TM_A + 8 * role;
-                                const uint64_t b0 = sdesc_kmajor_noswz(st, 128, 2048);
-#pragma unroll
-                                for (int ks = 0; ks < 4; ks++) mma_i8_ts(d, a0 + 16 * ks, b0 + 16 * ks, id, 1);
-                                if (last) tc_commit(&sh.a_empty[0]);
-#pragma unroll
-                                for (int ks = 4; ks < 8; ks++) mma_i8_ts(d, a0 + 16 * ks, b0 + 16 * ks, id, 1);
-                                if (last) tc_commit(&sh.a_empty[1]);
-                            } else {
-                                if (last) tc_commit(&sh.a_empty[0]);
-                                if constexpr (C::MIN) {
-                                    const uint32_t d = tmem + TM_MIN + tt * NTOK;
-                                    const uint32_t id = idesc_tf32(128, ntok);
-                                    const uint32_t ma = smem_u32(mina);
-                                    const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
-                                    const uint64_t a_lo = sdesc_kmajor_noswz(ma + 4096, 128, 256);
-                                    const uint64_t b_hi = sdesc_kmajor_noswz(st + C::B_Q, 128, SUMS_GROUP);
-                                    const uint64_t b_lo = sdesc_kmajor_noswz(st + C::B_Q + 256, 128, SUMS_GROUP);
-                                    mma_tf32_ss(d, a_hi, b_hi, id, s > un.sb0 ? 1u : 0u);
-                                    mma_tf32_ss(d, a_hi, b_lo, id, 1);
-                                    mma_tf32_ss(d, a_lo, b_hi, id, 1);
+            if (who < ISSUERS) {
+                uint32_t item = 0, sbc = 0, uc = 0;
+                for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
+                    const Unit un = unit_of(args, u);
+                    const int T = (un.len + NTOK - 1) / NTOK;
+                    for (int s = un.sb0; s < un.sb1; s++, sbc++, item += T) {
+#pragma unroll 1
+                        for (int half = 0; half < 2; half++) {
+                            if (!wait_bar_warp(sh, &sh.a_full[half], sbc & 1)) goto mma_done;
+                            for (int tt = 0; tt < T; tt++) {
+                                const uint32_t it = item + tt;
+                                if ((int)(it & 1) != who) continue;
+                                const uint32_t set = it & 1;
+                                const uint32_t bst = it % C::B_STAGES, bpar = (it / C::B_STAGES) & 1;
+                                const int ntok = min(NTOK, un.len - tt * NTOK);
+                                if (half == 0) {
+                                    if (!wait_bar_warp(sh, &sh.b_full[bst], bpar)) goto mma_done;
+                                    if (!wait_bar_warp(sh, &sh.acc_empty[set], (it >> 1) & 1)) goto mma_done;
+                                } else if (C::MIN && s == un.sb0) {
+                                    // a unit's first min-term MMAs overwrite the min accumulators:
+                                    // the previous unit's epilogue must have read them out
+                                    if (!wait_bar_warp(sh, &sh.min_empty, (uc & 1) ^ 1)) goto mma_done;
                                 }
-                                if (last) tc_commit(&sh.a_empty[1]);
+                                tc_fence_after();
+                                if (leader) {
+                                    const uint32_t st = smem_u32(b_stage + bst * C::B_STAGE);
+                                    const uint32_t id = QT == 12 ? idesc_i8(128, ntok, 0, 1) : idesc_i8(128, ntok, 1, 1);
+                                    const uint32_t d0 = tmem + TM_ACC + set * 2 * NTOK;
+                                    const uint32_t a0 = tmem + TM_A + 64 * half;
+                                    const uint64_t b0 = sdesc_kmajor_noswz(st, 128, 2048) + 64 * half;
+#pragma unroll
+                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0, a0 + 16 * ks, b0 + 16 * ks, id, 1);
+#pragma unroll
+                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0 + NTOK, a0 + 16 * ks + 8, b0 + 16 * ks, id, 1);
+                                    if (C::MIN && half == 1) {
+                                        const uint32_t d = tmem + TM_MIN + tt * NTOK;
+                                        const uint32_t idm = idesc_tf32(128, ntok);
+                                        const uint32_t ma = smem_u32(mina);
+                                        const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
+                                        const uint64_t a_lo = sdesc_kmajor_noswz(ma + 4096, 128, 256);
+                                        const uint64_t b_hi = sdesc_kmajor_noswz(st + C::B_Q, 128, SUMS_GROUP);
+                                        const uint64_t b_lo = sdesc_kmajor_noswz(st + C::B_Q + 256, 128, SUMS_GROUP);
+                                        mma_tf32_ss(d, a_hi, b_hi, idm, s > un.sb0 ? 1u : 0u);
+                                        mma_tf32_ss(d, a_hi, b_lo, idm, 1);
+                                        mma_tf32_ss(d, a_lo, b_hi, idm, 1);
+                                    }
+                                    if (half == 1) tc_commit(&sh.acc_full[set]);
+                                }
+                                __syncwarp();
                             }
-                            tc_commit(&sh.acc_full[r]);
+                            if (leader) tc_commit(&sh.a_empty[half]);
+                            __syncwarp();
                         }
-                        __syncwarp();
-                        if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
-                        if (++r == ACC_SETS) { r = 0; rph ^= 1; }
                     }
                 }
             }
@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             (void)wait_bar_warp(sh, &sh.final_bar[who], 0);
         }
     } else if (warp < 8) {
-        setmaxnreg_dec<88>();
+        setmaxnreg_dec<80>();
         // ============================================================ unpack
         // Per super-block: decode this row, then build the planes of K-steps 0-3 and
         // publish them together, then K-steps 4-7 (and the min-term A), so the MMAs of
@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
 #pragma unroll
                     for (int half = 0; half < 2; half++) {
                         if (!wait_bar_warp(sh, &sh.a_empty[half], (sbc & 1) ^ 1)) goto unpack_done;
-#pragma unroll 1
+#pragma unroll
                         for (int kq = 0; kq < 4; kq++) {
                             const int ks = 4 * half + kq;
                             const int h = ks >> 2, g = ks & 3;
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         }
     unpack_done:;
     } else {
-        setmaxnreg_inc<184>();
+        setmaxnreg_inc<192>();
         // ============================================================ epilogue
         const int quad = warp & 3;
         const int half = (warp - 8) >> 2;
@@ -547,6 +547,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         tc_fence_after();
                         const uint32_t acc_t = tmem + lane_off + TM_ACC + r * 2 * NTOK + half * HC;
                         const float* da = reinterpret_cast<const float*>(b_stage + bs * C::B_STAGE + C::B_Q + C::B_SUMS);
+                        // read both plane accumulators, preset them again and release them
+                        // to the MMA issuer before doing any arithmetic on the values
                         if (half * HC < ntok) {
                             uint32_t x0[HC], x1[HC];
                             load_cols(acc_t, x0);
@@ -554,6 +556,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                             tmem_wait_ld();
                             fill_cols(acc_t, MAGIC_BITS);
                             fill_cols(acc_t + NTOK, MAGIC_BITS);
+                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(&sh.acc_empty[r]);
                             if constexpr (DBG) {
 #pragma unroll
                                 for (int i = 0; i < HC; i++) {
@@ -575,10 +580,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                     acc[tt][i] = __ffma2_rn(__fmul2_rn(S, d2), dav, acc[tt][i]);
                                 }
                             }
+                        } else {
+                            tc_fence_before();
+                            mbar_arrive(&sh.acc_empty[r]);
                         }
-                        tmem_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(&sh.acc_empty[r]);
                         mbar_arrive(&sh.b_empty[bs]);
                         if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
                         if (++r == ACC_SETS) { r = 0; rph ^= 1; }
@@ -618,23 +623,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         }
                     }
                 } else {
-                    // this K-chunk's partial: [unit][128 rows][mu tokens]; a thread's
-                    // columns of one token tile are contiguous
-                    float* part = args.partials + ((size_t)u * TROWS + row) * args.mu;
+                    // this K-chunk's partial: [unit][mu/4][128 rows][4 tokens], so a thread's
+                    // 4 consecutive tokens are one 16-byte store and a warp's 32 rows 512
+                    // contiguous bytes (token counts are multiples of 16)
+                    float* part = args.partials + (size_t)u * args.mu * TROWS + row * 4;
 #pragma unroll
                     for (int tt = 0; tt < TMAX; tt++) {
-                        const int ml0 = tt * NTOK + half * HC;
-                        if (tt < T && ml0 < un.len) {
-                            if (ml0 + HC <= un.len) {
 #pragma unroll
-                                for (int j = 0; j < HC / 2; j += 2)
-                                    *reinterpret_cast<float4*>(part + ml0 + 2 * j) =
-                                        make_float4(acc[tt][j].x, acc[tt][j].y, acc[tt][j + 1].x, acc[tt][j + 1].y);
-                            } else {
-#pragma unroll
-                                for (int j = 0; j < HC / 2; j++)
-                                    if (ml0 + 2 * j < un.len) *reinterpret_cast<float2*>(part + ml0 + 2 * j) = acc[tt][j];
-                            }
+                        for (int q4 = 0; q4 < HC / 4; q4++) {
+                            const int ml = tt * NTOK + half * HC + 4 * q4;
+                            if (tt < T && ml < un.len)
+                                __stcg(reinterpret_cast<float4*>(part + (size_t)(ml / 4) * TROWS * 4),
+                                       make_float4(acc[tt][2 * q4].x, acc[tt][2 * q4].y, acc[tt][2 * q4 + 1].x,
+                                                   acc[tt][2 * q4 + 1].y));
                         }
                     }
                     __threadfence();
@@ -651,25 +652,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     }
                     if (!epi_sync(sh, epi_ph)) goto epi_done;
                     if (sh.last_flag) {
-                        // sum the chunk partials in chunk order; every load of a chunk is
-                        // issued before any is used
+                        // sum the chunk partials in chunk order; each token tile's 8 loads of
+                        // 16 bytes are issued before any is used
                         const int64_t u0 = u - un.chunk;
                         for (int c2 = 0; c2 < args.kc; c2++) {
-                            const float* part = args.partials + ((size_t)(u0 + c2) * TROWS + row) * args.mu;
-                            float2 pv[TMAX][HC / 2];
+                            const float* part = args.partials + (size_t)(u0 + c2) * args.mu * TROWS + row * 4;
 #pragma unroll
-                            for (int tt = 0; tt < TMAX; tt++)
+                            for (int tt = 0; tt < TMAX; tt++) {
+                                float4 pv[HC / 4];
 #pragma unroll
-                                for (int j = 0; j < HC / 2; j++) {
-                                    const int ml = tt * NTOK + half * HC + 2 * j;
-                                    pv[tt][j] = (tt < T && ml < un.len) ? __ldcg(reinterpret_cast<const float2*>(part + ml))
-                                                                        : make_float2(0.0f, 0.0f);
+                                for (int q4 = 0; q4 < HC / 4; q4++) {
+                                    const int ml = tt * NTOK + half * HC + 4 * q4;
+                                    pv[q4] = (tt < T && ml < un.len)
+                                                 ? __ldcg(reinterpret_cast<const float4*>(part + (size_t)(ml / 4) * TROWS * 4))
+                                                 : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                                 }
 #pragma unroll
-                            for (int tt = 0; tt < TMAX; tt++)
-#pragma unroll
-                                for (int j = 0; j < HC / 2; j++)
-                                    acc[tt][j] = c2 == 0 ? pv[tt][j] : __fadd2_rn(acc[tt][j], pv[tt][j]);
+                                for (int q4 = 0; q4 < HC / 4; q4++) {
+                                    const float2 lo = make_float2(pv[q4].x, pv[q4].y), hi = make_float2(pv[q4].z, pv[q4].w);
+                                    acc[tt][2 * q4] = c2 == 0 ? lo : __fadd2_rn(acc[tt][2 * q4], lo);
+                                    acc[tt][2 * q4 + 1] = c2 == 0 ? hi : __fadd2_rn(acc[tt][2 * q4 + 1], hi);
+                                }
+                            }
                         }
                         float* out = sg.out;
 #pragma unroll

@@ -28,6 +28,24 @@ int current_device(int* dev) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel on the stream finishes, and synchronises with it on the device
+// (pdl_wait) before touching memory that kernel can write.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 int launch_status() {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
@@ -41,17 +59,20 @@ int grid_for(int64_t work, int64_t per_block) {
 
 // K-chunks per tile.  A function of the tile count, the super-block count and the
 // SM count only (never of M or of a row list), so that every call on the same
-// weight shape sums the same partials in the same order.  Cost model in units of one
-// super-block of one tile: the busiest SM's share, plus one unit per chunk for
-// writing and re-reading its partial; chunks are at least 4 super-blocks long.
+// weight shape sums the same partials in the same order.  Cost model, in units of
+// one super-block of one tile, fitted to measured launch times at 128 canvas rows:
+// the busiest SM runs ceil(units / SMs) work units, each costing its super-blocks
+// plus 2.35 for the unit's start and drain, plus 2.7 more when the tile's K range is
+// split (partial write, arrival counter, and the last arriver's chunk sum); chunks
+// are at least 4 super-blocks long.
 int choose_kc(int64_t n_tiles, int64_t nsb, int sms) {
     int best = 1;
     int64_t best_cost = -1;
     for (int kc = 1; kc <= MAX_KC && kc <= nsb; kc++) {
         const int64_t len = (nsb + kc - 1) / kc;
         if (kc > 1 && len < 4) break;
-        const int64_t waves = (n_tiles * kc + sms - 1) / sms;
-        const int64_t cost = waves * (len + (kc > 1 ? 1 : 0));
+        const int64_t per_sm = (n_tiles * kc + sms - 1) / sms;
+        const int64_t cost = per_sm * (100 * len + 235 + (kc > 1 ? 270 : 0));
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best = kc;
@@ -108,7 +129,10 @@ int run_gemm(GemmArgs& a, cudaStream_t s) {
     }
     const int64_t units = (int64_t)a.n_tiles * a.n_st * a.kc;
     const int grid = (int)(units < g_num_sms[dev] ? units : g_num_sms[dev]);
-    qgemm_kernel<QT, DBG><<<grid, GEMM_THREADS, smem, s>>>(a);
+    if (launch_pdl(qgemm_kernel<QT, DBG>, dim3(grid), dim3(GEMM_THREADS), smem, s, a) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DLLM_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -184,7 +208,11 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     if ((rc = current_device(&dev))) return rc;
     const int64_t Mp = round_up(M, 16);
     dim3 grid((unsigned)(Mp / 8), (unsigned)(K / QK));
-    quantize_act_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, M, ldx, Mp, q, scale, sums);
+    if (launch_pdl(quantize_act_kernel, grid, dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), x, M, ldx, Mp, q,
+                   scale, sums) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DLLM_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -239,8 +267,11 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
         float* gs = reinterpret_cast<float*>(ws + p.gs_off);
         uint8_t* gu = ws + p.gu_off;
         const int64_t work = nsb * p.Mp * 21;
-        gather_rows_kernel<<<grid_for(work, 256), 256, 0, s>>>(q, scale, sums, M, round_up(M, 16), rows,
-                                                                (int32_t)n_rows, p.Mp, (int32_t)nsb, gq, gs, gu);
+        if (launch_pdl(gather_rows_kernel, dim3(grid_for(work, 256)), dim3(256), 0, s, q, scale, sums, M,
+                       round_up(M, 16), rows, (int32_t)n_rows, p.Mp, (int32_t)nsb, gq, gs, gu) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return DLLM_ERR_CUDA;
+        }
         if ((rc = launch_status())) return rc;
         a.q = gq;
         a.scale = gs;

@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const float* __restri
     __shared__ __align__(16) uint8_t tile[16 * 8 * 16];  // [chunk][row][16 B]
     __shared__ __align__(16) float tsum[4 * 8 * 4];      // [hi j0-3, hi j4-7, lo j0-3, lo j4-7][row][4]
     __shared__ float tscale[8];
+    pdl_trigger();
+    pdl_wait();  // x may be the output of the previous kernel on the stream
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t g = blockIdx.x, s = blockIdx.y;
     const int64_t m = 8 * g + w;

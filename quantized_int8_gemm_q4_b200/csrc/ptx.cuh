@@ -73,6 +73,19 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
+// Bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.  A
+// hint only: L2 is the coherence point, so a prefetch never exposes stale data.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch.  pdl_wait: block until the grids this one depends
+// on have completed and their memory operations are visible.  pdl_trigger: let the
+// grid that depends on this one be scheduled now (it still runs pdl_wait before
+// touching anything this grid writes).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -249,6 +249,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
+    // Everything above, and the producer's L2 prefetch of its first weight tiles, may
+    // overlap the previous kernel on the stream; every access to global memory that
+    // earlier work can write comes after pdl_wait in the role that makes it.
+    if (threadIdx.x == 0) pdl_trigger();
 
     if (warp < 4) {
         setmaxnreg_dec<48>();
@@ -259,6 +263,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             uint32_t w_iss = 0, w_php = 0, b_iss = 0, b_php = 0;
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
+            if (lane == 0 && blockIdx.x < n_units) {
+                const Unit un = unit_of(args, blockIdx.x);
+                const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
+                for (int s = un.sb0; s < un.sb1 && s < un.sb0 + C::W_STAGES; s++)
+                    prefetch_l2(wt + (size_t)s * C::TILE, C::TILE);
+            }
+            pdl_wait();
             for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
                 const Unit un = unit_of(args, u);
                 const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
@@ -509,6 +520,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     } else {
         setmaxnreg_inc<192>();
         // ============================================================ epilogue
+        pdl_wait();  // outputs, partials and counters may be in use by earlier work
         const int quad = warp & 3;
         const int half = (warp - 8) >> 2;
         const int row = quad * 32 + lane;
@@ -715,6 +727,8 @@ __global__ void gather_rows_kernel(const int8_t* __restrict__ q, const float* __
                                    const uint8_t* __restrict__ sums, int64_t M, int64_t Mp,
                                    const int32_t* __restrict__ rows, int32_t n_rows, int64_t Mp_r, int32_t nsb,
                                    int8_t* __restrict__ gq, float* __restrict__ gscale, uint8_t* __restrict__ gsums) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t total = (int64_t)nsb * Mp_r * 21;
     for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total; g += (int64_t)gridDim.x * blockDim.x) {
         const int c = (int)(g % 21);

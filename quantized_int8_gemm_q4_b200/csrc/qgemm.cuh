@@ -15,10 +15,10 @@
 //         0..105 (u8).  S = P0 + 8*P1.
 //   Q6_K: v = (q-32)*sc + 32896 lies in [28800, 36992]; plane 0 = (v & 255) - 128,
 //         plane 1 = (v >> 8) - 128 (both s8), and plane0 + 256*plane1 = (q-32)*sc.
-// Each plane accumulator stays within 2^22 in magnitude.  Tensor memory is preset to
-// the bit pattern of 1.5*2^23 before each super-block, so the int32 the MMAs leave
-// there, read as an f32, is exactly 1.5*2^23 + value, and the epilogue recovers S
-// with one FFMA and one FADD (packed f32x2), with no integer-to-float instruction.
+// Each plane accumulator stays within 2^22 in magnitude.  The first MMA of each
+// super-block overwrites it, and the epilogue adds the bit pattern of 1.5*2^23 to
+// the int32 it reads, which makes an f32 equal to exactly 1.5*2^23 + value; S then
+// takes one FFMA and one FADD (packed f32x2), with no integer-to-float instruction.
 // The epilogue then accumulates da * d * S in f32 registers.
 //
 // The min term (Q4_K), on the tf32 tensor pipe.  Its per-super-block factor
@@ -183,10 +183,6 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&x)[HC]) {
     tmem_ld16(taddr, x);
     tmem_ld16(taddr + 16, x + 16);
-}
-__device__ __forceinline__ void fill_cols(uint32_t taddr, uint32_t v) {
-    tmem_fill16(taddr, v);
-    tmem_fill16(taddr + 16, v);
 }
 
 struct Unit {
@@ -355,9 +351,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                     const uint32_t a0 = tmem + TM_A + 64 * half;
                                     const uint64_t b0 = sdesc_kmajor_noswz(st, 128, 2048) + 64 * half;
 #pragma unroll
-                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0, a0 + 16 * ks, b0 + 16 * ks, id, 1);
+                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0, a0 + 16 * ks, b0 + 16 * ks, id, half | ks ? 1u : 0u);
 #pragma unroll
-                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0 + NTOK, a0 + 16 * ks + 8, b0 + 16 * ks, id, 1);
+                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0 + NTOK, a0 + 16 * ks + 8, b0 + 16 * ks, id, half | ks ? 1u : 0u);
                                     if (C::MIN && half == 1) {
                                         const uint32_t d = tmem + TM_MIN + tt * NTOK;
                                         const uint32_t idm = idesc_tf32(128, ntok);
@@ -526,10 +522,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         const int row = quad * 32 + lane;
         const int etid = threadIdx.x - 256;  // 0..255
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        for (int r = 0; r < ACC_SETS; r++)
-            for (int a = 0; a < 2; a++) fill_cols(tmem + lane_off + TM_ACC + (r * 2 + a) * NTOK + half * HC, MAGIC_BITS);
-        tmem_wait_st();
-        tc_fence_before();
         for (int r = 0; r < ACC_SETS; r++) mbar_arrive(&sh.acc_empty[r]);
         const float2 k8 = make_float2(8.0f, 8.0f), k256 = make_float2(256.0f, 256.0f);
         const float2 m9 = make_float2(-9.0f * MAGIC, -9.0f * MAGIC);
@@ -559,16 +551,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         tc_fence_after();
                         const uint32_t acc_t = tmem + lane_off + TM_ACC + r * 2 * NTOK + half * HC;
                         const float* da = reinterpret_cast<const float*>(b_stage + bs * C::B_STAGE + C::B_Q + C::B_SUMS);
-                        // read both plane accumulators, preset them again and release them
-                        // to the MMA issuer before doing any arithmetic on the values
+                        // read both plane accumulators and release them to the MMA issuer
+                        // (the next super-block's first MMA overwrites them) before doing
+                        // any arithmetic on the values
                         if (half * HC < ntok) {
                             uint32_t x0[HC], x1[HC];
                             load_cols(acc_t, x0);
                             load_cols(acc_t + NTOK, x1);
                             tmem_wait_ld();
-                            fill_cols(acc_t, MAGIC_BITS);
-                            fill_cols(acc_t + NTOK, MAGIC_BITS);
-                            tmem_wait_st();
                             tc_fence_before();
                             mbar_arrive(&sh.acc_empty[r]);
                             if constexpr (DBG) {
@@ -577,15 +567,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                     const int64_t m = un.m0 + tt * NTOK + half * HC + i;
                                     if (half * HC + i < ntok && m < args.m_out) {
                                         const int64_t n = un.tile * TROWS + row;
-                                        const int32_t P0 = (int32_t)(x0[i] - MAGIC_BITS), P1 = (int32_t)(x1[i] - MAGIC_BITS);
+                                        const int32_t P0 = (int32_t)x0[i], P1 = (int32_t)x1[i];
                                         args.dbg_S[(m * args.dbg_N + n) * args.nsb + s] = P0 + (QT == 12 ? 8 : 256) * P1;
                                     }
                                 }
                             } else {
 #pragma unroll
                                 for (int i = 0; i < HC / 2; i++) {
-                                    const float2 X0 = make_float2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
-                                    const float2 X1 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+                                    // |P| < 2^22: adding the bits of 1.5*2^23 gives the f32 1.5*2^23 + P
+                                    const float2 X0 = make_float2(__uint_as_float(x0[2 * i] + MAGIC_BITS),
+                                                                  __uint_as_float(x0[2 * i + 1] + MAGIC_BITS));
+                                    const float2 X1 = make_float2(__uint_as_float(x1[2 * i] + MAGIC_BITS),
+                                                                  __uint_as_float(x1[2 * i + 1] + MAGIC_BITS));
                                     const float2 S = QT == 12 ? __fadd2_rn(__ffma2_rn(X1, k8, m9), X0)
                                                               : __fadd2_rn(__ffma2_rn(X1, k256, m257), X0);
                                     const float2 dav = *reinterpret_cast<const float2*>(da + half * HC + 2 * i);

@@ -68,9 +68,10 @@ constexpr int ACC_SETS = 2;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 
 // tensor-memory columns
-constexpr uint32_t TM_A = 0;      // 8 K-step slots x 16 columns (plane 0 | plane 1)
-constexpr uint32_t TM_ACC = 128;  // ACC_SETS x 2 planes x NTOK columns
-constexpr uint32_t TM_MIN = 384;  // TMAX x NTOK columns: f32 min-term accumulators (Q4_K)
+// tensor-memory columns: the A ring (RING halves of a super-block, each 4 K-step slots
+// of 16 columns: plane 0 | plane 1), then ACC_SETS x 2 planes x NTOK accumulator
+// columns, then (Q4_K) TMAX x NTOK f32 min-term accumulator columns
+constexpr uint32_t TM_A = 0;
 constexpr uint32_t TM_COLS = 512;
 
 // Activation "sums" operand of one super-block: per 8-row group 512 bytes =
@@ -89,6 +90,9 @@ struct GemmCfg<12> {  // Q4_K
     static constexpr int B_SUMS = NTOK / 8 * SUMS_GROUP;
     static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
     static constexpr int MINA = 2 * 4096;  // -dmin*m_j as [hi | lo], canonical K-major 128 rows x 32 B
+    static constexpr int RING = 2;         // A ring: one super-block (the min accumulators take the rest)
+    static constexpr uint32_t TM_ACC = 64 * RING;
+    static constexpr uint32_t TM_MIN = TM_ACC + ACC_SETS * 2 * NTOK;
 };
 template <>
 struct GemmCfg<14> {  // Q6_K
@@ -100,6 +104,9 @@ struct GemmCfg<14> {  // Q6_K
     static constexpr int B_SUMS = 0;
     static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
     static constexpr int MINA = 0;
+    static constexpr int RING = 4;  // A ring: two super-blocks, so the unpack runs one ahead
+    static constexpr uint32_t TM_ACC = 64 * RING;
+    static constexpr uint32_t TM_MIN = 0;
 };
 
 struct Segment {
@@ -131,7 +138,7 @@ struct GemmArgs {
 struct GemmShared {
     uint64_t w_full[8], w_empty[8];
     uint64_t b_full[8], b_empty[8];
-    uint64_t a_full[2], a_empty[2];  // A ring halves: K-steps 0-3, and 4-7 (+ the min-term A)
+    uint64_t a_full[4], a_empty[4];  // A ring slots: super-block halves (K-steps 0-3, 4-7 + the min-term A)
     uint64_t s_full[S_SLOTS], s_empty[S_SLOTS];
     uint64_t acc_full[ACC_SETS], acc_empty[ACC_SETS];
     uint64_t min_empty;
@@ -213,6 +220,14 @@ __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int64_t u) {
     return r;
 }
 
+template <int QT>
+constexpr bool tmem_fits() {
+    using C = GemmCfg<QT>;
+    return C::TM_ACC + ACC_SETS * 2 * NTOK + (C::MIN ? TMAX * NTOK : 0) <= TM_COLS &&
+           (!C::MIN || C::TM_MIN == C::TM_ACC + ACC_SETS * 2 * NTOK) && C::RING <= 4 && C::RING % 2 == 0;
+}
+static_assert(tmem_fits<12>() && tmem_fits<14>(), "tensor-memory columns over budget");
+
 template <int QT, bool DBG>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<QT>;
@@ -228,7 +243,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 128); }
         for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 256); }
-        for (int i = 0; i < 2; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], ISSUERS); }
+        for (int i = 0; i < C::RING; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], ISSUERS); }
         for (int i = 0; i < S_SLOTS; i++) { mbar_init(&sh.s_full[i], 128); mbar_init(&sh.s_empty[i], 256); }
         for (int i = 0; i < ACC_SETS; i++) { mbar_init(&sh.acc_full[i], 1); mbar_init(&sh.acc_empty[i], 256); }
         mbar_init(&sh.min_empty, 256);
@@ -328,7 +343,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     for (int s = un.sb0; s < un.sb1; s++, sbc++, item += T) {
 #pragma unroll 1
                         for (int half = 0; half < 2; half++) {
-                            if (!wait_bar_warp(sh, &sh.a_full[half], sbc & 1)) goto mma_done;
+                            const uint32_t hc = 2 * sbc + half, slot = hc % C::RING;
+                            if (!wait_bar_warp(sh, &sh.a_full[slot], (hc / C::RING) & 1)) goto mma_done;
                             for (int tt = 0; tt < T; tt++) {
                                 const uint32_t it = item + tt;
                                 if ((int)(it & 1) != who) continue;
@@ -347,15 +363,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 if (leader) {
                                     const uint32_t st = smem_u32(b_stage + bst * C::B_STAGE);
                                     const uint32_t id = QT == 12 ? idesc_i8(128, ntok, 0, 1) : idesc_i8(128, ntok, 1, 1);
-                                    const uint32_t d0 = tmem + TM_ACC + set * 2 * NTOK;
-                                    const uint32_t a0 = tmem + TM_A + 64 * half;
+                                    const uint32_t d0 = tmem + C::TM_ACC + set * 2 * NTOK;
+                                    const uint32_t a0 = tmem + TM_A + 64 * slot;
                                     const uint64_t b0 = sdesc_kmajor_noswz(st, 128, 2048) + 64 * half;
 #pragma unroll
                                     for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0, a0 + 16 * ks, b0 + 16 * ks, id, half | ks ? 1u : 0u);
 #pragma unroll
                                     for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0 + NTOK, a0 + 16 * ks + 8, b0 + 16 * ks, id, half | ks ? 1u : 0u);
                                     if (C::MIN && half == 1) {
-                                        const uint32_t d = tmem + TM_MIN + tt * NTOK;
+                                        const uint32_t d = tmem + C::TM_MIN + tt * NTOK;
                                         const uint32_t idm = idesc_tf32(128, ntok);
                                         const uint32_t ma = smem_u32(mina);
                                         const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
@@ -370,7 +386,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 }
                                 __syncwarp();
                             }
-                            if (leader) tc_commit(&sh.a_empty[half]);
+                            if (leader) tc_commit(&sh.a_empty[slot]);
                             __syncwarp();
                         }
                     }
@@ -421,7 +437,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
 #pragma unroll
                     for (int half = 0; half < 2; half++) {
-                        if (!wait_bar_warp(sh, &sh.a_empty[half], (sbc & 1) ^ 1)) goto unpack_done;
+                        const uint32_t hc = 2 * sbc + half, slot = hc % C::RING;
+                        if (!wait_bar_warp(sh, &sh.a_empty[slot], ((hc / C::RING) & 1) ^ 1)) goto unpack_done;
                         if (half == 1) {
                             // -dmin*m_j as tf32 hi + lo: row `row` of the canonical K-major
                             // layout (8-row groups of 256 bytes, two 16-byte K chunks)
@@ -452,12 +469,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                     v[i] = nib * lo3;
                                     v[8 + i] = nib * hi3;
                                 }
-                                tmem_st16(tmem + lane_off + TM_A + 16 * ks, v);
+                                tmem_st16(tmem + lane_off + TM_A + 64 * slot + 16 * (ks & 3), v);
                             }
                         }
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(&sh.a_full[half]);
+                        mbar_arrive(&sh.a_full[slot]);
                     }
                 } else {
                     const uint4 scv = *reinterpret_cast<const uint4*>(tl + Q6K_OFF_SC + 16 * row);
@@ -470,7 +487,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
 #pragma unroll
                     for (int half = 0; half < 2; half++) {
-                        if (!wait_bar_warp(sh, &sh.a_empty[half], (sbc & 1) ^ 1)) goto unpack_done;
+                        const uint32_t hc = 2 * sbc + half, slot = hc % C::RING;
+                        if (!wait_bar_warp(sh, &sh.a_empty[slot], ((hc / C::RING) & 1) ^ 1)) goto unpack_done;
 #pragma unroll
                         for (int kq = 0; kq < 4; kq++) {
                             const int ks = 4 * half + kq;
@@ -501,11 +519,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 v[i] = __byte_perm(pa, pb, 0x6420) ^ 0x80808080u;
                                 v[8 + i] = __byte_perm(pa, pb, 0x7531) ^ 0x80808080u;
                             }
-                            tmem_st16(tmem + lane_off + TM_A + 16 * ks, v);
+                            tmem_st16(tmem + lane_off + TM_A + 64 * slot + 16 * (ks & 3), v);
                         }
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(&sh.a_full[half]);
+                        mbar_arrive(&sh.a_full[slot]);
                     }
                 }
                 mbar_arrive(&sh.w_empty[ws]);
@@ -549,7 +567,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         if (!wait_bar_warp(sh, &sh.acc_full[r], rph)) goto epi_done;
                         if (!wait_bar_warp(sh, &sh.b_full[bs], bph)) goto epi_done;
                         tc_fence_after();
-                        const uint32_t acc_t = tmem + lane_off + TM_ACC + r * 2 * NTOK + half * HC;
+                        const uint32_t acc_t = tmem + lane_off + C::TM_ACC + r * 2 * NTOK + half * HC;
                         const float* da = reinterpret_cast<const float*>(b_stage + bs * C::B_STAGE + C::B_Q + C::B_SUMS);
                         // read both plane accumulators and release them to the MMA issuer
                         // (the next super-block's first MMA overwrites them) before doing
@@ -602,7 +620,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                 for (int tt = 0; tt < TMAX; tt++) {
                     if (tt < T && half * HC < un.len - tt * NTOK) {
                         uint32_t y[HC];
-                        load_cols(tmem + lane_off + TM_MIN + tt * NTOK + half * HC, y);
+                        load_cols(tmem + lane_off + C::TM_MIN + tt * NTOK + half * HC, y);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < HC / 2; i++)

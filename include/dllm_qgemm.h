@@ -148,8 +148,9 @@ int dllm_qgemm(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* 
  *   - Limit: a call whose scratch need (dllm_qgemm_workspace_bytes() for the same
  *     arguments) exceeds DLLM_NOALLOC_SCRATCH_BYTES returns DLLM_ERR_SCRATCH_LIMIT
  *     and launches nothing.  32 MiB holds every single projection of LLaDA-8B and
- *     Dream-7B on canvases of up to 128 rows (the largest, LLaDA-8B gate or up at
- *     128 rows, needs 18 MiB) and the output projection on up to 32 rows.
+ *     Dream-7B on canvases of up to 384 rows (the largest, Dream-7B's down
+ *     projection at 384 rows, needs 26.25 MiB) and the output projection on up to
+ *     32 rows.
  *   - Zero state: only the arrival counters must start at zero.  The call clears
  *     the counters it uses on `stream` (an asynchronous memset of at most a few KB)
  *     before its kernel runs, so nothing carries over between calls, including from

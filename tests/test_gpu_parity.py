@@ -307,6 +307,47 @@ def test_full_output_projection_rows_sampled():
     _sampled_parity(Q6, M, 126464, 4096, 3, rows=rows, n_samples=4, width=128)
 
 
+@pytest.mark.parametrize("M", [512, 1024])
+def test_full_ffn_canvas_sweep_sampled(M):
+    """LLaDA-8B FFN at the larger canvases of the sweep: gate/up (Q4_K) and down (Q6_K)
+    with several 128-row token super-tiles per weight tile."""
+    _sampled_parity(Q4, M, 12288, 4096, 5, n_samples=2, width=32)
+    _sampled_parity(Q6, M, 4096, 12288, 6, n_samples=2, width=32)
+
+
+def test_dream_qkv_fused_sampled():
+    """Dream-7B attention projections in one launch: Q N=3584 and K, V N=512 (28 Q heads,
+    4 KV heads) over K=3584 (14 super-blocks, so K-chunks of unequal length)."""
+    M, K, Nq, Nkv = 160, 3584, 3584, 512
+    x = synth.activations(M, K, 7)
+    act = gu.Act(x)
+    oq_, os_, _ = oracle.quantize_act(x)
+    ws_ = [synth.weights(Q4, n, K, 7, i) for i, n in enumerate((Nq, Nkv, Nkv))]
+    wd = [dllm.repack(Q4, w, w.shape[0], K) for w in ws_]
+    outs = [torch.empty((M, Nq), device="cuda"), torch.empty((M, Nkv), device="cuda"),
+            torch.empty((M, Nkv), device="cuda")]
+    wsb = dllm.dllm_qgemm_workspace_bytes(Q4, Nq + 2 * Nkv, K, M)
+    work = dllm.alloc_workspace(wsb)
+    dllm.dllm_qkv_qgemm(wd[0], wd[1], wd[2], Q4, Nq, Nkv, K, act.q, act.scale, act.sums, M, outs[0], Nq, outs[1],
+                        outs[2], Nkv, work, wsb)
+    rng = np.random.default_rng(7)
+    for w, o in zip(ws_, outs):
+        got = o.cpu().numpy()
+        N = w.shape[0]
+        for n0 in sorted(set([0, N - 64] + list(rng.integers(0, N - 64, 2)))):
+            _, ref, T = oracle.qgemm(Q4, w, N, K, oq_, os_, n0=int(n0), n1=int(n0) + 64)
+            ok, worst = gu.tol_ok(got[:, n0:n0 + 64], ref, T)
+            assert ok, (N, n0, worst)
+
+
+def test_dream_down_and_output_sampled():
+    """Dream-7B down projection (Q6_K, K=18944: 74 super-blocks) and output projection
+    (Q6_K, vocab 152064, K=3584) on 32 requested rows of a 160-row canvas."""
+    _sampled_parity(Q6, 160, 3584, 18944, 8, n_samples=2, width=32)
+    rows = synth.block_rows(160, 32, 9)
+    _sampled_parity(Q6, 160, 152064, 3584, 9, rows=rows, n_samples=3, width=128)
+
+
 # ------------------------------------------------------------------ split-K workspace contract
 
 def test_workspace_shared_across_calls_and_shapes():

@@ -164,6 +164,17 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def workload_config(model, L, n_layers, n_rows, world):
+    """The `config` object both arms report: the workload, not the implementation."""
+    gemms = step_gemms(model, L, n_layers)
+    return {"workload": f"{model.name}-shaped denoising step: {n_layers} layers (QKV, O, gate/up Q4_K; "
+                        f"down Q6_K) + output projection (Q6_K, {model.vocab} wide) on {n_rows} requested rows",
+            "canvas_tokens": L, "layers": n_layers,
+            "weight_bytes_per_step": int(sum(g.weight_bytes for g in gemms)),
+            "l2": "inputs larger than L2: every step streams all weights from HBM",
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
+
+
 # ---------------------------------------------------------------------------- ranks
 
 def max_over_ranks(value: float, world: int, device=None) -> float:
@@ -420,13 +431,8 @@ def run_ours(args, rank, world):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": f"{model.name}-shaped denoising step: {n_layers} layers (QKV, O, gate/up Q4_K; "
-                               f"down Q6_K) + output projection (Q6_K, {model.vocab} wide) on "
-                               f"{len(rows_np)} requested rows",
-                   "canvas_tokens": L, "layers": n_layers, "weight_bytes_per_step": int(wbytes_step),
-                   "l2": "inputs larger than L2: every step streams all weights from HBM",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                   "graph": f"CUDA graphs of {S} steps, replayed; no events inside the timed region"},
+        "config": dict(workload_config(model, L, n_layers, len(rows_np), world),
+                       graph=f"CUDA graphs of {S} steps, replayed; no events inside the timed region"),
         "weight_gbs": round(wbytes_step / (ms_step * 1e-3) / 1e9, 1),
         "step_roofline": {"t_star_ms": round(tstar * 1e3, 4), "frac": round(tstar * 1e3 / ms_step, 4),
                           "p_int8_tops": p_int8 / 1e12, "hbm_gbs": hbm_gbs},
@@ -503,7 +509,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": f"{model.name}-shaped denoising step (oracle sample)", "canvas_tokens": L},
+        "config": workload_config(model, L, model.n_layers, min(L, model.out_rows), args.gpus),
         "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": nt, "kind": "oracle",
                          "sample": f"per step: {ncols} of {p.N} output columns of the layer-0 Q projection, "
                                    f"M={L}, K={p.K}"},

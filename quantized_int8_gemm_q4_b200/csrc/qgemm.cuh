@@ -349,10 +349,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 const uint32_t it = item + tt;
                                 if ((int)(it & 1) != who) continue;
                                 const uint32_t set = it & 1;
-                                const uint32_t bst = it % C::B_STAGES, bpar = (it / C::B_STAGES) & 1;
+                                const uint32_t bst = it % C::B_STAGES;
                                 const int ntok = min(NTOK, un.len - tt * NTOK);
                                 if (half == 0) {
-                                    if (!wait_bar_warp(sh, &sh.b_full[bst], bpar)) goto mma_done;
+                                    // (the item's activation stage is full: the unpack waited for it
+                                    // before publishing the A-ring half waited on above)
                                     if (!wait_bar_warp(sh, &sh.acc_empty[set], (it >> 1) & 1)) goto mma_done;
                                 } else if (C::MIN && s == un.sb0) {
                                     // a unit's first min-term MMAs overwrite the min accumulators:
@@ -407,11 +408,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        uint32_t ws = 0, wph = 0, ss = 0, sph = 0, sbc = 0;
+        uint32_t ws = 0, wph = 0, ss = 0, sph = 0, sbc = 0, itm = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
             const Unit un = unit_of(args, u);
-            for (int s = un.sb0; s < un.sb1; s++, sbc++) {
+            const int T = (un.len + NTOK - 1) / NTOK;
+            for (int s = un.sb0; s < un.sb1; s++, sbc++, itm += T) {
                 if (!wait_bar_warp(sh, &sh.w_full[ws], wph)) goto unpack_done;
+                // the super-block's activation stages (one per token tile) are full before
+                // any half of its A ring is published, so the MMA issuer need not wait on them
+                for (int tt = 0; tt < T; tt++) {
+                    const uint32_t it = itm + tt;
+                    if (!wait_bar_warp(sh, &sh.b_full[it % C::B_STAGES], (it / C::B_STAGES) & 1)) goto unpack_done;
+                }
                 const uint8_t* tl = w_stage + ws * C::TILE;
                 if constexpr (QT == 12) {
                     const uint32_t b0 = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_SC + 12 * row);

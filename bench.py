@@ -98,10 +98,16 @@ def load_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(texts=None):
+    """Hash of the CUDA sources with `//` comments and blank lines removed, so that a
+    comment edit does not mark stored ncu counters as stale."""
+    import re
+    if texts is None:
+        texts = [p.read_text() for p in sorted((ROOT / "quantized_int8_gemm_q4_b200" / "csrc").glob("*.cu*"))]
     h = hashlib.sha256()
-    for p in sorted((ROOT / "quantized_int8_gemm_q4_b200" / "csrc").glob("*.cu*")):
-        h.update(p.read_bytes())
+    for t in texts:
+        code = [re.sub(r"\s*//.*$", "", line).rstrip() for line in t.splitlines()]
+        h.update("\n".join(line for line in code if line).encode())
     return h.hexdigest()[:16]
 
 

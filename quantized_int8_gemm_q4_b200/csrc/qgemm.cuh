@@ -39,11 +39,13 @@
 //               with its own accumulator set and a short wait/issue/commit loop
 //   warp 3      idle
 //   warps 4-7   unpack: thread = weight row; decode the super-block, build the two
-//               weight planes per K-step of 32 into tensor memory (the A operand),
-//               the min-term A operand into shared memory, and the f32 d
+//               weight planes per K-step of 32 into a tensor-memory ring of half
+//               super-blocks (the A operand), the min-term A operand into shared
+//               memory, and the f32 d; a half is published only once the
+//               super-block's activation stages have landed
 //   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each on half of
 //               the token columns; per super-block, read the two plane accumulators,
-//               preset them again, and accumulate the f32 result in registers
+//               release them to the issuer, and accumulate the f32 result in registers
 //
 // A work unit is (128 weight rows, up to 128 canvas rows, one K-chunk).  The number
 // of K-chunks per tile depends only on N, K and the SM count, never on M or on the

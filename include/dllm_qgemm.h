@@ -203,6 +203,13 @@ int dllm_debug_subblock_dots(const void* w, dllm_qtype t, int64_t N, int64_t K, 
 int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
                        const uint8_t* sums, int64_t M, int32_t* S, dllm_stream_t stream);
 
+/* Bounded-wait check: launches one CTA of the GEMM kernel whose producer issues no
+ * copy, so the first barrier wait of every other role runs out (after about 2 s).
+ * The kernel then records DLLM_ERR_TIMEOUT in the device error word, frees its tensor
+ * memory and returns; the context stays usable.  Returns the launch status; read the
+ * device status with dllm_get_device_status(). */
+int dllm_debug_bounded_wait(dllm_stream_t stream);
+
 /* int8 tensor-core throughput probe: on each of `ctas` CTAs, `issuers` warps (1..4)
  * each issue `iters` back-to-back tcgen05 kind::i8 MMAs of 128 x n x 32 into their own
  * n_acc accumulators, with A in tensor memory (a_from_tmem != 0) or shared memory.

@@ -553,6 +553,24 @@ int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
     return dispatch(a, t, true, s);
 }
 
+int dllm_debug_bounded_wait(dllm_stream_t stream) {
+    // One CTA of the Q4_K GEMM kernel on a one-tile problem whose producer issues
+    // nothing.  No pointer in the arguments is dereferenced: every other role's first
+    // wait runs out instead.
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.nseg = 1;
+    a.n_tiles = 1;
+    a.nsb = 1;
+    a.kc = 1;
+    a.Mp = 16;
+    a.m_out = 16;
+    a.n_st = 1;
+    a.mu = 16;
+    a.stall = 1;
+    return run_gemm<12, false>(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int issuers, int iters, int ctas,
                       unsigned long long* ns_out, dllm_stream_t stream) {
     if (n < 16 || n > 256 || n % 16 || n_acc < 1 || n_acc > 8 || issuers < 1 || issuers > 4 ||

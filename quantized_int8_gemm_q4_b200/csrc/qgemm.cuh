@@ -134,6 +134,7 @@ struct GemmArgs {
     uint32_t* counters;  // [n_tiles * n_st], when kc > 1
     float* partials;     // [units][mu/4][128 rows][4 tokens], when kc > 1
     int32_t* dbg_S;    // debug: per-super-block integer S instead of f32 (nullable)
+    int32_t stall;     // test: the producer issues nothing, so every other role's wait runs out
     int64_t dbg_N;
 };
 
@@ -276,14 +277,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             uint32_t w_iss = 0, w_php = 0, b_iss = 0, b_php = 0;
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
-            if (lane == 0 && blockIdx.x < n_units) {
+            const int64_t n_prod = args.stall ? 0 : n_units;
+            if (lane == 0 && blockIdx.x < n_prod) {
                 const Unit un = unit_of(args, blockIdx.x);
                 const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
                 for (int s = un.sb0; s < un.sb1 && s < un.sb0 + C::W_STAGES; s++)
                     prefetch_l2(wt + (size_t)s * C::TILE, C::TILE);
             }
             pdl_wait();
-            for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+            for (int64_t u = blockIdx.x; u < n_prod; u += gridDim.x) {
                 const Unit un = unit_of(args, u);
                 const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
                 const int T = (un.len + NTOK - 1) / NTOK;

@@ -30,7 +30,8 @@ DLLM_NOALLOC_SCRATCH_BYTES = 32 << 20
 EXPORTS = (
     "dllm_repacked_bytes", "dllm_repack_q4k", "dllm_repack_q6k", "dllm_act_bytes", "dllm_quantize_act",
     "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_get_device_status",
-    "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_bench_mma_i8",
+    "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_debug_bounded_wait",
+    "dllm_bench_mma_i8",
 )
 
 
@@ -69,6 +70,7 @@ def load() -> ctypes.CDLL:
         "dllm_status_string": [I],
         "dllm_debug_subblock_dots": [P, I, I64, I64, P, I64, P, P],
         "dllm_debug_sb_ints": [P, I, I64, I64, P, P, P, I64, P, P],
+        "dllm_debug_bounded_wait": [P],
         "dllm_bench_mma_i8": [I, I, I, I, I, I, P, P],
     }
     for name, args in sig.items():
@@ -175,6 +177,10 @@ def dllm_debug_subblock_dots(w, qtype: int, N: int, K: int, q, M: int, dots, str
 def dllm_debug_sb_ints(w, qtype: int, N: int, K: int, q, scale, sums, M: int, S, stream=None):
     _check(load().dllm_debug_sb_ints(_ptr(w), qtype, N, K, _ptr(q), _ptr(scale), _ptr(sums), M, _ptr(S),
                                      _stream(stream)), "dllm_debug_sb_ints")
+
+
+def dllm_debug_bounded_wait(stream=None):
+    _check(load().dllm_debug_bounded_wait(_stream(stream)), "dllm_debug_bounded_wait")
 
 
 def dllm_bench_mma_i8(n: int, n_acc: int, a_from_tmem: int, issuers: int, iters: int, ctas: int, ns_out,

@@ -1,0 +1,50 @@
+"""Failure detection on the device without faulting it: every barrier wait in the GEMM
+kernel is bounded, and a wait that runs out ends the kernel with DLLM_ERR_TIMEOUT in the
+device error word instead of hanging.  The test makes one run out (a producer that
+issues no copy, so nothing ever fills the rings), checks the reported status, and then
+checks that the context still computes correct results."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_int8_gemm_q4_b200 import dllm
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test run without a CUDA device")
+    from quantized_int8_gemm_q4_b200 import build
+    build.build()
+    dllm.load()
+    yield
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    t0 = time.monotonic()
+    dllm.dllm_debug_bounded_wait()
+    status = dllm.dllm_get_device_status()  # synchronizes the stream
+    elapsed = time.monotonic() - t0
+    assert status == dllm.DLLM_ERR_TIMEOUT, dllm.status_string(status)
+    assert 1.5 < elapsed < 60.0, elapsed  # the kernel's limit is 2 s
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK  # reading the word cleared it
+
+    # the same context still runs a split-K GEMM correctly
+    M, N, K = 48, 256, 4096
+    w, x = gu.make_case(dllm.DLLM_Q4_K, M, N, K, 77)
+    wd = dllm.repack(dllm.DLLM_Q4_K, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, dllm.DLLM_Q4_K, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    _, ref, T = oracle.qgemm(dllm.DLLM_Q4_K, w, N, K, oq, os_)
+    ok, worst = gu.tol_ok(out, ref, T)
+    assert ok, worst
+    assert np.isfinite(out).all()

@@ -25,6 +25,12 @@
  *     on the host before anything is launched.  Errors found on the device (a row
  *     index out of range, a bounded wait that ran out) set a per-device error word
  *     that dllm_get_device_status() reports and clears; the kernel never traps.
+ *   - dllm_quantize_act, dllm_qgemm and dllm_qkv_qgemm launch their kernels with
+ *     programmatic dependent launch: a kernel may start while the previous kernel on
+ *     the stream is finishing, and waits on the device for it to complete before
+ *     touching any memory that kernel can write.  Before that wait the GEMM only
+ *     prefetches its first weight tiles into L2, which is always safe.  Stream order
+ *     is preserved as usual.
  *   - N must be a multiple of 128 and K a multiple of 256.  Device pointers must be
  *     16-byte aligned.
  *   - Inputs must be finite.

@@ -127,9 +127,10 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  * bytes (that size may be 0, and then workspace may be NULL); otherwise the call
  * returns DLLM_ERR_WORKSPACE.  It holds the gathered rows and, when a tile's K range
  * is split over several CTAs, their partial sums and one arrival counter per tile.
- * It must be zero-filled before its first use; every call that completes leaves the
- * counters as it found them (a call that ends in DLLM_ERR_TIMEOUT may not, so zero
- * it again after one).  Calls that share a workspace must be ordered on one stream.
+ * It must be zero-filled before its first use.  Every call that completes leaves
+ * each counter at a multiple of 16, which is all the next call needs; a call that
+ * ends in DLLM_ERR_TIMEOUT may not, so zero the workspace again after one.  Calls that
+ * share a workspace must be ordered on one stream.
  * For dllm_qkv_qgemm pass N = Nq + 2*Nkv (Nq + Nkv without wv) and n_rows = 0.
  * ---------------------------------------------------------------------------- */
 int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, int64_t n_rows, size_t* bytes);

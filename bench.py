@@ -154,12 +154,19 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+        lines = Path(self.path).read_text().splitlines()
+        os.unlink(self.path)
+        return self.summarize(lines)
+
+    @staticmethod
+    def summarize(lines):
+        """Median SM clock, max clock and the throttle reasons seen, from nvidia-smi
+        csv lines (noheader, nounits) in FIELDS order."""
         rows = []
-        for line in Path(self.path).read_text().splitlines():
+        for line in lines:
             parts = [s.strip() for s in line.split(",")]
             if len(parts) >= 9:
                 rows.append(parts)
-        os.unlink(self.path)
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]

@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_qgemm.argtypes = [ctypes.c_int, P, I64, I64, P, P, I64, P, I64, I64, I64,
                                    P, P, P, I64, ctypes.c_int]
         L.oracle_sb_ints.argtypes = [ctypes.c_int, P, I64, I64, P, I64, P, P, P]
+        L.oracle_rmsnorm.argtypes = [P, I64, I64, I64, P, ctypes.c_float, ctypes.c_double, P]
+        L.oracle_swiglu.argtypes = [P, P, I64, I64, I64, ctypes.c_double, P]
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -153,3 +155,37 @@ def sb_ints(qtype: int, w: np.ndarray, N: int, K: int, q: np.ndarray):
     Smin = np.zeros((M, N, K // QK_K), np.int64)
     _chk(lib().oracle_sb_ints(qtype, _p(w), N, K, _p(q), M, _p(dots), _p(S), _p(Smin)))
     return dots, S, Smin
+
+
+def rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float, ss_scale: float = 1.0) -> np.ndarray:
+    """f32 [M][K] -> f32 [M][K]: f32((x * r) * gamma), r = 1/sqrt(ss/K + eps) in fp64.
+    ss_scale != 1 scales the sum of squares (tests use it to bracket summation order)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    g = np.ascontiguousarray(gamma, dtype=np.float32)
+    M, K = x.shape
+    assert g.shape == (K,)
+    y = np.zeros((M, K), np.float32)
+    _chk(lib().oracle_rmsnorm(_p(x), M, K, K, _p(g), float(eps), float(ss_scale), _p(y)))
+    return y
+
+
+def swiglu(gate: np.ndarray, up: np.ndarray, h_scale: float = 1.0) -> np.ndarray:
+    """f32 [M][K] x2 -> f32 [M][K]: f32((g / (1 + exp(-g))) * u) in fp64.
+    h_scale != 1 scales the fp64 value before rounding (tests use it to bracket exp)."""
+    g = np.ascontiguousarray(gate, dtype=np.float32)
+    u = np.ascontiguousarray(up, dtype=np.float32)
+    assert g.shape == u.shape
+    M, K = g.shape
+    h = np.zeros((M, K), np.float32)
+    _chk(lib().oracle_swiglu(_p(g), _p(u), M, K, K, float(h_scale), _p(h)))
+    return h
+
+
+def rmsnorm_quantize(x: np.ndarray, gamma: np.ndarray, eps: float):
+    """quantize_act(rmsnorm(x)): the definition the fused library kernel follows."""
+    return quantize_act(rmsnorm(x, gamma, eps))
+
+
+def swiglu_quantize(gate: np.ndarray, up: np.ndarray):
+    """quantize_act(swiglu(gate, up)): the definition the fused library kernel follows."""
+    return quantize_act(swiglu(gate, up))

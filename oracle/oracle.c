@@ -24,6 +24,11 @@
  *    a = scale[m][sb] * qa.  It is formed the way the method runs it: integer
  *    sub-block dots, integer per-super-block combinations, and one fp64
  *    combine per super-block, rounded to f32 once at the end.
+ *  - The steps either side of the quantizer in a forward pass (Architecture page,
+ *    "A forward pass", steps 2 and 4): RMSNorm of a projection input, and the
+ *    SwiGLU gate SiLU(g) * u between the gate/up and down projections.  Both are
+ *    formed in fp64 and rounded to f32 once; the fused library kernels quantize
+ *    that f32 exactly like oracle_quantize_act.
  *
  * Parity status: every function here is pinned by tests (gguf package decode,
  * brute-force fp64 dequantize-then-matmul, closed forms and invariants).
@@ -199,6 +204,60 @@ int oracle_quantize_act(const float *x, int64_t M, int64_t K, int64_t ldx,
                 for (int i = 0; i < 32; i++) t += qb[32 * j + i];
                 asum32[m * (K / 32) + s * 8 + j] = t;
             }
+        }
+    return 0;
+}
+
+/*
+ * RMSNorm (Architecture page, "A forward pass", steps 2 and 4: every layer
+ * normalises its attention input and its FFN input, and the final hidden state is
+ * normalised before the output projection).  The page names the step but gives no
+ * formula or precision.  Reading taken, the usual RMSNorm of both model families:
+ * y = x * r * gamma with r = 1 / sqrt(mean over the row of x^2 + eps).  It is
+ * evaluated in fp64 and rounded to f32 once, because the f32 activation quantizer
+ * consumes y:
+ *     ss = sum over the K elements of x_k * x_k   (each square exact in fp64)
+ *     r  = 1 / sqrt(ss / K + eps)
+ *     y  = f32((x * r) * gamma)
+ * ss_scale multiplies ss before use.  It is 1 for the definition.  Tests pass
+ * 1 +- delta to bracket the effect of any other summation order: r and y are
+ * monotone in ss, because every later step is one correctly rounded operation.
+ * x is [M][ldx] (ldx >= K), gamma is [K], y is [M][K].
+ */
+int oracle_rmsnorm(const float *x, int64_t M, int64_t K, int64_t ldx,
+                   const float *gamma, float eps, double ss_scale, float *y)
+{
+    if (K <= 0 || ldx < K || !(eps >= 0.0f)) return -1;
+    for (int64_t m = 0; m < M; m++) {
+        const float *xr = x + m * ldx;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; k++) ss += (double)xr[k] * (double)xr[k];
+        ss *= ss_scale;
+        double r = 1.0 / sqrt(ss / (double)K + (double)eps);
+        for (int64_t k = 0; k < K; k++)
+            y[m * K + k] = (float)(((double)xr[k] * r) * (double)gamma[k]);
+    }
+    return 0;
+}
+
+/*
+ * Gated FFN activation (Architecture page, "A forward pass", step 2: the FFN
+ * applies SiLU between the gate/up projections and the down projection).  Reading
+ * taken, the SwiGLU of both model families: h = SiLU(g) * u with
+ * SiLU(g) = g / (1 + e^-g).  Evaluated in fp64 and rounded to f32 once:
+ *     h = f32((g / (1 + exp(-g))) * u * h_scale)
+ * h_scale is 1 for the definition.  Tests pass 1 +- delta to bracket the last-place
+ * differences of another exp.  gate and up are [M][ld] (ld >= K), h is [M][K].
+ */
+int oracle_swiglu(const float *gate, const float *up, int64_t M, int64_t K, int64_t ld,
+                  double h_scale, float *h)
+{
+    if (K <= 0 || ld < K) return -1;
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t k = 0; k < K; k++) {
+            double g = gate[m * ld + k], u = up[m * ld + k];
+            double silu = g / (1.0 + exp(-g));
+            h[m * K + k] = (float)(silu * u * h_scale);
         }
     return 0;
 }

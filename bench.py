@@ -2,10 +2,12 @@
 """Benchmark: the projection GEMMs of one LLaDA-8B-shaped denoising step on B200.
 
 A step is one pass of the whole hot path over one synthetic canvas: for each of the
-32 layers, quantize the attention input once and run Q, K and V in one launch,
-quantize and run O, quantize once and run gate and up in one launch, quantize and
-run down (Q6_K); then quantize the final hidden state and run the 126464-wide output
-projection (Q6_K) on the 32 rows of the current block only.  Weights are random
+32 layers, RMSNorm and quantize the attention input once (one fused kernel) and run
+Q, K and V in one launch, quantize and run O, RMSNorm and quantize the FFN input once
+and run gate and up in one launch, apply SwiGLU to the gate/up outputs and quantize
+(one fused kernel) and run down (Q6_K); then RMSNorm and quantize the final hidden
+state and run the 126464-wide output projection (Q6_K) on the 32 rows of the current
+block only.  Weights are random
 (the GGUF Q4_K / Q6_K distributions of the synthetic workloads), drawn on the device,
 repacked once and kept resident (4.77 GB, far above the 126 MB L2, so every step
 streams them from HBM).
@@ -180,8 +182,10 @@ class ClockSampler:
 def workload_config(model, L, n_layers, n_rows, world):
     """The `config` object both arms report: the workload, not the implementation."""
     gemms = step_gemms(model, L, n_layers)
-    return {"workload": f"{model.name}-shaped denoising step: {n_layers} layers (QKV, O, gate/up Q4_K; "
-                        f"down Q6_K) + output projection (Q6_K, {model.vocab} wide) on {n_rows} requested rows",
+    return {"workload": f"{model.name}-shaped denoising step: {n_layers} layers (RMSNorm+quantize -> QKV, "
+                        f"quantize -> O, RMSNorm+quantize -> gate/up Q4_K, SwiGLU+quantize -> down Q6_K) + "
+                        f"final RMSNorm+quantize -> output projection (Q6_K, {model.vocab} wide) on {n_rows} "
+                        f"requested rows",
             "canvas_tokens": L, "layers": n_layers,
             "weight_bytes_per_step": int(sum(g.weight_bytes for g in gemms)),
             "l2": "inputs larger than L2: every step streams all weights from HBM",
@@ -245,16 +249,21 @@ def run_ours(args, rank, world):
     del g
     torch.cuda.synchronize()
 
-    # ---- activations (the f32 inputs of each projection), one contiguous buffer
-    sizes = [L * h, L * h, L * h, L * f, L * h]
+    # ---- the step's f32 inputs, one contiguous buffer: the residual stream entering
+    # each layer's attention and FFN norms, the attention output and the final hidden
+    # state.  The down projection's input is the SwiGLU of the gate/up outputs.
+    sizes = [L * h] * 4
     xin = torch.empty(sum(sizes), dtype=torch.float32, device=dev)
     views, off = [], 0
     for i, sz in enumerate(sizes):
         v = xin[off:off + sz].view(L, -1)
-        v.copy_(synth.device_activations(L, sz // L, seed, 100 + i, device=dev))
+        v.copy_(synth.device_activations(L, sz // L, seed, 100 + (4 if i == 3 else i), device=dev))
         views.append(v)
         off += sz
-    x_attn, x_o, x_ffn, x_down, x_fin = views
+    x_attn, x_o, x_ffn, x_fin = views
+    gam_host = synth.norm_weights(2 * n_layers + 1, h, seed)   # attn, ffn per layer; final
+    gam = torch.from_numpy(gam_host).to(dev)
+    eps = model.norm_eps
     act_h = dllm.alloc_act(L, h, dev)
     act_f = dllm.alloc_act(L, f, dev)
     o_q = torch.empty((L, model.q_out), device=dev)
@@ -287,7 +296,7 @@ def run_ours(args, rank, world):
 
         for l in range(n_layers):
             W = layers[l]
-            dllm.dllm_quantize_act(x_attn, L, h, h, *act_h)
+            dllm.dllm_rmsnorm_quantize(x_attn, L, h, h, gam[2 * l], eps, *act_h)
             mark()
             dllm.dllm_qkv_qgemm(W["q"], W["k"], W["v"], Q4, model.q_out, model.kv_out, h, *act_h, L,
                                 o_q, model.q_out, o_k, o_v, model.kv_out, ws, wsb)
@@ -296,15 +305,15 @@ def run_ours(args, rank, world):
             mark()
             dllm.dllm_qgemm(W["o"], Q4, h, h, *act_h, L, None, 0, o_o, h, ws, wsb)
             mark()
-            dllm.dllm_quantize_act(x_ffn, L, h, h, *act_h)
+            dllm.dllm_rmsnorm_quantize(x_ffn, L, h, h, gam[2 * l + 1], eps, *act_h)
             mark()
             dllm.dllm_qkv_qgemm(W["gate"], W["up"], None, Q4, f, f, h, *act_h, L, o_g, f, o_u, None, f, ws, wsb)
             mark()
-            dllm.dllm_quantize_act(x_down, L, f, f, *act_f)
+            dllm.dllm_swiglu_quantize(o_g, o_u, L, f, f, *act_f)
             mark()
             dllm.dllm_qgemm(W["down"], Q6, h, f, *act_f, L, None, 0, o_d, h, ws, wsb)
             mark()
-        dllm.dllm_quantize_act(x_fin, L, h, h, *act_h)
+        dllm.dllm_rmsnorm_quantize(x_fin, L, h, h, gam[2 * n_layers], eps, *act_h)
         mark()
         dllm.dllm_qgemm(w_out, Q6, model.vocab, h, *act_h, L, rows, len(rows_np), logits, model.vocab, ws, wsb)
         mark()
@@ -437,7 +446,7 @@ def run_ours(args, rank, world):
 
     cpu = None
     if rank == 0 and not args.no_cpu and cpu_sample:
-        cpu = cpu_baseline(model, L, cpu_sample, rows_np, seed)
+        cpu = cpu_baseline(model, L, cpu_sample, rows_np, seed, gam_host, n_layers)
 
     del gE, gS, g1
     result = {
@@ -456,38 +465,44 @@ def run_ours(args, rank, world):
     return result
 
 
-def cpu_baseline(model, L, sample, rows_np, seed, max_threads=None):
+def cpu_baseline(model, L, sample, rows_np, seed, gam, n_layers, max_threads=None):
     """The oracle, as it stands, on a bounded sample of the same step: the projection
-    sets of the first few layers and the output projection on the requested rows."""
+    sets of the first few layers (with their RMSNorm and SwiGLU quantizers) and the
+    output projection on the requested rows."""
     import oracle
     from quantized_int8_gemm_q4_b200 import synth
     nt = max_threads or oracle.max_threads()
-    h, f = model.hidden, model.ffn
+    h = model.hidden
+    eps = model.norm_eps
     x = {"attn": synth.activations(L, h, seed, 100), "o": synth.activations(L, h, seed, 101),
-         "ffn": synth.activations(L, h, seed, 102), "down": synth.activations(L, f, seed, 103),
-         "fin": synth.activations(L, h, seed, 104)}
-    src = {"q": "attn", "k": "attn", "v": "attn", "o": "o", "gate": "ffn", "up": "ffn", "down": "down"}
+         "ffn": synth.activations(L, h, seed, 102), "fin": synth.activations(L, h, seed, 104)}
     ops = 0
     t0 = time.perf_counter()
-    qa = {k: oracle.quantize_act(v)[:2] for k, v in x.items()}
     nl = 0
     for l, mats in sample.items():
         if l == "output":
             continue
         nl += 1
-        for name, (p, blocks) in mats.items():
-            q, s = qa[src[name]]
-            oracle.qgemm(p.qtype, blocks, p.N, p.K, q, s, nthreads=nt)
+        out = {}
+        qa = {"attn": oracle.rmsnorm_quantize(x["attn"], gam[2 * l], eps)[:2], "o": oracle.quantize_act(x["o"])[:2],
+              "ffn": oracle.rmsnorm_quantize(x["ffn"], gam[2 * l + 1], eps)[:2]}
+        for name, src in (("q", "attn"), ("k", "attn"), ("v", "attn"), ("o", "o"), ("gate", "ffn"), ("up", "ffn")):
+            p, blocks = mats[name]
+            out[name] = oracle.qgemm(p.qtype, blocks, p.N, p.K, *qa[src], nthreads=nt)[0]
             ops += 2 * L * p.N * p.K
+        p, blocks = mats["down"]
+        q, s, _ = oracle.swiglu_quantize(out["gate"], out["up"])
+        oracle.qgemm(p.qtype, blocks, p.N, p.K, q, s, nthreads=nt)
+        ops += 2 * L * p.N * p.K
     if "output" in sample:
-        q, s = qa["fin"]
+        q, s, _ = oracle.rmsnorm_quantize(x["fin"], gam[2 * n_layers], eps)
         oracle.qgemm(Q6, sample["output"], model.vocab, h, q, s, rows=rows_np, nthreads=nt)
         ops += 2 * len(rows_np) * model.vocab * h
     dt = time.perf_counter() - t0
     return {"value": round(ops / dt / 1e12, 6), "unit": UNIT, "cores": nt, "kind": "oracle",
             "seconds": round(dt, 2),
             "sample": f"{nl} of {model.n_layers} layers' projection sets + output projection on "
-                      f"{len(rows_np)} rows, canvas {L} (quantize included)"}
+                      f"{len(rows_np)} rows, canvas {L} (RMSNorm, SwiGLU and quantize included)"}
 
 
 # ---------------------------------------------------------------------------- reference arm

@@ -110,6 +110,41 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
                       uint8_t* sums, dllm_stream_t stream);
 
 /* ------------------------------------------------------------------------------
+ * Quantization fused with the step that produces its input (Architecture page,
+ * "A forward pass", steps 2 and 4).  Each layer runs RMSNorm before the Q/K/V and the
+ * gate/up projections, and the final hidden state is normalised before the output
+ * projection.  The FFN applies SiLU between gate/up and down.  The normalised or gated
+ * f32 value is quantized in registers and never stored.  q, scale and sums have
+ * exactly the layouts, sizes (dllm_act_bytes) and zero padding rows of
+ * dllm_quantize_act, and the GEMM entry points consume them unchanged.
+ *
+ * Arithmetic (the page names the steps without formulas; these are the readings the
+ * library implements).  Each value is formed in fp64 with correctly rounded
+ * operations and rounded to f32 once.  The f32 is then quantized exactly as in
+ * dllm_quantize_act.
+ *   RMSNorm: ss = sum over the row's K elements of x^2, r = 1 / sqrt(ss / K + eps),
+ *            y = f32((x * r) * gamma[k]).  The order of the fp64 sum is unspecified.
+ *            A different order can move y by one f32 rounding only when the fp64
+ *            value lies within about K * 2^-53 (relative) of a rounding boundary.
+ *   SwiGLU:  h = f32((g / (1 + exp(-g))) * u).  exp is CUDA's fp64 exp.
+ *
+ * dllm_rmsnorm_quantize: x f32 [M][ldx] (ldx >= K, ldx % 4 == 0), gamma f32 [K],
+ *   eps > 0 and finite (else DLLM_ERR_ARG; eps = 0 would make an all-zero row 0/0).
+ *   One CTA per canvas row (M rounded up to 16 CTAs).
+ * dllm_swiglu_quantize: gate, up f32 [M][ld] each (ld >= K, ld % 4 == 0).  They may
+ *   be two column ranges of one buffer, e.g. the out_q/out_k pair of dllm_qkv_qgemm
+ *   run on the gate and up weights with ld = 2 * K and up = gate + K.
+ * Inputs are only read; the caller owns every buffer.  Both launch with programmatic
+ * dependent launch, like dllm_quantize_act.  Errors: DLLM_ERR_ARG (sizes, eps, null),
+ * DLLM_ERR_ALIGN (a pointer not 16-byte aligned or a leading dimension not a multiple
+ * of 4), DLLM_ERR_UNSUPPORTED, DLLM_ERR_CUDA.
+ * ---------------------------------------------------------------------------- */
+int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, const float* gamma, float eps,
+                          int8_t* q, float* scale, uint8_t* sums, dllm_stream_t stream);
+int dllm_swiglu_quantize(const float* gate, const float* up, int64_t M, int64_t K, int64_t ld, int8_t* q,
+                         float* scale, uint8_t* sums, dllm_stream_t stream);
+
+/* ------------------------------------------------------------------------------
  * GEMM: out[i][n] for n in [0, N) of one repacked weight matrix `w` (from
  * dllm_repack_*), activations (q, scale, sums) of an M-row canvas from
  * dllm_quantize_act.

@@ -1,0 +1,151 @@
+// Activation quantization fused with the step that produces its input in a forward
+// pass (Architecture page, "A forward pass", steps 2 and 4): RMSNorm in front of the
+// Q/K/V, gate/up and output projections, and the SwiGLU gate SiLU(g) * u in front of
+// the down projection.  The f32 value each step produces is quantized in registers
+// and never written to memory; the outputs are those of quantize_act_kernel, in the
+// same layouts, so the GEMM consumes them unchanged.
+//
+// Precision: the normalised or gated value is formed in fp64 with explicitly rounded
+// operations (no contraction) and rounded to f32 once; that f32 is quantized with
+// quantize_act_kernel's arithmetic.  RMSNorm: ss = sum of x^2, r = 1/sqrt(ss/K + eps),
+// y = f32((x * r) * gamma).  SwiGLU: h = f32((g / (1 + exp(-g))) * u).
+#pragma once
+
+#include "layout.cuh"
+
+namespace dllm {
+
+// Quantizes the 8 values v[] that this lane holds of one 256-block (elements
+// 8 lane .. 8 lane + 7 of super-block s of canvas row m) and stores the codes, the
+// block scale and the two-float scaled sub-block sums in the layouts that
+// quantize_act_kernel writes (Mp = the canvas rounded up to 16 rows).  The whole warp
+// calls it for the same (m, s).  Arithmetic: amax by warp reduction, iscale = 127/amax
+// and scale = amax/127 as IEEE f32 divisions, code = round-half-even(v * iscale)
+// clamped to [-127, 127]; sum of each sub-block of 32 (lanes 4j..4j+3) times scale.
+__device__ __forceinline__ void quantize_store_lane(const float (&v)[8], int lane, int64_t m, int64_t s,
+                                                    int64_t Mp, int8_t* __restrict__ q,
+                                                    float* __restrict__ scale, uint8_t* __restrict__ sums) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float iscale = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    const float sc = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    uint32_t packed[2] = {0u, 0u};
+    int part = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        int t = __float2int_rn(__fmul_rn(v[i], iscale));
+        t = max(-127, min(127, t));
+        part += t;
+        packed[i >> 2] |= (uint32_t)(t & 255) << (8 * (i & 3));
+    }
+    const int64_t g = m >> 3;
+    const int r = (int)(m & 7);
+    const int64_t blk = s * (Mp / 8) + g;
+    // 16-byte chunk lane/2 of row r: [blk][chunk][8 rows][16 bytes], lane half (lane & 1)
+    *reinterpret_cast<uint2*>(q + (blk * 16 + (lane >> 1)) * 128 + r * 16 + (lane & 1) * 8) =
+        make_uint2(packed[0], packed[1]);
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    if ((lane & 3) == 0) {
+        const int j = lane >> 2;
+        float hi, lo;
+        split_tf32(__fmul_rn(sc, (float)part), hi, lo);
+        float* ts = reinterpret_cast<float*>(sums + blk * 512);
+        ts[((j >> 2) * 8 + r) * 4 + (j & 3)] = hi;
+        ts[((2 + (j >> 2)) * 8 + r) * 4 + (j & 3)] = lo;
+    }
+    if (lane == 0) scale[s * Mp + m] = sc;
+}
+
+__device__ __forceinline__ void load8(const float* __restrict__ p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+constexpr int FUSE_WARPS = 8;
+
+// RMSNorm + quantize.  One CTA of 8 warps per canvas row m in [0, Mp); warp w handles
+// super-blocks w, w + 8, ...  Pass 1 sums the squares in fp64 (each lane in element
+// order, then a fixed reduction tree); pass 2 re-reads the row (an L1 hit), normalises
+// and quantizes.  Rows M..Mp-1 are written as zeros.
+__global__ void __launch_bounds__(FUSE_WARPS * 32) rmsnorm_quantize_kernel(
+    const float* __restrict__ x, int64_t M, int64_t K, int64_t ldx, const float* __restrict__ gamma, float eps,
+    int64_t Mp, int8_t* __restrict__ q, float* __restrict__ scale, uint8_t* __restrict__ sums) {
+    __shared__ double red[FUSE_WARPS];
+    pdl_trigger();
+    pdl_wait();  // x may be the output of the previous kernel on the stream
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t m = blockIdx.x;
+    const int64_t nsb = K / QK;
+    const bool live = m < M;
+    const float* xr = x + m * ldx;
+    double ss = 0.0;
+    if (live) {
+#pragma unroll 2
+        for (int64_t s = w; s < nsb; s += FUSE_WARPS) {
+            float v[8];
+            load8(xr + s * QK + 8 * lane, v);
+#pragma unroll
+            for (int i = 0; i < 8; i++) ss = __dadd_rn(ss, __dmul_rn((double)v[i], (double)v[i]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+    if (lane == 0) red[w] = ss;
+    __syncthreads();
+    ss = red[0];
+#pragma unroll
+    for (int i = 1; i < FUSE_WARPS; i++) ss = __dadd_rn(ss, red[i]);
+    const double rn = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)eps)));
+    for (int64_t s = w; s < nsb; s += FUSE_WARPS) {
+        float v[8];
+        if (live) {
+            float xv[8], gv[8];
+            load8(xr + s * QK + 8 * lane, xv);
+            load8(gamma + s * QK + 8 * lane, gv);
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                v[i] = __double2float_rn(__dmul_rn(__dmul_rn((double)xv[i], rn), (double)gv[i]));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; i++) v[i] = 0.0f;
+        }
+        quantize_store_lane(v, lane, m, s, Mp, q, scale, sums);
+    }
+}
+
+// SwiGLU + quantize.  Grid (Mp, ceil(nsb / 8)); warp w of CTA (m, b) handles
+// super-block 8 b + w of canvas row m.  Rows M..Mp-1 are written as zeros.
+__global__ void __launch_bounds__(FUSE_WARPS * 32) swiglu_quantize_kernel(
+    const float* __restrict__ gate, const float* __restrict__ up, int64_t M, int64_t K, int64_t ld, int64_t Mp,
+    int8_t* __restrict__ q, float* __restrict__ scale, uint8_t* __restrict__ sums) {
+    pdl_trigger();
+    pdl_wait();  // gate and up are normally the output of the previous kernel
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t m = blockIdx.x;
+    const int64_t s = (int64_t)blockIdx.y * FUSE_WARPS + w;
+    if (s >= K / QK) return;  // whole warp: no collective below spans warps
+    float v[8];
+    if (m < M) {
+        float gv[8], uv[8];
+        load8(gate + m * ld + s * QK + 8 * lane, gv);
+        load8(up + m * ld + s * QK + 8 * lane, uv);
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const double g = gv[i];
+            const double silu = __ddiv_rn(g, __dadd_rn(1.0, exp(-g)));
+            v[i] = __double2float_rn(__dmul_rn(silu, (double)uv[i]));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; i++) v[i] = 0.0f;
+    }
+    quantize_store_lane(v, lane, m, s, Mp, q, scale, sums);
+}
+
+}  // namespace dllm

@@ -3,6 +3,7 @@
 #include <cstring>
 
 #include "../../include/dllm_qgemm.h"
+#include "actfuse.cuh"
 #include "layout.cuh"
 #include "qgemm.cuh"
 
@@ -210,6 +211,45 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     dim3 grid((unsigned)(Mp / 8), (unsigned)(K / QK));
     if (launch_pdl(quantize_act_kernel, grid, dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), x, M, ldx, Mp, q,
                    scale, sums) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DLLM_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, const float* gamma, float eps, int8_t* q,
+                          float* scale, uint8_t* sums, dllm_stream_t stream) {
+    if (!x || !gamma || M <= 0 || K <= 0 || K % QK || ldx < K) return DLLM_ERR_ARG;
+    if (!(eps > 0.0f) || !(eps < INFINITY)) return DLLM_ERR_ARG;
+    int rc = check_act(q, scale, sums, M);
+    if (rc) return rc;
+    if (!aligned16(x) || !aligned16(gamma) || ldx % 4) return DLLM_ERR_ALIGN;
+    if (M > (1LL << 31) - 16) return DLLM_ERR_ARG;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    const int64_t Mp = round_up(M, 16);
+    if (launch_pdl(rmsnorm_quantize_kernel, dim3((unsigned)Mp), dim3(FUSE_WARPS * 32), 0,
+                   reinterpret_cast<cudaStream_t>(stream), x, M, K, ldx, gamma, eps, Mp, q, scale, sums) !=
+        cudaSuccess) {
+        (void)cudaGetLastError();
+        return DLLM_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+int dllm_swiglu_quantize(const float* gate, const float* up, int64_t M, int64_t K, int64_t ld, int8_t* q, float* scale,
+                         uint8_t* sums, dllm_stream_t stream) {
+    if (!gate || !up || M <= 0 || K <= 0 || K % QK || ld < K) return DLLM_ERR_ARG;
+    int rc = check_act(q, scale, sums, M);
+    if (rc) return rc;
+    if (!aligned16(gate) || !aligned16(up) || ld % 4) return DLLM_ERR_ALIGN;
+    if (M > (1LL << 31) - 16 || K / QK > 65535LL * FUSE_WARPS) return DLLM_ERR_ARG;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    const int64_t Mp = round_up(M, 16);
+    const dim3 grid((unsigned)Mp, (unsigned)((K / QK + FUSE_WARPS - 1) / FUSE_WARPS));
+    if (launch_pdl(swiglu_quantize_kernel, grid, dim3(FUSE_WARPS * 32), 0, reinterpret_cast<cudaStream_t>(stream),
+                   gate, up, M, K, ld, Mp, q, scale, sums) != cudaSuccess) {
         (void)cudaGetLastError();
         return DLLM_ERR_CUDA;
     }

@@ -29,6 +29,7 @@ DLLM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 EXPORTS = (
     "dllm_repacked_bytes", "dllm_repack_q4k", "dllm_repack_q6k", "dllm_act_bytes", "dllm_quantize_act",
+    "dllm_rmsnorm_quantize", "dllm_swiglu_quantize",
     "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_get_device_status",
     "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_debug_bounded_wait",
     "dllm_bench_mma_i8",
@@ -62,6 +63,8 @@ def load() -> ctypes.CDLL:
         "dllm_repack_q6k": [P, I64, I64, P, P],
         "dllm_act_bytes": [I64, I64, PSZ, PSZ, PSZ],
         "dllm_quantize_act": [P, I64, I64, I64, P, P, P, P],
+        "dllm_rmsnorm_quantize": [P, I64, I64, I64, P, ctypes.c_float, P, P, P, P],
+        "dllm_swiglu_quantize": [P, P, I64, I64, I64, P, P, P, P],
         "dllm_qgemm_workspace_bytes": [I, I64, I64, I64, I64, PSZ],
         "dllm_qgemm": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P, SZ, P],
         "dllm_qgemm_noalloc": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P],
@@ -133,6 +136,16 @@ def dllm_act_bytes(M: int, K: int):
 def dllm_quantize_act(x, M: int, K: int, ldx: int, q, scale, sums, stream=None):
     _check(load().dllm_quantize_act(_ptr(x), M, K, ldx, _ptr(q), _ptr(scale), _ptr(sums), _stream(stream)),
            "dllm_quantize_act")
+
+
+def dllm_rmsnorm_quantize(x, M: int, K: int, ldx: int, gamma, eps: float, q, scale, sums, stream=None):
+    _check(load().dllm_rmsnorm_quantize(_ptr(x), M, K, ldx, _ptr(gamma), float(eps), _ptr(q), _ptr(scale),
+                                        _ptr(sums), _stream(stream)), "dllm_rmsnorm_quantize")
+
+
+def dllm_swiglu_quantize(gate, up, M: int, K: int, ld: int, q, scale, sums, stream=None):
+    _check(load().dllm_swiglu_quantize(_ptr(gate), _ptr(up), M, K, ld, _ptr(q), _ptr(scale), _ptr(sums),
+                                       _stream(stream)), "dllm_swiglu_quantize")
 
 
 def dllm_qgemm_workspace_bytes(qtype: int, N: int, K: int, M: int, n_rows: int = 0) -> int:

@@ -68,6 +68,11 @@ def activations(M: int, K: int, seed, *sub) -> np.ndarray:
     return _rng(seed, 8, *sub).standard_normal((M, K), dtype=np.float32)
 
 
+def norm_weights(n: int, K: int, seed, *sub) -> np.ndarray:
+    """f32 [n, K] RMSNorm gains, uniform in [0.5, 1.5) (trained gains sit around 1)."""
+    return (_rng(seed, 10, *sub).random((n, K)) + 0.5).astype(np.float32)
+
+
 def block_rows(M: int, n_rows: int, seed, *sub, block: int | None = None) -> np.ndarray:
     """n_rows distinct canvas rows in random order, drawn from one 32-row window
     [32 + 32b, 64 + 32b) of an M-row canvas whose first 32 rows are the prompt."""
@@ -98,6 +103,7 @@ class Model:
     vocab: int
     out_rows: int = 32
     layer: tuple = field(default=())
+    norm_eps: float = 1e-5
 
 
 def llada_8b() -> Model:
@@ -113,7 +119,7 @@ def dream_7b() -> Model:
     return Model("dream-7b", h, f, 28, h, 512, 152064, 32,
                  (Proj("q", Q4_K, h, h), Proj("k", Q4_K, 512, h), Proj("v", Q4_K, 512, h),
                   Proj("o", Q4_K, h, h), Proj("gate", Q4_K, f, h), Proj("up", Q4_K, f, h),
-                  Proj("down", Q6_K, h, f)))
+                  Proj("down", Q6_K, h, f)), norm_eps=1e-6)
 
 
 MODELS = {"llada-8b": llada_8b, "dream-7b": dream_7b}

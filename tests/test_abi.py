@@ -30,7 +30,7 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for must in ("dllm_repack_q4k", "dllm_repack_q6k", "dllm_quantize_act", "dllm_qgemm", "dllm_qkv_qgemm",
-                 "dllm_get_device_status", "dllm_status_string", "dllm_debug_subblock_dots"):
+                 "dllm_rmsnorm_quantize", "dllm_swiglu_quantize", "dllm_get_device_status", "dllm_status_string", "dllm_debug_subblock_dots"):
         assert must in syms
 
 
@@ -101,6 +101,41 @@ def test_quantize_argument_checks(lib):
     assert f(_fake(A), 4, 256, 128, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
     assert f(_fake(A + 4), 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ALIGN
     assert f(_fake(A), 4, 256, 258, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ALIGN
+
+
+def test_fused_quantize_argument_checks(lib):
+    A = 0x10000
+    f = lib.dllm_rmsnorm_quantize
+    ok = (_fake(A), 4, 256, 256, _fake(A), 1e-5, _fake(A), _fake(A), _fake(A), None)
+
+    def rms(**kw):
+        a = list(ok)
+        for i, k in enumerate(("x", "M", "K", "ldx", "gamma", "eps", "q", "scale", "sums")):
+            if k in kw:
+                a[i] = kw[k]
+        return f(*a)
+    assert rms(x=None) == dllm.DLLM_ERR_ARG
+    assert rms(gamma=None) == dllm.DLLM_ERR_ARG
+    assert rms(K=300, ldx=300) == dllm.DLLM_ERR_ARG
+    assert rms(ldx=128) == dllm.DLLM_ERR_ARG
+    assert rms(M=0) == dllm.DLLM_ERR_ARG
+    assert rms(eps=0.0) == dllm.DLLM_ERR_ARG
+    assert rms(eps=-1e-5) == dllm.DLLM_ERR_ARG
+    assert rms(eps=float("inf")) == dllm.DLLM_ERR_ARG
+    assert rms(eps=float("nan")) == dllm.DLLM_ERR_ARG
+    assert rms(x=_fake(A + 4)) == dllm.DLLM_ERR_ALIGN
+    assert rms(gamma=_fake(A + 8)) == dllm.DLLM_ERR_ALIGN
+    assert rms(ldx=258) == dllm.DLLM_ERR_ALIGN
+    assert rms(q=_fake(A + 1)) == dllm.DLLM_ERR_ALIGN
+    g = lib.dllm_swiglu_quantize
+    assert g(None, _fake(A), 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert g(_fake(A), None, 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert g(_fake(A), _fake(A), 4, 256, 128, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert g(_fake(A), _fake(A), 4, 260, 512, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert g(_fake(A), _fake(A), 0, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
+    assert g(_fake(A), _fake(A + 4), 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ALIGN
+    assert g(_fake(A), _fake(A), 4, 256, 514, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ALIGN
+    assert g(_fake(A), _fake(A), 4, 256, 256, _fake(A), _fake(A + 2), _fake(A), None) == dllm.DLLM_ERR_ALIGN
 
 
 def test_repack_rejects_overlap(lib):

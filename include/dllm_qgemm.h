@@ -25,8 +25,8 @@
  *     on the host before anything is launched.  Errors found on the device (a row
  *     index out of range, a bounded wait that ran out) set a per-device error word
  *     that dllm_get_device_status() reports and clears; the kernel never traps.
- *   - dllm_quantize_act, dllm_qgemm and dllm_qkv_qgemm launch their kernels with
- *     programmatic dependent launch: a kernel may start while the previous kernel on
+ *   - dllm_quantize_act, dllm_rmsnorm_quantize, dllm_swiglu_quantize, dllm_qgemm and
+ *     dllm_qkv_qgemm launch their kernels with programmatic dependent launch: a kernel may start while the previous kernel on
  *     the stream is finishing, and waits on the device for it to complete before
  *     touching any memory that kernel can write.  Before that wait the GEMM only
  *     prefetches its first weight tiles into L2, which is always safe.  Stream order
@@ -130,7 +130,7 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  *
  * dllm_rmsnorm_quantize: x f32 [M][ldx] (ldx >= K, ldx % 4 == 0), gamma f32 [K],
  *   eps > 0 and finite (else DLLM_ERR_ARG; eps = 0 would make an all-zero row 0/0).
- *   One CTA per canvas row (M rounded up to 16 CTAs).
+ *   One CTA per canvas row (M rounded up to 16 CTAs), min(K/256, 32) warps.
  * dllm_swiglu_quantize: gate, up f32 [M][ld] each (ld >= K, ld % 4 == 0).  They may
  *   be two column ranges of one buffer, e.g. the out_q/out_k pair of dllm_qkv_qgemm
  *   run on the gate and up weights with ld = 2 * K and up = gate + K.

@@ -69,25 +69,34 @@ __device__ __forceinline__ void load8(const float* __restrict__ p, float (&v)[8]
 
 constexpr int FUSE_WARPS = 8;
 
-// RMSNorm + quantize.  One CTA of 8 warps per canvas row m in [0, Mp); warp w handles
-// super-blocks w, w + 8, ...  Pass 1 sums the squares in fp64 (each lane in element
-// order, then a fixed reduction tree); pass 2 re-reads the row (an L1 hit), normalises
-// and quantizes.  Rows M..Mp-1 are written as zeros.
-__global__ void __launch_bounds__(FUSE_WARPS * 32) rmsnorm_quantize_kernel(
+// RMSNorm + quantize.  One CTA per canvas row m in [0, Mp) with W = min(K/256, 32)
+// warps; warp w handles super-blocks w, w + W, ...  Pass 1 loads the warp's first
+// super-block of x and gamma into registers and sums the squares in fp64 (each lane in
+// element order, then a fixed reduction tree); pass 2 normalises and quantizes from the
+// registers, re-reading only super-blocks beyond the first (K > 8192).  Rows M..Mp-1
+// are written as zeros.
+constexpr int RMS_MAX_WARPS = 32;
+
+__global__ void __launch_bounds__(RMS_MAX_WARPS * 32) rmsnorm_quantize_kernel(
     const float* __restrict__ x, int64_t M, int64_t K, int64_t ldx, const float* __restrict__ gamma, float eps,
     int64_t Mp, int8_t* __restrict__ q, float* __restrict__ scale, uint8_t* __restrict__ sums) {
-    __shared__ double red[FUSE_WARPS];
+    __shared__ double red[RMS_MAX_WARPS];
     pdl_trigger();
-    pdl_wait();  // x may be the output of the previous kernel on the stream
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int W = blockDim.x >> 5;
     const int64_t m = blockIdx.x;
     const int64_t nsb = K / QK;
     const bool live = m < M;
     const float* xr = x + m * ldx;
+    float xv[8], gv[8];
+    pdl_wait();  // x may be the output of the previous kernel on the stream
+    load8(gamma + w * QK + 8 * lane, gv);
     double ss = 0.0;
     if (live) {
-#pragma unroll 2
-        for (int64_t s = w; s < nsb; s += FUSE_WARPS) {
+        load8(xr + w * QK + 8 * lane, xv);
+#pragma unroll
+        for (int i = 0; i < 8; i++) ss = __dadd_rn(ss, __dmul_rn((double)xv[i], (double)xv[i]));
+        for (int64_t s = w + W; s < nsb; s += W) {
             float v[8];
             load8(xr + s * QK + 8 * lane, v);
 #pragma unroll
@@ -99,22 +108,17 @@ __global__ void __launch_bounds__(FUSE_WARPS * 32) rmsnorm_quantize_kernel(
     if (lane == 0) red[w] = ss;
     __syncthreads();
     ss = red[0];
-#pragma unroll
-    for (int i = 1; i < FUSE_WARPS; i++) ss = __dadd_rn(ss, red[i]);
+    for (int i = 1; i < W; i++) ss = __dadd_rn(ss, red[i]);
     const double rn = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)eps)));
-    for (int64_t s = w; s < nsb; s += FUSE_WARPS) {
-        float v[8];
-        if (live) {
-            float xv[8], gv[8];
-            load8(xr + s * QK + 8 * lane, xv);
+    for (int64_t s = w; s < nsb; s += W) {
+        if (s != w) {
             load8(gamma + s * QK + 8 * lane, gv);
-#pragma unroll
-            for (int i = 0; i < 8; i++)
-                v[i] = __double2float_rn(__dmul_rn(__dmul_rn((double)xv[i], rn), (double)gv[i]));
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; i++) v[i] = 0.0f;
+            if (live) load8(xr + s * QK + 8 * lane, xv);
         }
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+            v[i] = live ? __double2float_rn(__dmul_rn(__dmul_rn((double)xv[i], rn), (double)gv[i])) : 0.0f;
         quantize_store_lane(v, lane, m, s, Mp, q, scale, sums);
     }
 }

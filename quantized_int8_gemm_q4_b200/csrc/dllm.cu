@@ -228,7 +228,8 @@ int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, con
     int dev;
     if ((rc = current_device(&dev))) return rc;
     const int64_t Mp = round_up(M, 16);
-    if (launch_pdl(rmsnorm_quantize_kernel, dim3((unsigned)Mp), dim3(FUSE_WARPS * 32), 0,
+    const int64_t warps = K / QK < RMS_MAX_WARPS ? K / QK : RMS_MAX_WARPS;
+    if (launch_pdl(rmsnorm_quantize_kernel, dim3((unsigned)Mp), dim3((unsigned)(warps * 32)), 0,
                    reinterpret_cast<cudaStream_t>(stream), x, M, K, ldx, gamma, eps, Mp, q, scale, sums) !=
         cudaSuccess) {
         (void)cudaGetLastError();

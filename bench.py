@@ -56,6 +56,8 @@ def parse():
     p.add_argument("--cpu-layers", type=int, default=16, help="layers in the oracle's timed sample")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--gather-last", action="store_true",
+                   help="the last layer's O and FFN, and the final norm, on the requested rows only")
     return p.parse_args()
 
 
@@ -79,14 +81,18 @@ class Gemm:
         return self.weight_bytes + self.M_act * self.K * per + self.M_out * self.N * 4
 
 
-def step_gemms(model, L, n_layers):
-    """The GEMM launches of one step, in order (QKV and gate/up are single launches)."""
-    h, f = model.hidden, model.ffn
-    per_layer = [Gemm("qkv", Q4, model.q_out + 2 * model.kv_out, h, L, L),
-                 Gemm("o", Q4, h, h, L, L),
-                 Gemm("gate_up", Q4, 2 * f, h, L, L),
-                 Gemm("down", Q6, h, f, L, L)]
-    return per_layer * n_layers + [Gemm("output", Q6, model.vocab, h, model.out_rows, model.out_rows)]
+def step_gemms(model, L, n_layers, gather_last=False):
+    """The GEMM launches of one step, in order (QKV and gate/up are single launches).
+    gather_last: past attention, the last layer runs on the requested rows only."""
+    h, f, R = model.hidden, model.ffn, min(L, model.out_rows)
+
+    def layer(m):
+        return [Gemm("qkv", Q4, model.q_out + 2 * model.kv_out, h, L, L),
+                Gemm("o", Q4, h, h, m, m),
+                Gemm("gate_up", Q4, 2 * f, h, m, m),
+                Gemm("down", Q6, h, f, m, m)]
+    last = layer(R if gather_last else L)
+    return layer(L) * (n_layers - 1) + last + [Gemm("output", Q6, model.vocab, h, R, R)]
 
 
 def roofline_time(gemms, hbm_gbs, p_int8):
@@ -179,13 +185,15 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def workload_config(model, L, n_layers, n_rows, world):
+def workload_config(model, L, n_layers, n_rows, world, gather_last=False):
     """The `config` object both arms report: the workload, not the implementation."""
-    gemms = step_gemms(model, L, n_layers)
+    gemms = step_gemms(model, L, n_layers, gather_last)
+    tail = (f"; past attention, the last layer and the final norm run on the {n_rows} requested rows only"
+            if gather_last else "")
     return {"workload": f"{model.name}-shaped denoising step: {n_layers} layers (RMSNorm+quantize -> QKV, "
                         f"quantize -> O, RMSNorm+quantize -> gate/up Q4_K, SwiGLU+quantize -> down Q6_K) + "
                         f"final RMSNorm+quantize -> output projection (Q6_K, {model.vocab} wide) on {n_rows} "
-                        f"requested rows",
+                        f"requested rows{tail}",
             "canvas_tokens": L, "layers": n_layers,
             "weight_bytes_per_step": int(sum(g.weight_bytes for g in gemms)),
             "l2": "inputs larger than L2: every step streams all weights from HBM",
@@ -277,12 +285,20 @@ def run_ours(args, rank, world):
                                                                                      dtype=np.int32)
     rows = torch.from_numpy(rows_np).to(dev)
     logits = torch.empty((len(rows_np), model.vocab), device=dev)
+    R = len(rows_np)
+    act_hr = dllm.alloc_act(R, h, dev)  # compact activations of the requested rows
+    act_fr = dllm.alloc_act(R, f, dev)
     # one zero-filled workspace, large enough for every GEMM of the step (stream-ordered)
     wsb = max(dllm.dllm_qgemm_workspace_bytes(Q4, model.q_out + 2 * model.kv_out, h, L),
               dllm.dllm_qgemm_workspace_bytes(Q4, h, h, L),
               dllm.dllm_qgemm_workspace_bytes(Q4, 2 * f, h, L),
               dllm.dllm_qgemm_workspace_bytes(Q6, h, f, L),
-              dllm.dllm_qgemm_workspace_bytes(Q6, model.vocab, h, L, len(rows_np)))
+              dllm.dllm_qgemm_workspace_bytes(Q6, model.vocab, h, L, len(rows_np)),
+              # the requested-rows shapes of --gather-last
+              dllm.dllm_qgemm_workspace_bytes(Q4, h, h, R),
+              dllm.dllm_qgemm_workspace_bytes(Q4, 2 * f, h, R),
+              dllm.dllm_qgemm_workspace_bytes(Q6, h, f, R),
+              dllm.dllm_qgemm_workspace_bytes(Q6, model.vocab, h, R))
     ws = dllm.alloc_workspace(max(wsb, 256), dev)
 
     def step(ev=None):
@@ -296,16 +312,33 @@ def run_ours(args, rank, world):
 
         for l in range(n_layers):
             W = layers[l]
-            dllm.dllm_rmsnorm_quantize(x_attn, L, h, h, gam[2 * l], eps, *act_h)
+            dllm.dllm_rmsnorm_quantize(x_attn, L, h, h, gam[2 * l], eps, None, 0, *act_h)
             mark()
             dllm.dllm_qkv_qgemm(W["q"], W["k"], W["v"], Q4, model.q_out, model.kv_out, h, *act_h, L,
                                 o_q, model.q_out, o_k, o_v, model.kv_out, ws, wsb)
             mark()
+            if args.gather_last and l == n_layers - 1:
+                # past attention only the requested positions continue: the attention output
+                # of those rows (compact), the FFN input gathered from the canvas by the norm
+                dllm.dllm_quantize_act(x_o, R, h, h, *act_hr)
+                mark()
+                dllm.dllm_qgemm(W["o"], Q4, h, h, *act_hr, R, None, 0, o_o, h, ws, wsb)
+                mark()
+                dllm.dllm_rmsnorm_quantize(x_ffn, L, h, h, gam[2 * l + 1], eps, rows, R, *act_hr)
+                mark()
+                dllm.dllm_qkv_qgemm(W["gate"], W["up"], None, Q4, f, f, h, *act_hr, R, o_g, f, o_u, None, f,
+                                    ws, wsb)
+                mark()
+                dllm.dllm_swiglu_quantize(o_g, o_u, R, f, f, *act_fr)
+                mark()
+                dllm.dllm_qgemm(W["down"], Q6, h, f, *act_fr, R, None, 0, o_d, h, ws, wsb)
+                mark()
+                continue
             dllm.dllm_quantize_act(x_o, L, h, h, *act_h)
             mark()
             dllm.dllm_qgemm(W["o"], Q4, h, h, *act_h, L, None, 0, o_o, h, ws, wsb)
             mark()
-            dllm.dllm_rmsnorm_quantize(x_ffn, L, h, h, gam[2 * l + 1], eps, *act_h)
+            dllm.dllm_rmsnorm_quantize(x_ffn, L, h, h, gam[2 * l + 1], eps, None, 0, *act_h)
             mark()
             dllm.dllm_qkv_qgemm(W["gate"], W["up"], None, Q4, f, f, h, *act_h, L, o_g, f, o_u, None, f, ws, wsb)
             mark()
@@ -313,13 +346,22 @@ def run_ours(args, rank, world):
             mark()
             dllm.dllm_qgemm(W["down"], Q6, h, f, *act_f, L, None, 0, o_d, h, ws, wsb)
             mark()
-        dllm.dllm_rmsnorm_quantize(x_fin, L, h, h, gam[2 * n_layers], eps, *act_h)
-        mark()
-        dllm.dllm_qgemm(w_out, Q6, model.vocab, h, *act_h, L, rows, len(rows_np), logits, model.vocab, ws, wsb)
-        mark()
+        if args.gather_last:
+            # the last layer's output exists for the requested rows only (compact)
+            dllm.dllm_rmsnorm_quantize(x_fin, R, h, h, gam[2 * n_layers], eps, None, 0, *act_hr)
+            mark()
+            dllm.dllm_qgemm(w_out, Q6, model.vocab, h, *act_hr, R, None, 0, logits, model.vocab, ws, wsb)
+            mark()
+        else:
+            dllm.dllm_rmsnorm_quantize(x_fin, L, h, h, gam[2 * n_layers], eps, None, 0, *act_h)
+            mark()
+            dllm.dllm_qgemm(w_out, Q6, model.vocab, h, *act_h, L, rows, len(rows_np), logits, model.vocab,
+                            ws, wsb)
+            mark()
 
-    launches_per_step = n_layers * 8 + 3  # + the row gather of the output projection
-    gemms = step_gemms(model, L, n_layers)
+    # + the row gather of the output projection, unless the final norm gathers the rows
+    launches_per_step = n_layers * 8 + (2 if args.gather_last else 3)
+    gemms = step_gemms(model, L, n_layers, args.gather_last)
 
     # eager warm-up of every kernel (attribute setup happens outside capture)
     step()
@@ -429,7 +471,7 @@ def run_ours(args, rank, world):
         e2e = {"value": ops_step / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": int(xin.numel() * 4), "d2h_bytes_per_step": int(logits.numel() * 4)}
 
-    traffic = stored_traffic(f"{args.model}_L{L}")
+    traffic = None if args.gather_last else stored_traffic(f"{args.model}_L{L}")
     roof = None
     if gemm_ms > 0:
         achieved = abytes_step / (gemm_ms * 1e-3) / 1e9
@@ -453,7 +495,7 @@ def run_ours(args, rank, world):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": dict(workload_config(model, L, n_layers, len(rows_np), world),
+        "config": dict(workload_config(model, L, n_layers, len(rows_np), world, args.gather_last),
                        graph=f"CUDA graphs of {S} steps, replayed; no events inside the timed region"),
         "weight_gbs": round(wbytes_step / (ms_step * 1e-3) / 1e9, 1),
         "step_roofline": {"t_star_ms": round(tstar * 1e3, 4), "frac": round(tstar * 1e3 / ms_step, 4),

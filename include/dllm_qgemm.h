@@ -130,7 +130,15 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  *
  * dllm_rmsnorm_quantize: x f32 [M][ldx] (ldx >= K, ldx % 4 == 0), gamma f32 [K],
  *   eps > 0 and finite (else DLLM_ERR_ARG; eps = 0 would make an all-zero row 0/0).
- *   One CTA per canvas row (M rounded up to 16 CTAs), min(K/256, 32) warps.
+ *   rows == NULL (n_rows = 0): all M canvas rows; the output has M rows.
+ *   rows != NULL: device int32 list of n_rows >= 1 canvas rows (any order, duplicates
+ *   allowed); output row i is canvas row rows[i] and the output has n_rows rows
+ *   (size it with dllm_act_bytes(n_rows, K)).  This is the final RMSNorm on the
+ *   requested rows only (Architecture page, "A forward pass", step 4), and the FFN
+ *   input of the last layer, where only the requested positions continue past attention
+ *   (step 3).  An entry outside [0, M) zero-fills its output row and sets
+ *   DLLM_ERR_ROW_RANGE in the device error word.
+ *   One CTA per output row (rounded up to 16 CTAs), min(K/256, 32) warps.
  * dllm_swiglu_quantize: gate, up f32 [M][ld] each (ld >= K, ld % 4 == 0).  They may
  *   be two column ranges of one buffer, e.g. the out_q/out_k pair of dllm_qkv_qgemm
  *   run on the gate and up weights with ld = 2 * K and up = gate + K.
@@ -140,7 +148,8 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  * of 4), DLLM_ERR_UNSUPPORTED, DLLM_ERR_CUDA.
  * ---------------------------------------------------------------------------- */
 int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, const float* gamma, float eps,
-                          int8_t* q, float* scale, uint8_t* sums, dllm_stream_t stream);
+                          const int32_t* rows, int64_t n_rows, int8_t* q, float* scale, uint8_t* sums,
+                          dllm_stream_t stream);
 int dllm_swiglu_quantize(const float* gate, const float* up, int64_t M, int64_t K, int64_t ld, int8_t* q,
                          float* scale, uint8_t* sums, dllm_stream_t stream);
 

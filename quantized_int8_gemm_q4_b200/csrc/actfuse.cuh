@@ -69,27 +69,39 @@ __device__ __forceinline__ void load8(const float* __restrict__ p, float (&v)[8]
 
 constexpr int FUSE_WARPS = 8;
 
-// RMSNorm + quantize.  One CTA per canvas row m in [0, Mp) with W = min(K/256, 32)
-// warps; warp w handles super-blocks w, w + W, ...  Pass 1 loads the warp's first
-// super-block of x and gamma into registers and sums the squares in fp64 (each lane in
-// element order, then a fixed reduction tree); pass 2 normalises and quantizes from the
-// registers, re-reading only super-blocks beyond the first (K > 8192).  Rows M..Mp-1
-// are written as zeros.
+// RMSNorm + quantize.  One CTA per output row m in [0, Mp) with W = min(K/256, 32)
+// warps; warp w handles super-blocks w, w + W, ...  Output row m reads canvas row
+// rows[m] when a row list is given (M is then the list's length and M_src the canvas
+// height), else canvas row m.  Pass 1 loads the warp's first super-block of x and gamma
+// into registers and sums the squares in fp64 (each lane in element order, then a
+// fixed reduction tree); pass 2 normalises and quantizes from the registers,
+// re-reading only super-blocks beyond the first (K > 8192).  Rows M..Mp-1, and rows
+// whose list entry is outside [0, M_src), are written as zeros; the latter also set
+// ERR_ROW_RANGE.
 constexpr int RMS_MAX_WARPS = 32;
 
 __global__ void __launch_bounds__(RMS_MAX_WARPS * 32) rmsnorm_quantize_kernel(
     const float* __restrict__ x, int64_t M, int64_t K, int64_t ldx, const float* __restrict__ gamma, float eps,
-    int64_t Mp, int8_t* __restrict__ q, float* __restrict__ scale, uint8_t* __restrict__ sums) {
+    const int32_t* __restrict__ rows, int64_t M_src, int64_t Mp, int8_t* __restrict__ q, float* __restrict__ scale,
+    uint8_t* __restrict__ sums) {
     __shared__ double red[RMS_MAX_WARPS];
     pdl_trigger();
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int W = blockDim.x >> 5;
     const int64_t m = blockIdx.x;
     const int64_t nsb = K / QK;
-    const bool live = m < M;
-    const float* xr = x + m * ldx;
     float xv[8], gv[8];
-    pdl_wait();  // x may be the output of the previous kernel on the stream
+    pdl_wait();  // x and rows may be outputs of the previous kernel on the stream
+    int64_t src = m;
+    if (rows != nullptr && m < M) {
+        src = rows[m];
+        if (src < 0 || src >= M_src) {
+            if (threadIdx.x == 0) set_err(ERR_ROW_RANGE);
+            src = -1;
+        }
+    }
+    const bool live = m < M && src >= 0;
+    const float* xr = x + (live ? src : 0) * ldx;
     load8(gamma + w * QK + 8 * lane, gv);
     double ss = 0.0;
     if (live) {

@@ -217,21 +217,24 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
     return launch_status();
 }
 
-int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, const float* gamma, float eps, int8_t* q,
-                          float* scale, uint8_t* sums, dllm_stream_t stream) {
+int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, const float* gamma, float eps,
+                          const int32_t* rows, int64_t n_rows, int8_t* q, float* scale, uint8_t* sums,
+                          dllm_stream_t stream) {
     if (!x || !gamma || M <= 0 || K <= 0 || K % QK || ldx < K) return DLLM_ERR_ARG;
     if (!(eps > 0.0f) || !(eps < INFINITY)) return DLLM_ERR_ARG;
-    int rc = check_act(q, scale, sums, M);
+    if (rows ? n_rows <= 0 : n_rows != 0) return DLLM_ERR_ARG;
+    const int64_t M_out = rows ? n_rows : M;
+    int rc = check_act(q, scale, sums, M_out);
     if (rc) return rc;
     if (!aligned16(x) || !aligned16(gamma) || ldx % 4) return DLLM_ERR_ALIGN;
-    if (M > (1LL << 31) - 16) return DLLM_ERR_ARG;
+    if (M_out > (1LL << 31) - 16) return DLLM_ERR_ARG;
     int dev;
     if ((rc = current_device(&dev))) return rc;
-    const int64_t Mp = round_up(M, 16);
+    const int64_t Mp = round_up(M_out, 16);
     const int64_t warps = K / QK < RMS_MAX_WARPS ? K / QK : RMS_MAX_WARPS;
     if (launch_pdl(rmsnorm_quantize_kernel, dim3((unsigned)Mp), dim3((unsigned)(warps * 32)), 0,
-                   reinterpret_cast<cudaStream_t>(stream), x, M, K, ldx, gamma, eps, Mp, q, scale, sums) !=
-        cudaSuccess) {
+                   reinterpret_cast<cudaStream_t>(stream), x, M_out, K, ldx, gamma, eps, rows, M, Mp, q, scale,
+                   sums) != cudaSuccess) {
         (void)cudaGetLastError();
         return DLLM_ERR_CUDA;
     }

@@ -63,7 +63,7 @@ def load() -> ctypes.CDLL:
         "dllm_repack_q6k": [P, I64, I64, P, P],
         "dllm_act_bytes": [I64, I64, PSZ, PSZ, PSZ],
         "dllm_quantize_act": [P, I64, I64, I64, P, P, P, P],
-        "dllm_rmsnorm_quantize": [P, I64, I64, I64, P, ctypes.c_float, P, P, P, P],
+        "dllm_rmsnorm_quantize": [P, I64, I64, I64, P, ctypes.c_float, P, I64, P, P, P, P],
         "dllm_swiglu_quantize": [P, P, I64, I64, I64, P, P, P, P],
         "dllm_qgemm_workspace_bytes": [I, I64, I64, I64, I64, PSZ],
         "dllm_qgemm": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P, SZ, P],
@@ -138,9 +138,10 @@ def dllm_quantize_act(x, M: int, K: int, ldx: int, q, scale, sums, stream=None):
            "dllm_quantize_act")
 
 
-def dllm_rmsnorm_quantize(x, M: int, K: int, ldx: int, gamma, eps: float, q, scale, sums, stream=None):
-    _check(load().dllm_rmsnorm_quantize(_ptr(x), M, K, ldx, _ptr(gamma), float(eps), _ptr(q), _ptr(scale),
-                                        _ptr(sums), _stream(stream)), "dllm_rmsnorm_quantize")
+def dllm_rmsnorm_quantize(x, M: int, K: int, ldx: int, gamma, eps: float, rows, n_rows: int, q, scale, sums,
+                          stream=None):
+    _check(load().dllm_rmsnorm_quantize(_ptr(x), M, K, ldx, _ptr(gamma), float(eps), _ptr(rows), n_rows, _ptr(q),
+                                        _ptr(scale), _ptr(sums), _stream(stream)), "dllm_rmsnorm_quantize")
 
 
 def dllm_swiglu_quantize(gate, up, M: int, K: int, ld: int, q, scale, sums, stream=None):

@@ -106,11 +106,11 @@ def test_quantize_argument_checks(lib):
 def test_fused_quantize_argument_checks(lib):
     A = 0x10000
     f = lib.dllm_rmsnorm_quantize
-    ok = (_fake(A), 4, 256, 256, _fake(A), 1e-5, _fake(A), _fake(A), _fake(A), None)
+    ok = (_fake(A), 4, 256, 256, _fake(A), 1e-5, None, 0, _fake(A), _fake(A), _fake(A), None)
 
     def rms(**kw):
         a = list(ok)
-        for i, k in enumerate(("x", "M", "K", "ldx", "gamma", "eps", "q", "scale", "sums")):
+        for i, k in enumerate(("x", "M", "K", "ldx", "gamma", "eps", "rows", "n_rows", "q", "scale", "sums")):
             if k in kw:
                 a[i] = kw[k]
         return f(*a)
@@ -127,6 +127,9 @@ def test_fused_quantize_argument_checks(lib):
     assert rms(gamma=_fake(A + 8)) == dllm.DLLM_ERR_ALIGN
     assert rms(ldx=258) == dllm.DLLM_ERR_ALIGN
     assert rms(q=_fake(A + 1)) == dllm.DLLM_ERR_ALIGN
+    assert rms(rows=_fake(A), n_rows=0) == dllm.DLLM_ERR_ARG      # a row list needs n_rows >= 1
+    assert rms(rows=_fake(A), n_rows=-3) == dllm.DLLM_ERR_ARG
+    assert rms(rows=None, n_rows=5) == dllm.DLLM_ERR_ARG          # n_rows without a list
     g = lib.dllm_swiglu_quantize
     assert g(None, _fake(A), 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
     assert g(_fake(A), None, 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG

@@ -52,3 +52,21 @@ def test_step_roofline_matches_the_stated_target():
     assert abs(t * 1e3 - 0.8618) < 5e-4
     ops = sum(g.ops for g in gemms)
     assert abs(ops / 1e12 - 1.82) < 0.01  # 1.82 T int8 ops per step at canvas 128
+
+
+def test_gather_last_step_shapes():
+    """--gather-last: past attention the last layer runs on the requested rows only."""
+    model = synth.MODELS["llada-8b"]()
+    full = bench.step_gemms(model, 128, model.n_layers)
+    g = bench.step_gemms(model, 128, model.n_layers, gather_last=True)
+    assert [x.name for x in g] == [x.name for x in full]
+    last = g[-5:-1]
+    assert [x.M_out for x in last] == [128, 32, 32, 32]       # QKV still on the canvas
+    assert all(a.M_out == b.M_out for a, b in zip(g[:-5], full[:-5]))
+    h, f = model.hidden, model.ffn
+    saved = 2 * (128 - 32) * (h * h + 2 * f * h + h * f)
+    assert sum(x.ops for x in full) - sum(x.ops for x in g) == saved
+    assert sum(x.weight_bytes for x in g) == sum(x.weight_bytes for x in full)
+    cfg = bench.workload_config(model, 128, model.n_layers, 32, 1, gather_last=True)
+    assert "requested rows only" in cfg["workload"]
+    assert "requested rows only" not in bench.workload_config(model, 128, model.n_layers, 32, 1)["workload"]

@@ -118,7 +118,7 @@ def _run_rms(x, gamma, eps, ldx=None):
     q, s, u = dllm.alloc_act(M, K)
     q.fill_(0x55)
     s.fill_(float("nan"))
-    dllm.dllm_rmsnorm_quantize(xd, M, K, ldx, gd, eps, q, s, u)
+    dllm.dllm_rmsnorm_quantize(xd, M, K, ldx, gd, eps, None, 0, q, s, u)
     return q, s, u
 
 
@@ -219,7 +219,7 @@ def test_chain_rmsnorm_qkv_and_gateup_swiglu_down():
     ws_b = max(dllm.dllm_qgemm_workspace_bytes(Q4, 2 * f, h, M), dllm.dllm_qgemm_workspace_bytes(Q6, h, f, M))
     ws = dllm.alloc_workspace(max(ws_b, 256))
     # the whole chain back to back on one stream (programmatic dependent launches)
-    dllm.dllm_rmsnorm_quantize(xd, M, h, h, gd, 1e-5, qh, sh, uh)
+    dllm.dllm_rmsnorm_quantize(xd, M, h, h, gd, 1e-5, None, 0, qh, sh, uh)
     dllm.dllm_qkv_qgemm(dg, du, None, Q4, f, f, h, qh, sh, uh, M, o_gu, 2 * f, o_gu[:, f:], None, 2 * f, ws, ws_b)
     dllm.dllm_swiglu_quantize(o_gu, o_gu[:, f:], M, f, 2 * f, qf, sf, uf)
     dllm.dllm_qgemm(dd, Q6, h, f, qf, sf, uf, M, None, 0, o_d, h, ws, ws_b)
@@ -241,23 +241,83 @@ def test_chain_rmsnorm_qkv_and_gateup_swiglu_down():
     assert ok, worst
 
 
+def _run_rms_rows(x, gamma, eps, rows):
+    M, K = x.shape
+    xd = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    gd = torch.from_numpy(gamma).cuda()
+    r = torch.from_numpy(np.asarray(rows, np.int32)).cuda()
+    n = len(rows)
+    q, s, u = dllm.alloc_act(n, K)
+    q.fill_(0x55)
+    s.fill_(float("nan"))
+    dllm.dllm_rmsnorm_quantize(xd, M, K, K, gd, eps, r, n, q, s, u)
+    return q, s, u
+
+
+def test_rmsnorm_quantize_rows():
+    """A row list: output row i is canvas row rows[i] (any order, duplicates), equal bit for
+    bit to that row of the full-canvas result."""
+    M, K = 160, 4096
+    x = _rms_rows(M, K, 47)
+    gamma = _gamma(K, 11)
+    rows = np.concatenate([synth.block_rows(M, 32, 48), [0, M - 1, 5, 5, 37]]).astype(np.int32)
+    n = len(rows)
+    q, s, u = _run_rms_rows(x, gamma, 1e-5, rows)
+    xr = np.ascontiguousarray(x[rows])
+    got = _host(q, s, u, n, K)
+    _compare(got, *_rms_bracket(xr, gamma, 1e-5), n, K)
+    full = _host(*_run_rms(x, gamma, 1e-5), M, K)
+    assert np.array_equal(got[0], full[0][rows])
+    assert np.array_equal(got[1].view(np.uint32), full[1][rows].view(np.uint32))
+    Mp = (n + 15) // 16 * 16
+    qa = q.cpu().numpy().reshape(K // 256, Mp // 8, 16, 8, 16).transpose(1, 3, 0, 2, 4).reshape(Mp, K)
+    assert not qa[n:].any()
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+
+def test_rmsnorm_quantize_row_out_of_range():
+    """An entry outside [0, M) zero-fills its output row and reports DLLM_ERR_ROW_RANGE;
+    the other rows are unaffected."""
+    M, K = 64, 1024
+    x = _rms_rows(M, K, 49)
+    gamma = _gamma(K, 12)
+    rows = np.array([3, M, 10, -1, 63], np.int32)
+    q, s, u = _run_rms_rows(x, gamma, 1e-5, rows)
+    assert dllm.dllm_get_device_status() == dllm.DLLM_ERR_ROW_RANGE
+    gq, gs, (hi, lo) = _host(q, s, u, len(rows), K)
+    for i in (1, 3):
+        assert not gq[i].any() and not gs[i].any() and not hi[i].any() and not lo[i].any()
+    ok = np.array([0, 2, 4])
+    xr = np.ascontiguousarray(x[rows[ok]])
+    sub = (gq[ok], gs[ok], (hi[ok], lo[ok]))
+    _compare(sub, *_rms_bracket(xr, gamma, 1e-5), len(ok), K)
+
+
 def test_final_rmsnorm_output_rows():
-    """Final RMSNorm -> quantize over the canvas, then the output projection on 32
-    requested rows only."""
+    """Final RMSNorm -> quantize on the 32 requested rows only (a compact activation),
+    then the output projection on that activation, with no row list."""
     M, h, V = 96, 1024, 2048
     x = _rms_rows(M, h, 45)
     gamma = _gamma(h, 10)
     w = synth.weights(Q6, V, h, 54)
     wd = dllm.repack(Q6, w, V, h)
-    q, s, u = _run_rms(x, gamma, 1e-6)
     rows = synth.block_rows(M, 32, 46)
-    r = torch.from_numpy(rows).cuda()
+    q, s, u = _run_rms_rows(x, gamma, 1e-6, rows)
     out = torch.empty((32, V), device="cuda")
-    wsb = dllm.dllm_qgemm_workspace_bytes(Q6, V, h, M, 32)
+    wsb = dllm.dllm_qgemm_workspace_bytes(Q6, V, h, 32)
     ws = dllm.alloc_workspace(max(wsb, 256))
-    dllm.dllm_qgemm(wd, Q6, V, h, q, s, u, M, r, 32, out, V, ws, wsb)
-    _compare(_host(q, s, u, M, h), *_rms_bracket(x, gamma, 1e-6), M, h)
-    oq, os_, _ = oracle.rmsnorm_quantize(x, gamma, 1e-6)
-    _, ref, T = oracle.qgemm(Q6, w, V, h, oq, os_, rows=rows)
+    dllm.dllm_qgemm(wd, Q6, V, h, q, s, u, 32, None, 0, out, V, ws, wsb)
+    xr = np.ascontiguousarray(x[rows])
+    _compare(_host(q, s, u, 32, h), *_rms_bracket(xr, gamma, 1e-6), 32, h)
+    oq, os_, _ = oracle.rmsnorm_quantize(xr, gamma, 1e-6)
+    _, ref, T = oracle.qgemm(Q6, w, V, h, oq, os_)
     ok, worst = gu.tol_ok(out.cpu().numpy(), ref, T)
     assert ok, worst
+    # the same logits as normalising the whole canvas and gathering rows in the GEMM
+    qa, sa, ua = _run_rms(x, gamma, 1e-6)
+    r = torch.from_numpy(rows).cuda()
+    out2 = torch.empty((32, V), device="cuda")
+    wsb2 = dllm.dllm_qgemm_workspace_bytes(Q6, V, h, M, 32)
+    ws2 = dllm.alloc_workspace(max(wsb2, 256))
+    dllm.dllm_qgemm(wd, Q6, V, h, qa, sa, ua, M, r, 32, out2, V, ws2, wsb2)
+    assert torch.equal(out, out2)

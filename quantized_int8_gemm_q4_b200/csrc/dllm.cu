@@ -14,7 +14,7 @@ namespace {
 constexpr int MAX_DEV = 64;
 int g_dev_checked[MAX_DEV];  // 0 unknown, 1 sm_100, -1 other
 int g_num_sms[MAX_DEV];
-bool g_attr_done[MAX_DEV][4];
+bool g_attr_done[MAX_DEV][8];
 
 int current_device(int* dev) {
     if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= MAX_DEV) return DLLM_ERR_CUDA;
@@ -84,9 +84,32 @@ int choose_kc(int64_t n_tiles, int64_t nsb, int sms) {
 
 struct Plan {
     int kc, n_st, mu;
+    int full_tiles, tail_k, tail_big;  // tail split (tail_k > 0), see GemmArgs
+    bool split;        // some tile's K range is cut: counters and partials in use
+    int64_t n_units;
     int64_t Mp;        // activation rows seen by the GEMM
     size_t ctr_off, part_off, gq_off, gs_off, gu_off, bytes;
 };
+
+int64_t uniform_cost(int64_t n_tiles, int64_t nsb, int kc, int sms) {
+    const int64_t len = (nsb + kc - 1) / kc;
+    return (n_tiles * kc + sms - 1) / sms * (100 * len + 235 + (kc > 1 ? 270 : 0));
+}
+
+// Tail split, in the cost units of choose_kc: every CTA runs full_tiles / SMs whole
+// tiles, then one piece of a tail tile.  Applies when the tiles left after the whole
+// rounds can each be cut into 2..15 pieces of at least 4 super-blocks that number
+// exactly one per SM.  Returns the cost, or -1 when it does not apply.
+int64_t tail_plan(int64_t n_tiles, int64_t nsb, int sms, int* full_tiles, int* tail_k, int* tail_big) {
+    const int64_t rounds = n_tiles / sms, n_tail = n_tiles - rounds * sms;
+    if (n_tail == 0) return -1;
+    const int64_t k = sms / n_tail, big = sms - k * n_tail;
+    if (k < 2 || k + (big > 0) > 15 || nsb / (k + (big > 0)) < 4) return -1;
+    *full_tiles = (int)(rounds * sms);
+    *tail_k = (int)k;
+    *tail_big = (int)big;
+    return rounds * (100 * nsb + 235) + 100 * ((nsb + k - 1) / k) + 235 + 270;
+}
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -95,13 +118,23 @@ Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
     const int64_t nsb = K / QK;
     p.Mp = round_up(n_rows > 0 ? n_rows : M, 16);
     p.kc = choose_kc(n_tiles, nsb, sms);
+    p.full_tiles = p.tail_k = p.tail_big = 0;
+    const int64_t tail_cost = tail_plan(n_tiles, nsb, sms, &p.full_tiles, &p.tail_k, &p.tail_big);
+    const int64_t tail_units = (n_tiles / sms + 1) * sms * ((p.Mp + UNIT_TOKENS - 1) / UNIT_TOKENS);
+    if (tail_cost < 0 || tail_cost >= uniform_cost(n_tiles, nsb, p.kc, sms) || tail_units >= (1LL << 31) ||
+        nsb * 16 >= (1LL << 31))
+        p.full_tiles = p.tail_k = p.tail_big = 0;
+    if (p.tail_k > 0) p.kc = 1;
+    p.split = p.kc > 1 || p.tail_k > 0;
     p.n_st = (int)((p.Mp + UNIT_TOKENS - 1) / UNIT_TOKENS);
     p.mu = (int)round_up((p.Mp + p.n_st - 1) / p.n_st, 16);
+    p.n_units = p.tail_k > 0 ? (int64_t)(p.full_tiles + sms) * p.n_st : n_tiles * p.n_st * p.kc;
     size_t off = 0;
     p.ctr_off = off;
     off += align256((size_t)n_tiles * p.n_st * 4);
     p.part_off = off;
     if (p.kc > 1) off += align256((size_t)n_tiles * p.n_st * p.kc * p.mu * TROWS * 4);
+    if (p.tail_k > 0) off += align256((size_t)sms * p.n_st * p.mu * TROWS * 4);
     p.gq_off = p.gs_off = p.gu_off = off;
     if (n_rows > 0) {
         p.gq_off = off;
@@ -111,26 +144,26 @@ Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
         p.gu_off = off;
         off += align256((size_t)nsb * p.Mp * 64);
     }
-    p.bytes = (p.kc > 1 || n_rows > 0) ? off : 0;
+    p.bytes = (p.split || n_rows > 0) ? off : 0;
     return p;
 }
 
-template <int QT, bool DBG>
+template <int QT, bool DBG, bool TAIL>
 int run_gemm(GemmArgs& a, cudaStream_t s) {
     int dev;
     int rc = current_device(&dev);
     if (rc) return rc;
     constexpr size_t smem = gemm_smem_bytes<QT>();
-    const int slot = (QT == 12 ? 0 : 2) + (DBG ? 1 : 0);
+    const int slot = (QT == 12 ? 0 : 4) + (DBG ? 2 : 0) + (TAIL ? 1 : 0);
     if (!g_attr_done[dev][slot]) {
-        if (cudaFuncSetAttribute(qgemm_kernel<QT, DBG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        if (cudaFuncSetAttribute(qgemm_kernel<QT, DBG, TAIL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return DLLM_ERR_CUDA;
         g_attr_done[dev][slot] = true;
     }
-    const int64_t units = (int64_t)a.n_tiles * a.n_st * a.kc;
+    const int64_t units = a.n_units;
     const int grid = (int)(units < g_num_sms[dev] ? units : g_num_sms[dev]);
-    if (launch_pdl(qgemm_kernel<QT, DBG>, dim3(grid), dim3(GEMM_THREADS), smem, s, a) != cudaSuccess) {
+    if (launch_pdl(qgemm_kernel<QT, DBG, TAIL>, dim3(grid), dim3(GEMM_THREADS), smem, s, a) != cudaSuccess) {
         (void)cudaGetLastError();
         return DLLM_ERR_CUDA;
     }
@@ -287,6 +320,9 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
     Plan p = make_plan(N_total / TROWS, K, M, rows ? n_rows : 0, g_num_sms[dev]);
     if (dbg) {  // integers per super-block: no chunk partials to combine
         p.kc = 1;
+        p.full_tiles = p.tail_k = p.tail_big = 0;
+        p.split = false;
+        p.n_units = (N_total / TROWS) * p.n_st;
         if (!rows) p.bytes = 0;
     }
     if (p.bytes > 0 && (!workspace || workspace_bytes < p.bytes)) return DLLM_ERR_WORKSPACE;
@@ -294,6 +330,10 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
     const int64_t nsb = K / QK;
     a.nsb = (int32_t)nsb;
     a.kc = p.kc;
+    a.full_tiles = p.full_tiles;
+    a.tail_k = p.tail_k;
+    a.tail_big = p.tail_big;
+    a.n_units = p.n_units;
     a.n_st = p.n_st;
     a.mu = p.mu;
     a.Mp = p.Mp;
@@ -302,7 +342,7 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
     a.scale = scale;
     a.sums = sums;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if (p.kc > 1) {
+    if (p.split) {
         a.counters = reinterpret_cast<uint32_t*>(ws + p.ctr_off);
         a.partials = reinterpret_cast<float*>(ws + p.part_off);
     }
@@ -325,8 +365,13 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
 }
 
 static int dispatch(GemmArgs& a, dllm_qtype t, bool dbg, cudaStream_t s) {
-    if (t == DLLM_Q4_K) return dbg ? run_gemm<12, true>(a, s) : run_gemm<12, false>(a, s);
-    return dbg ? run_gemm<14, true>(a, s) : run_gemm<14, false>(a, s);
+    // the debug integers never split K (uniform plan, one chunk)
+    if (t == DLLM_Q4_K) {
+        if (dbg) return run_gemm<12, true, false>(a, s);
+        return a.tail_k > 0 ? run_gemm<12, false, true>(a, s) : run_gemm<12, false, false>(a, s);
+    }
+    if (dbg) return run_gemm<14, true, false>(a, s);
+    return a.tail_k > 0 ? run_gemm<14, false, true>(a, s) : run_gemm<14, false, false>(a, s);
 }
 
 int dllm_qgemm(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* q, const float* scale,
@@ -418,7 +463,7 @@ int dllm_qgemm_noalloc(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
     if (p.bytes > DLLM_NOALLOC_SCRATCH_BYTES) return DLLM_ERR_SCRATCH_LIMIT;
     uint8_t* scratch;
     if ((rc = noalloc_scratch(dev, &scratch))) return rc;
-    if (p.kc > 1) {
+    if (p.split) {
         const size_t ctr_bytes = (size_t)(N / TROWS) * p.n_st * 4;
         if (cudaMemsetAsync(scratch + p.ctr_off, 0, ctr_bytes, reinterpret_cast<cudaStream_t>(stream)) !=
             cudaSuccess)
@@ -607,12 +652,13 @@ int dllm_debug_bounded_wait(dllm_stream_t stream) {
     a.n_tiles = 1;
     a.nsb = 1;
     a.kc = 1;
+    a.n_units = 1;
     a.Mp = 16;
     a.m_out = 16;
     a.n_st = 1;
     a.mu = 16;
     a.stall = 1;
-    return run_gemm<12, false>(a, reinterpret_cast<cudaStream_t>(stream));
+    return run_gemm<12, false, false>(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int issuers, int iters, int ctas,

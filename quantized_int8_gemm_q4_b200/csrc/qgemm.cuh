@@ -123,7 +123,13 @@ struct GemmArgs {
     int nseg;
     int32_t n_tiles;   // total 128-row tiles over all segments
     int32_t nsb;       // K / 256
-    int32_t kc;        // K-chunks per tile
+    int32_t kc;        // K-chunks per tile (uniform split: tail_k == 0)
+    // Tail split (tail_k > 0): tiles [0, full_tiles) run whole, one round of one tile per
+    // CTA at a time; each remaining tile is cut into K-pieces so that the pieces fill
+    // exactly one more unit per CTA: the first tail_big of them into tail_k + 1 pieces,
+    // the others into tail_k.
+    int32_t full_tiles, tail_k, tail_big;
+    int64_t n_units;   // work units of the launch (token super-tiles included)
     const int8_t* q;   // tiled activations
     const float* scale;
     const uint8_t* sums;
@@ -200,26 +206,59 @@ struct Unit {
     int64_t tile;   // tile index inside the segment
     int32_t gtile;  // global tile index
     int32_t st;     // token super-tile
-    int32_t chunk;  // K-chunk
+    int32_t chunk;  // K-piece of the tile
     int64_t m0;     // first token of the super-tile
     int32_t len;    // tokens in the super-tile (multiple of 16)
     int32_t sb0, sb1;
+    int32_t np;        // K-pieces of the tile (1: the unit writes the output itself)
+    int64_t slot0;     // partial-sum slot of the tile's piece 0 (same super-tile)
+    int32_t pstride;   // slot distance between consecutive pieces
 };
 
+template <bool TAIL>
 __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int64_t u) {
     Unit r;
-    r.chunk = (int32_t)(u % a.kc);
-    const int64_t ts = u / a.kc;
-    r.st = (int32_t)(ts % a.n_st);
-    r.gtile = (int32_t)(ts / a.n_st);
+    if constexpr (!TAIL) {
+        r.chunk = (int32_t)(u % a.kc);
+        const int64_t ts = u / a.kc;
+        r.st = (int32_t)(ts % a.n_st);
+        r.gtile = (int32_t)(ts / a.n_st);
+        r.sb0 = (int32_t)((int64_t)r.chunk * a.nsb / a.kc);
+        r.sb1 = (int32_t)((int64_t)(r.chunk + 1) * a.nsb / a.kc);
+        r.np = a.kc;
+        r.slot0 = u - r.chunk;  // partial slots are unit indices
+        r.pstride = 1;
+    } else {
+        // unit u = (tile piece cu, super-tile st), st fastest; partial slots count the
+        // tail units only.  32-bit arithmetic: the host keeps n_units below 2^31 here.
+        const uint32_t uu = (uint32_t)u, nst = (uint32_t)a.n_st;
+        const uint32_t cu = uu / nst;
+        r.st = (int32_t)(uu - cu * nst);
+        if (cu < (uint32_t)a.full_tiles) {
+            r.gtile = (int32_t)cu;
+            r.chunk = 0;
+            r.np = 1;
+        } else {
+            const uint32_t i = cu - (uint32_t)a.full_tiles;
+            const uint32_t big = (uint32_t)a.tail_big * (uint32_t)(a.tail_k + 1);
+            const uint32_t np = i < big ? (uint32_t)a.tail_k + 1 : (uint32_t)a.tail_k;
+            const uint32_t i2 = i < big ? i : i - big;
+            const uint32_t j = i2 / np;
+            r.np = (int32_t)np;
+            r.chunk = (int32_t)(i2 - j * np);
+            r.gtile = a.full_tiles + (int32_t)(i < big ? j : (uint32_t)a.tail_big + j);
+        }
+        r.sb0 = (int32_t)((uint32_t)r.chunk * (uint32_t)a.nsb / (uint32_t)r.np);
+        r.sb1 = (int32_t)((uint32_t)(r.chunk + 1) * (uint32_t)a.nsb / (uint32_t)r.np);
+        r.slot0 = (int64_t)((cu - (uint32_t)r.chunk - (uint32_t)a.full_tiles) * nst + (uint32_t)r.st);
+        r.pstride = a.n_st;
+    }
     r.seg = 0;
     if (a.nseg > 1 && r.gtile >= a.seg[1].tile0) r.seg = 1;
     if (a.nseg > 2 && r.gtile >= a.seg[2].tile0) r.seg = 2;
     r.tile = r.gtile - a.seg[r.seg].tile0;
     r.m0 = (int64_t)r.st * a.mu;
     r.len = (int32_t)min((int64_t)a.mu, a.Mp - r.m0);
-    r.sb0 = (int32_t)((int64_t)r.chunk * a.nsb / a.kc);
-    r.sb1 = (int32_t)((int64_t)(r.chunk + 1) * a.nsb / a.kc);
     return r;
 }
 
@@ -231,7 +270,7 @@ constexpr bool tmem_fits() {
 }
 static_assert(tmem_fits<12>() && tmem_fits<14>(), "tensor-memory columns over budget");
 
-template <int QT, bool DBG>
+template <int QT, bool DBG, bool TAIL>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<QT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -241,7 +280,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     GemmShared& sh = *reinterpret_cast<GemmShared*>(mina + C::MINA);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n_units = (int64_t)args.n_tiles * args.n_st * args.kc;
+    const int64_t n_units = args.n_units;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 128); }
@@ -279,14 +318,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             const uint64_t pol_a = policy_evict_last();
             const int64_t n_prod = args.stall ? 0 : n_units;
             if (lane == 0 && blockIdx.x < n_prod) {
-                const Unit un = unit_of(args, blockIdx.x);
+                const Unit un = unit_of<TAIL>(args, blockIdx.x);
                 const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
                 for (int s = un.sb0; s < un.sb1 && s < un.sb0 + C::W_STAGES; s++)
                     prefetch_l2(wt + (size_t)s * C::TILE, C::TILE);
             }
             pdl_wait();
             for (int64_t u = blockIdx.x; u < n_prod; u += gridDim.x) {
-                const Unit un = unit_of(args, u);
+                const Unit un = unit_of<TAIL>(args, u);
                 const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
                 const int T = (un.len + NTOK - 1) / NTOK;
                 for (int s = un.sb0; s < un.sb1; s++) {
@@ -342,7 +381,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             if (who < ISSUERS) {
                 uint32_t item = 0, sbc = 0, uc = 0;
                 for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
-                    const Unit un = unit_of(args, u);
+                    const Unit un = unit_of<TAIL>(args, u);
                     const int T = (un.len + NTOK - 1) / NTOK;
                     for (int s = un.sb0; s < un.sb1; s++, sbc++, item += T) {
 #pragma unroll 1
@@ -414,7 +453,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         uint32_t ws = 0, wph = 0, ss = 0, sph = 0, sbc = 0, itm = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const Unit un = unit_of(args, u);
+            const Unit un = unit_of<TAIL>(args, u);
             const int T = (un.len + NTOK - 1) / NTOK;
             for (int s = un.sb0; s < un.sb1; s++, sbc++, itm += T) {
                 if (!wait_bar_warp(sh, &sh.w_full[ws], wph)) goto unpack_done;
@@ -558,7 +597,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         const float2 m257 = make_float2(-257.0f * MAGIC, -257.0f * MAGIC);
         uint32_t bs = 0, bph = 0, r = 0, rph = 0, ss = 0, sph = 0, epi_ph = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const Unit un = unit_of(args, u);
+            const Unit un = unit_of<TAIL>(args, u);
             const int T = (un.len + NTOK - 1) / NTOK;
             const Segment& sg = args.seg[un.seg];
             float2 acc[TMAX][HC / 2];
@@ -644,7 +683,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             }
             if constexpr (!DBG) {
                 const int64_t n = un.tile * TROWS + row;
-                if (args.kc == 1) {
+                // uniform split: every tile has kc pieces and partial slots are unit indices
+                const int np = TAIL ? un.np : args.kc;
+                if (np == 1) {
                     float* out = sg.out;
 #pragma unroll
                     for (int tt = 0; tt < TMAX; tt++) {
@@ -661,7 +702,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     // this K-chunk's partial: [unit][mu/4][128 rows][4 tokens], so a thread's
                     // 4 consecutive tokens are one 16-byte store and a warp's 32 rows 512
                     // contiguous bytes (token counts are multiples of 16)
-                    float* part = args.partials + (size_t)u * args.mu * TROWS + row * 4;
+                    const int64_t my_slot = TAIL ? un.slot0 + (int64_t)un.chunk * un.pstride : u;
+                    float* part = args.partials + (size_t)my_slot * args.mu * TROWS + row * 4;
 #pragma unroll
                     for (int tt = 0; tt < TMAX; tt++) {
 #pragma unroll
@@ -678,20 +720,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     if (etid == 0) {
                         uint32_t* ctr = args.counters + (size_t)un.gtile * args.n_st + un.st;
                         const uint32_t old = atomicAdd(ctr, 1u);
-                        // counters advance by 16 per call and tile: the last of the kc
-                        // arrivals tops the counter up to the next multiple of 16
-                        const int last = (int)(old & 15u) == args.kc - 1;
-                        if (last) atomicAdd(ctr, (uint32_t)(16 - args.kc));
+                        // counters advance by 16 per call and split tile: the last of the
+                        // np arrivals tops the counter up to the next multiple of 16
+                        const int last = (int)(old & 15u) == np - 1;
+                        if (last) atomicAdd(ctr, (uint32_t)(16 - np));
                         __threadfence();
                         sh.last_flag = last;
                     }
                     if (!epi_sync(sh, epi_ph)) goto epi_done;
                     if (sh.last_flag) {
-                        // sum the chunk partials in chunk order; each token tile's 8 loads of
+                        // sum the piece partials in piece order; each token tile's 8 loads of
                         // 16 bytes are issued before any is used
-                        const int64_t u0 = u - un.chunk;
-                        for (int c2 = 0; c2 < args.kc; c2++) {
-                            const float* part = args.partials + (size_t)(u0 + c2) * args.mu * TROWS + row * 4;
+                        for (int c2 = 0; c2 < np; c2++) {
+                            const int64_t slot = TAIL ? un.slot0 + (int64_t)c2 * un.pstride : u - un.chunk + c2;
+                            const float* part = args.partials + (size_t)slot * args.mu * TROWS + row * 4;
 #pragma unroll
                             for (int tt = 0; tt < TMAX; tt++) {
                                 float4 pv[HC / 4];

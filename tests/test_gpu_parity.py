@@ -395,3 +395,62 @@ def test_workspace_too_small_is_rejected():
     small = dllm.alloc_workspace(wsb - 256)
     with pytest.raises(dllm.DllmError):
         dllm.dllm_qgemm(wd, Q4, N, K, act.q, act.scale, act.sums, M, None, 0, out, N, small, wsb - 256)
+
+
+# ------------------------------------------------------------------ tail split
+# 192 tiles of 128 rows on B200's 148 SMs: one round of whole tiles, then the 44 tiles
+# left are cut into 148 K-pieces (3 or 4 per tile), one more unit per SM, summed by the
+# last arriving piece in piece order.
+
+TAIL_N = 192 * 128
+
+
+@pytest.mark.parametrize("qtype,M", [(Q4, 16), (Q4, 160), (Q6, 48)])
+def test_tail_split_parity(qtype, M):
+    N, K = TAIL_N, 4096
+    w, x = gu.make_case(qtype, M, N, K, 42)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, qtype, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    _, ref, T = oracle.qgemm(qtype, w, N, K, oq, os_)
+    ok, worst = gu.tol_ok(out, ref, T)
+    assert ok, worst
+
+
+def test_tail_split_independent_of_M_and_rows():
+    """The K pieces depend on the weight shape only: the same rows at another canvas
+    height, or gathered by a row list, give the same bits."""
+    N, K, M = TAIL_N, 4096, 160
+    w, x = gu.make_case(Q4, M, N, K, 43)
+    wd = dllm.repack(Q4, w, N, K)
+    full = gu.gemm(wd, Q4, N, K, gu.Act(x))
+    part = gu.gemm(wd, Q4, N, K, gu.Act(x[:16].copy()))
+    assert torch.equal(part, full[:16])
+    rows = synth.block_rows(M, 32, 44)
+    act = gu.Act(x)
+    got = gu.gemm(wd, Q4, N, K, act, rows=rows)
+    assert torch.equal(got, full[torch.from_numpy(rows).long().cuda()])
+    again = gu.gemm(wd, Q4, N, K, act)
+    assert torch.equal(again, full)
+
+
+def test_tail_split_gate_up_in_one_launch():
+    """gate and up (2 x 12288 rows) in one launch, as the step runs them."""
+    M, F, K = 32, 12288, 4096
+    wg = synth.weights(Q4, F, K, 45)
+    wu = synth.weights(Q4, F, K, 46)
+    x = synth.activations(M, K, 45)
+    dg, du = dllm.repack(Q4, wg, F, K), dllm.repack(Q4, wu, F, K)
+    act = gu.Act(x)
+    og = torch.empty((M, F), device="cuda")
+    ou = torch.empty((M, F), device="cuda")
+    wsb = dllm.dllm_qgemm_workspace_bytes(Q4, 2 * F, K, M)
+    ws = dllm.alloc_workspace(max(wsb, 256))
+    dllm.dllm_qkv_qgemm(dg, du, None, Q4, F, F, K, act.q, act.scale, act.sums, M, og, F, ou, None, F, ws, wsb)
+    oq, os_, _ = oracle.quantize_act(x)
+    for w, o in ((wg, og), (wu, ou)):
+        _, ref, T = oracle.qgemm(Q4, w, F, K, oq, os_)
+        ok, worst = gu.tol_ok(o.cpu().numpy(), ref, T)
+        assert ok, worst
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK

@@ -261,6 +261,16 @@ int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
  * device status with dllm_get_device_status(). */
 int dllm_debug_bounded_wait(dllm_stream_t stream);
 
+/* The work split the GEMM would use for a weight of n_tiles 128-row tiles, K inputs,
+ * an M-row canvas (n_rows requested rows, 0 for all) on a device with `sms` SMs.
+ * Host only: no device is touched.  out (host, 8 entries) receives kc (K-chunks per
+ * tile of the uniform split), full_tiles, tail_k and tail_big (the tail split: tiles
+ * [0, full_tiles) whole, the first tail_big of the rest in tail_k + 1 K-pieces, the
+ * others in tail_k; tail_k = 0 means the uniform split), n_units, n_st (token
+ * super-tiles), mu (tokens per super-tile) and the workspace bytes.  The pages have no
+ * counterpart; the split is this library's scheduling.  DLLM_ERR_ARG on bad sizes. */
+int dllm_debug_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms, int64_t* out);
+
 /* int8 tensor-core throughput probe: on each of `ctas` CTAs, `issuers` warps (1..4)
  * each issue `iters` back-to-back tcgen05 kind::i8 MMAs of 128 x n x 32 into their own
  * n_acc accumulators, with A in tensor memory (a_from_tmem != 0) or shared memory.

@@ -661,6 +661,22 @@ int dllm_debug_bounded_wait(dllm_stream_t stream) {
     return run_gemm<12, false, false>(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int dllm_debug_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms, int64_t* out) {
+    if (n_tiles <= 0 || n_tiles > (1LL << 30) || K <= 0 || K % QK || K / QK > (1 << 20) || M <= 0 ||
+        M > (1LL << 31) || n_rows < 0 || n_rows > 32 || sms <= 0 || sms > 4096 || !out)
+        return DLLM_ERR_ARG;
+    const Plan p = make_plan(n_tiles, K, M, n_rows, sms);
+    out[0] = p.kc;
+    out[1] = p.full_tiles;
+    out[2] = p.tail_k;
+    out[3] = p.tail_big;
+    out[4] = p.n_units;
+    out[5] = p.n_st;
+    out[6] = p.mu;
+    out[7] = (int64_t)p.bytes;
+    return DLLM_OK;
+}
+
 int dllm_bench_mma_i8(int n, int n_acc, int a_from_tmem, int issuers, int iters, int ctas,
                       unsigned long long* ns_out, dllm_stream_t stream) {
     if (n < 16 || n > 256 || n % 16 || n_acc < 1 || n_acc > 8 || issuers < 1 || issuers > 4 ||

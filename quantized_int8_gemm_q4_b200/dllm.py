@@ -32,7 +32,7 @@ EXPORTS = (
     "dllm_rmsnorm_quantize", "dllm_swiglu_quantize",
     "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_get_device_status",
     "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_debug_bounded_wait",
-    "dllm_bench_mma_i8",
+    "dllm_bench_mma_i8", "dllm_debug_plan",
 )
 
 
@@ -75,6 +75,7 @@ def load() -> ctypes.CDLL:
         "dllm_debug_sb_ints": [P, I, I64, I64, P, P, P, I64, P, P],
         "dllm_debug_bounded_wait": [P],
         "dllm_bench_mma_i8": [I, I, I, I, I, I, P, P],
+        "dllm_debug_plan": [I64, I64, I64, I64, I, ctypes.POINTER(ctypes.c_int64)],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -231,3 +232,11 @@ def alloc_act(M: int, K: int, device="cuda"):
     return (torch.empty(qb, dtype=torch.int8, device=device),
             torch.empty(sb // 4, dtype=torch.float32, device=device),
             torch.empty(ub // 4, dtype=torch.float32, device=device))
+
+
+def dllm_debug_plan(n_tiles: int, K: int, M: int, n_rows: int, sms: int) -> dict:
+    """The GEMM's work split for a shape (host only): see include/dllm_qgemm.h."""
+    out = (ctypes.c_int64 * 8)()
+    _check(load().dllm_debug_plan(n_tiles, K, M, n_rows, sms, out), "dllm_debug_plan")
+    keys = ("kc", "full_tiles", "tail_k", "tail_big", "n_units", "n_st", "mu", "bytes")
+    return dict(zip(keys, list(out)))

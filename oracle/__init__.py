@@ -20,10 +20,13 @@ HERE = Path(__file__).resolve().parent
 SRC = HERE / "oracle.c"
 LIB = HERE / "_build" / "liboracle.so"
 
+Q8_0 = 8
 Q4_K = 12
+Q5_K = 13
 Q6_K = 14
 QK_K = 256
-BLOCK_BYTES = {Q4_K: 144, Q6_K: 210}
+# bytes per 256 weights of a row: one K-quant super-block, or eight 34-byte Q8_0 blocks
+BLOCK_BYTES = {Q4_K: 144, Q5_K: 176, Q6_K: 210, Q8_0: 272}
 
 _lib = None
 
@@ -50,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.oracle_q4k_decode.argtypes = [P, P, P, P, P, P]
         L.oracle_q6k_decode.argtypes = [P, P, P, P]
+        L.oracle_q5k_decode.argtypes = [P, P, P, P, P, P]
+        L.oracle_q80_decode.argtypes = [P, P, P]
         L.oracle_dequant.argtypes = [ctypes.c_int, P, I64, I64, P]
         L.oracle_quantize_act.argtypes = [P, I64, I64, I64, P, P, P]
         L.oracle_qgemm.argtypes = [ctypes.c_int, P, I64, I64, P, P, I64, P, I64, I64, I64,
@@ -92,6 +97,29 @@ def q4k_decode(block: np.ndarray):
     return float(d[0]), float(dmin[0]), sc, mn, q
 
 
+def q5k_decode(block: np.ndarray):
+    """One 176-byte Q5_K block -> (d, dmin, sc[8], m[8], q[256] in [0,31])."""
+    b = np.ascontiguousarray(block, dtype=np.uint8)
+    assert b.size == 176
+    d = np.zeros(1, np.float64)
+    dmin = np.zeros(1, np.float64)
+    sc = np.zeros(8, np.uint8)
+    mn = np.zeros(8, np.uint8)
+    q = np.zeros(256, np.uint8)
+    lib().oracle_q5k_decode(_p(b), _p(d), _p(dmin), _p(sc), _p(mn), _p(q))
+    return float(d[0]), float(dmin[0]), sc, mn, q
+
+
+def q80_decode(block: np.ndarray):
+    """One 34-byte Q8_0 block -> (d, q[32] int8)."""
+    b = np.ascontiguousarray(block, dtype=np.uint8)
+    assert b.size == 34
+    d = np.zeros(1, np.float64)
+    q = np.zeros(32, np.int8)
+    lib().oracle_q80_decode(_p(b), _p(d), _p(q))
+    return float(d[0]), q
+
+
 def q6k_decode(block: np.ndarray):
     """One 210-byte Q6_K block -> (d, sc[16] int8, q[256] in [0,63])."""
     b = np.ascontiguousarray(block, dtype=np.uint8)
@@ -104,7 +132,7 @@ def q6k_decode(block: np.ndarray):
 
 
 def dequant(qtype: int, w: np.ndarray, N: int, K: int) -> np.ndarray:
-    """Row-major [N][K/256] blocks -> fp64 [N][K]."""
+    """Row-major blocks ([N][K/256] super-blocks, or [N][K/32] Q8_0 blocks) -> fp64 [N][K]."""
     w = np.ascontiguousarray(w, dtype=np.uint8)
     assert w.size == N * (K // QK_K) * BLOCK_BYTES[qtype]
     out = np.zeros((N, K), np.float64)
@@ -149,7 +177,7 @@ def sb_ints(qtype: int, w: np.ndarray, N: int, K: int, q: np.ndarray):
     w = np.ascontiguousarray(w, dtype=np.uint8)
     q = np.ascontiguousarray(q, dtype=np.int8)
     M = q.shape[0]
-    nsub = K // 32 if qtype == Q4_K else K // 16
+    nsub = K // 16 if qtype == Q6_K else K // 32
     dots = np.zeros((M, N, nsub), np.int32)
     S = np.zeros((M, N, K // QK_K), np.int64)
     Smin = np.zeros((M, N, K // QK_K), np.int64)

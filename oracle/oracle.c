@@ -13,7 +13,9 @@
  *    test oracle; the heatdrop repository card ("Key highlights") names the gguf
  *    package's dequantization as the external correctness reference.  The byte
  *    layouts themselves are not on the pages; they are the GGUF block formats
- *    (144-byte Q4_K, 210-byte Q6_K), restated below in our own words.
+ *    (144-byte Q4_K, 210-byte Q6_K), restated below in our own words.  Q5_K
+ *    (176 bytes) and Q8_0 (34-byte blocks of 32), the other formats the same row
+ *    lists, are decoded too: the oracle side of the next formats.
  *  - Activations are quantized to int8 with one f32 scale per 256 elements
  *    (Architecture page, "Source map", kernels/qgemm.mojo row).  The pages do
  *    not fix the rounding; the reading used here is: amax over the block,
@@ -43,7 +45,22 @@
 
 #define QK 256
 #define Q4K_BYTES 144
+#define Q5K_BYTES 176
 #define Q6K_BYTES 210
+#define Q80_BYTES 34     /* one Q8_0 block: 32 weights */
+
+/* Bytes of one 256-weight span of a row, for each supported GGML type id:
+ * 8 = Q8_0 (eight 34-byte blocks), 12 = Q4_K, 13 = Q5_K, 14 = Q6_K. */
+static int span_bytes(int qtype)
+{
+    switch (qtype) {
+    case 8: return 8 * Q80_BYTES;
+    case 12: return Q4K_BYTES;
+    case 13: return Q5K_BYTES;
+    case 14: return Q6K_BYTES;
+    default: return 0;
+    }
+}
 
 /* IEEE 754 binary16 -> double, from the format definition: 1 sign bit,
  * 5 exponent bits (bias 15), 10 fraction bits; exponent 0 is subnormal,
@@ -78,13 +95,9 @@ static uint16_t rd16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); 
  *          both in byte order.
  *   weight value: d * sc_j * q - dmin * m_j.
  */
-void oracle_q4k_decode(const uint8_t *blk, double *d, double *dmin,
-                       uint8_t sc[8], uint8_t mn[8], uint8_t q[256])
+/* The eight 6-bit scales and mins of a Q4_K or Q5_K block, from its 12 packed bytes. */
+static void scales_mins_6bit(const uint8_t *b, uint8_t sc[8], uint8_t mn[8])
 {
-    const uint8_t *b = blk + 4;
-    const uint8_t *qs = blk + 16;
-    *d = oracle_f16_to_f64(rd16(blk));
-    *dmin = oracle_f16_to_f64(rd16(blk + 2));
     for (int j = 0; j < 8; j++) {
         if (j < 4) {
             sc[j] = b[j] & 63;
@@ -94,11 +107,60 @@ void oracle_q4k_decode(const uint8_t *blk, double *d, double *dmin,
             mn[j] = (uint8_t)((b[j + 4] >> 4) | ((b[j] >> 6) << 4));
         }
     }
+}
+
+void oracle_q4k_decode(const uint8_t *blk, double *d, double *dmin,
+                       uint8_t sc[8], uint8_t mn[8], uint8_t q[256])
+{
+    const uint8_t *qs = blk + 16;
+    *d = oracle_f16_to_f64(rd16(blk));
+    *dmin = oracle_f16_to_f64(rd16(blk + 2));
+    scales_mins_6bit(blk + 4, sc, mn);
     for (int c = 0; c < 4; c++)
         for (int l = 0; l < 32; l++) {
             q[64 * c + l] = qs[32 * c + l] & 15;
             q[64 * c + 32 + l] = qs[32 * c + l] >> 4;
         }
+}
+
+/*
+ * Q5_K super-block (176 bytes, 256 weights in 8 sub-blocks of 32): the Q4_K block
+ * with a fifth bit per quant.  This is the GGUF definition; the pages list Q5_K among
+ * the formats (Architecture page, "Source map", quant/kquants.mojo row).
+ *   [0,2)    d     f16
+ *   [2,4)    dmin  f16
+ *   [4,16)   the eight 6-bit scales and mins, packed as in Q4_K
+ *   [16,48)  qh: 32 bytes; bit j of qh[l] is the fifth bit of element l of sub-block j
+ *   [48,176) qs: 128 bytes of low nibbles, in four 32-byte chunks as in Q4_K
+ *            (chunk c: sub-block 2c in the low nibbles, 2c+1 in the high nibbles)
+ *   q in [0, 31]; weight value: d * sc_j * q - dmin * m_j.
+ */
+void oracle_q5k_decode(const uint8_t *blk, double *d, double *dmin,
+                       uint8_t sc[8], uint8_t mn[8], uint8_t q[256])
+{
+    const uint8_t *qh = blk + 16;
+    const uint8_t *qs = blk + 48;
+    *d = oracle_f16_to_f64(rd16(blk));
+    *dmin = oracle_f16_to_f64(rd16(blk + 2));
+    scales_mins_6bit(blk + 4, sc, mn);
+    for (int c = 0; c < 4; c++)
+        for (int l = 0; l < 32; l++) {
+            int j0 = 2 * c, j1 = 2 * c + 1;
+            q[32 * j0 + l] = (uint8_t)((qs[32 * c + l] & 15) | (((qh[l] >> j0) & 1) << 4));
+            q[32 * j1 + l] = (uint8_t)((qs[32 * c + l] >> 4) | (((qh[l] >> j1) & 1) << 4));
+        }
+}
+
+/*
+ * Q8_0 block (34 bytes, 32 weights): d (f16) then 32 signed 8-bit quants;
+ * weight value: d * q.  GGUF definition; the pages list Q8_0 among the formats
+ * (Architecture page, "Source map", quant/kquants.mojo row).  A 256-weight span of a
+ * row is eight consecutive blocks.
+ */
+void oracle_q80_decode(const uint8_t *blk, double *d, int8_t q[32])
+{
+    *d = oracle_f16_to_f64(rd16(blk));
+    for (int i = 0; i < 32; i++) q[i] = (int8_t)blk[2 + i];
 }
 
 /*
@@ -130,13 +192,14 @@ void oracle_q6k_decode(const uint8_t *blk, double *d, int8_t sc[16], uint8_t q[2
             }
 }
 
-/* Dequantize a row-major [N][K/256] matrix of blocks to fp64 [N][K].
- * qtype: 12 = Q4_K, 14 = Q6_K (the GGML type ids). */
+/* Dequantize a row-major matrix of blocks ([N][K/256] super-blocks, or [N][K/32]
+ * Q8_0 blocks) to fp64 [N][K].  qtype: 8 = Q8_0, 12 = Q4_K, 13 = Q5_K, 14 = Q6_K (the
+ * GGML type ids). */
 int oracle_dequant(int qtype, const uint8_t *w, int64_t N, int64_t K, double *out)
 {
-    if (K % QK) return -1;
+    if (K % QK || !span_bytes(qtype)) return -1;
     int64_t nsb = K / QK;
-    int bb = qtype == 12 ? Q4K_BYTES : Q6K_BYTES;
+    int bb = span_bytes(qtype);
     for (int64_t n = 0; n < N; n++)
         for (int64_t s = 0; s < nsb; s++) {
             const uint8_t *blk = w + (n * nsb + s) * bb;
@@ -148,6 +211,12 @@ int oracle_dequant(int qtype, const uint8_t *w, int64_t N, int64_t K, double *ou
                 oracle_q4k_decode(blk, &d, &dmin, sc, mn, q);
                 for (int i = 0; i < QK; i++)
                     o[i] = d * sc[i / 32] * q[i] - dmin * mn[i / 32];
+            } else if (qtype == 13) {
+                double d, dmin;
+                uint8_t sc[8], mn[8];
+                oracle_q5k_decode(blk, &d, &dmin, sc, mn, q);
+                for (int i = 0; i < QK; i++)
+                    o[i] = d * sc[i / 32] * q[i] - dmin * mn[i / 32];
             } else if (qtype == 14) {
                 double d;
                 int8_t sc[16];
@@ -155,7 +224,12 @@ int oracle_dequant(int qtype, const uint8_t *w, int64_t N, int64_t K, double *ou
                 for (int i = 0; i < QK; i++)
                     o[i] = d * sc[i / 16] * ((int)q[i] - 32);
             } else {
-                return -1;
+                for (int b = 0; b < 8; b++) {
+                    double d;
+                    int8_t q8[32];
+                    oracle_q80_decode(blk + b * Q80_BYTES, &d, q8);
+                    for (int i = 0; i < 32; i++) o[32 * b + i] = d * q8[i];
+                }
             }
         }
     return 0;
@@ -264,23 +338,39 @@ int oracle_swiglu(const float *gate, const float *up, int64_t M, int64_t K, int6
 
 /* Decoded form of one weight row: all super-blocks, kept as integers. */
 typedef struct {
-    double *d, *dmin;     /* [nsb] */
-    int32_t *sc, *mn;     /* [nsb][nsub] (mn unused for Q6_K) */
-    int32_t *q;           /* [K]: Q4_K q in [0,15]; Q6_K (q - 32) in [-32,31] */
+    double *d, *dmin;     /* [nsb] (Q8_0: unused) */
+    double *dsub;         /* [nsb][8]: Q8_0 block scales (other types: unused) */
+    int32_t *sc, *mn;     /* [nsb][nsub] (mn unused for Q6_K and Q8_0; sc = 1 for Q8_0) */
+    int32_t *q;           /* [K]: Q4_K q in [0,15]; Q5_K q in [0,31]; Q6_K (q - 32) in
+                             [-32,31]; Q8_0 q in [-128,127] */
 } row_t;
+
+static int subblocks(int qtype) { return qtype == 14 ? 16 : 8; }
 
 static void decode_row(int qtype, const uint8_t *wrow, int64_t nsb, row_t *r)
 {
     for (int64_t s = 0; s < nsb; s++) {
         uint8_t q[256];
-        if (qtype == 12) {
+        if (qtype == 12 || qtype == 13) {
             uint8_t sc[8], mn[8];
-            oracle_q4k_decode(wrow + s * Q4K_BYTES, &r->d[s], &r->dmin[s], sc, mn, q);
+            if (qtype == 12)
+                oracle_q4k_decode(wrow + s * Q4K_BYTES, &r->d[s], &r->dmin[s], sc, mn, q);
+            else
+                oracle_q5k_decode(wrow + s * Q5K_BYTES, &r->d[s], &r->dmin[s], sc, mn, q);
             for (int j = 0; j < 8; j++) {
                 r->sc[s * 8 + j] = sc[j];
                 r->mn[s * 8 + j] = mn[j];
             }
             for (int i = 0; i < QK; i++) r->q[s * QK + i] = q[i];
+        } else if (qtype == 8) {
+            r->d[s] = r->dmin[s] = 0.0;
+            for (int b = 0; b < 8; b++) {
+                int8_t q8[32];
+                oracle_q80_decode(wrow + s * 8 * Q80_BYTES + b * Q80_BYTES, &r->dsub[s * 8 + b], q8);
+                r->sc[s * 8 + b] = 1;
+                r->mn[s * 8 + b] = 0;
+                for (int i = 0; i < 32; i++) r->q[s * QK + 32 * b + i] = q8[i];
+            }
         } else {
             int8_t sc[16];
             oracle_q6k_decode(wrow + s * Q6K_BYTES, &r->d[s], sc, q);
@@ -297,20 +387,23 @@ static void decode_row(int qtype, const uint8_t *wrow, int64_t nsb, row_t *r)
  *          asum_j = sum_{i in sub-block j} a_i               (int32)
  *          S      = sum_j sc_j * dot_j,  Smin = sum_j m_j * asum_j   (int64)
  *          acc   += da * (d * S - dmin * Smin)               (fp64)
+ *   Q5_K:  as Q4_K, with q in [0,31]
  *   Q6_K:  dot_j  = sum_{i in sub-block j} (q_i - 32) * a_i  (16 terms)
  *          S      = sum_j sc_j * dot_j;  acc += da * d * S
+ *   Q8_0:  dot_b  = sum_{i in block b} q_i * a_i (32 terms);  acc += da * sum_b d_b * dot_b
  * T accumulates sum_sb |da| * (|d| * sum_j |sc_j dot_j| + |dmin| * sum_j |m_j asum_j|),
  * the scale of the rounding error any f32 evaluation order can make.
  */
 static void one_output(int qtype, const row_t *r, int64_t nsb, const int8_t *a,
                        const float *da, double *acc_out, double *T_out)
 {
-    int nsub = qtype == 12 ? 8 : 16;
+    int nsub = subblocks(qtype);
     int sub = QK / nsub;
+    int has_min = qtype == 12 || qtype == 13;
     double acc = 0.0, T = 0.0;
     for (int64_t s = 0; s < nsb; s++) {
         int64_t S = 0, Smin = 0;
-        double Sabs = 0.0, Mabs = 0.0;
+        double Sabs = 0.0, Mabs = 0.0, part8 = 0.0, abs8 = 0.0;
         for (int j = 0; j < nsub; j++) {
             int32_t dot = 0, asum = 0;
             for (int i = 0; i < sub; i++) {
@@ -318,16 +411,26 @@ static void one_output(int qtype, const row_t *r, int64_t nsb, const int8_t *a,
                 dot += r->q[k] * (int32_t)a[k];
                 asum += a[k];
             }
+            if (qtype == 8) {
+                part8 += r->dsub[s * 8 + j] * (double)dot;
+                abs8 += fabs(r->dsub[s * 8 + j] * (double)dot);
+                continue;
+            }
             int64_t t = (int64_t)r->sc[s * nsub + j] * dot;
             S += t;
             Sabs += fabs((double)t);
-            if (qtype == 12) {
+            if (has_min) {
                 int64_t u = (int64_t)r->mn[s * nsub + j] * asum;
                 Smin += u;
                 Mabs += fabs((double)u);
             }
         }
         double das = (double)da[s];
+        if (qtype == 8) {
+            acc += das * part8;
+            T += fabs(das) * abs8;
+            continue;
+        }
         acc += das * (r->d[s] * (double)S - r->dmin[s] * (double)Smin);
         T += fabs(das) * (fabs(r->d[s]) * Sabs + fabs(r->dmin[s]) * Mabs);
     }
@@ -350,15 +453,15 @@ int oracle_qgemm(int qtype, const uint8_t *w, int64_t N, int64_t K,
                  const int32_t *rows, int64_t n_rows, int64_t n0, int64_t n1,
                  float *out, double *out64, double *T, int64_t ldo, int nthreads)
 {
-    if ((qtype != 12 && qtype != 14) || K % QK || n0 < 0 || n1 > N || n0 > n1) return -1;
+    if (!span_bytes(qtype) || K % QK || n0 < 0 || n1 > N || n0 > n1) return -1;
     int64_t nsb = K / QK;
     int64_t n_out = rows ? n_rows : M;
     if (ldo < n1 - n0) return -1;
     if (rows)
         for (int64_t i = 0; i < n_rows; i++)
             if (rows[i] < 0 || rows[i] >= M) return -1;
-    int bb = qtype == 12 ? Q4K_BYTES : Q6K_BYTES;
-    int nsub = qtype == 12 ? 8 : 16;
+    int bb = span_bytes(qtype);
+    int nsub = subblocks(qtype);
     if (nthreads <= 0) nthreads = 1;
     (void)nthreads;
 #pragma omp parallel num_threads(nthreads)
@@ -366,6 +469,7 @@ int oracle_qgemm(int qtype, const uint8_t *w, int64_t N, int64_t K,
         row_t r;
         r.d = malloc(sizeof(double) * nsb);
         r.dmin = malloc(sizeof(double) * nsb);
+        r.dsub = malloc(sizeof(double) * nsb * 8);
         r.sc = malloc(sizeof(int32_t) * nsb * nsub);
         r.mn = malloc(sizeof(int32_t) * nsb * nsub);
         r.q = malloc(sizeof(int32_t) * K);
@@ -381,29 +485,32 @@ int oracle_qgemm(int qtype, const uint8_t *w, int64_t N, int64_t K,
                 if (T) T[i * ldo + (n - n0)] = t;
             }
         }
-        free(r.d); free(r.dmin); free(r.sc); free(r.mn); free(r.q);
+        free(r.d); free(r.dmin); free(r.dsub); free(r.sc); free(r.mn); free(r.q);
     }
     return 0;
 }
 
 /*
  * Integer intermediates, for bit-exact comparison:
- *   dots[m][n][j]  per-sub-block dot products (Q4_K: K/32 of sum q*a with
- *                  q in [0,15]; Q6_K: K/16 of sum (q-32)*a)
+ *   dots[m][n][j]  per-sub-block dot products (Q4_K / Q5_K: K/32 of sum q*a;
+ *                  Q6_K: K/16 of sum (q-32)*a; Q8_0: K/32 of sum q*a per block)
  *   S[m][n][sb], Smin[m][n][sb]  the per-super-block integer combinations
- *                  (Smin is 0 for Q6_K).  Any pointer may be NULL.
+ *                  (Smin is 0 for Q6_K and Q8_0; for Q8_0, whose blocks carry their
+ *                  own f16 scales, S is the plain sum of its eight dots).
+ *   Any pointer may be NULL.
  */
 int oracle_sb_ints(int qtype, const uint8_t *w, int64_t N, int64_t K,
                    const int8_t *q, int64_t M, int32_t *dots, int64_t *S, int64_t *Smin)
 {
-    if ((qtype != 12 && qtype != 14) || K % QK) return -1;
+    if (!span_bytes(qtype) || K % QK) return -1;
     int64_t nsb = K / QK;
-    int nsub = qtype == 12 ? 8 : 16;
+    int nsub = subblocks(qtype);
     int sub = QK / nsub;
-    int bb = qtype == 12 ? Q4K_BYTES : Q6K_BYTES;
+    int bb = span_bytes(qtype);
     row_t r;
     r.d = malloc(sizeof(double) * nsb);
     r.dmin = malloc(sizeof(double) * nsb);
+    r.dsub = malloc(sizeof(double) * nsb * 8);
     r.sc = malloc(sizeof(int32_t) * nsb * nsub);
     r.mn = malloc(sizeof(int32_t) * nsb * nsub);
     r.q = malloc(sizeof(int32_t) * K);
@@ -422,14 +529,14 @@ int oracle_sb_ints(int qtype, const uint8_t *w, int64_t N, int64_t K,
                     }
                     if (dots) dots[(m * N + n) * (nsb * nsub) + s * nsub + j] = dot;
                     Ss += (int64_t)r.sc[s * nsub + j] * dot;
-                    if (qtype == 12) Sm += (int64_t)r.mn[s * nsub + j] * asum;
+                    if (qtype == 12 || qtype == 13) Sm += (int64_t)r.mn[s * nsub + j] * asum;
                 }
                 if (S) S[(m * N + n) * nsb + s] = Ss;
                 if (Smin) Smin[(m * N + n) * nsb + s] = Sm;
             }
         }
     }
-    free(r.d); free(r.dmin); free(r.sc); free(r.mn); free(r.q);
+    free(r.d); free(r.dmin); free(r.dsub); free(r.sc); free(r.mn); free(r.q);
     return 0;
 }
 

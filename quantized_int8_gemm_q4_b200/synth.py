@@ -12,6 +12,10 @@ Distributions (the synthetic stand-ins for real GGUF weights, which are not used
   * Q6_K: the 128 low-bit bytes and 64 high-bit bytes are uniform random bytes,
     so every 6-bit quant is uniform on 0..63; the 16 int8 scales are uniform on
     -32..31 (configurable); d as above.
+  * Q5_K: as Q4_K, plus 32 uniform random bytes of fifth bits, so every 5-bit quant
+    is uniform on 0..31.
+  * Q8_0: every 34-byte block has d uniform on [1e-4, 1e-3] rounded to f16 and 32
+    int8 quants uniform on -127..127.
   * Activations: f32 standard normal.
 """
 from __future__ import annotations
@@ -20,10 +24,12 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
+Q8_0 = 8
 Q4_K = 12
+Q5_K = 13
 Q6_K = 14
 QK_K = 256
-BLOCK_BYTES = {Q4_K: 144, Q6_K: 210}
+BLOCK_BYTES = {Q4_K: 144, Q5_K: 176, Q6_K: 210, Q8_0: 272}  # bytes per 256 weights
 
 
 def _rng(seed, *sub):
@@ -59,8 +65,32 @@ def q6k_weights(N: int, K: int, seed, *sub, sc_lo: int = -32, sc_hi: int = 31) -
     return blk.reshape(N, K // QK_K, 210)
 
 
+def q5k_weights(N: int, K: int, seed, *sub) -> np.ndarray:
+    """uint8 [N, K/256, 176] GGUF Q5_K blocks: d | dmin | 12 scale bytes | 32 qh | 128 qs."""
+    assert K % QK_K == 0
+    nb = N * (K // QK_K)
+    rng = _rng(seed, 5, *sub)
+    blk = np.empty((nb, 176), np.uint8)
+    blk[:, 0:2] = _f16_bytes(rng, nb)
+    blk[:, 2:4] = _f16_bytes(rng, nb)
+    blk[:, 4:176] = rng.integers(0, 256, size=(nb, 172), dtype=np.uint8)
+    return blk.reshape(N, K // QK_K, 176)
+
+
+def q80_weights(N: int, K: int, seed, *sub) -> np.ndarray:
+    """uint8 [N, K/256, 272]: per 256 weights, eight GGUF Q8_0 blocks d | 32 int8."""
+    assert K % QK_K == 0
+    nb = N * (K // 32)
+    rng = _rng(seed, 11, *sub)
+    blk = np.empty((nb, 34), np.uint8)
+    blk[:, 0:2] = _f16_bytes(rng, nb, 1e-4, 1e-3)
+    blk[:, 2:34] = rng.integers(-127, 128, size=(nb, 32)).astype(np.int8).view(np.uint8)
+    return blk.reshape(N, K // QK_K, 272)
+
+
 def weights(qtype: int, N: int, K: int, seed, *sub) -> np.ndarray:
-    return q4k_weights(N, K, seed, *sub) if qtype == Q4_K else q6k_weights(N, K, seed, *sub)
+    gen = {Q4_K: q4k_weights, Q5_K: q5k_weights, Q6_K: q6k_weights, Q8_0: q80_weights}[qtype]
+    return gen(N, K, seed, *sub)
 
 
 def activations(M: int, K: int, seed, *sub) -> np.ndarray:

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
         L.oracle_sb_ints.argtypes = [ctypes.c_int, P, I64, I64, P, I64, P, P, P]
         L.oracle_rmsnorm.argtypes = [P, I64, I64, I64, P, ctypes.c_float, ctypes.c_double, P]
         L.oracle_swiglu.argtypes = [P, P, I64, I64, I64, ctypes.c_double, P]
+        L.oracle_attention.argtypes = [P, P, P, I64, I64, I64, I64, I64, P, ctypes.c_int]
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -217,3 +218,18 @@ def rmsnorm_quantize(x: np.ndarray, gamma: np.ndarray, eps: float):
 def swiglu_quantize(gate: np.ndarray, up: np.ndarray):
     """quantize_act(swiglu(gate, up)): the definition the fused library kernel follows."""
     return quantize_act(swiglu(gate, up))
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """Bidirectional attention, fp64: q [Lq][H][dh], k and v [Lk][Hkv][dh] -> o [Lq][H][dh].
+    Head h attends with key/value head h // (H / Hkv)."""
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    Lq, H, dh = q.shape
+    Lk, Hkv, dh2 = k.shape
+    assert v.shape == k.shape and dh2 == dh
+    o = np.zeros((Lq, H, dh), np.float64)
+    nt = max_threads() if nthreads is None else nthreads
+    _chk(lib().oracle_attention(_p(q), _p(k), _p(v), Lq, Lk, H, Hkv, dh, _p(o), nt))
+    return o

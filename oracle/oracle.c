@@ -26,6 +26,8 @@
  *    a = scale[m][sb] * qa.  It is formed the way the method runs it: integer
  *    sub-block dots, integer per-super-block combinations, and one fp64
  *    combine per super-block, rounded to f32 once at the end.
+ *  - Bidirectional attention over the canvas (the next step the GPU path will
+ *    take on; no kernel yet), in fp64, with grouped key/value heads.
  *  - The steps either side of the quantizer in a forward pass (Architecture page,
  *    "A forward pass", steps 2 and 4): RMSNorm of a projection input, and the
  *    SwiGLU gate SiLU(g) * u between the gate/up and down projections.  Both are
@@ -537,6 +539,58 @@ int oracle_sb_ints(int qtype, const uint8_t *w, int64_t N, int64_t K,
         }
     }
     free(r.d); free(r.dmin); free(r.dsub); free(r.sc); free(r.mn); free(r.q);
+    return 0;
+}
+
+/*
+ * Bidirectional attention over the canvas (Architecture page, "A forward pass",
+ * step 2: attention runs over all L positions with no mask; heatdrop card, "Key
+ * highlights": the GPU path runs it as an online-softmax attention on f16 tensor
+ * cores).  For query row i and head h, whose key/value head is g = h / (H / Hkv):
+ *     o[i][h] = sum_j softmax_j( q[i][h] . k[j][g] / sqrt(dh) ) v[j][g]
+ * over every key row j, evaluated in fp64 (the largest logit is subtracted before
+ * exp, which leaves softmax unchanged).  q is [Lq][H][dh], k and v are [Lk][Hkv][dh]
+ * (f32), o is [Lq][H][dh] (fp64).  Lq < Lk covers the last layer, where only the
+ * requested rows continue but attend to the whole canvas.  H must be a multiple of Hkv.
+ */
+int oracle_attention(const float *q, const float *k, const float *v, int64_t Lq, int64_t Lk,
+                     int64_t H, int64_t Hkv, int64_t dh, double *o, int nthreads)
+{
+    if (Lq <= 0 || Lk <= 0 || H <= 0 || Hkv <= 0 || dh <= 0 || H % Hkv) return -1;
+    int64_t group = H / Hkv;
+    double scale = 1.0 / sqrt((double)dh);
+    if (nthreads <= 0) nthreads = 1;
+    (void)nthreads;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double *logit = malloc(sizeof(double) * Lk);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < Lq * H; t++) {
+            int64_t i = t / H, h = t % H, g = h / group;
+            const float *qi = q + (i * H + h) * dh;
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < Lk; j++) {
+                const float *kj = k + (j * Hkv + g) * dh;
+                double dot = 0.0;
+                for (int64_t c = 0; c < dh; c++) dot += (double)qi[c] * (double)kj[c];
+                logit[j] = dot * scale;
+                if (logit[j] > mx) mx = logit[j];
+            }
+            double den = 0.0;
+            for (int64_t j = 0; j < Lk; j++) {
+                logit[j] = exp(logit[j] - mx);
+                den += logit[j];
+            }
+            double *oi = o + (i * H + h) * dh;
+            for (int64_t c = 0; c < dh; c++) oi[c] = 0.0;
+            for (int64_t j = 0; j < Lk; j++) {
+                const float *vj = v + (j * Hkv + g) * dh;
+                double w = logit[j] / den;
+                for (int64_t c = 0; c < dh; c++) oi[c] += w * (double)vj[c];
+            }
+        }
+        free(logit);
+    }
     return 0;
 }
 

@@ -259,7 +259,7 @@ int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, con
     const int64_t M_out = rows ? n_rows : M;
     int rc = check_act(q, scale, sums, M_out);
     if (rc) return rc;
-    if (!aligned16(x) || !aligned16(gamma) || ldx % 4) return DLLM_ERR_ALIGN;
+    if (!aligned16(x) || !aligned16(gamma) || ldx % 4 || (rows && !aligned16(rows))) return DLLM_ERR_ALIGN;
     if (M_out > (1LL << 31) - 16) return DLLM_ERR_ARG;
     int dev;
     if ((rc = current_device(&dev))) return rc;

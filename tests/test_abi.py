@@ -130,6 +130,7 @@ def test_fused_quantize_argument_checks(lib):
     assert rms(rows=_fake(A), n_rows=0) == dllm.DLLM_ERR_ARG      # a row list needs n_rows >= 1
     assert rms(rows=_fake(A), n_rows=-3) == dllm.DLLM_ERR_ARG
     assert rms(rows=None, n_rows=5) == dllm.DLLM_ERR_ARG          # n_rows without a list
+    assert rms(rows=_fake(A + 4), n_rows=2) == dllm.DLLM_ERR_ALIGN
     g = lib.dllm_swiglu_quantize
     assert g(None, _fake(A), 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG
     assert g(_fake(A), None, 4, 256, 256, _fake(A), _fake(A), _fake(A), None) == dllm.DLLM_ERR_ARG

@@ -95,6 +95,69 @@ def step_gemms(model, L, n_layers, gather_last=False):
     return layer(L) * (n_layers - 1) + last + [Gemm("output", Q6, model.vocab, h, R, R)]
 
 
+# bytes written per activation element by every quantizer: the int8 code, plus the f32
+# scale per 256 and the two-float scaled sum per 32 (4/256 + 64/256)
+ACT_OUT_BYTES = 1 + 4 / 256 + 64 / 256
+
+
+def act_kernel_plan(model, L, n_layers, gather_last=False):
+    """The quantizer launch in front of each GEMM of the step, in launch order:
+    (kernel, rows, K).  Same order as step_gemms."""
+    h, f, R = model.hidden, model.ffn, min(L, model.out_rows)
+    plan = []
+    for l in range(n_layers):
+        m = R if gather_last and l == n_layers - 1 else L
+        plan += [("rmsnorm_quantize", L, h), ("quantize_act", m, h), ("rmsnorm_quantize", m, h),
+                 ("swiglu_quantize", m, f)]
+    plan.append(("rmsnorm_quantize", R if gather_last else L, h))
+    return plan
+
+
+def act_bytes(kernel, M, K):
+    """Algorithmic bytes of one quantizer launch: f32 inputs read (x; gate and up), the
+    gains of RMSNorm, and the quantized activation written."""
+    read = {"rmsnorm_quantize": 4, "quantize_act": 4, "swiglu_quantize": 8}[kernel]
+    return M * K * (read + ACT_OUT_BYTES) + (K * 4 if kernel == "rmsnorm_quantize" else 0)
+
+
+def act_rooflines(durations_ms, plan, hbm_gbs):
+    """Per quantizer kernel: launches timed, mean duration, achieved GB/s of algorithmic
+    bytes and its fraction of hbm_gbs.  durations_ms[a] is launch a's time (None if not
+    timed)."""
+    agg = {}
+    for (kernel, M, K), d in zip(plan, durations_ms):
+        if d is None or d <= 0:
+            continue
+        a = agg.setdefault(kernel, [0, 0.0, 0.0])
+        a[0] += 1
+        a[1] += d
+        a[2] += act_bytes(kernel, M, K)
+    out = {}
+    for kernel, (n, ms, nbytes) in sorted(agg.items()):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[kernel] = {"launches_timed": n, "mean_us": round(ms * 1e3 / n, 3), "achieved_gbs": round(gbs, 1),
+                       "frac": round(gbs / hbm_gbs, 4)}
+    return out
+
+
+def split_durations(evs, n_marks):
+    """Per-launch times from S steps of events: evs[i][j] is recorded after the j-th
+    launch of step i, a quantizer at even j and its GEMM at odd j.  Returns the GEMM ms
+    per step, the quantizer ms per step, and each quantizer's mean ms (None for the
+    step's first quantizer, which has no mark before it)."""
+    S = len(evs)
+    gemm_ms = quant_ms = 0.0
+    act = [0.0] * (n_marks // 2)
+    for e in evs:
+        for j in range(0, n_marks, 2):
+            if j > 0:
+                d = e[j - 1].elapsed_time(e[j])
+                quant_ms += d
+                act[j // 2] += d
+            gemm_ms += e[j].elapsed_time(e[j + 1])
+    return gemm_ms / S, quant_ms / S, [None] + [x / S for x in act[1:]]
+
+
 def roofline_time(gemms, hbm_gbs, p_int8):
     return sum(max(g.bytes / (hbm_gbs * 1e9), g.ops / p_int8) for g in gemms)
 
@@ -426,17 +489,7 @@ def run_ours(args, rank, world):
     with torch.cuda.stream(s):
         gE.replay()
     torch.cuda.synchronize()
-    gemm_ms = 0.0
-    quant_ms = 0.0
-    for i in range(S):
-        e = evs[i]
-        # marks: after each quantize (even index), after each GEMM (odd index)
-        for j in range(0, n_marks, 2):
-            if j > 0:
-                quant_ms += e[j - 1].elapsed_time(e[j])
-            gemm_ms += e[j].elapsed_time(e[j + 1])
-    gemm_ms /= S
-    quant_ms /= S
+    gemm_ms, quant_ms, act_launch_ms = split_durations(evs, n_marks)
     assert dllm.dllm_get_device_status() == dllm.DLLM_OK
 
     ms_step = elapsed_ms / args.steps
@@ -486,6 +539,15 @@ def run_ours(args, rank, world):
                 "durations": f"CUDA events on the launching stream around every GEMM launch, over {S} "
                              "graph-replayed steps right after the timed region"}
 
+    # the quantizers' own rooflines (the step's first quantizer has no mark before it)
+    try:
+        hbm_for_act, _ = load_peaks()
+        act = act_rooflines(act_launch_ms, act_kernel_plan(model, L, n_layers, args.gather_last), hbm_for_act)
+        act["durations"] = ("CUDA events from the previous GEMM's end to the quantizer's end, in the same "
+                            "second pass; they include each launch's event cost")
+    except Exception as ex:  # a report, never a reason to lose the bench line
+        act = {"error": repr(ex)}
+
     cpu = None
     if rank == 0 and not args.no_cpu and cpu_sample:
         cpu = cpu_baseline(model, L, cpu_sample, rows_np, seed, gam_host, n_layers)
@@ -501,7 +563,7 @@ def run_ours(args, rank, world):
         "step_roofline": {"t_star_ms": round(tstar * 1e3, 4), "frac": round(tstar * 1e3 / ms_step, 4),
                           "p_int8_tops": p_int8 / 1e12, "hbm_gbs": hbm_gbs},
         "gemm_ms_per_step": round(gemm_ms, 4), "quantize_ms_per_step": round(quant_ms, 4),
-        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "roofline": roof, "act_kernels": act, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
     return result

@@ -70,3 +70,56 @@ def test_gather_last_step_shapes():
     cfg = bench.workload_config(model, 128, model.n_layers, 32, 1, gather_last=True)
     assert "requested rows only" in cfg["workload"]
     assert "requested rows only" not in bench.workload_config(model, 128, model.n_layers, 32, 1)["workload"]
+
+
+def test_act_kernel_plan_matches_the_gemms():
+    model = synth.MODELS["llada-8b"]()
+    for gl in (False, True):
+        plan = bench.act_kernel_plan(model, 128, model.n_layers, gl)
+        gemms = bench.step_gemms(model, 128, model.n_layers, gl)
+        assert len(plan) == len(gemms) == 129
+        # each quantizer feeds the GEMM after it: same K and same activation rows
+        for (kind, M, K), g in zip(plan, gemms):
+            assert K == g.K
+            assert M == g.M_act or (g.name == "output" and not gl)  # the output GEMM gathers rows
+    kinds = [k for k, _, _ in bench.act_kernel_plan(model, 128, 2)]
+    assert kinds == ["rmsnorm_quantize", "quantize_act", "rmsnorm_quantize", "swiglu_quantize"] * 2 + \
+        ["rmsnorm_quantize"]
+
+
+def test_act_rooflines():
+    model = synth.MODELS["llada-8b"]()
+    plan = bench.act_kernel_plan(model, 128, 1)
+    # 2.78 MB of RMSNorm traffic in 5 us is 555.6 GB/s; swiglu 14.57 MB in 10 us
+    d = [None, 0.004, 0.005, 0.010, 0.005]
+    r = bench.act_rooflines(d, plan, 6527.8)
+    rms = bench.act_bytes("rmsnorm_quantize", 128, 4096)
+    assert abs(rms - 2777088) < 1   # 2 MiB of x + 16 KiB of gains + 0.64 MiB written
+    assert r["rmsnorm_quantize"]["launches_timed"] == 2
+    assert abs(r["rmsnorm_quantize"]["achieved_gbs"] - rms * 2 / 10e-6 / 1e9) < 0.1
+    sw = bench.act_bytes("swiglu_quantize", 128, 12288)
+    assert abs(r["swiglu_quantize"]["achieved_gbs"] - sw / 10e-6 / 1e9) < 0.1
+    assert r["quantize_act"]["mean_us"] == 4.0
+    assert abs(r["quantize_act"]["frac"] - r["quantize_act"]["achieved_gbs"] / 6527.8) < 1e-4
+
+
+def test_split_durations_from_events():
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    # two steps of 3 (quantizer, GEMM) pairs: quantizers take 1, 2, 3 ms, GEMMs 10, 20, 30
+    def step(t0):
+        marks, t = [], t0
+        for q, g in ((1, 10), (2, 20), (3, 30)):
+            t += q
+            marks.append(Ev(t))
+            t += g
+            marks.append(Ev(t))
+        return marks
+    gemm, quant, per = bench.split_durations([step(0.0), step(100.0)], 6)
+    assert gemm == 60.0 and quant == 5.0   # the first quantizer of a step is not timed
+    assert per == [None, 2.0, 3.0]

@@ -88,7 +88,7 @@ struct Plan {
     bool split;        // some tile's K range is cut: counters and partials in use
     int64_t n_units;
     int64_t Mp;        // activation rows seen by the GEMM
-    size_t ctr_off, part_off, gq_off, gs_off, gu_off, bytes;
+    size_t ctr_off, ctr_bytes, part_off, gq_off, gs_off, gu_off, bytes;
 };
 
 int64_t uniform_cost(int64_t n_tiles, int64_t nsb, int kc, int sms) {
@@ -131,7 +131,8 @@ Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
     p.n_units = p.tail_k > 0 ? (int64_t)(p.full_tiles + sms) * p.n_st : n_tiles * p.n_st * p.kc;
     size_t off = 0;
     p.ctr_off = off;
-    off += align256((size_t)n_tiles * p.n_st * 4);
+    p.ctr_bytes = (size_t)n_tiles * p.n_st * 4;  // one arrival counter per (tile, token super-tile)
+    off += align256(p.ctr_bytes);
     p.part_off = off;
     if (p.kc > 1) off += align256((size_t)n_tiles * p.n_st * p.kc * p.mu * TROWS * 4);
     if (p.tail_k > 0) off += align256((size_t)sms * p.n_st * p.mu * TROWS * 4);
@@ -463,12 +464,9 @@ int dllm_qgemm_noalloc(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
     if (p.bytes > DLLM_NOALLOC_SCRATCH_BYTES) return DLLM_ERR_SCRATCH_LIMIT;
     uint8_t* scratch;
     if ((rc = noalloc_scratch(dev, &scratch))) return rc;
-    if (p.split) {
-        const size_t ctr_bytes = (size_t)(N / TROWS) * p.n_st * 4;
-        if (cudaMemsetAsync(scratch + p.ctr_off, 0, ctr_bytes, reinterpret_cast<cudaStream_t>(stream)) !=
-            cudaSuccess)
-            return DLLM_ERR_CUDA;
-    }
+    if (p.split &&
+        cudaMemsetAsync(scratch + p.ctr_off, 0, p.ctr_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return DLLM_ERR_CUDA;
     return dllm_qgemm(w, t, N, K, q, scale, sums, M, rows, n_rows, out, ldo, scratch, DLLM_NOALLOC_SCRATCH_BYTES,
                       stream);
 }

@@ -15,11 +15,12 @@
 //         0..105 (u8).  S = P0 + 8*P1.
 //   Q6_K: v = (q-32)*sc + 32896 lies in [28800, 36992]; plane 0 = (v & 255) - 128,
 //         plane 1 = (v >> 8) - 128 (both s8), and plane0 + 256*plane1 = (q-32)*sc.
-// Each plane accumulator stays within 2^22 in magnitude.  The first MMA of each
-// super-block overwrites it, and the epilogue adds the bit pattern of 1.5*2^23 to
-// the int32 it reads, which makes an f32 equal to exactly 1.5*2^23 + value; S then
-// takes one FFMA and one FADD (packed f32x2), with no integer-to-float instruction.
-// The epilogue then accumulates da * d * S in f32 registers.
+// Each plane sum stays within 2^22 in magnitude.  Each plane has its own int32
+// accumulator in tensor memory, preset to the bit pattern of 1.5*2^23 (MAGIC): after
+// a super-block's MMAs it holds the bits of the f32 1.5*2^23 + P exactly, so the
+// epilogue needs no integer-to-float instruction.  It forms S with one FFMA and one
+// FADD (packed f32x2), accumulates da * d * S in f32 registers, and writes the preset
+// back before releasing the accumulator.
 //
 // The min term (Q4_K), on the tf32 tensor pipe.  Its per-super-block factor
 // dmin[n] * da[m] is a product of a row term and a column term, so
@@ -27,25 +28,31 @@
 // a GEMM with one K step per sub-block.  Both operands are split as hi + lo with hi
 // exact in tf32 (-dmin m_j is exact in hi + lo; da*sum32_j loses at most 2^-22 of
 // itself), and hi*hi + hi*lo + lo*hi accumulate in an f32 tensor-memory accumulator
-// over the whole K range, read once per work unit.  Its error is below 2^-21 of the
-// min term's magnitude, inside the 1e-6 * sum|terms| tolerance.
+// over the whole K range of a work unit, read once per unit.  The dropped lo*lo
+// product and the split lose at most 2^-21 of each product's magnitude; the f32
+// accumulation over the unit's K/32 sub-block steps adds at most (K/32) * 2^-24 of
+// the running sum of magnitudes (about 2^-17 at K = 4096); both bounds are relative to
+// the min term's own sum of |terms|, a part of the 1e-6 * sum|terms| tolerance.
 //
-// Roles (16 warps, one CTA per SM, persistent over work units):
-//   warp 0      producer: bulk copies of weight tiles and activation tiles into
-//               shared-memory rings
-//   warps 1-2   MMA issue (warp 1 also allocates tensor memory).  One thread can
-//               issue a tcgen05.mma only every ~28 ns, longer than a 64-token MMA
-//               takes, so the two token tiles of a super-block go to two warps, each
-//               with its own accumulator set and a short wait/issue/commit loop
+// Pipeline (16 warps, one CTA per SM, persistent over work units).  Per super-block
+// the MMAs run plane-major: the 8 K-steps of plane 0 into accumulator P0, then the 8
+// of plane 1 into P1, then (Q4_K) the 3 min-term MMAs.  Every MMA covers all of the
+// unit's tokens (N <= 128; at N = 128 one int8 MMA takes ~64 cycles, the pipe's full
+// rate).  So each plane accumulator is drained by the epilogue while the other plane's
+// MMAs run, and the tensor pipe never waits for an epilogue hand-off.
+//   warp 0      weight producer: bulk copies of weight tiles into a shared-memory
+//               ring.  Weights are never written by the kernels this library chains
+//               with programmatic dependent launch, so these copies start before the
+//               dependency wait.
+//   warp 1      MMA issuer (one thread) and tensor-memory allocation
+//   warp 2      activation producer: bulk copies of activation tiles (int8 codes,
+//               scales, scaled sums), after the dependency wait
 //   warp 3      idle
-//   warps 4-7   unpack: thread = weight row; decode the super-block, build the two
-//               weight planes per K-step of 32 into a tensor-memory ring of half
-//               super-blocks (the A operand), the min-term A operand into shared
-//               memory, and the f32 d; a half is published only once the
-//               super-block's activation stages have landed
-//   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each on half of
-//               the token columns; per super-block, read the two plane accumulators,
-//               release them to the issuer, and accumulate the f32 result in registers
+//   warps 4-7   unpack: thread = weight row; per quarter super-block (two K-steps)
+//               build both weight planes into a tensor-memory ring (the A operand),
+//               the min-term A operand (Q4_K) into shared memory, and the f32 d
+//   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each on 64 of the
+//               token columns
 //
 // A work unit is (128 weight rows, up to 128 canvas rows, one K-chunk).  The number
 // of K-chunks per tile depends only on N, K and the SM count, never on M or on the
@@ -60,25 +67,27 @@ constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float MAGIC = 12582912.0f;
 constexpr int GEMM_THREADS = 512;
 constexpr int UNIT_TOKENS = 128;
-constexpr int NTOK = 64;                           // token columns per MMA and per accumulator
-constexpr int TMAX = UNIT_TOKENS / NTOK;           // token tiles per unit
-constexpr int HC = NTOK / 2;                       // token columns per epilogue warp
+constexpr int EPI_COLS = 64;                       // token columns per epilogue thread
 constexpr int MAX_KC = 16;                         // K-chunks per tile, at most
-constexpr int ISSUERS = 2;                         // MMA-issuing warps
 constexpr int S_SLOTS = 4;                         // d ring (unpack -> epilogue)
-constexpr int ACC_SETS = 2;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
-
-// tensor-memory columns
-// tensor-memory columns: the A ring (RING halves of a super-block, each 4 K-step slots
-// of 16 columns: plane 0 | plane 1), then ACC_SETS x 2 planes x NTOK accumulator
-// columns, then (Q4_K) TMAX x NTOK f32 min-term accumulator columns
-constexpr uint32_t TM_A = 0;
-constexpr uint32_t TM_COLS = 512;
+// Registers per thread of each warpgroup after setmaxnreg: producers and issuer,
+// unpack, and the two epilogue warpgroups.  setmaxnreg.inc draws on the registers the
+// CTA was launched with (512 threads x 128), so the split must not exceed them, or the
+// increasing warps would wait for registers that never come free.
+constexpr int REG_CTRL = 40, REG_UNPACK = 56, REG_EPI = 208;
+static_assert(128 * REG_CTRL + 128 * REG_UNPACK + 256 * REG_EPI <= 65536, "register split over the launch budget");
+static_assert(REG_CTRL % 8 == 0 && REG_UNPACK % 8 == 0 && REG_EPI % 8 == 0 && REG_CTRL >= 24, "setmaxnreg counts");
 
 // Activation "sums" operand of one super-block: per 8-row group 512 bytes =
 // [hi j0-3 | hi j4-7 | lo j0-3 | lo j4-7] x [8 rows x 16 bytes].
 constexpr int SUMS_GROUP = 512;
+
+// Tensor-memory columns: the A ring (A_SLOTS quarter super-blocks; a quarter is two
+// K-steps of 16 columns, [plane 0: 8 | plane 1: 8]), then the plane accumulators P0
+// and P1 (128 token columns each), then (Q4_K) the f32 min-term accumulator.
+constexpr uint32_t TM_COLS = 512;
+constexpr uint32_t TM_A = 0;
 
 template <int QT>
 struct GemmCfg;
@@ -87,29 +96,44 @@ struct GemmCfg<12> {  // Q4_K
     static constexpr int TILE = Q4K_TILE;
     static constexpr bool MIN = true;
     static constexpr int W_STAGES = 4;
-    static constexpr int B_STAGES = 4;
-    static constexpr int B_Q = NTOK * 256;
-    static constexpr int B_SUMS = NTOK / 8 * SUMS_GROUP;
-    static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
+    static constexpr int B_STAGES = 3;
+    static constexpr int B_Q = UNIT_TOKENS * 256;
+    static constexpr int B_SUMS = UNIT_TOKENS / 8 * SUMS_GROUP;
+    static constexpr int B_STAGE = B_Q + B_SUMS + UNIT_TOKENS * 4;
     static constexpr int MINA = 2 * 4096;  // -dmin*m_j as [hi | lo], canonical K-major 128 rows x 32 B
-    static constexpr int RING = 2;         // A ring: one super-block (the min accumulators take the rest)
-    static constexpr uint32_t TM_ACC = 64 * RING;
-    static constexpr uint32_t TM_MIN = TM_ACC + ACC_SETS * 2 * NTOK;
+    static constexpr int MINA_BUFS = 2;
+    static constexpr int A_SLOTS = 4;      // one super-block
+    static constexpr uint32_t TM_P0 = TM_A + 32 * A_SLOTS;
+    static constexpr uint32_t TM_P1 = TM_P0 + UNIT_TOKENS;
+    static constexpr uint32_t TM_MIN = TM_P1 + UNIT_TOKENS;
+    static constexpr uint32_t TM_END = TM_MIN + UNIT_TOKENS;
 };
 template <>
 struct GemmCfg<14> {  // Q6_K
     static constexpr int TILE = Q6K_TILE;
     static constexpr bool MIN = false;
-    static constexpr int W_STAGES = 3;
-    static constexpr int B_STAGES = 4;
-    static constexpr int B_Q = NTOK * 256;
+    static constexpr int W_STAGES = 4;
+    static constexpr int B_STAGES = 3;
+    static constexpr int B_Q = UNIT_TOKENS * 256;
     static constexpr int B_SUMS = 0;
-    static constexpr int B_STAGE = B_Q + B_SUMS + NTOK * 4;
+    static constexpr int B_STAGE = B_Q + B_SUMS + UNIT_TOKENS * 4;
     static constexpr int MINA = 0;
-    static constexpr int RING = 4;  // A ring: two super-blocks, so the unpack runs one ahead
-    static constexpr uint32_t TM_ACC = 64 * RING;
+    static constexpr int MINA_BUFS = 0;
+    static constexpr int A_SLOTS = 8;      // two super-blocks: the unpack runs one ahead
+    static constexpr uint32_t TM_P0 = TM_A + 32 * A_SLOTS;
+    static constexpr uint32_t TM_P1 = TM_P0 + UNIT_TOKENS;
     static constexpr uint32_t TM_MIN = 0;
+    static constexpr uint32_t TM_END = TM_P1 + UNIT_TOKENS;
 };
+static_assert(GemmCfg<12>::TM_END <= TM_COLS && GemmCfg<14>::TM_END <= TM_COLS, "tensor-memory columns over budget");
+
+// K-step (of 32) that sub-position kk of quarter q holds.  Q4_K: the quarter is one
+// 32-byte nibble chunk, K-steps 2q (low nibbles) and 2q+1 (high nibbles).  Q6_K: the
+// two K-steps that share their low-bit bytes, 4h + g and 4h + g + 2 (h = q/2, g = q%2).
+template <int QT>
+__host__ __device__ constexpr int kstep_of(int q, int kk) {
+    return QT == 12 ? 2 * q + kk : 4 * (q >> 1) + (q & 1) + 2 * kk;
+}
 
 struct Segment {
     const uint8_t* w;  // repacked weights
@@ -140,18 +164,19 @@ struct GemmArgs {
     uint32_t* counters;  // [n_tiles * n_st], when kc > 1
     float* partials;     // [units][mu/4][128 rows][4 tokens], when kc > 1
     int32_t* dbg_S;    // debug: per-super-block integer S instead of f32 (nullable)
-    int32_t stall;     // test: the producer issues nothing, so every other role's wait runs out
+    int32_t stall;     // test: the producers issue nothing, so every other role's wait runs out
     int64_t dbg_N;
 };
 
 struct GemmShared {
-    uint64_t w_full[8], w_empty[8];
-    uint64_t b_full[8], b_empty[8];
-    uint64_t a_full[4], a_empty[4];  // A ring slots: super-block halves (K-steps 0-3, 4-7 + the min-term A)
+    uint64_t w_full[4], w_empty[4];
+    uint64_t b_full[3], b_empty[3];
+    uint64_t a_full[8], a_empty[8];   // A ring slots: quarter super-blocks
+    uint64_t p_full[2], p_empty[2];   // plane accumulators P0, P1
+    uint64_t m_full[2], m_empty[2];   // min-term A operand buffers (Q4_K)
+    uint64_t min_full, min_empty;     // min-term accumulator (Q4_K), once per unit
     uint64_t s_full[S_SLOTS], s_empty[S_SLOTS];
-    uint64_t acc_full[ACC_SETS], acc_empty[ACC_SETS];
-    uint64_t min_empty;
-    uint64_t final_bar[4];
+    uint64_t final_bar;
     uint64_t epi_bar;
     uint32_t tmem_base;
     volatile int abort_flag;
@@ -180,6 +205,19 @@ __device__ __forceinline__ bool wait_bar_warp(GemmShared& sh, uint64_t* bar, uin
     const bool ok = wait_bar(sh, bar, parity);
     return __all_sync(0xffffffffu, ok);
 }
+// Drain wait of an aborting CTA: waits for the CTA's own asynchronous work (bulk copies
+// into its shared memory, MMAs on its tensor memory) regardless of the abort flag,
+// bounded by its own limit.  True if the phase completed.
+__device__ __forceinline__ bool drain_bar(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, 200000u)) {
+        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            set_err(ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
 // Bounded barrier among the 256 epilogue threads.
 __device__ __forceinline__ bool epi_sync(GemmShared& sh, uint32_t& phase) {
     mbar_arrive(&sh.epi_bar);
@@ -194,11 +232,6 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-// This warp's HC = 32 consecutive accumulator columns.
-__device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&x)[HC]) {
-    tmem_ld16(taddr, x);
-    tmem_ld16(taddr + 16, x + 16);
 }
 
 struct Unit {
@@ -262,13 +295,33 @@ __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int64_t u) {
     return r;
 }
 
-template <int QT>
-constexpr bool tmem_fits() {
-    using C = GemmCfg<QT>;
-    return C::TM_ACC + ACC_SETS * 2 * NTOK + (C::MIN ? TMAX * NTOK : 0) <= TM_COLS &&
-           (!C::MIN || C::TM_MIN == C::TM_ACC + ACC_SETS * 2 * NTOK) && C::RING <= 4 && C::RING % 2 == 0;
+// 64 consecutive accumulator columns of this warp's 32 lanes.
+__device__ __forceinline__ void load_cols64(uint32_t taddr, uint32_t (&x)[EPI_COLS]) {
+    tmem_ld16(taddr, x);
+    tmem_ld16(taddr + 16, x + 16);
+    tmem_ld16(taddr + 32, x + 32);
+    tmem_ld16(taddr + 48, x + 48);
 }
-static_assert(tmem_fits<12>() && tmem_fits<14>(), "tensor-memory columns over budget");
+// Write the MAGIC preset into 64 consecutive accumulator columns of this warp's lanes.
+__device__ __forceinline__ void preset_cols64(uint32_t taddr) {
+    uint32_t m[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) m[i] = MAGIC_BITS;
+    tmem_st16(taddr, m);
+    tmem_st16(taddr + 16, m);
+    tmem_st16(taddr + 32, m);
+    tmem_st16(taddr + 48, m);
+}
+
+// Store the first cnt of this thread's EPI_COLS accumulated outputs: column j goes to
+// p + j * ld (one output row per token; the warp's 32 lanes are 32 consecutive n).
+__device__ __forceinline__ void store_cols(float* p, int64_t ld, int cnt, const float2 (&acc)[EPI_COLS / 2]) {
+#pragma unroll
+    for (int j = 0; j < EPI_COLS; j++) {
+        if (j < cnt) *p = j & 1 ? acc[j / 2].y : acc[j / 2].x;
+        p += ld;
+    }
+}
 
 template <int QT, bool DBG, bool TAIL>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmArgs args) {
@@ -277,19 +330,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     uint8_t* w_stage = smem_raw;
     uint8_t* b_stage = w_stage + C::W_STAGES * C::TILE;
     uint8_t* mina = b_stage + C::B_STAGES * C::B_STAGE;
-    GemmShared& sh = *reinterpret_cast<GemmShared*>(mina + C::MINA);
+    GemmShared& sh = *reinterpret_cast<GemmShared*>(mina + C::MINA_BUFS * C::MINA);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n_units = args.n_units;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 128); }
-        for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 256); }
-        for (int i = 0; i < C::RING; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], ISSUERS); }
-        for (int i = 0; i < S_SLOTS; i++) { mbar_init(&sh.s_full[i], 128); mbar_init(&sh.s_empty[i], 256); }
-        for (int i = 0; i < ACC_SETS; i++) { mbar_init(&sh.acc_full[i], 1); mbar_init(&sh.acc_empty[i], 256); }
+        // an activation stage is released by the issuer's commit (its MMAs are done)
+        // and by the 256 epilogue threads (the scales are read)
+        for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 257); }
+        for (int i = 0; i < C::A_SLOTS; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], 1); }
+        for (int i = 0; i < 2; i++) { mbar_init(&sh.p_full[i], 1); mbar_init(&sh.p_empty[i], 256); }
+        for (int i = 0; i < 2; i++) { mbar_init(&sh.m_full[i], 128); mbar_init(&sh.m_empty[i], 1); }
+        mbar_init(&sh.min_full, 1);
         mbar_init(&sh.min_empty, 256);
-        for (int i = 0; i < 4; i++) mbar_init(&sh.final_bar[i], 1);
+        for (int i = 0; i < S_SLOTS; i++) { mbar_init(&sh.s_full[i], 128); mbar_init(&sh.s_empty[i], 256); }
+        mbar_init(&sh.final_bar, 1);
         mbar_init(&sh.epi_bar, 256);
         sh.abort_flag = 0;
         fence_mbar_init();
@@ -302,167 +359,154 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
-    // Everything above, and the producer's L2 prefetch of its first weight tiles, may
-    // overlap the previous kernel on the stream; every access to global memory that
-    // earlier work can write comes after pdl_wait in the role that makes it.
+    // Everything above, and the weight copies, may overlap the previous kernel on the
+    // stream; every access to global memory that earlier work can write comes after
+    // pdl_wait in the role that makes it.
     if (threadIdx.x == 0) pdl_trigger();
 
     if (warp < 4) {
-        setmaxnreg_dec<48>();
-        if (warp == 0) {
-            // ======================================================== producer
-            uint32_t ws = 0, wph = 0, bs = 0, bph = 0;
-            // stages with a copy issued (bit i) and the phase it completes (bit i)
-            uint32_t w_iss = 0, w_php = 0, b_iss = 0, b_php = 0;
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_a = policy_evict_last();
+        setmaxnreg_dec<REG_CTRL>();
+        if (warp == 0 || warp == 2) {
+            // ======================================================== producers
+            // warp 0: weight tiles; warp 2: activation tiles.  Stages with a copy issued
+            // (bit i) and the phase that copy completes (bit i), for the abort drain.
+            const bool wprod = warp == 0;
+            uint32_t st = 0, ph = 0, iss = 0, php = 0;
+            const uint64_t pol = wprod ? policy_evict_first() : policy_evict_last();
             const int64_t n_prod = args.stall ? 0 : n_units;
-            if (lane == 0 && blockIdx.x < n_prod) {
-                const Unit un = unit_of<TAIL>(args, blockIdx.x);
-                const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
-                for (int s = un.sb0; s < un.sb1 && s < un.sb0 + C::W_STAGES; s++)
-                    prefetch_l2(wt + (size_t)s * C::TILE, C::TILE);
-            }
-            pdl_wait();
+            const int NST = wprod ? C::W_STAGES : C::B_STAGES;
+            uint64_t* full = wprod ? sh.w_full : sh.b_full;
+            uint64_t* empty = wprod ? sh.w_empty : sh.b_empty;
+            if (!wprod) pdl_wait();
             for (int64_t u = blockIdx.x; u < n_prod; u += gridDim.x) {
                 const Unit un = unit_of<TAIL>(args, u);
                 const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
-                const int T = (un.len + NTOK - 1) / NTOK;
                 for (int s = un.sb0; s < un.sb1; s++) {
-                    if (!wait_bar_warp(sh, &sh.w_empty[ws], wph ^ 1)) goto prod_done;
+                    if (!wait_bar_warp(sh, &empty[st], ph ^ 1)) goto prod_done;
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&sh.w_full[ws], C::TILE);
-                        bulk_g2s_hint(w_stage + ws * C::TILE, wt + (size_t)s * C::TILE, C::TILE, &sh.w_full[ws],
-                                      pol_w);
-                    }
-                    w_iss |= 1u << ws;
-                    w_php = (w_php & ~(1u << ws)) | (wph << ws);
-                    if (++ws == C::W_STAGES) { ws = 0; wph ^= 1; }
-                    for (int tt = 0; tt < T; tt++) {
-                        const int64_t t0 = un.m0 + (int64_t)tt * NTOK;
-                        const int ntok = min(NTOK, un.len - tt * NTOK);
-                        if (!wait_bar_warp(sh, &sh.b_empty[bs], bph ^ 1)) goto prod_done;
-                        if (lane == 0) {
-                            uint8_t* st = b_stage + bs * C::B_STAGE;
+                        if (wprod) {
+                            mbar_arrive_expect_tx(&full[st], C::TILE);
+                            bulk_g2s_hint(w_stage + st * C::TILE, wt + (size_t)s * C::TILE, C::TILE, &full[st], pol);
+                        } else {
+                            uint8_t* bs = b_stage + st * C::B_STAGE;
+                            const int64_t t0 = un.m0;
+                            const uint32_t ntok = (uint32_t)un.len;
                             const uint32_t sums_bytes = C::B_SUMS ? ntok / 8 * SUMS_GROUP : 0;
-                            mbar_arrive_expect_tx(&sh.b_full[bs], ntok * 256 + sums_bytes + ntok * 4);
-                            bulk_g2s_hint(st, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256, &sh.b_full[bs],
-                                          pol_a);
+                            mbar_arrive_expect_tx(&full[st], ntok * 256 + sums_bytes + ntok * 4);
+                            bulk_g2s_hint(bs, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256, &full[st], pol);
                             if (C::B_SUMS)
-                                bulk_g2s_hint(st + C::B_Q, args.sums + ((size_t)s * args.Mp + t0) / 8 * SUMS_GROUP,
-                                              sums_bytes, &sh.b_full[bs], pol_a);
-                            bulk_g2s_hint(st + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
-                                          &sh.b_full[bs], pol_a);
+                                bulk_g2s_hint(bs + C::B_Q, args.sums + ((size_t)s * args.Mp + t0) / 8 * SUMS_GROUP,
+                                              sums_bytes, &full[st], pol);
+                            bulk_g2s_hint(bs + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
+                                          &full[st], pol);
                         }
-                        b_iss |= 1u << bs;
-                        b_php = (b_php & ~(1u << bs)) | (bph << bs);
-                        if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
                     }
+                    iss |= 1u << st;
+                    php = (php & ~(1u << st)) | (ph << st);
+                    if (++st == (uint32_t)NST) { st = 0; ph ^= 1; }
                 }
             }
         prod_done:
             if (sh.abort_flag) {  // never leave with bulk copies in flight into this CTA's shared memory
-                for (int i = 0; i < C::W_STAGES; i++)
-                    if ((w_iss >> i) & 1u) (void)wait_bar(sh, &sh.w_full[i], (w_php >> i) & 1u);
-                for (int i = 0; i < C::B_STAGES; i++)
-                    if ((b_iss >> i) & 1u) (void)wait_bar(sh, &sh.b_full[i], (b_php >> i) & 1u);
+                for (int i = 0; i < NST; i++)
+                    if ((iss >> i) & 1u) (void)drain_bar(&full[i], (php >> i) & 1u);
             }
-        } else {
-            // ======================================================== MMA issuers
-            // The (super-block, token tile) items of this CTA alternate between warps 1
-            // and 2, and item i owns accumulator set i % 2; with two token tiles each
-            // issuer owns one tile.  Per super-block an issuer waits for each half of
-            // the A ring, issues its item's MMAs on that half (both planes; the min
-            // term with the second half), and commits once to the half's release
-            // barrier, so every release takes one arrival from each issuer.  Warp 3
-            // issues nothing.
-            const int who = warp - 1;
+        } else if (warp == 1) {
+            // ======================================================== MMA issuer
             const bool leader = lane == 0;
-            if (who < ISSUERS) {
-                uint32_t item = 0, sbc = 0, uc = 0;
-                for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
-                    const Unit un = unit_of<TAIL>(args, u);
-                    const int T = (un.len + NTOK - 1) / NTOK;
-                    for (int s = un.sb0; s < un.sb1; s++, sbc++, item += T) {
+            constexpr uint32_t ASG = QT == 12 ? 0 : 1;  // plane operand type: u8 (Q4_K), s8 (Q6_K)
+            uint32_t sbc = 0, uc = 0;
+            for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
+                const Unit un = unit_of<TAIL>(args, u);
+                const uint32_t ntok = (uint32_t)un.len;
+                const uint32_t id = idesc_i8(128, (int)ntok, (int)ASG, 1);
+                for (int s = un.sb0; s < un.sb1; s++, sbc++) {
+                    const uint32_t bst = sbc % C::B_STAGES;
+                    if (!wait_bar_warp(sh, &sh.b_full[bst], (sbc / C::B_STAGES) & 1)) goto mma_done;
+                    const uint32_t stg = smem_u32(b_stage + bst * C::B_STAGE);
+                    const uint64_t bdesc = sdesc_kmajor_noswz(stg, 128, 2048);
+                    // ---- plane 0: waits for its accumulator to be drained and preset, and
+                    // for each quarter of the A ring to be published
+                    if (!wait_bar_warp(sh, &sh.p_empty[0], sbc & 1)) goto mma_done;
 #pragma unroll 1
-                        for (int half = 0; half < 2; half++) {
-                            const uint32_t hc = 2 * sbc + half, slot = hc % C::RING;
-                            if (!wait_bar_warp(sh, &sh.a_full[slot], (hc / C::RING) & 1)) goto mma_done;
-                            for (int tt = 0; tt < T; tt++) {
-                                const uint32_t it = item + tt;
-                                if ((int)(it & 1) != who) continue;
-                                const uint32_t set = it & 1;
-                                const uint32_t bst = it % C::B_STAGES;
-                                const int ntok = min(NTOK, un.len - tt * NTOK);
-                                if (half == 0) {
-                                    // (the item's activation stage is full: the unpack waited for it
-                                    // before publishing the A-ring half waited on above)
-                                    if (!wait_bar_warp(sh, &sh.acc_empty[set], (it >> 1) & 1)) goto mma_done;
-                                } else if (C::MIN && s == un.sb0) {
-                                    // a unit's first min-term MMAs overwrite the min accumulators:
-                                    // the previous unit's epilogue must have read them out
-                                    if (!wait_bar_warp(sh, &sh.min_empty, (uc & 1) ^ 1)) goto mma_done;
-                                }
-                                tc_fence_after();
-                                if (leader) {
-                                    const uint32_t st = smem_u32(b_stage + bst * C::B_STAGE);
-                                    const uint32_t id = QT == 12 ? idesc_i8(128, ntok, 0, 1) : idesc_i8(128, ntok, 1, 1);
-                                    const uint32_t d0 = tmem + C::TM_ACC + set * 2 * NTOK;
-                                    const uint32_t a0 = tmem + TM_A + 64 * slot;
-                                    const uint64_t b0 = sdesc_kmajor_noswz(st, 128, 2048) + 64 * half;
+                    for (int q = 0; q < 4; q++) {
+                        const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
+                        if (!wait_bar_warp(sh, &sh.a_full[sl], (qc / C::A_SLOTS) & 1)) goto mma_done;
+                        tc_fence_after();
+                        if (leader) {
 #pragma unroll
-                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0, a0 + 16 * ks, b0 + 16 * ks, id, half | ks ? 1u : 0u);
-#pragma unroll
-                                    for (int ks = 0; ks < 4; ks++) mma_i8_ts(d0 + NTOK, a0 + 16 * ks + 8, b0 + 16 * ks, id, half | ks ? 1u : 0u);
-                                    if (C::MIN && half == 1) {
-                                        const uint32_t d = tmem + C::TM_MIN + tt * NTOK;
-                                        const uint32_t idm = idesc_tf32(128, ntok);
-                                        const uint32_t ma = smem_u32(mina);
-                                        const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
-                                        const uint64_t a_lo = sdesc_kmajor_noswz(ma + 4096, 128, 256);
-                                        const uint64_t b_hi = sdesc_kmajor_noswz(st + C::B_Q, 128, SUMS_GROUP);
-                                        const uint64_t b_lo = sdesc_kmajor_noswz(st + C::B_Q + 256, 128, SUMS_GROUP);
-                                        mma_tf32_ss(d, a_hi, b_hi, idm, s > un.sb0 ? 1u : 0u);
-                                        mma_tf32_ss(d, a_hi, b_lo, idm, 1);
-                                        mma_tf32_ss(d, a_lo, b_hi, idm, 1);
-                                    }
-                                    if (half == 1) tc_commit(&sh.acc_full[set]);
-                                }
-                                __syncwarp();
-                            }
-                            if (leader) tc_commit(&sh.a_empty[slot]);
-                            __syncwarp();
+                            for (int kk = 0; kk < 2; kk++)
+                                mma_i8_ts(tmem + C::TM_P0, tmem + TM_A + 32 * sl + 16 * kk,
+                                          bdesc + 16 * kstep_of<QT>(q, kk), id, 1u);
                         }
+                        __syncwarp();
                     }
+                    if (leader) tc_commit(&sh.p_full[0]);
+                    __syncwarp();
+                    // ---- plane 1; each quarter slot is released once its plane-1 MMAs finish
+                    if (!wait_bar_warp(sh, &sh.p_empty[1], sbc & 1)) goto mma_done;
+                    tc_fence_after();
+                    if (leader) {
+#pragma unroll 1
+                        for (int q = 0; q < 4; q++) {
+                            const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
+#pragma unroll
+                            for (int kk = 0; kk < 2; kk++)
+                                mma_i8_ts(tmem + C::TM_P1, tmem + TM_A + 32 * sl + 16 * kk + 8,
+                                          bdesc + 16 * kstep_of<QT>(q, kk), id, 1u);
+                            tc_commit(&sh.a_empty[sl]);
+                        }
+                        tc_commit(&sh.p_full[1]);
+                    }
+                    __syncwarp();
+                    if constexpr (C::MIN) {
+                        // ---- min term: (-dmin m_j) x (da sum32_j), three tf32 products
+                        const uint32_t mb = sbc & 1;
+                        if (!wait_bar_warp(sh, &sh.m_full[mb], (sbc >> 1) & 1)) goto mma_done;
+                        // a unit's first min-term MMA overwrites the accumulator: the previous
+                        // unit's epilogue must have read it out
+                        if (s == un.sb0 && !wait_bar_warp(sh, &sh.min_empty, (uc & 1) ^ 1)) goto mma_done;
+                        tc_fence_after();
+                        if (leader) {
+                            const uint32_t idm = idesc_tf32(128, (int)ntok);
+                            const uint32_t ma = smem_u32(mina + mb * C::MINA);
+                            const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
+                            const uint64_t a_lo = sdesc_kmajor_noswz(ma + 4096, 128, 256);
+                            const uint64_t b_hi = sdesc_kmajor_noswz(stg + C::B_Q, 128, SUMS_GROUP);
+                            const uint64_t b_lo = sdesc_kmajor_noswz(stg + C::B_Q + 256, 128, SUMS_GROUP);
+                            mma_tf32_ss(tmem + C::TM_MIN, a_hi, b_hi, idm, s > un.sb0 ? 1u : 0u);
+                            mma_tf32_ss(tmem + C::TM_MIN, a_hi, b_lo, idm, 1u);
+                            mma_tf32_ss(tmem + C::TM_MIN, a_lo, b_hi, idm, 1u);
+                            tc_commit(&sh.m_empty[mb]);
+                            if (s == un.sb1 - 1) tc_commit(&sh.min_full);
+                        }
+                        __syncwarp();
+                    }
+                    if (leader) tc_commit(&sh.b_empty[bst]);
+                    __syncwarp();
                 }
             }
         mma_done:
             // every MMA this warp issued has completed before tensor memory is freed
-            if (leader) tc_commit(&sh.final_bar[who]);
+            if (leader) tc_commit(&sh.final_bar);
             __syncwarp();
-            (void)wait_bar_warp(sh, &sh.final_bar[who], 0);
+            (void)drain_bar(&sh.final_bar, 0);
+            __syncwarp();
         }
     } else if (warp < 8) {
-        setmaxnreg_dec<80>();
+        setmaxnreg_dec<REG_UNPACK>();
         // ============================================================ unpack
-        // Per super-block: decode this row, then build the planes of K-steps 0-3 and
-        // publish them together, then K-steps 4-7 (and the min-term A), so the MMAs of
-        // a super-block can start while the second half is still being built.
+        // Per super-block: decode this row's scales, hand d to the epilogue and (Q4_K)
+        // the min-term A operand to the issuer, then build the two weight planes of
+        // each quarter (two K-steps) and publish it as soon as its ring slot is free.
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        uint32_t ws = 0, wph = 0, ss = 0, sph = 0, sbc = 0, itm = 0;
+        uint32_t ws = 0, wph = 0, ss = 0, sph = 0, sbc = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
             const Unit un = unit_of<TAIL>(args, u);
-            const int T = (un.len + NTOK - 1) / NTOK;
-            for (int s = un.sb0; s < un.sb1; s++, sbc++, itm += T) {
+            for (int s = un.sb0; s < un.sb1; s++, sbc++) {
                 if (!wait_bar_warp(sh, &sh.w_full[ws], wph)) goto unpack_done;
-                // the super-block's activation stages (one per token tile) are full before
-                // any half of its A ring is published, so the MMA issuer need not wait on them
-                for (int tt = 0; tt < T; tt++) {
-                    const uint32_t it = itm + tt;
-                    if (!wait_bar_warp(sh, &sh.b_full[it % C::B_STAGES], (it / C::B_STAGES) & 1)) goto unpack_done;
-                }
                 const uint8_t* tl = w_stage + ws * C::TILE;
                 if constexpr (QT == 12) {
                     const uint32_t b0 = *reinterpret_cast<const uint32_t*>(tl + Q4K_OFF_SC + 12 * row);
@@ -486,46 +530,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     sh.dd[ss][row] = d;
                     mbar_arrive(&sh.s_full[ss]);
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
+                    {
+                        // -dmin*m_j as tf32 hi + lo: row `row` of the canonical K-major layout
+                        // (8-row groups of 256 bytes, two 16-byte K chunks)
+                        const uint32_t mb = sbc & 1;
+                        if (!wait_bar_warp(sh, &sh.m_empty[mb], ((sbc >> 1) & 1) ^ 1)) goto unpack_done;
+                        float hi[8], lo[8];
 #pragma unroll
-                    for (int half = 0; half < 2; half++) {
-                        const uint32_t hc = 2 * sbc + half, slot = hc % C::RING;
-                        if (!wait_bar_warp(sh, &sh.a_empty[slot], ((hc / C::RING) & 1) ^ 1)) goto unpack_done;
-                        if (half == 1) {
-                            // -dmin*m_j as tf32 hi + lo: row `row` of the canonical K-major
-                            // layout (8-row groups of 256 bytes, two 16-byte K chunks)
-                            float hi[8], lo[8];
+                        for (int j = 0; j < 8; j++) split_tf32(nmin[j], hi[j], lo[j]);
+                        uint8_t* base = mina + mb * C::MINA + (row >> 3) * 256 + (row & 7) * 16;
+                        *reinterpret_cast<float4*>(base) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<float4*>(base + 128) = make_float4(hi[4], hi[5], hi[6], hi[7]);
+                        *reinterpret_cast<float4*>(base + 4096) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+                        *reinterpret_cast<float4*>(base + 4096 + 128) = make_float4(lo[4], lo[5], lo[6], lo[7]);
+                        fence_proxy_async_smem();
+                        mbar_arrive(&sh.m_full[mb]);
+                    }
+#pragma unroll 1
+                    for (int q = 0; q < 4; q++) {
+                        const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
+                        if (!wait_bar_warp(sh, &sh.a_empty[sl], ((qc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
+                        // 32-byte quant chunk q: sub-block 2q in the low nibbles, 2q+1 in the high
+                        const uint4 p0 = *reinterpret_cast<const uint4*>(tl + ((2 * q) * TROWS + row) * 16);
+                        const uint4 p1 = *reinterpret_cast<const uint4*>(tl + ((2 * q + 1) * TROWS + row) * 16);
+                        const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                        const uint32_t sca = q == 0 ? sc[0] : q == 1 ? sc[2] : q == 2 ? sc[4] : sc[6];
+                        const uint32_t scb = q == 0 ? sc[1] : q == 1 ? sc[3] : q == 2 ? sc[5] : sc[7];
 #pragma unroll
-                            for (int j = 0; j < 8; j++) split_tf32(nmin[j], hi[j], lo[j]);
-                            uint8_t* base = mina + (row >> 3) * 256 + (row & 7) * 16;
-                            *reinterpret_cast<float4*>(base) = make_float4(hi[0], hi[1], hi[2], hi[3]);
-                            *reinterpret_cast<float4*>(base + 128) = make_float4(hi[4], hi[5], hi[6], hi[7]);
-                            *reinterpret_cast<float4*>(base + 4096) = make_float4(lo[0], lo[1], lo[2], lo[3]);
-                            *reinterpret_cast<float4*>(base + 4096 + 128) = make_float4(lo[4], lo[5], lo[6], lo[7]);
-                            fence_proxy_async_smem();
-                        }
+                        for (int kk = 0; kk < 2; kk++) {
+                            const uint32_t s6 = kk ? scb : sca;
+                            const uint32_t lo3 = s6 & 7, hi3 = s6 >> 3;
+                            uint32_t v[16];
 #pragma unroll
-                        for (int cc = 0; cc < 2; cc++) {
-                            const int c = 2 * half + cc;  // 32-byte quant chunk: sub-blocks 2c, 2c+1
-                            const uint4 p0 = *reinterpret_cast<const uint4*>(tl + ((2 * c) * TROWS + row) * 16);
-                            const uint4 p1 = *reinterpret_cast<const uint4*>(tl + ((2 * c + 1) * TROWS + row) * 16);
-                            const uint32_t wv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-                            for (int h = 0; h < 2; h++) {
-                                const int ks = 2 * c + h;
-                                const uint32_t lo3 = sc[ks] & 7, hi3 = sc[ks] >> 3;
-                                uint32_t v[16];
-#pragma unroll
-                                for (int i = 0; i < 8; i++) {
-                                    const uint32_t nib = (wv[i] >> (4 * h)) & 0x0F0F0F0Fu;
-                                    v[i] = nib * lo3;
-                                    v[8 + i] = nib * hi3;
-                                }
-                                tmem_st16(tmem + lane_off + TM_A + 64 * slot + 16 * (ks & 3), v);
+                            for (int i = 0; i < 8; i++) {
+                                const uint32_t nib = (wv[i] >> (4 * kk)) & 0x0F0F0F0Fu;
+                                v[i] = nib * lo3;
+                                v[8 + i] = nib * hi3;
                             }
+                            tmem_st16(tmem + lane_off + TM_A + 32 * sl + 16 * kk, v);
                         }
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(&sh.a_full[slot]);
+                        mbar_arrive(&sh.a_full[sl]);
                     }
                 } else {
                     const uint4 scv = *reinterpret_cast<const uint4*>(tl + Q6K_OFF_SC + 16 * row);
@@ -536,26 +582,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     sh.dd[ss][row] = d;
                     mbar_arrive(&sh.s_full[ss]);
                     if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
+#pragma unroll 1
+                    for (int q = 0; q < 4; q++) {
+                        const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
+                        if (!wait_bar_warp(sh, &sh.a_empty[sl], ((qc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
+                        // K-steps 4h + g and 4h + g + 2 share their low-bit bytes (low and high
+                        // nibbles) and the half's high-bit bytes
+                        const int h = q >> 1, g = q & 1;
+                        const int lp = 2 * (2 * h + g);  // low-bit piece index
+                        const uint4 l0 = *reinterpret_cast<const uint4*>(tl + (lp * TROWS + row) * 16);
+                        const uint4 l1 = *reinterpret_cast<const uint4*>(tl + ((lp + 1) * TROWS + row) * 16);
+                        const uint4 h0 =
+                            *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h) * TROWS + row) * 16);
+                        const uint4 h1 =
+                            *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h + 1) * TROWS + row) * 16);
+                        const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+                        const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+                        // scale bytes 2ks, 2ks+1 of K-step ks = 4h + g + 2kk sit in word 2h + kk at
+                        // bit offset 16g
+                        const uint32_t swq[2] = {h ? scw[2] : scw[0], h ? scw[3] : scw[1]};
 #pragma unroll
-                    for (int half = 0; half < 2; half++) {
-                        const uint32_t hc = 2 * sbc + half, slot = hc % C::RING;
-                        if (!wait_bar_warp(sh, &sh.a_empty[slot], ((hc / C::RING) & 1) ^ 1)) goto unpack_done;
-#pragma unroll
-                        for (int kq = 0; kq < 4; kq++) {
-                            const int ks = 4 * half + kq;
-                            const int h = ks >> 2, g = ks & 3;
-                            const int lp = 2 * (2 * h + (g & 1));  // low-bit piece index
-                            const uint4 l0 = *reinterpret_cast<const uint4*>(tl + (lp * TROWS + row) * 16);
-                            const uint4 l1 = *reinterpret_cast<const uint4*>(tl + ((lp + 1) * TROWS + row) * 16);
-                            const uint4 h0 =
-                                *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h) * TROWS + row) * 16);
-                            const uint4 h1 =
-                                *reinterpret_cast<const uint4*>(tl + Q6K_OFF_QH + ((2 * h + 1) * TROWS + row) * 16);
-                            const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-                            const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-                            const int sh_lo = 4 * (g >> 1), sh_hi = 2 * g;
-                            const int32_t sca = (int32_t)(int8_t)((scw[ks >> 1] >> (16 * (ks & 1))) & 0xFF);
-                            const int32_t scb = (int32_t)(int8_t)((scw[ks >> 1] >> (16 * (ks & 1) + 8)) & 0xFF);
+                        for (int kk = 0; kk < 2; kk++) {
+                            const int G = g + 2 * kk;
+                            const int sh_lo = 4 * kk, sh_hi = 2 * G;
+                            const int32_t sca = (int32_t)(int8_t)((swq[kk] >> (16 * g)) & 0xFF);
+                            const int32_t scb = (int32_t)(int8_t)((swq[kk] >> (16 * g + 8)) & 0xFF);
                             const uint32_t adda = (uint32_t)(32896 - 32 * sca) * 0x10001u;
                             const uint32_t addb = (uint32_t)(32896 - 32 * scb) * 0x10001u;
                             uint32_t v[16];
@@ -570,11 +621,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 v[i] = __byte_perm(pa, pb, 0x6420) ^ 0x80808080u;
                                 v[8 + i] = __byte_perm(pa, pb, 0x7531) ^ 0x80808080u;
                             }
-                            tmem_st16(tmem + lane_off + TM_A + 64 * slot + 16 * (ks & 3), v);
+                            tmem_st16(tmem + lane_off + TM_A + 32 * sl + 16 * kk, v);
                         }
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(&sh.a_full[slot]);
+                        mbar_arrive(&sh.a_full[sl]);
                     }
                 }
                 mbar_arrive(&sh.w_empty[ws]);
@@ -583,121 +634,132 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         }
     unpack_done:;
     } else {
-        setmaxnreg_inc<192>();
+        setmaxnreg_inc<REG_EPI>();
         // ============================================================ epilogue
-        pdl_wait();  // outputs, partials and counters may be in use by earlier work
         const int quad = warp & 3;
         const int half = (warp - 8) >> 2;
         const int row = quad * 32 + lane;
         const int etid = threadIdx.x - 256;  // 0..255
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        for (int r = 0; r < ACC_SETS; r++) mbar_arrive(&sh.acc_empty[r]);
-        const float2 k8 = make_float2(8.0f, 8.0f), k256 = make_float2(256.0f, 256.0f);
-        const float2 m9 = make_float2(-9.0f * MAGIC, -9.0f * MAGIC);
-        const float2 m257 = make_float2(-257.0f * MAGIC, -257.0f * MAGIC);
-        uint32_t bs = 0, bph = 0, r = 0, rph = 0, ss = 0, sph = 0, epi_ph = 0;
-        for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const Unit un = unit_of<TAIL>(args, u);
-            const int T = (un.len + NTOK - 1) / NTOK;
-            const Segment& sg = args.seg[un.seg];
-            float2 acc[TMAX][HC / 2];
+        const uint32_t col0 = (uint32_t)(half * EPI_COLS);
+        // initial preset of both plane accumulators (this warp's lanes and columns)
+        preset_cols64(tmem + lane_off + C::TM_P0 + col0);
+        preset_cols64(tmem + lane_off + C::TM_P1 + col0);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh.p_empty[0]);
+        mbar_arrive(&sh.p_empty[1]);
+        pdl_wait();  // outputs, partials and counters may be in use by earlier work
+        const float2 kP = QT == 12 ? make_float2(8.0f, 8.0f) : make_float2(256.0f, 256.0f);
+        const float2 mP = QT == 12 ? make_float2(-9.0f * MAGIC, -9.0f * MAGIC)
+                                   : make_float2(-257.0f * MAGIC, -257.0f * MAGIC);
+        uint32_t ss = 0, sph = 0, sbc = 0, uc = 0, epi_ph = 0;
+        for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
+            int sb_first, sb_end, ulen;
+            {
+                const Unit u0 = unit_of<TAIL>(args, u);
+                sb_first = u0.sb0;
+                sb_end = u0.sb1;
+                ulen = u0.len;
+            }
+            const bool live = (int)col0 < ulen;  // this thread has token columns in the unit
+            float2 acc[EPI_COLS / 2];
 #pragma unroll
-            for (int t = 0; t < TMAX; t++)
-#pragma unroll
-                for (int j = 0; j < HC / 2; j++) acc[t][j] = make_float2(0.0f, 0.0f);
-            for (int s = un.sb0; s < un.sb1; s++) {
+            for (int j = 0; j < EPI_COLS / 2; j++) acc[j] = make_float2(0.0f, 0.0f);
+            for (int s = sb_first; s < sb_end; s++, sbc++) {
+                const uint32_t bst = sbc % C::B_STAGES;
+                // ---- plane 0: read, preset, release; keep the raw f32 bits 1.5*2^23 + P0
+                uint32_t x0[EPI_COLS];
+                if (!wait_bar_warp(sh, &sh.p_full[0], sbc & 1)) goto epi_done;
+                tc_fence_after();
+                if (live) {
+                    load_cols64(tmem + lane_off + C::TM_P0 + col0, x0);
+                    tmem_wait_ld();
+                    preset_cols64(tmem + lane_off + C::TM_P0 + col0);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(&sh.p_empty[0]);
                 if (!wait_bar_warp(sh, &sh.s_full[ss], sph)) goto epi_done;
                 const float dv = sh.dd[ss][row];
                 mbar_arrive(&sh.s_empty[ss]);
                 if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
                 const float2 d2 = make_float2(dv, dv);
+                // ---- plane 1, in four chunks of 16 columns
+                if (!wait_bar_warp(sh, &sh.p_full[1], sbc & 1)) goto epi_done;
+                if (!wait_bar_warp(sh, &sh.b_full[bst], (sbc / C::B_STAGES) & 1)) goto epi_done;
+                tc_fence_after();
+                if (live) {
+                    const float* da =
+                        reinterpret_cast<const float*>(b_stage + bst * C::B_STAGE + C::B_Q + C::B_SUMS) + col0;
 #pragma unroll
-                for (int tt = 0; tt < TMAX; tt++) {
-                    if (tt < T) {
-                        const int ntok = min(NTOK, un.len - tt * NTOK);
-                        if (!wait_bar_warp(sh, &sh.acc_full[r], rph)) goto epi_done;
-                        if (!wait_bar_warp(sh, &sh.b_full[bs], bph)) goto epi_done;
-                        tc_fence_after();
-                        const uint32_t acc_t = tmem + lane_off + C::TM_ACC + r * 2 * NTOK + half * HC;
-                        const float* da = reinterpret_cast<const float*>(b_stage + bs * C::B_STAGE + C::B_Q + C::B_SUMS);
-                        // read both plane accumulators and release them to the MMA issuer
-                        // (the next super-block's first MMA overwrites them) before doing
-                        // any arithmetic on the values
-                        if (half * HC < ntok) {
-                            uint32_t x0[HC], x1[HC];
-                            load_cols(acc_t, x0);
-                            load_cols(acc_t + NTOK, x1);
-                            tmem_wait_ld();
-                            tc_fence_before();
-                            mbar_arrive(&sh.acc_empty[r]);
-                            if constexpr (DBG) {
+                    for (int c = 0; c < 4; c++) {
+                        uint32_t x1[16];
+                        tmem_ld16(tmem + lane_off + C::TM_P1 + col0 + 16 * c, x1);
+                        tmem_wait_ld();
+                        if constexpr (DBG) {
+                            const Unit un = unit_of<TAIL>(args, u);
 #pragma unroll
-                                for (int i = 0; i < HC; i++) {
-                                    const int64_t m = un.m0 + tt * NTOK + half * HC + i;
-                                    if (half * HC + i < ntok && m < args.m_out) {
-                                        const int64_t n = un.tile * TROWS + row;
-                                        const int32_t P0 = (int32_t)x0[i], P1 = (int32_t)x1[i];
-                                        args.dbg_S[(m * args.dbg_N + n) * args.nsb + s] = P0 + (QT == 12 ? 8 : 256) * P1;
-                                    }
-                                }
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < HC / 2; i++) {
-                                    // |P| < 2^22: adding the bits of 1.5*2^23 gives the f32 1.5*2^23 + P
-                                    const float2 X0 = make_float2(__uint_as_float(x0[2 * i] + MAGIC_BITS),
-                                                                  __uint_as_float(x0[2 * i + 1] + MAGIC_BITS));
-                                    const float2 X1 = make_float2(__uint_as_float(x1[2 * i] + MAGIC_BITS),
-                                                                  __uint_as_float(x1[2 * i + 1] + MAGIC_BITS));
-                                    const float2 S = QT == 12 ? __fadd2_rn(__ffma2_rn(X1, k8, m9), X0)
-                                                              : __fadd2_rn(__ffma2_rn(X1, k256, m257), X0);
-                                    const float2 dav = *reinterpret_cast<const float2*>(da + half * HC + 2 * i);
-                                    acc[tt][i] = __ffma2_rn(__fmul2_rn(S, d2), dav, acc[tt][i]);
+                            for (int i = 0; i < 16; i++) {
+                                const int ml = (int)col0 + 16 * c + i;
+                                const int64_t m = un.m0 + ml;
+                                if (ml < un.len && m < args.m_out) {
+                                    const int64_t n = un.tile * TROWS + row;
+                                    const int32_t P0 = (int32_t)(x0[16 * c + i] - MAGIC_BITS);
+                                    const int32_t P1 = (int32_t)(x1[i] - MAGIC_BITS);
+                                    args.dbg_S[(m * args.dbg_N + n) * args.nsb + s] = P0 + (QT == 12 ? 8 : 256) * P1;
                                 }
                             }
                         } else {
-                            tc_fence_before();
-                            mbar_arrive(&sh.acc_empty[r]);
+#pragma unroll
+                            for (int i = 0; i < 8; i++) {
+                                const float2 X0 = make_float2(__uint_as_float(x0[16 * c + 2 * i]),
+                                                              __uint_as_float(x0[16 * c + 2 * i + 1]));
+                                const float2 X1 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+                                // 8*P1 - M (or 256*P1 - M) exactly unless it is large, then + (M + P0)
+                                const float2 S = __fadd2_rn(__ffma2_rn(X1, kP, mP), X0);
+                                const float2 dav = *reinterpret_cast<const float2*>(da + 16 * c + 2 * i);
+                                acc[8 * c + i] = __ffma2_rn(__fmul2_rn(S, d2), dav, acc[8 * c + i]);
+                            }
                         }
-                        mbar_arrive(&sh.b_empty[bs]);
-                        if (++bs == C::B_STAGES) { bs = 0; bph ^= 1; }
-                        if (++r == ACC_SETS) { r = 0; rph ^= 1; }
                     }
+                    preset_cols64(tmem + lane_off + C::TM_P1 + col0);
+                    tmem_wait_st();
                 }
+                tc_fence_before();
+                mbar_arrive(&sh.p_empty[1]);
+                mbar_arrive(&sh.b_empty[bst]);
             }
             if constexpr (C::MIN) {
-                // the min-term accumulators: complete, since every tile's last MMAs were
-                // covered by the accumulator barriers waited on above
+                // the unit's min-term accumulator, complete once min_full flips
+                if (!wait_bar_warp(sh, &sh.min_full, uc & 1)) goto epi_done;
+                tc_fence_after();
+                if (live) {
 #pragma unroll
-                for (int tt = 0; tt < TMAX; tt++) {
-                    if (tt < T && half * HC < un.len - tt * NTOK) {
-                        uint32_t y[HC];
-                        load_cols(tmem + lane_off + C::TM_MIN + tt * NTOK + half * HC, y);
+                    for (int c = 0; c < 4; c++) {
+                        uint32_t y[16];
+                        tmem_ld16(tmem + lane_off + C::TM_MIN + col0 + 16 * c, y);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < HC / 2; i++)
-                            acc[tt][i] = __fadd2_rn(acc[tt][i], make_float2(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1])));
+                        for (int i = 0; i < 8; i++)
+                            acc[8 * c + i] = __fadd2_rn(acc[8 * c + i],
+                                                        make_float2(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1])));
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(&sh.min_empty);
             }
             if constexpr (!DBG) {
+                const Unit un = unit_of<TAIL>(args, u);
+                const Segment& sg = args.seg[un.seg];
                 const int64_t n = un.tile * TROWS + row;
                 // uniform split: every tile has kc pieces and partial slots are unit indices
                 const int np = TAIL ? un.np : args.kc;
+                // output rows of this thread: canvas rows m0 + col0 + j for j < cnt
+                const int64_t mfirst = un.m0 + col0;
+                const int cnt = (int)min((int64_t)min(EPI_COLS, un.len - (int)col0), args.m_out - mfirst);
                 if (np == 1) {
-                    float* out = sg.out;
-#pragma unroll
-                    for (int tt = 0; tt < TMAX; tt++) {
-                        if (tt < T) {
-#pragma unroll
-                            for (int j = 0; j < HC; j++) {
-                                const int64_t m = un.m0 + tt * NTOK + half * HC + j;
-                                if (m < args.m_out && m < un.m0 + un.len)
-                                    out[m * sg.ldo + n] = j & 1 ? acc[tt][j / 2].y : acc[tt][j / 2].x;
-                            }
-                        }
-                    }
+                    if (cnt > 0) store_cols(sg.out + mfirst * sg.ldo + n, sg.ldo, cnt, acc);
                 } else {
                     // this K-chunk's partial: [unit][mu/4][128 rows][4 tokens], so a thread's
                     // 4 consecutive tokens are one 16-byte store and a warp's 32 rows 512
@@ -705,15 +767,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     const int64_t my_slot = TAIL ? un.slot0 + (int64_t)un.chunk * un.pstride : u;
                     float* part = args.partials + (size_t)my_slot * args.mu * TROWS + row * 4;
 #pragma unroll
-                    for (int tt = 0; tt < TMAX; tt++) {
-#pragma unroll
-                        for (int q4 = 0; q4 < HC / 4; q4++) {
-                            const int ml = tt * NTOK + half * HC + 4 * q4;
-                            if (tt < T && ml < un.len)
-                                __stcg(reinterpret_cast<float4*>(part + (size_t)(ml / 4) * TROWS * 4),
-                                       make_float4(acc[tt][2 * q4].x, acc[tt][2 * q4].y, acc[tt][2 * q4 + 1].x,
-                                                   acc[tt][2 * q4 + 1].y));
-                        }
+                    for (int q4 = 0; q4 < EPI_COLS / 4; q4++) {
+                        const int ml = (int)col0 + 4 * q4;
+                        if (ml < un.len)
+                            __stcg(reinterpret_cast<float4*>(part + (size_t)(ml / 4) * TROWS * 4),
+                                   make_float4(acc[2 * q4].x, acc[2 * q4].y, acc[2 * q4 + 1].x, acc[2 * q4 + 1].y));
                     }
                     __threadfence();
                     if (!epi_sync(sh, epi_ph)) goto epi_done;
@@ -728,43 +786,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         sh.last_flag = last;
                     }
                     if (!epi_sync(sh, epi_ph)) goto epi_done;
-                    if (sh.last_flag) {
-                        // sum the piece partials in piece order; each token tile's 8 loads of
-                        // 16 bytes are issued before any is used
+                    if (sh.last_flag && live) {
+                        // sum the piece partials in piece order, four 16-byte loads in flight
+                        // at a time
                         for (int c2 = 0; c2 < np; c2++) {
                             const int64_t slot = TAIL ? un.slot0 + (int64_t)c2 * un.pstride : u - un.chunk + c2;
-                            const float* part = args.partials + (size_t)slot * args.mu * TROWS + row * 4;
+                            const float* pp = args.partials + (size_t)slot * args.mu * TROWS + row * 4;
 #pragma unroll
-                            for (int tt = 0; tt < TMAX; tt++) {
-                                float4 pv[HC / 4];
+                            for (int c4 = 0; c4 < EPI_COLS / 16; c4++) {
+                                float4 pv[4];
 #pragma unroll
-                                for (int q4 = 0; q4 < HC / 4; q4++) {
-                                    const int ml = tt * NTOK + half * HC + 4 * q4;
-                                    pv[q4] = (tt < T && ml < un.len)
-                                                 ? __ldcg(reinterpret_cast<const float4*>(part + (size_t)(ml / 4) * TROWS * 4))
+                                for (int q4 = 0; q4 < 4; q4++) {
+                                    const int ml = (int)col0 + 16 * c4 + 4 * q4;
+                                    pv[q4] = ml < un.len
+                                                 ? __ldcg(reinterpret_cast<const float4*>(pp + (size_t)(ml / 4) * TROWS * 4))
                                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                                 }
 #pragma unroll
-                                for (int q4 = 0; q4 < HC / 4; q4++) {
+                                for (int q4 = 0; q4 < 4; q4++) {
+                                    const int a2 = 8 * c4 + 2 * q4;
                                     const float2 lo = make_float2(pv[q4].x, pv[q4].y), hi = make_float2(pv[q4].z, pv[q4].w);
-                                    acc[tt][2 * q4] = c2 == 0 ? lo : __fadd2_rn(acc[tt][2 * q4], lo);
-                                    acc[tt][2 * q4 + 1] = c2 == 0 ? hi : __fadd2_rn(acc[tt][2 * q4 + 1], hi);
+                                    acc[a2] = c2 == 0 ? lo : __fadd2_rn(acc[a2], lo);
+                                    acc[a2 + 1] = c2 == 0 ? hi : __fadd2_rn(acc[a2 + 1], hi);
                                 }
                             }
                         }
-                        float* out = sg.out;
-#pragma unroll
-                        for (int tt = 0; tt < TMAX; tt++) {
-                            if (tt < T) {
-#pragma unroll
-                                for (int j = 0; j < HC; j++) {
-                                    const int ml = tt * NTOK + half * HC + j;
-                                    const int64_t m = un.m0 + ml;
-                                    if (ml < un.len && m < args.m_out)
-                                        out[m * sg.ldo + n] = j & 1 ? acc[tt][j / 2].y : acc[tt][j / 2].x;
-                                }
-                            }
-                        }
+                        if (cnt > 0) store_cols(sg.out + mfirst * sg.ldo + n, sg.ldo, cnt, acc);
                     }
                 }
             }
@@ -782,8 +829,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
 template <int QT>
 constexpr size_t gemm_smem_bytes() {
     using C = GemmCfg<QT>;
-    return (size_t)C::W_STAGES * C::TILE + (size_t)C::B_STAGES * C::B_STAGE + C::MINA + sizeof(GemmShared);
+    return (size_t)C::W_STAGES * C::TILE + (size_t)C::B_STAGES * C::B_STAGE + (size_t)C::MINA_BUFS * C::MINA +
+           sizeof(GemmShared);
 }
+static_assert(gemm_smem_bytes<12>() <= 232448 && gemm_smem_bytes<14>() <= 232448, "shared memory over budget");
 
 // Gather the requested canvas rows of a tiled activation into a compact tiled
 // activation of Mp_r rows (rows past n_rows are zero).  One thread per 16-byte

@@ -296,6 +296,62 @@ def test_full_qkv_shape_sampled():
     _sampled_parity(Q4, 160, 12288, 4096, 1)
 
 
+def test_config1_qkv_three_segments_and_o_sampled():
+    """The attention-projection workload exactly as named: a 160-token canvas
+    (32 prompt + 128 masked), one quantized activation shared by Q, K and V through
+    dllm_qkv_qgemm with three 4096 x 4096 Q4_K segments, then O (4096 x 4096, Q4_K) on a
+    second quantized activation; sampled output columns of every projection against the
+    oracle."""
+    M, K, N = 160, 4096, 4096
+    xa, xo = synth.activations(M, K, 1, 0), synth.activations(M, K, 1, 1)
+    wq, wk, wv, wo = (synth.weights(Q4, N, K, 1, i) for i in range(4))
+    dq, dk, dv, do = (dllm.repack(Q4, w, N, K) for w in (wq, wk, wv, wo))
+    act, act_o = gu.Act(xa), gu.Act(xo)
+    outs = [torch.full((M, N), float("nan"), device="cuda") for _ in range(3)]
+    wsb = dllm.dllm_qgemm_workspace_bytes(Q4, 3 * N, K, M)
+    work = dllm.alloc_workspace(max(wsb, 256))
+    dllm.dllm_qkv_qgemm(dq, dk, dv, Q4, N, N, K, act.q, act.scale, act.sums, M, outs[0], N, outs[1], outs[2], N,
+                        work, wsb)
+    o_out = gu.gemm(do, Q4, N, K, act_o).cpu().numpy()
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    qa, sa, _ = oracle.quantize_act(xa)
+    qo, so, _ = oracle.quantize_act(xo)
+    rng = np.random.default_rng(11)
+    cases = [(w, o.cpu().numpy(), qa, sa) for w, o in zip((wq, wk, wv), outs)] + [(wo, o_out, qo, so)]
+    for w, out, q_, s_ in cases:
+        for n0 in sorted({0, N - 64, int(rng.integers(0, N - 64))}):
+            _, ref, T = oracle.qgemm(Q4, w, N, K, q_, s_, n0=n0, n1=n0 + 64)
+            ok, worst = gu.tol_ok(out[:, n0:n0 + 64], ref, T)
+            assert ok, (n0, worst)
+
+
+@pytest.mark.parametrize("K", [4096, 3584])
+@pytest.mark.parametrize("dd", ["random", "min_dominant"])
+def test_min_term_worst_case_long_k(K, dd):
+    """The Q4_K min term at its largest over a whole LLaDA-8B / Dream-7B K range: every
+    6-bit scale and min 63, every quant 15, and each canvas row constant (+-3.0, so every
+    code is +-127 and every per-32 sum is 32 * 127 with one sign per row).  The min-term
+    accumulator then grows monotonically over K/32 sub-block steps (128 at K = 4096, 112
+    at K = 3584), against a d-term of the opposite sign.  min_dominant sets d = 1e-3 and
+    dmin = 1e-2 in every block, so that the two terms nearly cancel and the tolerance is
+    set by 1e-6 * sum|terms|."""
+    M, N = 16, 256
+    w = synth.q4k_weights(N, K, 35).copy()
+    w[..., 4:144] = 0xFF
+    if dd == "min_dominant":
+        w[..., 0:2] = np.frombuffer(np.float16(1e-3).tobytes(), np.uint8)
+        w[..., 2:4] = np.frombuffer(np.float16(1e-2).tobytes(), np.uint8)
+    x = np.full((M, K), 3.0, np.float32)
+    x[::2] *= -1
+    wd = dllm.repack(Q4, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, Q4, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    _, ref, T = oracle.qgemm(Q4, w, N, K, oq, os_)
+    ok, worst = gu.tol_ok(out, ref, T)
+    assert ok, worst
+
+
 def test_full_ffn_shapes_sampled():
     _sampled_parity(Q4, 256, 12288, 4096, 2, width=32)
     _sampled_parity(Q6, 160, 4096, 12288, 2, width=32)

@@ -1,8 +1,8 @@
 """dllm_qgemm_noalloc: the GEMM with its scratch in the library's fixed device array
 instead of a caller workspace.  Each case calls it twice in a row through the C-ABI
-and compares both results with dllm_qgemm on a caller-owned workspace, within the
-parity tolerance |a - b| <= max(1e-5 |b|, 1e-6 T) (T from the oracle where it runs,
-else the largest |b| of the row).  The file is named to be collected last, so the
+and compares both results with dllm_qgemm on a caller-owned workspace and with the
+oracle (in full, or on sampled column ranges for the full-size shapes), within the
+parity tolerance |a - b| <= max(1e-5 |b|, 1e-6 T), T the oracle's sum of |terms|.  The file is named to be collected last, so the
 cases also run after every other GPU test has used the library in the same process.
 """
 import numpy as np
@@ -98,28 +98,59 @@ def test_noalloc_matches_workspace_entry(qtype, M, N, K, rows):
         _close(got, ref64, T)
 
 
+def _sampled_oracle(out, w, qtype, N, K, oq, os_, rows, width, seed):
+    """Column ranges (first, last, random) of `out` against the oracle, with its T."""
+    rng = np.random.default_rng(seed)
+    for n0 in sorted({0, N - width, int(rng.integers(0, N - width))}):
+        _, ref64, T = oracle.qgemm(qtype, w, N, K, oq, os_, rows=rows, n0=n0, n1=n0 + width)
+        _close(out[:, n0:n0 + width], ref64, T)
+
+
 @pytest.mark.gpu
 def test_noalloc_output_projection_full_vocab():
     """LLaDA-8B output projection (126464 x 4096, Q6_K) on 32 requested rows of a
-    128-row canvas: the gathered rows live in the fixed scratch."""
+    128-row canvas: the gathered rows live in the fixed scratch.  Both calls are
+    checked against the existing entry point in full and against the oracle on sampled
+    column ranges."""
     if not torch.cuda.is_available():
         pytest.fail("GPU test run without a CUDA device")
     qtype, N, K, M = Q6, 126464, 4096, 128
-    wd = dllm.repack(qtype, synth.device_weights(qtype, N, K, 93), N, K)
+    wg = synth.device_weights(qtype, N, K, 93)
+    wd = dllm.repack(qtype, wg, N, K)
+    w_host = wg.cpu().numpy().reshape(N, K // 256, 210)
+    del wg
     x = synth.device_activations(M, K, 93)
-    q, s, u = dllm.alloc_act(M, K)
-    dllm.dllm_quantize_act(x, M, K, K, q, s, u)
-
-    class _A:
-        pass
-    act = _A()
-    act.M, act.q, act.scale, act.sums = M, q, s, u
+    act = gu.Act(x.cpu().numpy())
     rows = synth.block_rows(M, 32, 93)
     rows_t = torch.tensor(np.asarray(rows, np.int32), device="cuda")
     ref = _existing(wd, qtype, N, K, act, rows_t, 32, 32)
-    T = np.repeat(np.max(np.abs(ref), axis=1, keepdims=True), N, axis=1).astype(np.float64)
+    oq, os_, _ = act.host()
     for got in _noalloc_twice(wd, qtype, N, K, act, rows_t, 32, 32):
-        _close(got, ref, T)
+        assert np.array_equal(got, ref)  # same plan and arithmetic: the same bits
+        _sampled_oracle(got, w_host, qtype, N, K, oq, os_, rows, 128, 93)
+
+
+@pytest.mark.gpu
+def test_noalloc_tail_split_plan():
+    """A weight whose 192 tiles leave 44 over after one round on 148 SMs: the tail
+    split (44 tiles cut into 148 K-pieces) keeps its arrival counters and K-piece
+    partials in the fixed scratch, which the entry point clears before each call."""
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test run without a CUDA device")
+    qtype, M, N, K = Q4, 128, 24576, 4096
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = dllm.dllm_debug_plan(N // 128, K, M, 0, sms)
+    if sms == 148:
+        assert plan["tail_k"] > 0, plan
+    assert plan["bytes"] <= dllm.DLLM_NOALLOC_SCRATCH_BYTES
+    w, x = gu.make_case(qtype, M, N, K, 94)
+    wd = dllm.repack(qtype, w, N, K)
+    act = gu.Act(x)
+    ref = _existing(wd, qtype, N, K, act, None, 0, M)
+    oq, os_, _ = act.host()
+    for got in _noalloc_twice(wd, qtype, N, K, act, None, 0, M):
+        assert np.array_equal(got, ref)
+        _sampled_oracle(got, w, qtype, N, K, oq, os_, None, 64, 94)
 
 
 @pytest.mark.gpu

@@ -160,6 +160,11 @@ int run_gemm(GemmArgs& a, cudaStream_t s) {
         if (cudaFuncSetAttribute(qgemm_kernel<QT, DBG, TAIL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return DLLM_ERR_CUDA;
+        // the warpgroups' setmaxnreg split must fit in the registers the CTA launches with
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, qgemm_kernel<QT, DBG, TAIL>) != cudaSuccess) return DLLM_ERR_CUDA;
+        if (fa.numRegs * GEMM_THREADS < REG_SPLIT_TOTAL || fa.maxThreadsPerBlock < GEMM_THREADS)
+            return DLLM_ERR_UNSUPPORTED;
         g_attr_done[dev][slot] = true;
     }
     const int64_t units = a.n_units;

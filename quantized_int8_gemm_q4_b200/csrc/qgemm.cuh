@@ -34,7 +34,7 @@
 // the running sum of magnitudes (about 2^-17 at K = 4096); both bounds are relative to
 // the min term's own sum of |terms|, a part of the 1e-6 * sum|terms| tolerance.
 //
-// Pipeline (16 warps, one CTA per SM, persistent over work units).  Per super-block
+// Pipeline (20 warps, one CTA per SM, persistent over work units).  Per super-block
 // the MMAs run plane-major: the 8 K-steps of plane 0 into accumulator P0, then the 8
 // of plane 1 into P1, then (Q4_K) the 3 min-term MMAs.  Every MMA covers all of the
 // unit's tokens (N <= 128; at N = 128 one int8 MMA takes ~64 cycles, the pipe's full
@@ -44,14 +44,15 @@
 //               ring.  Weights are never written by the kernels this library chains
 //               with programmatic dependent launch, so these copies start before the
 //               dependency wait.
-//   warp 1      MMA issuer (one thread) and tensor-memory allocation
+//   warp 1      MMA issuer of plane 0 (one thread) and tensor-memory allocation
 //   warp 2      activation producer: bulk copies of activation tiles (int8 codes,
 //               scales, scaled sums), after the dependency wait
-//   warp 3      idle
-//   warps 4-7   unpack: thread = weight row; per quarter super-block (two K-steps)
-//               build both weight planes into a tensor-memory ring (the A operand),
-//               the min-term A operand (Q4_K) into shared memory, and the f32 d
-//   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each on 64 of the
+//   warp 3      MMA issuer of plane 1 and of the min term (one thread)
+//   warps 4-11  unpack, two groups of four: thread = weight row; each group builds
+//               one quarter super-block (two K-steps, both weight planes) of every
+//               half super-block into a tensor-memory ring (the A operand); group 0
+//               also writes the min-term A operand (Q4_K) to shared memory and the f32 d
+//   warps 12-19 epilogue: two warps per tensor-memory lane quadrant, each on 64 of the
 //               token columns
 //
 // A work unit is (128 weight rows, up to 128 canvas rows, one K-chunk).  The number
@@ -65,27 +66,31 @@ namespace dllm {
 
 constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float MAGIC = 12582912.0f;
-constexpr int GEMM_THREADS = 512;
+constexpr int GEMM_THREADS = 640;
 constexpr int UNIT_TOKENS = 128;
 constexpr int EPI_COLS = 64;                       // token columns per epilogue thread
 constexpr int MAX_KC = 16;                         // K-chunks per tile, at most
 constexpr int S_SLOTS = 4;                         // d ring (unpack -> epilogue)
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
-// Registers per thread of each warpgroup after setmaxnreg: producers and issuer,
-// unpack, and the two epilogue warpgroups.  setmaxnreg.inc draws on the registers the
-// CTA was launched with (512 threads x 128), so the split must not exceed them, or the
-// increasing warps would wait for registers that never come free.
-constexpr int REG_CTRL = 40, REG_UNPACK = 56, REG_EPI = 208;
-static_assert(128 * REG_CTRL + 128 * REG_UNPACK + 256 * REG_EPI <= 65536, "register split over the launch budget");
+// Registers per thread of each warpgroup after setmaxnreg: producers and issuers (one
+// warpgroup), unpack (two) and epilogue (two).  setmaxnreg.inc draws on the registers the
+// CTA was launched with (640 threads x the kernel's register count), so the split must
+// not exceed them, or the increasing warps would wait for registers that never come
+// free.  REG_LAUNCH_MIN is the launch count the split assumes; the host checks the
+// compiled kernel's count against it before the first launch.
+constexpr int REG_CTRL = 48, REG_UNPACK = 64, REG_EPI = 152;
+constexpr int REG_SPLIT_TOTAL = 128 * REG_CTRL + 256 * REG_UNPACK + 256 * REG_EPI;
+constexpr int REG_LAUNCH_MIN = 96;
+static_assert(REG_SPLIT_TOTAL <= 640 * REG_LAUNCH_MIN && 640 * REG_LAUNCH_MIN <= 65536, "register split over the launch budget");
 static_assert(REG_CTRL % 8 == 0 && REG_UNPACK % 8 == 0 && REG_EPI % 8 == 0 && REG_CTRL >= 24, "setmaxnreg counts");
 
 // Activation "sums" operand of one super-block: per 8-row group 512 bytes =
 // [hi j0-3 | hi j4-7 | lo j0-3 | lo j4-7] x [8 rows x 16 bytes].
 constexpr int SUMS_GROUP = 512;
 
-// Tensor-memory columns: the A ring (A_SLOTS quarter super-blocks; a quarter is two
-// K-steps of 16 columns, [plane 0: 8 | plane 1: 8]), then the plane accumulators P0
-// and P1 (128 token columns each), then (Q4_K) the f32 min-term accumulator.
+// Tensor-memory columns: the A ring (A_SLOTS half super-blocks; a half is four K-steps
+// of 16 columns, [plane 0: 8 | plane 1: 8]), then the plane accumulators P0 and P1 (128
+// token columns each), then (Q4_K) the f32 min-term accumulator.
 constexpr uint32_t TM_COLS = 512;
 constexpr uint32_t TM_A = 0;
 
@@ -102,8 +107,8 @@ struct GemmCfg<12> {  // Q4_K
     static constexpr int B_STAGE = B_Q + B_SUMS + UNIT_TOKENS * 4;
     static constexpr int MINA = 2 * 4096;  // -dmin*m_j as [hi | lo], canonical K-major 128 rows x 32 B
     static constexpr int MINA_BUFS = 2;
-    static constexpr int A_SLOTS = 4;      // one super-block
-    static constexpr uint32_t TM_P0 = TM_A + 32 * A_SLOTS;
+    static constexpr int A_SLOTS = 2;      // one super-block
+    static constexpr uint32_t TM_P0 = TM_A + 64 * A_SLOTS;
     static constexpr uint32_t TM_P1 = TM_P0 + UNIT_TOKENS;
     static constexpr uint32_t TM_MIN = TM_P1 + UNIT_TOKENS;
     static constexpr uint32_t TM_END = TM_MIN + UNIT_TOKENS;
@@ -119,8 +124,8 @@ struct GemmCfg<14> {  // Q6_K
     static constexpr int B_STAGE = B_Q + B_SUMS + UNIT_TOKENS * 4;
     static constexpr int MINA = 0;
     static constexpr int MINA_BUFS = 0;
-    static constexpr int A_SLOTS = 8;      // two super-blocks: the unpack runs one ahead
-    static constexpr uint32_t TM_P0 = TM_A + 32 * A_SLOTS;
+    static constexpr int A_SLOTS = 4;      // two super-blocks: the unpack runs one ahead
+    static constexpr uint32_t TM_P0 = TM_A + 64 * A_SLOTS;
     static constexpr uint32_t TM_P1 = TM_P0 + UNIT_TOKENS;
     static constexpr uint32_t TM_MIN = 0;
     static constexpr uint32_t TM_END = TM_P1 + UNIT_TOKENS;
@@ -171,7 +176,7 @@ struct GemmArgs {
 struct GemmShared {
     uint64_t w_full[4], w_empty[4];
     uint64_t b_full[3], b_empty[3];
-    uint64_t a_full[8], a_empty[8];   // A ring slots: quarter super-blocks
+    uint64_t a_full[4], a_empty[4];   // A ring slots: half super-blocks
     uint64_t p_full[2], p_empty[2];   // plane accumulators P0, P1
     uint64_t m_full[2], m_empty[2];   // min-term A operand buffers (Q4_K)
     uint64_t min_full, min_empty;     // min-term accumulator (Q4_K), once per unit
@@ -336,17 +341,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     const int64_t n_units = args.n_units;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 128); }
-        // an activation stage is released by the issuer's commit (its MMAs are done)
-        // and by the 256 epilogue threads (the scales are read)
-        for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 257); }
-        for (int i = 0; i < C::A_SLOTS; i++) { mbar_init(&sh.a_full[i], 128); mbar_init(&sh.a_empty[i], 1); }
+        for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 256); }
+        // an activation stage is released by a commit from each issuer (their MMAs are
+        // done) and by the 256 epilogue threads (the scales are read)
+        for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 258); }
+        for (int i = 0; i < C::A_SLOTS; i++) { mbar_init(&sh.a_full[i], 256); mbar_init(&sh.a_empty[i], 2); }
         for (int i = 0; i < 2; i++) { mbar_init(&sh.p_full[i], 1); mbar_init(&sh.p_empty[i], 256); }
         for (int i = 0; i < 2; i++) { mbar_init(&sh.m_full[i], 128); mbar_init(&sh.m_empty[i], 1); }
         mbar_init(&sh.min_full, 1);
         mbar_init(&sh.min_empty, 256);
         for (int i = 0; i < S_SLOTS; i++) { mbar_init(&sh.s_full[i], 128); mbar_init(&sh.s_empty[i], 256); }
-        mbar_init(&sh.final_bar, 1);
+        mbar_init(&sh.final_bar, 2);
         mbar_init(&sh.epi_bar, 256);
         sh.abort_flag = 0;
         fence_mbar_init();
@@ -368,22 +373,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         setmaxnreg_dec<REG_CTRL>();
         if (warp == 0 || warp == 2) {
             // ======================================================== producers
-            // warp 0: weight tiles; warp 2: activation tiles.  Stages with a copy issued
-            // (bit i) and the phase that copy completes (bit i), for the abort drain.
+            // warp 0: weight tiles; warp 2: activation tiles.  A thread keeps only one bulk
+            // copy in flight at a time (its copies run one after another, each costing a
+            // full memory latency), so every ring stage has lanes of its own: weight
+            // stage i is lane i; activation stage i is lanes 3i (codes; it also arms the
+            // barrier with the stage's byte count), 3i+1 (scaled sums, Q4_K) and 3i+2
+            // (scales).  The lanes of one stage agree on each wait, so they issue all of a
+            // stage's copies or none.
             const bool wprod = warp == 0;
-            uint32_t st = 0, ph = 0, iss = 0, php = 0;
-            const uint64_t pol = wprod ? policy_evict_first() : policy_evict_last();
-            const int64_t n_prod = args.stall ? 0 : n_units;
             const int NST = wprod ? C::W_STAGES : C::B_STAGES;
+            const int st = wprod ? lane : lane / 3;
+            const int part = wprod ? 0 : lane % 3;
+            const bool active = st < NST && (wprod || C::B_SUMS || part != 1);
+            const uint32_t smask = wprod ? 0u : (C::B_SUMS ? 7u : 5u) << (3 * st);
             uint64_t* full = wprod ? sh.w_full : sh.b_full;
             uint64_t* empty = wprod ? sh.w_empty : sh.b_empty;
+            uint32_t ph = 0;
+            bool inflight = false;  // a copy of this lane's stage has been issued and not waited for
             if (!wprod) pdl_wait();
-            for (int64_t u = blockIdx.x; u < n_prod; u += gridDim.x) {
-                const Unit un = unit_of<TAIL>(args, u);
-                const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
-                for (int s = un.sb0; s < un.sb1; s++) {
-                    if (!wait_bar_warp(sh, &empty[st], ph ^ 1)) goto prod_done;
-                    if (lane == 0) {
+            if (active) {
+                const uint64_t pol = wprod ? policy_evict_first() : policy_evict_last();
+                const int64_t n_prod = args.stall ? 0 : n_units;
+                uint32_t g = 0;  // super-blocks of this CTA so far
+                for (int64_t u = blockIdx.x; u < n_prod; u += gridDim.x) {
+                    const Unit un = unit_of<TAIL>(args, u);
+                    const uint8_t* wt = args.seg[un.seg].w + (size_t)un.tile * args.nsb * C::TILE;
+                    for (int s = un.sb0; s < un.sb1; s++, g++) {
+                        if ((int)(g % NST) != st) continue;
+                        bool ok = wait_bar(sh, &empty[st], ph ^ 1);
+                        if (!wprod) ok = __all_sync(smask, ok);
+                        if (!ok) goto prod_done;
                         if (wprod) {
                             mbar_arrive_expect_tx(&full[st], C::TILE);
                             bulk_g2s_hint(w_stage + st * C::TILE, wt + (size_t)s * C::TILE, C::TILE, &full[st], pol);
@@ -392,28 +411,35 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                             const int64_t t0 = un.m0;
                             const uint32_t ntok = (uint32_t)un.len;
                             const uint32_t sums_bytes = C::B_SUMS ? ntok / 8 * SUMS_GROUP : 0;
-                            mbar_arrive_expect_tx(&full[st], ntok * 256 + sums_bytes + ntok * 4);
-                            bulk_g2s_hint(bs, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256, &full[st], pol);
-                            if (C::B_SUMS)
+                            if (part == 0) mbar_arrive_expect_tx(&full[st], ntok * 256 + sums_bytes + ntok * 4);
+                            __syncwarp(smask);  // the stage's byte count is armed before any of its copies lands
+                            if (part == 0)
+                                bulk_g2s_hint(bs, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256, &full[st], pol);
+                            else if (part == 1)
                                 bulk_g2s_hint(bs + C::B_Q, args.sums + ((size_t)s * args.Mp + t0) / 8 * SUMS_GROUP,
                                               sums_bytes, &full[st], pol);
-                            bulk_g2s_hint(bs + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
-                                          &full[st], pol);
+                            else
+                                bulk_g2s_hint(bs + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
+                                              &full[st], pol);
                         }
+                        inflight = true;
+                        ph ^= 1;
                     }
-                    iss |= 1u << st;
-                    php = (php & ~(1u << st)) | (ph << st);
-                    if (++st == (uint32_t)NST) { st = 0; ph ^= 1; }
                 }
             }
         prod_done:
-            if (sh.abort_flag) {  // never leave with bulk copies in flight into this CTA's shared memory
-                for (int i = 0; i < NST; i++)
-                    if ((iss >> i) & 1u) (void)drain_bar(&full[i], (php >> i) & 1u);
-            }
-        } else if (warp == 1) {
-            // ======================================================== MMA issuer
+            // never leave with bulk copies in flight into this CTA's shared memory: the
+            // stage's last phase completes once every copy of it has landed
+            if (sh.abort_flag && inflight && (wprod || part == 0)) (void)drain_bar(&full[st], ph ^ 1);
+        } else {
+            // ======================================================== MMA issuers
+            // One thread issues a tcgen05 instruction only every ~50-100 cycles, about
+            // the time an N = 128 int8 MMA takes, so the work is split between two warps:
+            // warp 1 issues plane 0 into P0; warp 3 issues plane 1 into P1 and the
+            // min-term MMAs.  Both read the same A-ring halves and activation stage, so
+            // each of those is released by a commit from each issuer.
             const bool leader = lane == 0;
+            const int plane = warp == 1 ? 0 : 1;
             constexpr uint32_t ASG = QT == 12 ? 0 : 1;  // plane operand type: u8 (Q4_K), s8 (Q6_K)
             uint32_t sbc = 0, uc = 0;
             for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
@@ -423,83 +449,75 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                 for (int s = un.sb0; s < un.sb1; s++, sbc++) {
                     const uint32_t bst = sbc % C::B_STAGES;
                     if (!wait_bar_warp(sh, &sh.b_full[bst], (sbc / C::B_STAGES) & 1)) goto mma_done;
+                    // this plane's accumulator has been drained and preset by the epilogue
+                    if (!wait_bar_warp(sh, &sh.p_empty[plane], sbc & 1)) goto mma_done;
                     const uint32_t stg = smem_u32(b_stage + bst * C::B_STAGE);
                     const uint64_t bdesc = sdesc_kmajor_noswz(stg, 128, 2048);
-                    // ---- plane 0: waits for its accumulator to be drained and preset, and
-                    // for each quarter of the A ring to be published
-                    if (!wait_bar_warp(sh, &sh.p_empty[0], sbc & 1)) goto mma_done;
 #pragma unroll 1
-                    for (int q = 0; q < 4; q++) {
-                        const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
-                        if (!wait_bar_warp(sh, &sh.a_full[sl], (qc / C::A_SLOTS) & 1)) goto mma_done;
+                    for (int hh = 0; hh < 2; hh++) {
+                        const uint32_t hc = 2 * sbc + hh, sl = hc % C::A_SLOTS;
+                        if (!wait_bar_warp(sh, &sh.a_full[sl], (hc / C::A_SLOTS) & 1)) goto mma_done;
                         tc_fence_after();
                         if (leader) {
 #pragma unroll
-                            for (int kk = 0; kk < 2; kk++)
-                                mma_i8_ts(tmem + C::TM_P0, tmem + TM_A + 32 * sl + 16 * kk,
+                            for (int kq = 0; kq < 4; kq++) {
+                                const int q = 2 * hh + (kq >> 1), kk = kq & 1;
+                                mma_i8_ts(tmem + (plane ? C::TM_P1 : C::TM_P0), tmem + TM_A + 64 * sl + 16 * kq + 8 * plane,
                                           bdesc + 16 * kstep_of<QT>(q, kk), id, 1u);
-                        }
-                        __syncwarp();
-                    }
-                    if (leader) tc_commit(&sh.p_full[0]);
-                    __syncwarp();
-                    // ---- plane 1; each quarter slot is released once its plane-1 MMAs finish
-                    if (!wait_bar_warp(sh, &sh.p_empty[1], sbc & 1)) goto mma_done;
-                    tc_fence_after();
-                    if (leader) {
-#pragma unroll 1
-                        for (int q = 0; q < 4; q++) {
-                            const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
-#pragma unroll
-                            for (int kk = 0; kk < 2; kk++)
-                                mma_i8_ts(tmem + C::TM_P1, tmem + TM_A + 32 * sl + 16 * kk + 8,
-                                          bdesc + 16 * kstep_of<QT>(q, kk), id, 1u);
+                            }
                             tc_commit(&sh.a_empty[sl]);
                         }
-                        tc_commit(&sh.p_full[1]);
+                        __syncwarp();
                     }
+                    if (leader) tc_commit(&sh.p_full[plane]);
                     __syncwarp();
                     if constexpr (C::MIN) {
-                        // ---- min term: (-dmin m_j) x (da sum32_j), three tf32 products
-                        const uint32_t mb = sbc & 1;
-                        if (!wait_bar_warp(sh, &sh.m_full[mb], (sbc >> 1) & 1)) goto mma_done;
-                        // a unit's first min-term MMA overwrites the accumulator: the previous
-                        // unit's epilogue must have read it out
-                        if (s == un.sb0 && !wait_bar_warp(sh, &sh.min_empty, (uc & 1) ^ 1)) goto mma_done;
-                        tc_fence_after();
-                        if (leader) {
-                            const uint32_t idm = idesc_tf32(128, (int)ntok);
-                            const uint32_t ma = smem_u32(mina + mb * C::MINA);
-                            const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
-                            const uint64_t a_lo = sdesc_kmajor_noswz(ma + 4096, 128, 256);
-                            const uint64_t b_hi = sdesc_kmajor_noswz(stg + C::B_Q, 128, SUMS_GROUP);
-                            const uint64_t b_lo = sdesc_kmajor_noswz(stg + C::B_Q + 256, 128, SUMS_GROUP);
-                            mma_tf32_ss(tmem + C::TM_MIN, a_hi, b_hi, idm, s > un.sb0 ? 1u : 0u);
-                            mma_tf32_ss(tmem + C::TM_MIN, a_hi, b_lo, idm, 1u);
-                            mma_tf32_ss(tmem + C::TM_MIN, a_lo, b_hi, idm, 1u);
-                            tc_commit(&sh.m_empty[mb]);
-                            if (s == un.sb1 - 1) tc_commit(&sh.min_full);
+                        if (plane == 1) {
+                            // ---- min term: (-dmin m_j) x (da sum32_j), three tf32 products
+                            const uint32_t mb = sbc & 1;
+                            if (!wait_bar_warp(sh, &sh.m_full[mb], (sbc >> 1) & 1)) goto mma_done;
+                            // a unit's first min-term MMA overwrites the accumulator: the
+                            // previous unit's epilogue must have read it out
+                            if (s == un.sb0 && !wait_bar_warp(sh, &sh.min_empty, (uc & 1) ^ 1)) goto mma_done;
+                            tc_fence_after();
+                            if (leader) {
+                                const uint32_t idm = idesc_tf32(128, (int)ntok);
+                                const uint32_t ma = smem_u32(mina + mb * C::MINA);
+                                const uint64_t a_hi = sdesc_kmajor_noswz(ma, 128, 256);
+                                const uint64_t a_lo = sdesc_kmajor_noswz(ma + 4096, 128, 256);
+                                const uint64_t b_hi = sdesc_kmajor_noswz(stg + C::B_Q, 128, SUMS_GROUP);
+                                const uint64_t b_lo = sdesc_kmajor_noswz(stg + C::B_Q + 256, 128, SUMS_GROUP);
+                                mma_tf32_ss(tmem + C::TM_MIN, a_hi, b_hi, idm, s > un.sb0 ? 1u : 0u);
+                                mma_tf32_ss(tmem + C::TM_MIN, a_hi, b_lo, idm, 1u);
+                                mma_tf32_ss(tmem + C::TM_MIN, a_lo, b_hi, idm, 1u);
+                                tc_commit(&sh.m_empty[mb]);
+                                if (s == un.sb1 - 1) tc_commit(&sh.min_full);
+                            }
+                            __syncwarp();
                         }
-                        __syncwarp();
                     }
                     if (leader) tc_commit(&sh.b_empty[bst]);
                     __syncwarp();
                 }
             }
         mma_done:
-            // every MMA this warp issued has completed before tensor memory is freed
+            // every MMA this warp issued has completed before tensor memory is freed (the
+            // barrier takes one commit from each issuer)
             if (leader) tc_commit(&sh.final_bar);
             __syncwarp();
             (void)drain_bar(&sh.final_bar, 0);
             __syncwarp();
         }
-    } else if (warp < 8) {
+    } else if (warp < 12) {
         setmaxnreg_dec<REG_UNPACK>();
         // ============================================================ unpack
-        // Per super-block: decode this row's scales, hand d to the epilogue and (Q4_K)
-        // the min-term A operand to the issuer, then build the two weight planes of
-        // each quarter (two K-steps) and publish it as soon as its ring slot is free.
+        // Two groups of four warps (one warp per lane quadrant each).  Per super-block
+        // both decode this row's scales; group 0 hands d to the epilogue and (Q4_K) the
+        // min-term A operand to the issuer.  In each half super-block, group g builds the
+        // two weight planes of quarter 2*half + g (two K-steps); the half is published
+        // once both groups have stored theirs.
         const int quad = warp & 3;
+        const int grp = (warp - 4) >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         uint32_t ws = 0, wph = 0, ss = 0, sph = 0, sbc = 0;
@@ -526,11 +544,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         nmin[j] = -dmin * (float)m_lo;
                         nmin[j + 4] = -dmin * (float)m_hi;
                     }
-                    if (!wait_bar_warp(sh, &sh.s_empty[ss], sph ^ 1)) goto unpack_done;
-                    sh.dd[ss][row] = d;
-                    mbar_arrive(&sh.s_full[ss]);
-                    if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
-                    {
+                    if (grp == 0) {
+                        if (!wait_bar_warp(sh, &sh.s_empty[ss], sph ^ 1)) goto unpack_done;
+                        sh.dd[ss][row] = d;
+                        mbar_arrive(&sh.s_full[ss]);
+                        if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
                         // -dmin*m_j as tf32 hi + lo: row `row` of the canonical K-major layout
                         // (8-row groups of 256 bytes, two 16-byte K chunks)
                         const uint32_t mb = sbc & 1;
@@ -547,9 +565,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         mbar_arrive(&sh.m_full[mb]);
                     }
 #pragma unroll 1
-                    for (int q = 0; q < 4; q++) {
-                        const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
-                        if (!wait_bar_warp(sh, &sh.a_empty[sl], ((qc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
+                    for (int hh = 0; hh < 2; hh++) {
+                        const int q = 2 * hh + grp;
+                        const uint32_t hc = 2 * sbc + hh, sl = hc % C::A_SLOTS;
+                        if (!wait_bar_warp(sh, &sh.a_empty[sl], ((hc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
                         // 32-byte quant chunk q: sub-block 2q in the low nibbles, 2q+1 in the high
                         const uint4 p0 = *reinterpret_cast<const uint4*>(tl + ((2 * q) * TROWS + row) * 16);
                         const uint4 p1 = *reinterpret_cast<const uint4*>(tl + ((2 * q + 1) * TROWS + row) * 16);
@@ -567,7 +586,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 v[i] = nib * lo3;
                                 v[8 + i] = nib * hi3;
                             }
-                            tmem_st16(tmem + lane_off + TM_A + 32 * sl + 16 * kk, v);
+                            tmem_st16(tmem + lane_off + TM_A + 64 * sl + 32 * grp + 16 * kk, v);
                         }
                         tmem_wait_st();
                         tc_fence_before();
@@ -578,14 +597,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     const uint32_t scw[4] = {scv.x, scv.y, scv.z, scv.w};
                     const float d = __half2float(
                         __ushort_as_half(*reinterpret_cast<const unsigned short*>(tl + Q6K_OFF_D + 2 * row)));
-                    if (!wait_bar_warp(sh, &sh.s_empty[ss], sph ^ 1)) goto unpack_done;
-                    sh.dd[ss][row] = d;
-                    mbar_arrive(&sh.s_full[ss]);
-                    if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
+                    if (grp == 0) {
+                        if (!wait_bar_warp(sh, &sh.s_empty[ss], sph ^ 1)) goto unpack_done;
+                        sh.dd[ss][row] = d;
+                        mbar_arrive(&sh.s_full[ss]);
+                        if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
+                    }
 #pragma unroll 1
-                    for (int q = 0; q < 4; q++) {
-                        const uint32_t qc = 4 * sbc + q, sl = qc % C::A_SLOTS;
-                        if (!wait_bar_warp(sh, &sh.a_empty[sl], ((qc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
+                    for (int hh = 0; hh < 2; hh++) {
+                        const int q = 2 * hh + grp;
+                        const uint32_t hc = 2 * sbc + hh, sl = hc % C::A_SLOTS;
+                        if (!wait_bar_warp(sh, &sh.a_empty[sl], ((hc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
                         // K-steps 4h + g and 4h + g + 2 share their low-bit bytes (low and high
                         // nibbles) and the half's high-bit bytes
                         const int h = q >> 1, g = q & 1;
@@ -621,7 +643,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 v[i] = __byte_perm(pa, pb, 0x6420) ^ 0x80808080u;
                                 v[8 + i] = __byte_perm(pa, pb, 0x7531) ^ 0x80808080u;
                             }
-                            tmem_st16(tmem + lane_off + TM_A + 32 * sl + 16 * kk, v);
+                            tmem_st16(tmem + lane_off + TM_A + 64 * sl + 32 * grp + 16 * kk, v);
                         }
                         tmem_wait_st();
                         tc_fence_before();
@@ -637,9 +659,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         setmaxnreg_inc<REG_EPI>();
         // ============================================================ epilogue
         const int quad = warp & 3;
-        const int half = (warp - 8) >> 2;
+        const int half = (warp - 12) >> 2;
         const int row = quad * 32 + lane;
-        const int etid = threadIdx.x - 256;  // 0..255
+        const int etid = threadIdx.x - 384;  // 0..255
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t col0 = (uint32_t)(half * EPI_COLS);
         // initial preset of both plane accumulators (this warp's lanes and columns)
@@ -650,9 +672,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         mbar_arrive(&sh.p_empty[0]);
         mbar_arrive(&sh.p_empty[1]);
         pdl_wait();  // outputs, partials and counters may be in use by earlier work
+        // plane 1 carries weight 8 (Q4_K) or 256 (Q6_K): kP * (M + P1) - kP * M = kP * P1
         const float2 kP = QT == 12 ? make_float2(8.0f, 8.0f) : make_float2(256.0f, 256.0f);
-        const float2 mP = QT == 12 ? make_float2(-9.0f * MAGIC, -9.0f * MAGIC)
-                                   : make_float2(-257.0f * MAGIC, -257.0f * MAGIC);
+        const float2 nkM = QT == 12 ? make_float2(-8.0f * MAGIC, -8.0f * MAGIC)
+                                    : make_float2(-256.0f * MAGIC, -256.0f * MAGIC);
+        const float2 nM = make_float2(-MAGIC, -MAGIC);
         uint32_t ss = 0, sph = 0, sbc = 0, uc = 0, epi_ph = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, uc++) {
             int sb_first, sb_end, ulen;
@@ -668,37 +692,35 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             for (int j = 0; j < EPI_COLS / 2; j++) acc[j] = make_float2(0.0f, 0.0f);
             for (int s = sb_first; s < sb_end; s++, sbc++) {
                 const uint32_t bst = sbc % C::B_STAGES;
-                // ---- plane 0: read, preset, release; keep the raw f32 bits 1.5*2^23 + P0
-                uint32_t x0[EPI_COLS];
-                if (!wait_bar_warp(sh, &sh.p_full[0], sbc & 1)) goto epi_done;
-                tc_fence_after();
-                if (live) {
-                    load_cols64(tmem + lane_off + C::TM_P0 + col0, x0);
-                    tmem_wait_ld();
-                    preset_cols64(tmem + lane_off + C::TM_P0 + col0);
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                mbar_arrive(&sh.p_empty[0]);
                 if (!wait_bar_warp(sh, &sh.s_full[ss], sph)) goto epi_done;
                 const float dv = sh.dd[ss][row];
                 mbar_arrive(&sh.s_empty[ss]);
                 if (++ss == S_SLOTS) { ss = 0; sph ^= 1; }
                 const float2 d2 = make_float2(dv, dv);
-                // ---- plane 1, in four chunks of 16 columns
-                if (!wait_bar_warp(sh, &sh.p_full[1], sbc & 1)) goto epi_done;
                 if (!wait_bar_warp(sh, &sh.b_full[bst], (sbc / C::B_STAGES) & 1)) goto epi_done;
-                tc_fence_after();
-                if (live) {
-                    const float* da =
-                        reinterpret_cast<const float*>(b_stage + bst * C::B_STAGE + C::B_Q + C::B_SUMS) + col0;
-#pragma unroll
-                    for (int c = 0; c < 4; c++) {
-                        uint32_t x1[16];
-                        tmem_ld16(tmem + lane_off + C::TM_P1 + col0 + 16 * c, x1);
+                const float* da = reinterpret_cast<const float*>(b_stage + bst * C::B_STAGE + C::B_Q + C::B_SUMS) + col0;
+                if constexpr (DBG) {
+                    // the integer S of every element: both planes, exactly
+                    uint32_t x0[EPI_COLS];
+                    if (!wait_bar_warp(sh, &sh.p_full[0], sbc & 1)) goto epi_done;
+                    tc_fence_after();
+                    if (live) {
+                        load_cols64(tmem + lane_off + C::TM_P0 + col0, x0);
                         tmem_wait_ld();
-                        if constexpr (DBG) {
-                            const Unit un = unit_of<TAIL>(args, u);
+                        preset_cols64(tmem + lane_off + C::TM_P0 + col0);
+                        tmem_wait_st();
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&sh.p_empty[0]);
+                    if (!wait_bar_warp(sh, &sh.p_full[1], sbc & 1)) goto epi_done;
+                    tc_fence_after();
+                    if (live) {
+                        const Unit un = unit_of<TAIL>(args, u);
+#pragma unroll
+                        for (int c = 0; c < 4; c++) {
+                            uint32_t x1[16];
+                            tmem_ld16(tmem + lane_off + C::TM_P1 + col0 + 16 * c, x1);
+                            tmem_wait_ld();
 #pragma unroll
                             for (int i = 0; i < 16; i++) {
                                 const int ml = (int)col0 + 16 * c + i;
@@ -710,24 +732,48 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                     args.dbg_S[(m * args.dbg_N + n) * args.nsb + s] = P0 + (QT == 12 ? 8 : 256) * P1;
                                 }
                             }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 8; i++) {
-                                const float2 X0 = make_float2(__uint_as_float(x0[16 * c + 2 * i]),
-                                                              __uint_as_float(x0[16 * c + 2 * i + 1]));
-                                const float2 X1 = make_float2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
-                                // 8*P1 - M (or 256*P1 - M) exactly unless it is large, then + (M + P0)
-                                const float2 S = __fadd2_rn(__ffma2_rn(X1, kP, mP), X0);
-                                const float2 dav = *reinterpret_cast<const float2*>(da + 16 * c + 2 * i);
-                                acc[8 * c + i] = __ffma2_rn(__fmul2_rn(S, d2), dav, acc[8 * c + i]);
-                            }
                         }
+                        preset_cols64(tmem + lane_off + C::TM_P1 + col0);
+                        tmem_wait_st();
                     }
-                    preset_cols64(tmem + lane_off + C::TM_P1 + col0);
-                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&sh.p_empty[1]);
+                } else {
+                    // each plane on its own: acc += da * d * (weight of the plane) * P, where
+                    // P comes exactly out of the f32 1.5*2^23 + P; two chunks of 32 columns
+#pragma unroll
+                    for (int pl = 0; pl < 2; pl++) {
+                        if (!wait_bar_warp(sh, &sh.p_full[pl], sbc & 1)) goto epi_done;
+                        tc_fence_after();
+                        if (live) {
+                            const uint32_t tp = tmem + lane_off + (pl ? C::TM_P1 : C::TM_P0) + col0;
+#pragma unroll
+                            for (int c = 0; c < 2; c++) {
+                                uint32_t x[32];
+                                tmem_ld16(tp + 32 * c, x);
+                                tmem_ld16(tp + 32 * c + 16, x + 16);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int i4 = 0; i4 < 8; i4++) {
+                                    const float4 dv4 = *reinterpret_cast<const float4*>(da + 32 * c + 4 * i4);
+#pragma unroll
+                                    for (int h2 = 0; h2 < 2; h2++) {
+                                        const int i = 2 * i4 + h2;
+                                        const float2 X = make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
+                                        const float2 T = pl ? __ffma2_rn(X, kP, nkM) : __fadd2_rn(X, nM);
+                                        const float2 dd = __fmul2_rn(d2, h2 ? make_float2(dv4.z, dv4.w)
+                                                                            : make_float2(dv4.x, dv4.y));
+                                        acc[16 * c + i] = __ffma2_rn(T, dd, acc[16 * c + i]);
+                                    }
+                                }
+                            }
+                            preset_cols64(tp);
+                            tmem_wait_st();
+                        }
+                        tc_fence_before();
+                        mbar_arrive(&sh.p_empty[pl]);
+                    }
                 }
-                tc_fence_before();
-                mbar_arrive(&sh.p_empty[1]);
                 mbar_arrive(&sh.b_empty[bst]);
             }
             if constexpr (C::MIN) {

@@ -170,11 +170,16 @@ int dllm_swiglu_quantize(const float* gate, const float* up, int64_t M, int64_t 
  * workspace: device scratch owned by the caller, at least dllm_qgemm_workspace_bytes()
  * bytes (that size may be 0, and then workspace may be NULL); otherwise the call
  * returns DLLM_ERR_WORKSPACE.  It holds the gathered rows and, when a tile's K range
- * is split over several CTAs, their partial sums and one arrival counter per tile.
- * It must be zero-filled before its first use.  Every call that completes leaves
- * each counter at a multiple of 16, which is all the next call needs; a call that
- * ends in DLLM_ERR_TIMEOUT may not, so zero the workspace again after one.  Calls that
- * share a workspace must be ordered on one stream.
+ * is split over several CTAs, their partial sums and one arrival counter per tile and
+ * token super-tile.  The counters are the only contents that carry over between calls:
+ * they occupy a fixed prefix (the first 64 KiB, or 4 bytes per tile and super-tile when
+ * a call needs more) that no call's partial sums or gathered rows overlap, so one
+ * workspace can serve calls of different shapes, provided each of them needs at most
+ * 64 KiB of counters (ceil(N/128) x ceil(M/128) <= 16384).  It must be zero-filled
+ * before its first use.  Every call that completes leaves each counter at a multiple of
+ * 16, which is all the next call needs; a call that ends in DLLM_ERR_TIMEOUT may not, so
+ * zero the workspace again after one.  Calls that share a workspace must be ordered on
+ * one stream.
  * For dllm_qkv_qgemm pass N = Nq + 2*Nkv (Nq + Nkv without wv) and n_rows = 0.
  * ---------------------------------------------------------------------------- */
 int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, int64_t n_rows, size_t* bytes);

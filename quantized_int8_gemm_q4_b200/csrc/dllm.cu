@@ -113,6 +113,11 @@ int64_t tail_plan(int64_t n_tiles, int64_t nsb, int sms, int* full_tiles, int* t
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// The arrival counters are the only workspace contents that persist from one call to
+// the next, so they sit in a fixed prefix that no call's partial sums or gathered rows
+// ever overlap, whatever its shape: calls of different shapes can share a workspace.
+constexpr size_t CTR_REGION = (size_t)64 << 10;
+
 Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
     Plan p;
     const int64_t nsb = K / QK;
@@ -132,7 +137,7 @@ Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
     size_t off = 0;
     p.ctr_off = off;
     p.ctr_bytes = (size_t)n_tiles * p.n_st * 4;  // one arrival counter per (tile, token super-tile)
-    off += align256(p.ctr_bytes);
+    off += p.ctr_bytes > CTR_REGION ? align256(p.ctr_bytes) : CTR_REGION;
     p.part_off = off;
     if (p.kc > 1) off += align256((size_t)n_tiles * p.n_st * p.kc * p.mu * TROWS * 4);
     if (p.tail_k > 0) off += align256((size_t)sms * p.n_st * p.mu * TROWS * 4);

@@ -123,3 +123,29 @@ def test_split_durations_from_events():
     gemm, quant, per = bench.split_durations([step(0.0), step(100.0)], 6)
     assert gemm == 60.0 and quant == 5.0   # the first quantizer of a step is not timed
     assert per == [None, 2.0, 3.0]
+
+
+def test_parity_sample_covers_full_layers_and_sixty_fourths():
+    model = synth.MODELS["llada-8b"]()
+    smp = bench.parity_sample(model, model.n_layers, 6, 4)
+    full = {l for (l, n), (a, b) in smp.items() if n == "down"}
+    assert full == {0, 1, 2, 3, 4, 31}
+    for l in range(model.n_layers):
+        for p in model.layer:
+            if l in full:
+                assert smp[(l, p.name)] == (0, p.N)
+            elif p.name == "down":
+                assert (l, p.name) not in smp
+            else:
+                a, b = smp[(l, p.name)]
+                assert b - a == p.N // 64 and 0 <= a and b <= p.N
+    assert bench.parity_sample(model, model.n_layers, 6, 4) == smp  # seeded
+
+
+def test_parity_ratio_is_the_tolerance():
+    import numpy as np
+    ref = np.array([[100.0, -2.0, 0.0]])
+    T = np.array([[100.0, 1e6, 10.0]])
+    got = ref + np.array([[1e-3, 0.5, 5e-6]])
+    # 1e-3 / (1e-5*100) = 1, 0.5 / (1e-6*1e6) = 0.5, 5e-6 / (1e-6*10) = 0.5
+    assert abs(bench.parity_ratio(got.astype(np.float32), ref, T) - 1.0) < 1e-3

@@ -437,6 +437,39 @@ def test_workspace_shared_across_calls_and_shapes():
     assert np.all(ctr % 16 == 0) and np.all(ctr > 0)
 
 
+def test_workspace_shared_by_tail_split_and_uniform_split():
+    """The step's own mix on one workspace: a 4096-row projection whose 32 tiles split K
+    four ways (O, down) between launches of a 192-tile gate/up whose 44 leftover tiles
+    are cut into K-pieces (tail split, arrival counters up to tile 191).  The partial
+    sums of the small calls must never land on the counters of the large one: every
+    repetition gives the same bits, within the oracle's bound."""
+    M, K, F = 128, 4096, 12288
+    x = synth.activations(M, K, 71)
+    act = gu.Act(x)
+    oq, os_, _ = oracle.quantize_act(x)
+    wo = synth.weights(Q4, K, K, 71, 0)
+    wg, wu = synth.weights(Q4, F, K, 71, 1), synth.weights(Q4, F, K, 71, 2)
+    do, dg, du = dllm.repack(Q4, wo, K, K), dllm.repack(Q4, wg, F, K), dllm.repack(Q4, wu, F, K)
+    wsb = max(dllm.dllm_qgemm_workspace_bytes(Q4, K, K, M), dllm.dllm_qgemm_workspace_bytes(Q4, 2 * F, K, M))
+    ws = dllm.alloc_workspace(wsb)
+    og, ou, oo = (torch.empty((M, n), device="cuda") for n in (F, F, K))
+    first = None
+    for rep in range(4):
+        dllm.dllm_qgemm(do, Q4, K, K, act.q, act.scale, act.sums, M, None, 0, oo, K, ws, wsb)
+        dllm.dllm_qkv_qgemm(dg, du, None, Q4, F, F, K, act.q, act.scale, act.sums, M, og, F, ou, None, F, ws, wsb)
+        got = [t.cpu().numpy() for t in (oo, og, ou)]
+        if first is None:
+            first = got
+            for w, o, n in ((wo, got[0], K), (wg, got[1], F), (wu, got[2], F)):
+                for n0 in (0, n - 256, n // 2):
+                    _, ref, T = oracle.qgemm(Q4, w, n, K, oq, os_, n0=n0, n1=n0 + 256)
+                    assert gu.tol_ok(o[:, n0:n0 + 256], ref, T)[0], n0
+        else:
+            for a, b in zip(first, got):
+                assert np.array_equal(a, b)
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+
 def test_workspace_too_small_is_rejected():
     M, N, K = 32, 256, 2048
     w, x = gu.make_case(Q4, M, N, K, 71)

@@ -59,6 +59,11 @@ def parse():
                         "sampled on 1/64 of their output columns")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--config", choices=["c1", "c2", "c3", "act"], default=None,
+                   help="time one of the single-GEMM workloads instead of the step: c1 attention projections "
+                        "(QKV in one launch + O, 160 rows), c2 FFN (gate/up + down) over canvases 160..1024, "
+                        "c3 output projection on 1..32 requested rows, act the fused quantizers at the step's "
+                        "canvas and at 2^24 elements; one JSON line per case")
     p.add_argument("--gather-last", action="store_true",
                    help="the last layer's O and FFN, and the final norm, on the requested rows only")
     return p.parse_args()
@@ -749,6 +754,158 @@ def measure_int8_peak(dllm, torch, dev, iters=8192):
     return 2 * 128 * 256 * 32 * iters * ctas / t
 
 
+# ---------------------------------------------------------------------------- single-GEMM configs
+
+def config_cases(name, model):
+    """(label, [Gemm per launch], M canvas, rows) of a single-GEMM workload."""
+    h, f = model.hidden, model.ffn
+    if name == "c1":
+        M = 160
+        return [("qkv+o", [Gemm("qkv", Q4, model.q_out + 2 * model.kv_out, h, M, M), Gemm("o", Q4, h, h, M, M)],
+                 M, None)]
+    if name == "c2":
+        return [(f"ffn M={M}", [Gemm("gate_up", Q4, 2 * f, h, M, M), Gemm("down", Q6, h, f, M, M)], M, None)
+                for M in (160, 256, 512, 1024)]
+    return [(f"output rows={R}", [Gemm("output", Q6, model.vocab, h, R, R)], 160, R) for R in (1, 2, 4, 8, 16, 32)]
+
+
+def run_act_config(args, dllm, torch, dev, model):
+    """Device time of the three quantizer kernels at the step's canvas and at 2^24
+    elements (inputs beyond L2 at the large size), against their algorithmic bytes."""
+    hbm_gbs, peak_kind = load_peaks()
+    lines = []
+    h, f, eps = model.hidden, model.ffn, model.norm_eps
+    for M in (args.canvas, 4096):
+        for kernel, K in (("quantize_act", h), ("rmsnorm_quantize", h), ("swiglu_quantize", f)):
+            Mk = M if kernel != "swiglu_quantize" else max(1, M * h // f)  # same element count at 2^24
+            if M == args.canvas:
+                Mk = M
+            x = torch.randn((Mk, K), device=dev)
+            u = torch.randn((Mk, K), device=dev)
+            gam = torch.rand(K, device=dev) + 0.5
+            q, sc, su = dllm.alloc_act(Mk, K, dev)
+
+            def run():
+                if kernel == "quantize_act":
+                    dllm.dllm_quantize_act(x, Mk, K, K, q, sc, su)
+                elif kernel == "rmsnorm_quantize":
+                    dllm.dllm_rmsnorm_quantize(x, Mk, K, K, gam, eps, None, 0, q, sc, su)
+                else:
+                    dllm.dllm_swiglu_quantize(x, u, Mk, K, K, q, sc, su)
+            for _ in range(3):
+                run()
+            torch.cuda.synchronize()
+            reps = 50
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                run()
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            nbytes = act_bytes(kernel, Mk, K)
+            gbs = nbytes / (us * 1e-6) / 1e9
+            lines.append({"metric": "GB/s of algorithmic bytes (% of HBM)", "config": {
+                "workload": "act", "kernel": kernel, "rows": Mk, "K": K, "elements": Mk * K},
+                "us": round(us, 2), "bytes": int(nbytes), "achieved_gbs": round(gbs, 1),
+                "frac": round(gbs / hbm_gbs, 4), "hbm_gbs": hbm_gbs, "hbm_source": peak_kind,
+                "timing": f"CUDA events over {reps} back-to-back launches"})
+            assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+            del x, u, q, sc, su
+    return lines
+
+
+def run_config(args):
+    """Device time of each launch of a single-GEMM workload, weights rotated over enough
+    copies to exceed L2, against t* = max(bytes / HBM, ops / int8 peak) per launch."""
+    import torch
+    from quantized_int8_gemm_q4_b200 import build, dllm, synth
+    build.build()
+    dllm.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    model = synth.MODELS[args.model]()
+    if args.config == "act":
+        return run_act_config(args, dllm, torch, dev, model)
+    hbm_gbs, peak_kind = load_peaks()
+    p_meas = measure_int8_peak(dllm, torch, dev)
+    lines = []
+    for label, gemms, M, R in config_cases(args.config, model):
+        mats = []  # per launch: list of weight-copy tuples
+        for gi, g in enumerate(gemms):
+            parts = ([(model.q_out, 0), (model.kv_out, 1), (model.kv_out, 2)] if g.name == "qkv" else
+                     [(model.ffn, 0), (model.ffn, 1)] if g.name == "gate_up" else [(g.N, 0)])
+            wbytes = sum(dllm.dllm_repacked_bytes(g.qtype, n, g.K) for n, _ in parts)
+            copies = max(1, min(8, int(3 * 126e6 // wbytes) + 1))
+            cps = []
+            for c in range(copies):
+                ws_ = []
+                for n, pi in parts:
+                    gg = synth.device_weights(g.qtype, n, g.K, 4, gi, pi, c, device=dev)
+                    w = torch.empty(dllm.dllm_repacked_bytes(g.qtype, n, g.K), dtype=torch.uint8, device=dev)
+                    (dllm.dllm_repack_q4k if g.qtype == Q4 else dllm.dllm_repack_q6k)(gg, n, g.K, w)
+                    del gg
+                    ws_.append(w)
+                cps.append(ws_)
+            mats.append(cps)
+        acts = {}
+        for g in gemms:
+            if g.K not in acts:
+                x = synth.device_activations(M, g.K, 4, g.K, device=dev)
+                acts[g.K] = dllm.alloc_act(M, g.K, dev)
+                dllm.dllm_quantize_act(x, M, g.K, g.K, *acts[g.K])
+        rows = torch.from_numpy(synth.block_rows(M, R, 4)).to(dev) if R else None
+        outs = [torch.empty((R or M, g.N), device=dev) for g in gemms]
+        wsb = max(dllm.dllm_qgemm_workspace_bytes(g.qtype, g.N, g.K, M, R or 0) for g in gemms)
+        work = dllm.alloc_workspace(max(wsb, 256), dev)
+
+        def launch(gi, i):
+            g, w = gemms[gi], mats[gi][i % len(mats[gi])]
+            o = outs[gi]
+            if g.name == "qkv":
+                dllm.dllm_qkv_qgemm(w[0], w[1], w[2], Q4, model.q_out, model.kv_out, g.K, *acts[g.K], M,
+                                    o[:, :model.q_out], g.N, o[:, model.q_out:model.q_out + model.kv_out],
+                                    o[:, model.q_out + model.kv_out:], g.N, work, wsb)
+            elif g.name == "gate_up":
+                dllm.dllm_qkv_qgemm(w[0], w[1], None, Q4, model.ffn, model.ffn, g.K, *acts[g.K], M,
+                                    o[:, :model.ffn], g.N, o[:, model.ffn:], None, g.N, work, wsb)
+            else:
+                dllm.dllm_qgemm(w[0], g.qtype, g.N, g.K, *acts[g.K], M, rows, R or 0, o, g.N, work, wsb)
+        reps = max(20, args.steps)
+        res = []
+        for gi, g in enumerate(gemms):
+            for i in range(5):
+                launch(gi, i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(reps):
+                launch(gi, i)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            t_hbm = g.bytes / (hbm_gbs * 1e9) * 1e6
+            t_tc = g.ops / p_meas * 1e6 if p_meas else g.ops / P_INT8_NOMINAL * 1e6
+            tstar = max(t_hbm, t_tc)
+            res.append({"launch": g.name, "N": g.N, "K": g.K, "rows_out": g.M_out, "us": round(us, 2),
+                        "t_star_us": round(tstar, 2), "frac": round(tstar / us, 4),
+                        "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                        "int8_tops": round(g.ops / (us * 1e-6) / 1e12, 1),
+                        "weight_gbs": round(g.weight_bytes / (us * 1e-6) / 1e9, 1)})
+        assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+        tot_us = sum(r["us"] for r in res)
+        tot_star = sum(r["t_star_us"] for r in res)
+        lines.append({"metric": METRIC, "config": {"workload": args.config, "case": label, "canvas_tokens": M,
+                                                    "model": model.name},
+                      "launches": res, "us": round(tot_us, 2), "t_star_us": round(tot_star, 2),
+                      "frac": round(tot_star / tot_us, 4), "hbm_gbs": hbm_gbs, "hbm_source": peak_kind,
+                      "p_int8_tops_measured": round(p_meas / 1e12, 1) if p_meas else None,
+                      "timing": f"CUDA events over {reps} launches, weights rotated over copies beyond L2"})
+        del mats, outs, work
+        torch.cuda.empty_cache()
+    return lines
+
+
 # ---------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -796,6 +953,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.config:
+        for line in run_config(args):
+            print(json.dumps(line), flush=True)
         return
     if world > 1:
         import datetime

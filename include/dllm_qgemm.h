@@ -237,6 +237,30 @@ int dllm_qkv_qgemm(const void* wq, const void* wk, const void* wv, dllm_qtype t,
                    int64_t ldo_q, float* ok, float* ov, int64_t ldo_kv, void* workspace, size_t workspace_bytes,
                    dllm_stream_t stream);
 
+/* ------------------------------------------------------------------------------
+ * Attention: bidirectional (no mask) softmax attention over the canvas, the step
+ * between the Q/K/V and the output projections (Architecture page, "A forward
+ * pass", step 2: attention runs over all L positions with no mask; heatdrop card,
+ * "Key highlights": f16 tensor cores with an online softmax).
+ *
+ *   o[i][h][:] = sum_j softmax_j( q[i][h] . k[j][g] / sqrt(dh) ) v[j][g][:],
+ *   g = h / (H / Hkv)   (grouped-query attention when Hkv < H)
+ *
+ * q: f16 [Lq][H][dh]; k, v: f16 [Lk][Hkv][dh] (contiguous, 16-byte aligned; q and k
+ * as they come out of RoPE); o: f32 [Lq][H][dh], written, may not overlap the inputs.
+ * dh must be 128 (LLaDA-8B and Dream-7B).  Lq == 0 is a no-op; Lk must be >= 1.
+ * Arithmetic: Q K^T on f16 tensor cores with f32 accumulation; the softmax in f32
+ * with base-2 exponents and a running maximum raised only when a block maximum
+ * exceeds it by more than 2^8; the weights rounded to f16 for P V on the tensor
+ * cores (f32 accumulation), the normaliser summed in f32 before that rounding, so each
+ * normalised weight is off by at most about 2^-11 of itself plus the f32 effects.
+ * One CTA per (128 queries, head), programmatic dependent launch like the GEMM.
+ * Errors: DLLM_ERR_ARG (sizes, dh != 128, H % Hkv, null), DLLM_ERR_ALIGN,
+ * DLLM_ERR_UNSUPPORTED, DLLM_ERR_CUDA; DLLM_ERR_TIMEOUT in the device error word.
+ * ---------------------------------------------------------------------------- */
+int dllm_attention(const void* q, const void* k, const void* v, int64_t Lq, int64_t Lk, int64_t H, int64_t Hkv,
+                   int64_t dh, float* o, dllm_stream_t stream);
+
 /* Synchronizes `stream`, then returns and clears the device error word
  * (DLLM_OK, DLLM_ERR_ROW_RANGE or DLLM_ERR_TIMEOUT). */
 int dllm_get_device_status(dllm_stream_t stream);

@@ -4,6 +4,7 @@
 
 #include "../../include/dllm_qgemm.h"
 #include "actfuse.cuh"
+#include "attention.cuh"
 #include "layout.cuh"
 #include "qgemm.cuh"
 
@@ -15,6 +16,7 @@ constexpr int MAX_DEV = 64;
 int g_dev_checked[MAX_DEV];  // 0 unknown, 1 sm_100, -1 other
 int g_num_sms[MAX_DEV];
 bool g_attr_done[MAX_DEV][8];
+bool g_att_attr_done[MAX_DEV];
 
 int current_device(int* dev) {
     if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= MAX_DEV) return DLLM_ERR_CUDA;
@@ -45,6 +47,38 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (the
+// library does not link the driver API).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static const EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeTiledFn) nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// A [rows][heads][128] f16 tensor as the 3-D tensor (head dim, head, row) with boxes of
+// 64 head-dim values x 1 head x 128 rows, 128-byte swizzled (half a tile).
+bool encode_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t heads) {
+    const EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)ATT_DH, (cuuint64_t)heads, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)ATT_DH * 2, (cuuint64_t)(heads * ATT_DH * 2)};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)ATT_BK};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int launch_status() {
@@ -479,6 +513,34 @@ int dllm_qgemm_noalloc(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
         return DLLM_ERR_CUDA;
     return dllm_qgemm(w, t, N, K, q, scale, sums, M, rows, n_rows, out, ldo, scratch, DLLM_NOALLOC_SCRATCH_BYTES,
                       stream);
+}
+
+int dllm_attention(const void* q, const void* k, const void* v, int64_t Lq, int64_t Lk, int64_t H, int64_t Hkv,
+                   int64_t dh, float* o, dllm_stream_t stream) {
+    if (Lq < 0 || Lk < 0 || H <= 0 || Hkv <= 0 || H % Hkv || dh != ATT_DH) return DLLM_ERR_ARG;
+    if (Lq == 0) return DLLM_OK;
+    if (!q || !k || !v || !o || Lk == 0) return DLLM_ERR_ARG;
+    if (Lq > (1LL << 30) || Lk > (1LL << 30) || H > 65535) return DLLM_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DLLM_ERR_ALIGN;
+    int dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    if (!g_att_attr_done[dev]) {
+        if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATT_SMEM) !=
+            cudaSuccess)
+            return DLLM_ERR_CUDA;
+        g_att_attr_done[dev] = true;
+    }
+    CUtensorMap tq, tk, tv;
+    if (!encode_head_rows(&tq, q, Lq, H) || !encode_head_rows(&tk, k, Lk, Hkv) || !encode_head_rows(&tv, v, Lk, Hkv))
+        return DLLM_ERR_CUDA;
+    const dim3 grid((unsigned)((Lq + ATT_BQ - 1) / ATT_BQ), (unsigned)H);
+    if (launch_pdl(attention_kernel, grid, dim3(ATT_THREADS), ATT_SMEM, reinterpret_cast<cudaStream_t>(stream), tq,
+                   tk, tv, o, (int)Lq, (int)Lk, (int)H, (int)(H / Hkv)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DLLM_ERR_CUDA;
+    }
+    return launch_status();
 }
 
 int dllm_get_device_status(dllm_stream_t stream) {

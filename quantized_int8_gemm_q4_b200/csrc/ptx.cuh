@@ -64,6 +64,17 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
+// Tensor copy (TMA) of one 3-D box described by the tensor map at `tmap` (a
+// __grid_constant__ kernel parameter) into shared memory, completing `bar`'s
+// transaction count.  The innermost coordinate x times the element size must be a
+// multiple of 16 bytes; out-of-range parts of the box are filled with zeros.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
 // Bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.  A
 // hint only: L2 is the coherence point, so a prefetch never exposes stale data.
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
@@ -152,6 +163,22 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_noswz(uint32_t saddr, uint32_t 
     return d;                // base offset 0, layout type 0 (no swizzle)
 }
 
+// Shared-memory matrix descriptor for the 128-byte swizzled canonical layouts (rows
+// of 128 bytes whose 16-byte chunks are XOR-ed with the row index mod 8, in atoms of
+// 8 rows = 1024 bytes, the pattern TMA writes with 128-byte swizzling; atoms 1024-byte
+// aligned).  K-major: sbo = distance between 8-row atoms, lbo unused; a K step inside
+// the 128-byte row advances the start address.  MN-major: lbo = distance between
+// atoms along M/N (64 16-bit elements each), sbo = distance between 8-row groups along K.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;  // layout type: 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor for kind::i8: int32 accumulator, K-major A and B.
 // a_signed / b_signed select s8 (1) or u8 (0) per operand.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N, int a_signed, int b_signed) {
@@ -170,6 +197,21 @@ __device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, ui
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor for kind::f16 with f16 A and B: f32 accumulator, K-major A and B.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// D[tmem] (+)= A[smem] * B[smem]^T in f16 (K = 16 per instruction), f32 accumulation.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }

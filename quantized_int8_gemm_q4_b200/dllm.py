@@ -30,7 +30,8 @@ DLLM_NOALLOC_SCRATCH_BYTES = 32 << 20
 EXPORTS = (
     "dllm_repacked_bytes", "dllm_repack_q4k", "dllm_repack_q6k", "dllm_act_bytes", "dllm_quantize_act",
     "dllm_rmsnorm_quantize", "dllm_swiglu_quantize",
-    "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_get_device_status",
+    "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_attention",
+    "dllm_get_device_status",
     "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_debug_bounded_wait",
     "dllm_bench_mma_i8", "dllm_debug_plan",
 )
@@ -69,6 +70,7 @@ def load() -> ctypes.CDLL:
         "dllm_qgemm": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P, SZ, P],
         "dllm_qgemm_noalloc": [P, I, I64, I64, P, P, P, I64, P, I64, P, I64, P],
         "dllm_qkv_qgemm": [P, P, P, I, I64, I64, I64, P, P, P, I64, P, I64, P, P, I64, P, SZ, P],
+        "dllm_attention": [P, P, P, I64, I64, I64, I64, I64, P, P],
         "dllm_get_device_status": [P],
         "dllm_status_string": [I],
         "dllm_debug_subblock_dots": [P, I, I64, I64, P, I64, P, P],
@@ -174,6 +176,11 @@ def dllm_qkv_qgemm(wq, wk, wv, qtype: int, Nq: int, Nkv: int, K: int, q, scale, 
     _check(load().dllm_qkv_qgemm(_ptr(wq), _ptr(wk), _ptr(wv), qtype, Nq, Nkv, K, _ptr(q), _ptr(scale), _ptr(sums),
                                  M, _ptr(oq), ldo_q, _ptr(ok), _ptr(ov), ldo_kv, _ptr(workspace), workspace_bytes,
                                  _stream(stream)), "dllm_qkv_qgemm")
+
+
+def dllm_attention(q, k, v, Lq: int, Lk: int, H: int, Hkv: int, dh: int, o, stream=None):
+    _check(load().dllm_attention(_ptr(q), _ptr(k), _ptr(v), Lq, Lk, H, Hkv, dh, _ptr(o), _stream(stream)),
+           "dllm_attention")
 
 
 def dllm_get_device_status(stream=None) -> int:

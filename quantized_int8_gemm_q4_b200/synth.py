@@ -17,6 +17,11 @@ Distributions (the synthetic stand-ins for real GGUF weights, which are not used
   * Q8_0: every 34-byte block has d uniform on [1e-4, 1e-3] rounded to f16 and 32
     int8 quants uniform on -127..127.
   * Activations: f32 standard normal.
+  * Attention inputs: q, k, v standard normal rounded to f16, q and k times a
+    spread factor (1 gives logits q.k/sqrt(128) of unit standard deviation; larger
+    factors give the peaked softmax rows of a trained model); optionally the key
+    rows grow linearly in norm along the sequence (each block of 128 keys then
+    raises the running maximum of the rows whose query leans the same way).
 """
 from __future__ import annotations
 
@@ -96,6 +101,17 @@ def weights(qtype: int, N: int, K: int, seed, *sub) -> np.ndarray:
 def activations(M: int, K: int, seed, *sub) -> np.ndarray:
     """f32 [M, K] standard normal."""
     return _rng(seed, 8, *sub).standard_normal((M, K), dtype=np.float32)
+
+
+def attention_inputs(Lq: int, Lk: int, H: int, Hkv: int, dh: int, seed, *sub, spread: float = 1.0,
+                     key_growth: float = 0.0):
+    """f16 q [Lq][H][dh], k and v [Lk][Hkv][dh]."""
+    rng = _rng(seed, 11, *sub)
+    q = (rng.standard_normal((Lq, H, dh)) * spread).astype(np.float16)
+    k = rng.standard_normal((Lk, Hkv, dh)) * spread
+    k *= (1.0 + key_growth * np.arange(Lk))[:, None, None]
+    v = rng.standard_normal((Lk, Hkv, dh)).astype(np.float16)
+    return q, k.astype(np.float16), v
 
 
 def norm_weights(n: int, K: int, seed, *sub) -> np.ndarray:

@@ -33,6 +33,18 @@ int main(void)
            dllm_rmsnorm_quantize((const float*)0x10000, 4, 256, 256, (const float*)0x10000, 0.0f, NULL, 0,
                                  (int8_t*)0x10000, (float*)0x10000, (uint8_t*)0x10000, NULL));
 
+    /* attention: argument errors and the empty query set, all decided on the host */
+    {
+        const void* d = (const void*)0x10000;
+        float* o = (float*)0x10000;
+        printf("attn_dh64 %d\n", dllm_attention(d, d, d, 4, 4, 2, 2, 64, o, NULL));
+        printf("attn_group %d\n", dllm_attention(d, d, d, 4, 4, 3, 2, 128, o, NULL));
+        printf("attn_no_keys %d\n", dllm_attention(d, d, d, 4, 0, 2, 2, 128, o, NULL));
+        printf("attn_null %d\n", dllm_attention(NULL, d, d, 4, 4, 2, 2, 128, o, NULL));
+        printf("attn_align %d\n", dllm_attention((const char*)d + 2, d, d, 4, 4, 2, 2, 128, o, NULL));
+        printf("attn_empty %d\n", dllm_attention(NULL, NULL, NULL, 0, 0, 2, 2, 128, NULL, NULL));
+    }
+
     const char* s = dllm_status_string(DLLM_ERR_ROW_RANGE);
     printf("status_row_range_nonempty %d\n", s != NULL && strlen(s) > 0);
     return 0;

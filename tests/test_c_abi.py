@@ -47,3 +47,9 @@ def test_plan_from_c(results):
     assert results["plan_rc"] == 0
     assert (results["plan_kc"], results["plan_full_tiles"], results["plan_tail_k"], results["plan_tail_big"]) == \
         (1, 148, 3, 16)
+
+
+def test_attention_rejections(results):
+    assert results["attn_dh64"] == -1 and results["attn_group"] == -1 and results["attn_no_keys"] == -1
+    assert results["attn_null"] == -1 and results["attn_align"] == -2
+    assert results["attn_empty"] == 0  # no queries: nothing to do, nothing launched

@@ -42,6 +42,9 @@ PEAKS_FILE = ROOT / "MEASURED_PEAKS.json"
 TRAFFIC_FILE = ROOT / "profiles" / "qgemm_dram_traffic.json"
 FALLBACK_HBM_GBS = 6650.0
 P_INT8_NOMINAL = 4.5e15  # dense int8 tensor ops/s of a B200 (datasheet)
+FALLBACK_BF16_TFLOPS = 1590.0  # dense bf16 (= f16) tensor TFLOP/s measured earlier on this machine (burst)
+# special-function unit: 16 ex2 per clock per SM x 148 SMs x 1.965 GHz (max SM clock)
+SFU_EX2_PER_S = 16 * 148 * 1.965e9
 Q4, Q6 = 12, 14
 
 
@@ -59,11 +62,12 @@ def parse():
                         "sampled on 1/64 of their output columns")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
-    p.add_argument("--config", choices=["c1", "c2", "c3", "act"], default=None,
+    p.add_argument("--config", choices=["c1", "c2", "c3", "act", "attn"], default=None,
                    help="time one of the single-GEMM workloads instead of the step: c1 attention projections "
                         "(QKV in one launch + O, 160 rows), c2 FFN (gate/up + down) over canvases 160..1024, "
                         "c3 output projection on 1..32 requested rows, act the fused quantizers at the step's "
-                        "canvas and at 2^24 elements; one JSON line per case")
+                        "canvas and at 2^24 elements, attn the bidirectional attention over canvases 128..4096; "
+                        "one JSON line per case")
     p.add_argument("--gather-last", action="store_true",
                    help="the last layer's O and FFN, and the final norm, on the requested rows only")
     return p.parse_args()
@@ -168,6 +172,15 @@ def split_durations(evs, n_marks):
 
 def roofline_time(gemms, hbm_gbs, p_int8):
     return sum(max(g.bytes / (hbm_gbs * 1e9), g.ops / p_int8) for g in gemms)
+
+
+def load_tensor_peak():
+    """Dense bf16 tensor TFLOP/s (the f16 rate is the same): burst figure."""
+    if PEAKS_FILE.exists():
+        d = json.loads(PEAKS_FILE.read_text())
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def load_peaks():
@@ -815,6 +828,60 @@ def run_act_config(args, dllm, torch, dev, model):
     return lines
 
 
+def run_attn_config(args, dllm, torch, dev, model):
+    """Device time of dllm_attention per launch at the model's head layout, canvases
+    128..1024 (the step sweep) and 4096, inputs rotated over copies beyond L2, against
+    t* = max(FLOPs / f16 tensor peak, exponentials / special-function-unit rate)."""
+    from quantized_int8_gemm_q4_b200 import synth
+    peak_tf, peak_kind = load_tensor_peak()
+    H, Hkv, dh = model.heads, model.kv_heads, model.hidden // model.heads
+    lines = []
+    for L in (128, 256, 512, 1024, 4096):
+        nbytes = 2 * (L * H * dh + 2 * L * Hkv * dh)
+        copies = max(1, min(16, int(3 * 126e6 // nbytes) + 1))
+        ins = [synth.device_attention_inputs(L, L, H, Hkv, dh, 6, L, c, device=dev) for c in range(copies)]
+        o = torch.empty((L, H, dh), dtype=torch.float32, device=dev)
+
+        def run(i):
+            q, k, v = ins[i % copies]
+            dllm.dllm_attention(q, k, v, L, L, H, Hkv, dh, o)
+        for i in range(5):
+            run(i)
+        torch.cuda.synchronize()
+        # the launches replayed from a CUDA graph: device time, not host launch time
+        reps = max(20, min(args.steps, 200))
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(reps):
+                run(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        del g
+        flops = 4.0 * L * L * dh * H
+        t_tc = flops / (peak_tf * 1e12) * 1e6
+        t_sfu = L * L * H / SFU_EX2_PER_S * 1e6
+        tstar = max(t_tc, t_sfu)
+        lines.append({"metric": "f16 tensor TFLOP/s of dllm_attention (% of t*)", "config": {
+            "workload": "attn", "model": model.name, "Lq": L, "Lk": L, "heads": H, "kv_heads": Hkv, "dh": dh},
+            "us": round(us, 2), "tflops": round(flops / (us * 1e-6) / 1e12, 1), "t_star_us": round(tstar, 2),
+            "bound": "tensor" if t_tc >= t_sfu else "sfu", "frac": round(tstar / us, 4),
+            "peak_tflops": peak_tf, "peak_source": peak_kind, "ctas": -(-L // 128) * H,
+            "timing": f"CUDA events around one replay of a graph of {reps} launches, inputs rotated over "
+                      f"{copies} copies beyond L2"})
+        del ins, o
+        torch.cuda.empty_cache()
+    return lines
+
+
 def run_config(args):
     """Device time of each launch of a single-GEMM workload, weights rotated over enough
     copies to exceed L2, against t* = max(bytes / HBM, ops / int8 peak) per launch."""
@@ -827,6 +894,8 @@ def run_config(args):
     model = synth.MODELS[args.model]()
     if args.config == "act":
         return run_act_config(args, dllm, torch, dev, model)
+    if args.config == "attn":
+        return run_attn_config(args, dllm, torch, dev, model)
     hbm_gbs, peak_kind = load_peaks()
     p_meas = measure_int8_peak(dllm, torch, dev)
     lines = []

@@ -4,20 +4,27 @@
 //
 //   o[i][h][:] = sum_j softmax_j(q[i][h] . k[j][g] / sqrt(dh)) v[j][g],  g = h / (H / Hkv)
 //
-// One CTA per (query tile of 128 rows, head), 7 warps:
-//   warp 5      TMA producer of Q (once) and of K key blocks of 128 (two slots)
-//   warp 6      TMA producer of V key blocks (two slots); rows past Lk (and query
+// One CTA per (query tile of 128 rows, head), 12 warps:
+//   warp 9      TMA producer of Q (once) and of K key blocks of 128 (two slots)
+//   warp 10     TMA producer of V key blocks (two slots); rows past Lk (and query
 //               rows past Lq) arrive as zeros
-//   warp 4      one thread issues the MMAs and allocates tensor memory:
-//               S(kb) = Q K(kb)^T   tcgen05 kind::f16, f32 in tensor memory (two slots
-//                                   of 128 lanes x 128 key columns)
-//               O += P(kb) V(kb)    kind::f16, f32 in tensor memory (128 x dh)
-//               S(kb + 1) is issued before P(kb) is waited for, so the tensor core
-//               works on the next block while the softmax threads work on this one
-//   warps 0-3   softmax, thread = query row = tensor-memory lane: block maximum,
-//               running maximum m (base-2 exponents), P = 2^(S c - m) rounded to f16
-//               into one of two shared-memory slots, running sum l; O is rescaled in
-//               tensor memory only when m is raised.  At the end O / l is stored.
+//   warp 8      one thread issues S(kb) = Q K(kb)^T (tcgen05 kind::f16, f32 in tensor
+//               memory, two slots of 128 lanes x 128 key columns), as soon as K(kb) is
+//               in and the softmax of block kb - 2 has left the slot; the warp
+//               allocates tensor memory.  So the tensor core computes the next block's
+//               scores while the softmax threads work on this one.
+//   warp 11     one thread issues O += P(kb) V(kb) (kind::f16 with P read from tensor
+//               memory, f32 in tensor memory, 128 x dh).  Two issuing threads,
+//               because one thread issues a 128 x 128 x 16 MMA no faster than the
+//               tensor core runs it.
+//   warps 0-7   softmax, query row = tensor-memory lane 32 (w % 4) + lane; warps w and
+//               w + 4 take key columns (and head-dim columns of O) 0..63 and 64..127
+//               of the same rows and swap their half-block maxima through shared
+//               memory and a named barrier of the two warps: running maximum m (base-2
+//               exponents), P = 2^(S c - m) rounded to f16 into one of two
+//               tensor-memory slots, running half sums of P; O is rescaled in tensor
+//               memory only when m is raised.  At the end the two halves of l are
+//               added and O / l is stored.
 // Keys beyond Lk score -inf; query rows beyond Lq are not stored.
 //
 // Shared-memory tiles:
@@ -29,10 +36,8 @@
 //            bytes are the MN-major swizzled B operand of P V: 64 head-dim values per
 //            atom row, the second box 16 KB further along N, 1024 bytes between groups
 //            of 8 keys (2048 per K step of 16 keys).  So V needs no transpose.
-//   P        no swizzle, element (r, c) at ((r/8)*16 + c/8)*128 + (r%8)*16 + (c%8)*2,
-//            written by the softmax threads (a quarter warp stores 128 contiguous
-//            bytes): K-major, 128 bytes between core matrices along K, 2048 between
-//            8-row groups.
+// P lives in tensor memory, one row per lane, two f16 keys per 32-bit column: the A
+// operand of P V read from tensor memory (8 columns per K step of 16 keys).
 #pragma once
 #include <cuda.h>
 
@@ -43,11 +48,20 @@ namespace dllm {
 constexpr int ATT_DH = 128;       // head dimension (LLaDA-8B: 4096 / 32, Dream-7B: 3584 / 28)
 constexpr int ATT_BQ = 128;       // queries per CTA (tensor-memory lanes)
 constexpr int ATT_BK = 128;       // keys per block
-constexpr int ATT_THREADS = 224;  // warps 0-3 softmax and output, warp 4 MMA issue, 5 Q and K, 6 V
+constexpr int ATT_SOFTMAX_WARPS = 8;            // two per query-row quadrant, one per half of the columns
+constexpr int ATT_MMA_WARP = ATT_SOFTMAX_WARPS;  // one thread issues Q K^T; the warp owns tensor memory
+constexpr int ATT_K_WARP = ATT_MMA_WARP + 1;     // TMA producer of Q and K
+constexpr int ATT_V_WARP = ATT_MMA_WARP + 2;     // TMA producer of V
+constexpr int ATT_PV_WARP = ATT_MMA_WARP + 3;    // one thread issues P V
+constexpr int ATT_THREADS = 32 * (ATT_SOFTMAX_WARPS + 4);
 constexpr int ATT_TILE = 128 * ATT_DH * 2;  // one 128 x 128 f16 tile, 32 KB
-constexpr uint32_t ATT_TM_COLS = 512;       // S blocks: columns 0..127 and 128..255, O: 256..383
+// Tensor memory: S slots at columns 0..127 and 128..255 (f32), O at 256..383 (f32), P
+// slots at 384..447 and 448..511 (f16 pairs, 128 keys per row).
+constexpr uint32_t ATT_TM_COLS = 512;
 constexpr uint32_t ATT_TM_O = 256;
-constexpr size_t ATT_SMEM = 7 * (size_t)ATT_TILE + 256;  // Q, K x2, V x2, P x2, barriers
+constexpr uint32_t ATT_TM_P = 384;
+// Q, K x2, V x2, barriers and tensor-memory address, exchange values [2][2][128]
+constexpr size_t ATT_SMEM = 5 * (size_t)ATT_TILE + 256 + 4 * 128 * 4;
 // log2(e) / sqrt(128): scores times this are base-2 exponents.
 constexpr float ATT_C = 0.12751743082459868f;
 // The running maximum is raised (and O, l rescaled) only when a block maximum exceeds
@@ -56,12 +70,10 @@ constexpr float ATT_C = 0.12751743082459868f;
 constexpr float ATT_RESCALE_LOG2 = 8.0f;
 constexpr uint64_t ATT_WAIT_NS = 2000000000ull;
 
-// Byte offset of element (r, c) of the P tile.
-__device__ __forceinline__ uint32_t att_off(int r, int c) {
-    return (uint32_t)(((r >> 3) * (ATT_DH / 8) + (c >> 3)) * 128 + (r & 7) * 16 + (c & 7) * 2);
-}
-
+// Bounded wait on a phase; the first poll does not read the timer (most waits in the
+// pipeline find the phase already complete).
 __device__ __forceinline__ bool att_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (globaltimer_ns() - t0 > ATT_WAIT_NS) {
@@ -100,16 +112,14 @@ __device__ __forceinline__ float att_ex2(float x) {
 }
 
 
-// Descriptors of the tiles.
-__device__ __forceinline__ uint64_t att_qk_desc(const uint8_t* t, int kk) {
-    return sdesc_sw128(smem_u32(t + (kk >> 2) * 16384 + (kk & 3) * 32), 16, 1024);
-}
-__device__ __forceinline__ uint64_t att_v_desc(const uint8_t* t, int kk) {
-    return sdesc_sw128(smem_u32(t + kk * 2048), 16384, 1024);
-}
-__device__ __forceinline__ uint64_t att_p_desc(const uint8_t* t, int kk) {
-    return sdesc_kmajor_noswz(smem_u32(t + kk * 256), 128, 2048);
-}
+// Descriptors of the tiles at their first K step; a K step adds a constant to the
+// start-address field (16-byte units, no carry out of it: shared memory < 256 KB).
+//   Q, K: 128-byte swizzled K-major; K step kk at byte (kk / 4) * 16384 + (kk % 4) * 32
+//   V:    128-byte swizzled MN-major; K step kk (16 keys) at byte kk * 2048
+__device__ __forceinline__ uint64_t att_qk_desc(const uint8_t* t) { return sdesc_sw128(smem_u32(t), 16, 1024); }
+__device__ __forceinline__ uint64_t att_v_desc(const uint8_t* t) { return sdesc_sw128(smem_u32(t), 16384, 1024); }
+__host__ __device__ constexpr uint64_t att_qk_step(int kk) { return (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2); }
+__host__ __device__ constexpr uint64_t att_v_step(int kk) { return (uint64_t)(kk * 128); }
 
 // Tensor maps over q: f16 [Lq][H][128], k, v: f16 [Lk][Hkv][128] as 3-D tensors
 // (head dim, head, row) with boxes of 8 x 1 x 128; o: f32 [Lq][H][128]; group = H / Hkv.
@@ -120,7 +130,8 @@ __device__ __forceinline__ uint64_t att_p_desc(const uint8_t* t, int kk) {
 //   k_full[b], v_full[b]   TMA transaction count of the 32 KB tile
 //   k_empty[b]             commit after Q K^T(kb): the K slot may be refilled
 //   s_full[b]              the same commit: S(kb) is ready
-//   p_full[b]              softmax threads, after P(kb) is in shared memory
+//   p_full[b]              softmax threads, after P(kb) is in tensor memory (and S(kb)
+//                          read, so the S slot may take block kb + 2)
 //   o_done[b], v_empty[b]  commit after P V(kb): O holds blocks 0..kb, and the P and
 //                          V slots may be refilled
 // A wait on "use u of slot b" takes parity (u >> 1) & 1; no barrier can run two uses
@@ -133,8 +144,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     uint8_t* const sQ = smem;
     uint8_t* const sK = smem + ATT_TILE;      // two slots
     uint8_t* const sV = smem + 3 * ATT_TILE;  // two slots
-    uint8_t* const sP = smem + 5 * ATT_TILE;  // two slots
-    uint64_t* const bars = reinterpret_cast<uint64_t*>(smem + 7 * ATT_TILE);
+    uint64_t* const bars = reinterpret_cast<uint64_t*>(smem + 5 * ATT_TILE);
     uint64_t* const q_full = bars;
     uint64_t* const k_full = bars + 1;
     uint64_t* const v_full = bars + 3;
@@ -145,6 +155,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     uint64_t* const o_done = bars + 13;
     uint64_t* const fin = bars + 15;
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    float* const xval = reinterpret_cast<float*>(smem + 5 * ATT_TILE + 256);  // [2][half][row]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q0 = blockIdx.x * ATT_BQ, h = blockIdx.y, hk = h / group;
@@ -158,13 +169,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             mbar_init(&k_empty[b], 1);
             mbar_init(&v_empty[b], 1);
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], ATT_BQ);
+            mbar_init(&p_full[b], 32 * ATT_SOFTMAX_WARPS);
             mbar_init(&o_done[b], 1);
         }
-        mbar_init(fin, 1);
+        mbar_init(fin, 2);
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == ATT_MMA_WARP) {
         tmem_alloc(tmem_slot, ATT_TM_COLS);
         tmem_relinquish();
     }
@@ -174,9 +185,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t tm = *tmem_slot;
     pdl_wait();  // q, k, v may come from the previous kernel on the stream
 
-    if (warp >= 5) {
+    if (warp == ATT_K_WARP || warp == ATT_V_WARP) {
         // ---------------------------------------------------------------- TMA producers
-        const bool is_k = warp == 5;
+        const bool is_k = warp == ATT_K_WARP;
         if (is_k) {
             if (lane == 0) mbar_arrive_expect_tx(q_full, ATT_TILE);
             __syncwarp();
@@ -202,38 +213,27 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (is_k) drain_wait(q_full, 0);
         }
         __syncwarp();
-    } else if (warp == 4) {
-        // ---------------------------------------------------------------- MMA issue
+    } else if (warp == ATT_MMA_WARP) {
+        // ---------------------------------------------------------------- Q K^T issue
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_f16(ATT_BQ, ATT_BK);
-            constexpr uint32_t ID_O = idesc_f16(ATT_BQ, ATT_DH) | (1u << 16);  // B (V) MN-major
-            // S[b] = Q K^T for key block kb: 8 steps of K = 16 along the head dimension.
-            auto issue_s = [&](int kb) -> bool {
+            const uint64_t dq = att_qk_desc(sQ), dk0 = att_qk_desc(sK), dk1 = att_qk_desc(sK + ATT_TILE);
+            bool ok = att_wait(q_full, 0);
+            for (int kb = 0; ok && kb < nkb; kb++) {
                 const int b = kb & 1;
-                if (!att_wait(&k_full[b], (kb >> 1) & 1)) return false;
+                // S slot b was last read by the softmax of block kb - 2 (P(kb - 2) marks it)
+                if (!att_wait(&k_full[b], (kb >> 1) & 1)) break;
+                if (kb >= 2 && !att_wait(&p_full[b], ((kb - 2) >> 1) & 1)) break;
                 tc_fence_after();
+                // S[b] = Q K^T for key block kb: 8 steps of K = 16 along the head dimension.
+                const uint32_t d = tm + b * ATT_BK;
+                const uint64_t dk = b ? dk1 : dk0;
+                mma_f16_ss(d, dq, dk, ID_S, 0);
 #pragma unroll
-                for (int kk = 0; kk < ATT_DH / 16; kk++)
-                    mma_f16_ss(tm + b * ATT_BK, att_qk_desc(sQ, kk), att_qk_desc(sK + b * ATT_TILE, kk), ID_S,
-                               kk > 0);
+                for (int kk = 1; kk < ATT_DH / 16; kk++)
+                    mma_f16_ss(d, dq + att_qk_step(kk), dk + att_qk_step(kk), ID_S, 1);
                 tc_commit(&s_full[b]);
                 tc_commit(&k_empty[b]);
-                return true;
-            };
-            bool ok = att_wait(q_full, 0) && issue_s(0);
-            for (int kb = 0; ok && kb < nkb; kb++) {
-                // S for the next block runs while the softmax threads work on this one.
-                if (kb + 1 < nkb && !issue_s(kb + 1)) break;
-                const int b = kb & 1;
-                if (!att_wait(&p_full[b], (kb >> 1) & 1) || !att_wait(&v_full[b], (kb >> 1) & 1)) break;
-                tc_fence_after();
-                // O += P V: 8 steps of K = 16 keys.
-#pragma unroll
-                for (int kk = 0; kk < ATT_BK / 16; kk++)
-                    mma_f16_ss(tm + ATT_TM_O, att_p_desc(sP + b * ATT_TILE, kk), att_v_desc(sV + b * ATT_TILE, kk),
-                               ID_O, (kb | kk) != 0);
-                tc_commit(&o_done[b]);
-                tc_commit(&v_empty[b]);
             }
             // Every MMA issued above completes before the tensor memory is released,
             // also when a wait ran out.
@@ -241,44 +241,94 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             drain_wait(fin, 0);
         }
         __syncwarp();
+    } else if (warp == ATT_PV_WARP) {
+        // ---------------------------------------------------------------- P V issue
+        if (lane == 0) {
+            constexpr uint32_t ID_O = idesc_f16(ATT_BQ, ATT_DH) | (1u << 16);  // B (V) MN-major
+            const uint64_t dv0 = att_v_desc(sV), dv1 = att_v_desc(sV + ATT_TILE);
+            for (int kb = 0; kb < nkb; kb++) {
+                const int b = kb & 1;
+                if (!att_wait(&p_full[b], (kb >> 1) & 1) || !att_wait(&v_full[b], (kb >> 1) & 1)) break;
+                tc_fence_after();
+                // O += P V: 8 steps of K = 16 keys (P from tensor memory, 8 columns a step).
+                const uint32_t pa = tm + ATT_TM_P + 64 * b;
+                const uint64_t dv = b ? dv1 : dv0;
+                mma_f16_ts(tm + ATT_TM_O, pa, dv, ID_O, kb > 0);
+#pragma unroll
+                for (int kk = 1; kk < ATT_BK / 16; kk++)
+                    mma_f16_ts(tm + ATT_TM_O, pa + 8 * kk, dv + att_v_step(kk), ID_O, 1);
+                tc_commit(&o_done[b]);
+                tc_commit(&v_empty[b]);
+            }
+            tc_commit(fin);
+            drain_wait(fin, 0);
+        }
+        __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax, output
-        const int row = threadIdx.x;  // query q0 + row, tensor-memory lane row
-        const uint32_t tl = tm + ((uint32_t)(warp * 32) << 16);
+        const int qd = warp & 3, hf = warp >> 2;
+        const int row = 32 * qd + lane;  // query q0 + row, tensor-memory lane row
+        const int c0 = 64 * hf;          // this half's key columns of S, head-dim columns of O
+        const uint32_t tl = tm + ((uint32_t)(32 * qd) << 16);
+        // Swap x with the thread of the other half that owns the same row, at exchange u,
+        // through named barrier 1 + qd of the quadrant's two warps.  The barrier also
+        // ANDs the two warps' ok flags, so a wait that ran out in either warp stops
+        // both at the same exchange: neither is left waiting at the barrier.
+        auto swap = [&](int u, float x, float& other, bool ok_in) -> bool {
+            xval[((u & 1) * 2 + hf) * 128 + row] = x;
+            if (!named_barrier_and(1 + qd, 64, ok_in)) return false;
+            other = xval[((u & 1) * 2 + (hf ^ 1)) * 128 + row];
+            return true;
+        };
         float m = -INFINITY, l = 0.0f;
         bool ok = true;
         for (int kb = 0; kb < nkb; kb++) {
             const int b = kb & 1;
-            ok = __all_sync(~0u, att_wait(&s_full[b], (kb >> 1) & 1));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t sr[ATT_BK];
+            ok = ok && __all_sync(~0u, att_wait(&s_full[b], (kb >> 1) & 1));  // ok is warp-uniform
+            uint32_t sr[64];
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < ATT_BK / 16; j++) tmem_ld16(tl + b * ATT_BK + 16 * j, sr + 16 * j);
-            tmem_wait_ld();
-            // block maximum over the valid keys (eight independent chains)
-            const int kvalid = Lk - kb * ATT_BK;  // >= 1
+                for (int j = 0; j < 4; j++) tmem_ld16(tl + b * ATT_BK + c0 + 16 * j, sr + 16 * j);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; j++) sr[j] = 0u;
+            }
+            // half-block maximum over the valid keys (eight independent chains); -inf
+            // when this half lies past Lk
+            const int kvalid = Lk - kb * ATT_BK - c0;
             float mx[8];
 #pragma unroll
             for (int e = 0; e < 8; e++) mx[e] = -INFINITY;
+            if (kvalid >= 64) {  // uniform across the CTA: no masking
 #pragma unroll
-            for (int j = 0; j < ATT_BK; j++) {
-                const float x = j < kvalid ? __uint_as_float(sr[j]) : -INFINITY;
-                sr[j] = __float_as_uint(x);
-                mx[j & 7] = fmaxf(mx[j & 7], x);
+                for (int j = 0; j < 64; j++) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sr[j]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; j++) {
+                    const float x = j < kvalid ? __uint_as_float(sr[j]) : -INFINITY;
+                    sr[j] = __float_as_uint(x);
+                    mx[j & 7] = fmaxf(mx[j & 7], x);
+                }
             }
-            const float bm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+            const float hm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            const float mc = bm * ATT_C;
+            float om;
+            if (!swap(kb, hm, om, ok)) {
+                ok = false;
+                break;
+            }
+            const float mc = fmaxf(hm, om) * ATT_C;  // finite: the block has a valid key
             const bool raise = kb == 0 || mc > m + ATT_RESCALE_LOG2;
             const float m_new = raise ? mc : m;
             // P(kb) = 2^(s c - m_new) in f16 pairs; l sums the unrounded weights.
-            uint32_t pk[ATT_BK / 2];
+            uint32_t pk[32];
             float ps[8];
 #pragma unroll
             for (int e = 0; e < 8; e++) ps[e] = 0.0f;
 #pragma unroll
-            for (int j = 0; j < ATT_BK; j += 2) {
+            for (int j = 0; j < 64; j += 2) {
                 const float p0 = att_ex2(fmaf(__uint_as_float(sr[j]), ATT_C, -m_new));
                 const float p1 = att_ex2(fmaf(__uint_as_float(sr[j + 1]), ATT_C, -m_new));
                 ps[(j >> 1) & 7] += p0 + p1;
@@ -286,51 +336,56 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
             }
             const float ls = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+            // After a wait below runs out, the loop goes on to the next exchange (where
+            // both warps stop) without touching tensor memory or the P slot.
             if (kb >= 2) {
                 // P V(kb - 2) has read this P slot
                 ok = __all_sync(~0u, att_wait(&o_done[b], ((kb - 2) >> 1) & 1));
-                if (!ok) break;
+                if (!ok) continue;
                 tc_fence_after();
             }
             if (kb >= 1 && __any_sync(~0u, raise)) {
                 // O must hold blocks 0..kb-1 before it is rescaled to the new maximum
                 ok = __all_sync(~0u, att_wait(&o_done[b ^ 1], ((kb - 1) >> 1) & 1));
-                if (!ok) break;
+                if (!ok) continue;
                 tc_fence_after();
                 const float alpha = raise ? att_ex2(m - m_new) : 1.0f;
                 l *= alpha;
 #pragma unroll 1
-                for (int j = 0; j < ATT_DH / 16; j++) {
+                for (int j = 0; j < 4; j++) {
                     uint32_t t[16];
-                    tmem_ld16(tl + ATT_TM_O + 16 * j, t);
+                    tmem_ld16(tl + ATT_TM_O + c0 + 16 * j, t);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; e++) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
-                    tmem_st16(tl + ATT_TM_O + 16 * j, t);
+                    tmem_st16(tl + ATT_TM_O + c0 + 16 * j, t);
                 }
                 tmem_wait_st();
             }
             l += ls;
             m = m_new;
-            uint8_t* const pt = sP + b * ATT_TILE;
-#pragma unroll
-            for (int c8 = 0; c8 < ATT_BK / 8; c8++)
-                *reinterpret_cast<uint4*>(pt + att_off(row, 8 * c8)) =
-                    make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
-            fence_proxy_async_smem();
+            // this half's 64 keys = 32 columns of the P slot
+            const uint32_t pt = tl + ATT_TM_P + 64 * b + 32 * hf;
+            tmem_st16(pt, pk);
+            tmem_st16(pt + 16, pk + 16);
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[b]);
         }
+        // Both warps of the quadrant reach the final exchange: either both left the
+        // loop at the same exchange, or both finished it.
         if (ok) ok = __all_sync(~0u, att_wait(&o_done[(nkb - 1) & 1], ((nkb - 1) >> 1) & 1));
+        float lo = 0.0f;
+        ok = swap(nkb, l, lo, ok);
         if (ok) {
             tc_fence_after();
             const int qi = q0 + row;
-            const float inv = 1.0f / l;
-            float* dst = o + ((int64_t)qi * H + h) * ATT_DH;
+            const float inv = 1.0f / (l + lo);
+            float* dst = o + ((int64_t)qi * H + h) * ATT_DH + c0;
 #pragma unroll 1
-            for (int j = 0; j < ATT_DH / 16; j++) {
+            for (int j = 0; j < 4; j++) {
                 uint32_t t[16];
-                tmem_ld16(tl + ATT_TM_O + 16 * j, t);
+                tmem_ld16(tl + ATT_TM_O + c0 + 16 * j, t);
                 tmem_wait_ld();
                 if (qi < Lq) {
 #pragma unroll
@@ -344,7 +399,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == ATT_MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tm, ATT_TM_COLS);
     }

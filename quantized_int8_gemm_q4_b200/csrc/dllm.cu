@@ -81,6 +81,28 @@ bool encode_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t he
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The last few encoded maps, per host thread (a layer's q, k and v, a few layers deep):
+// encoding costs about as much host time as the launch itself.
+bool cached_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t heads) {
+    struct Entry {
+        const void* base;
+        int64_t rows, heads;
+        CUtensorMap map;
+    };
+    constexpr int N = 12;
+    thread_local Entry cache[N] = {};
+    thread_local int next = 0;
+    for (int i = 0; i < N; i++)
+        if (cache[i].base == base && cache[i].rows == rows && cache[i].heads == heads) {
+            *m = cache[i].map;
+            return true;
+        }
+    if (!encode_head_rows(m, base, rows, heads)) return false;
+    cache[next] = {base, rows, heads, *m};
+    next = (next + 1) % N;
+    return true;
+}
+
 int launch_status() {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
@@ -532,7 +554,7 @@ int dllm_attention(const void* q, const void* k, const void* v, int64_t Lq, int6
         g_att_attr_done[dev] = true;
     }
     CUtensorMap tq, tk, tv;
-    if (!encode_head_rows(&tq, q, Lq, H) || !encode_head_rows(&tk, k, Lk, Hkv) || !encode_head_rows(&tv, v, Lk, Hkv))
+    if (!cached_head_rows(&tq, q, Lq, H) || !cached_head_rows(&tk, k, Lk, Hkv) || !cached_head_rows(&tv, v, Lk, Hkv))
         return DLLM_ERR_CUDA;
     const dim3 grid((unsigned)((Lq + ATT_BQ - 1) / ATT_BQ), (unsigned)H);
     if (launch_pdl(attention_kernel, grid, dim3(ATT_THREADS), ATT_SMEM, reinterpret_cast<cudaStream_t>(stream), tq,

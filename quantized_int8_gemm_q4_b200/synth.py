@@ -150,6 +150,11 @@ class Model:
     out_rows: int = 32
     layer: tuple = field(default=())
     norm_eps: float = 1e-5
+    heads: int = 32  # attention heads; head dim = hidden / heads = 128 for both models
+
+    @property
+    def kv_heads(self) -> int:
+        return self.kv_out // (self.hidden // self.heads)
 
 
 def llada_8b() -> Model:
@@ -165,7 +170,7 @@ def dream_7b() -> Model:
     return Model("dream-7b", h, f, 28, h, 512, 152064, 32,
                  (Proj("q", Q4_K, h, h), Proj("k", Q4_K, 512, h), Proj("v", Q4_K, 512, h),
                   Proj("o", Q4_K, h, h), Proj("gate", Q4_K, f, h), Proj("up", Q4_K, f, h),
-                  Proj("down", Q6_K, h, f)), norm_eps=1e-6)
+                  Proj("down", Q6_K, h, f)), norm_eps=1e-6, heads=28)
 
 
 MODELS = {"llada-8b": llada_8b, "dream-7b": dream_7b}
@@ -210,3 +215,13 @@ def device_activations(M: int, K: int, seed, *sub, device="cuda"):
     import torch
     g = _torch_gen(device, seed, 8, *sub)
     return torch.randn((M, K), generator=g, device=device, dtype=torch.float32)
+
+
+def device_attention_inputs(Lq: int, Lk: int, H: int, Hkv: int, dh: int, seed, *sub, device="cuda"):
+    """f16 q [Lq][H][dh], k and v [Lk][Hkv][dh], standard normal, drawn on the device."""
+    import torch
+    g = _torch_gen(device, seed, 11, *sub)
+    q = torch.randn((Lq, H, dh), generator=g, device=device).to(torch.float16)
+    k = torch.randn((Lk, Hkv, dh), generator=g, device=device).to(torch.float16)
+    v = torch.randn((Lk, Hkv, dh), generator=g, device=device).to(torch.float16)
+    return q, k, v

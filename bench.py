@@ -68,6 +68,10 @@ def parse():
                         "c3 output projection on 1..32 requested rows, act the fused quantizers at the step's "
                         "canvas and at 2^24 elements, attn the bidirectional attention over canvases 128..4096; "
                         "one JSON line per case")
+    p.add_argument("--parallel", choices=["replicas", "nsplit"], default="replicas",
+                   help="with several ranks: replicas (each GPU runs the whole step, weak scaling) or nsplit "
+                        "(each GPU owns 1/N of every projection's weight rows, outputs all-gathered over NCCL, "
+                        "strong scaling)")
     p.add_argument("--gather-last", action="store_true",
                    help="the last layer's O and FFN, and the final norm, on the requested rows only")
     return p.parse_args()
@@ -656,6 +660,114 @@ def run_ours(args, rank, world):
     return result
 
 
+def run_nsplit(args, rank, world):
+    """The step with every projection column-parallel over the ranks (nsplit module):
+    each rank repacks its rows of every weight matrix; per layer it quantizes its own
+    copy of the inputs, runs its rows of QKV, O, gate/up and down, and all-gathers the
+    f32 outputs (the down input: its SwiGLU K-slice, quantized, is gathered instead).
+    Eager launches timed with CUDA events; max over ranks."""
+    import torch
+    from quantized_int8_gemm_q4_b200 import build, dllm, nsplit, synth
+
+    build.build()
+    dllm.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    model = synth.MODELS[args.model]()
+    n_layers = args.layers or model.n_layers
+    L, h, f = args.canvas, model.hidden, model.ffn
+    seed = 4
+
+    def shard(qt, N, K, *sub):
+        n0, n1, _ = nsplit.shard_rows(N, world, rank)
+        g = synth.device_weights(qt, N, K, seed, *sub, device=dev).view(N, -1)[n0:n1].contiguous().view(-1)
+        return nsplit.ColumnParallelQGemm(g, qt, N, K, world, rank, dev)
+
+    layers = []
+    for l in range(n_layers):
+        layers.append({p.name: shard(p.qtype, p.N, p.K, l, pi) for pi, p in enumerate(model.layer)})
+    out_proj = shard(Q6, model.vocab, h, 999, 0)
+    torch.cuda.synchronize()
+    x = {n: synth.device_activations(L, h, seed, 100 + i, device=dev) for i, n in enumerate(("attn", "o", "ffn"))}
+    x_fin = synth.device_activations(L, h, seed, 104, device=dev)
+    gam = torch.from_numpy(synth.norm_weights(2 * n_layers + 1, h, seed)).to(dev)
+    rows = torch.from_numpy(synth.block_rows(L, model.out_rows, seed)).to(dev)
+    R = rows.numel()
+    act_h, act_r = dllm.alloc_act(L, h, dev), dllm.alloc_act(R, h, dev)
+    k0, k1 = nsplit.shard_k(f, world, rank)
+    act_fl, act_f = dllm.alloc_act(L, k1 - k0, dev), dllm.alloc_act(L, f, dev)
+    P = layers[0]
+    bufs = {}
+    for name, cp, M in [(n, P[n], L) for n in ("q", "k", "v", "o", "gate", "up", "down")] + [("out", out_proj, R)]:
+        bufs[name] = (torch.zeros((M, cp.Wp), device=dev), torch.empty((M, cp.N), device=dev),
+                      torch.empty((world * M, cp.Wp), device=dev))
+    wsb = max(max(cp.workspace_bytes(L) for cp in P.values()), out_proj.workspace_bytes(R), 256)
+    ws = dllm.alloc_workspace(wsb, dev)
+    gl, ul = bufs["gate"][0], bufs["up"][0]
+    fs = k1 - k0  # this rank's gate/up columns are the down input's K-slice
+
+    def proj(cp, name, act, M):
+        loc, full, scr = bufs[name]
+        cp(act, M, full, loc, scr, ws, wsb)
+
+    def step():
+        for l in range(n_layers):
+            W = layers[l]
+            dllm.dllm_rmsnorm_quantize(x["attn"], L, h, h, gam[2 * l], model.norm_eps, None, 0, *act_h)
+            for n in ("q", "k", "v"):
+                proj(W[n], n, act_h, L)
+            dllm.dllm_quantize_act(x["o"], L, h, h, *act_h)
+            proj(W["o"], "o", act_h, L)
+            dllm.dllm_rmsnorm_quantize(x["ffn"], L, h, h, gam[2 * l + 1], model.norm_eps, None, 0, *act_h)
+            W["gate"].local(act_h, L, gl, ws, wsb)
+            W["up"].local(act_h, L, ul, ws, wsb)
+            dllm.dllm_swiglu_quantize(gl, ul, L, fs, W["gate"].Wp, *act_fl)
+            nsplit.gather_act_k(act_fl, act_f, world)
+            proj(W["down"], "down", act_f, L)
+        dllm.dllm_rmsnorm_quantize(x_fin, L, h, h, gam[2 * n_layers], model.norm_eps, rows, R, *act_r)
+        proj(out_proj, "out", act_r, R)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_step = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    gemms = step_gemms(model, L, n_layers)
+    ops_step = sum(g.ops for g in gemms)
+    cfg = workload_config(model, L, n_layers, R, world)
+    cfg["parallelism"] = f"nsplit x{world}: weight rows column-parallel, f32 outputs all-gathered (NCCL)"
+    cfg["graph"] = "eager launches (collectives in the step)"
+    # our kernels per rank and step: per layer 4 quantizers + 7 GEMMs; the final norm and
+    # the output projection (the gathers are NCCL / copy kernels, not counted)
+    per_rank_launches = n_layers * 11 + 2
+    return {
+        "metric": METRIC, "value": round(ops_step / (ms_step * 1e-3) / 1e12, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": cfg,
+        "roofline": None, "cpu_baseline": None, "e2e": None,
+        "parity": {"checked": False, "reason": "the split's gather logic is checked against the oracle by "
+                                              "tests/test_nsplit.py; the GEMMs are the step's own kernels"},
+        "clocks": clocks, "gpu_launches": per_rank_launches * args.steps,
+    }
+
+
 def parity_sample(model, n_layers, full_layers, seed):
     """The oracle's sample of the step, as (layer, projection) -> output column range
     [n0, n1): the first full_layers - 1 layers and the last in full, every other layer's
@@ -1034,7 +1146,7 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    res = run_ours(args, rank, world)
+    res = run_nsplit(args, rank, world) if args.parallel == "nsplit" else run_ours(args, rank, world)
     if rank == 0:
         print(json.dumps(res), flush=True)
     par = res.get("parity") or {}

@@ -47,8 +47,14 @@ extern "C" {
 
 typedef struct CUstream_st* dllm_stream_t; /* a cudaStream_t; NULL = legacy default stream */
 
-/* GGML type ids of the two weight formats. */
-typedef enum { DLLM_Q4_K = 12, DLLM_Q6_K = 14 } dllm_qtype;
+/* GGML type ids of the weight formats.  Q5_K (mojo-dllm Architecture page, "Source map",
+ * quant/kquants.mojo row) runs on the Q4_K kernel in an exact split form: dllm_repack_q5k
+ * turns each 176-byte Q5_K super-block into two Q4_K-form super-blocks of a matrix twice
+ * as wide, the low nibbles (d, dmin, the same scales) and the fifth bits as 0/1 nibbles
+ * (16*d, dmin 0, the same scales), since d*sc*q - dmin*m = (d*sc*q4 - dmin*m) +
+ * (16d)*sc*b exactly.  It keeps 2 x 144 bytes per 256 weights resident (9 bits per
+ * weight, 1.64 x the GGUF size) and streams them at the Q4_K kernel's rate. */
+typedef enum { DLLM_Q4_K = 12, DLLM_Q5_K = 13, DLLM_Q6_K = 14 } dllm_qtype;
 
 enum {
     DLLM_OK = 0,
@@ -80,6 +86,12 @@ enum {
 int dllm_repacked_bytes(dllm_qtype t, int64_t N, int64_t K, size_t* out_bytes); /* host pointer */
 int dllm_repack_q4k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
 int dllm_repack_q6k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
+/* Q5_K: gguf_blocks is [N][K/256] 176-byte blocks; dst receives the Q4_K tile layout of
+ * the split form, [N/128][2K/256] tiles of 18432 bytes (super-block s of a row at tile
+ * column s for its low nibbles and K/256 + s for its fifth bits).  dllm_repacked_bytes
+ * gives the size.  dllm_qgemm / dllm_qkv_qgemm / dllm_qgemm_noalloc take t = DLLM_Q5_K
+ * with the ordinary K-wide activations. */
+int dllm_repack_q5k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
 
 /* ------------------------------------------------------------------------------
  * Activations: int8 with one f32 scale per 256 elements, plus scaled per-32 sums

@@ -174,9 +174,11 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // ever overlap, whatever its shape: calls of different shapes can share a workspace.
 constexpr size_t CTR_REGION = (size_t)64 << 10;
 
-Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
+// K: the weight matrix's width in the kernel's form (2K for Q5_K); K_act: the
+// activation width (the gathered requested rows are K_act wide).
+Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms, int64_t K_act) {
     Plan p;
-    const int64_t nsb = K / QK;
+    const int64_t nsb = K / QK, nsb_act = K_act / QK;
     p.Mp = round_up(n_rows > 0 ? n_rows : M, 16);
     p.kc = choose_kc(n_tiles, nsb, sms);
     p.full_tiles = p.tail_k = p.tail_big = 0;
@@ -200,11 +202,11 @@ Plan make_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms) {
     p.gq_off = p.gs_off = p.gu_off = off;
     if (n_rows > 0) {
         p.gq_off = off;
-        off += align256((size_t)p.Mp * K);
+        off += align256((size_t)p.Mp * K_act);
         p.gs_off = off;
-        off += align256((size_t)nsb * p.Mp * 4);
+        off += align256((size_t)nsb_act * p.Mp * 4);
         p.gu_off = off;
-        off += align256((size_t)nsb * p.Mp * 64);
+        off += align256((size_t)nsb_act * p.Mp * 64);
     }
     p.bytes = (p.split || n_rows > 0) ? off : 0;
     return p;
@@ -237,8 +239,15 @@ int run_gemm(GemmArgs& a, cudaStream_t s) {
     return launch_status();
 }
 
+// Q5_K runs on the Q4_K kernel in its exact two-super-block form (see repack_q5k_kernel):
+// weight width 2K, 2 x 144 repacked bytes per 256 weights.
+int64_t kernel_k(dllm_qtype t, int64_t K) { return t == DLLM_Q5_K ? 2 * K : K; }
+size_t repacked_per_sb(dllm_qtype t) {
+    return t == DLLM_Q4_K ? Q4K_BLOCK : t == DLLM_Q5_K ? 2 * Q4K_BLOCK : Q6K_BLOCK;
+}
+
 int check_shape(dllm_qtype t, int64_t N, int64_t K) {
-    if (t != DLLM_Q4_K && t != DLLM_Q6_K) return DLLM_ERR_ARG;
+    if (t != DLLM_Q4_K && t != DLLM_Q5_K && t != DLLM_Q6_K) return DLLM_ERR_ARG;
     if (N <= 0 || K <= 0 || N % TROWS || K % QK) return DLLM_ERR_ARG;
     if (N / TROWS > (1LL << 30) || K / QK > (1 << 20)) return DLLM_ERR_ARG;
     return DLLM_OK;
@@ -258,7 +267,7 @@ int dllm_repacked_bytes(dllm_qtype t, int64_t N, int64_t K, size_t* out_bytes) {
     int rc = check_shape(t, N, K);
     if (rc) return rc;
     if (!out_bytes) return DLLM_ERR_ARG;
-    *out_bytes = (size_t)N * (size_t)(K / QK) * (t == DLLM_Q4_K ? Q4K_BLOCK : Q6K_BLOCK);
+    *out_bytes = (size_t)N * (size_t)(K / QK) * repacked_per_sb(t);
     return DLLM_OK;
 }
 
@@ -267,16 +276,19 @@ static int repack(dllm_qtype t, const void* src, int64_t N, int64_t K, void* dst
     if (rc) return rc;
     if (!src || !dst) return DLLM_ERR_ARG;
     if (!aligned16(dst)) return DLLM_ERR_ALIGN;
-    const size_t bytes = (size_t)N * (K / QK) * (t == DLLM_Q4_K ? Q4K_BLOCK : Q6K_BLOCK);
+    const size_t bytes = (size_t)N * (K / QK) * repacked_per_sb(t);
+    const size_t src_bytes = (size_t)N * (K / QK) * (t == DLLM_Q4_K ? Q4K_BLOCK : t == DLLM_Q5_K ? Q5K_BLOCK : Q6K_BLOCK);
     const uint8_t* s8 = static_cast<const uint8_t*>(src);
     const uint8_t* d8 = static_cast<const uint8_t*>(dst);
-    if (s8 < d8 + bytes && d8 < s8 + bytes) return DLLM_ERR_ARG;
+    if (s8 < d8 + bytes && d8 < s8 + src_bytes) return DLLM_ERR_ARG;
     int dev;
     if ((rc = current_device(&dev))) return rc;
     const int64_t chunks = (int64_t)(bytes / 16);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (t == DLLM_Q4_K)
         repack_q4k_kernel<<<grid_for(chunks, 256), 256, 0, s>>>(s8, N, K / QK, static_cast<uint8_t*>(dst));
+    else if (t == DLLM_Q5_K)
+        repack_q5k_kernel<<<grid_for(chunks, 256), 256, 0, s>>>(s8, N, K / QK, static_cast<uint8_t*>(dst));
     else
         repack_q6k_kernel<<<grid_for(chunks, 256), 256, 0, s>>>(s8, N, K / QK, static_cast<uint8_t*>(dst));
     return launch_status();
@@ -287,6 +299,9 @@ int dllm_repack_q4k(const void* g, int64_t N, int64_t K, void* dst, dllm_stream_
 }
 int dllm_repack_q6k(const void* g, int64_t N, int64_t K, void* dst, dllm_stream_t s) {
     return repack(DLLM_Q6_K, g, N, K, dst, s);
+}
+int dllm_repack_q5k(const void* g, int64_t N, int64_t K, void* dst, dllm_stream_t s) {
+    return repack(DLLM_Q5_K, g, N, K, dst, s);
 }
 
 int dllm_act_bytes(int64_t M, int64_t K, size_t* q_bytes, size_t* scale_bytes, size_t* sums_bytes) {
@@ -366,7 +381,7 @@ int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, in
     if (M <= 0 || n_rows < 0 || n_rows > 32 || !bytes) return DLLM_ERR_ARG;
     int dev;
     if ((rc = current_device(&dev))) return rc;
-    *bytes = make_plan(N / TROWS, K, M, n_rows, g_num_sms[dev]).bytes;
+    *bytes = make_plan(N / TROWS, kernel_k(t, K), M, n_rows, g_num_sms[dev], K).bytes;
     return DLLM_OK;
 }
 
@@ -384,7 +399,8 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
     if (workspace && !aligned16(workspace)) return DLLM_ERR_ALIGN;
     int dev;
     if ((rc = current_device(&dev))) return rc;
-    Plan p = make_plan(N_total / TROWS, K, M, rows ? n_rows : 0, g_num_sms[dev]);
+    if (dbg && t == DLLM_Q5_K) return DLLM_ERR_ARG;  // the integer debug view covers Q4_K and Q6_K
+    Plan p = make_plan(N_total / TROWS, kernel_k(t, K), M, rows ? n_rows : 0, g_num_sms[dev], K);
     if (dbg) {  // integers per super-block: no chunk partials to combine
         p.kc = 1;
         p.full_tiles = p.tail_k = p.tail_big = 0;
@@ -394,8 +410,9 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
     }
     if (p.bytes > 0 && (!workspace || workspace_bytes < p.bytes)) return DLLM_ERR_WORKSPACE;
     memset(&a, 0, sizeof(a));
-    const int64_t nsb = K / QK;
-    a.nsb = (int32_t)nsb;
+    const int64_t nsb = K / QK;  // activation super-blocks
+    a.nsb = (int32_t)(kernel_k(t, K) / QK);
+    a.nsb_act = (int32_t)nsb;
     a.kc = p.kc;
     a.full_tiles = p.full_tiles;
     a.tail_k = p.tail_k;
@@ -432,8 +449,8 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
 }
 
 static int dispatch(GemmArgs& a, dllm_qtype t, bool dbg, cudaStream_t s) {
-    // the debug integers never split K (uniform plan, one chunk)
-    if (t == DLLM_Q4_K) {
+    // the debug integers never split K (uniform plan, one chunk); Q5_K runs as Q4_K
+    if (t == DLLM_Q4_K || t == DLLM_Q5_K) {
         if (dbg) return run_gemm<12, true, false>(a, s);
         return a.tail_k > 0 ? run_gemm<12, false, true>(a, s) : run_gemm<12, false, false>(a, s);
     }
@@ -526,7 +543,7 @@ int dllm_qgemm_noalloc(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
     if (M > (1LL << 31)) return DLLM_ERR_ARG;
     int dev;
     if ((rc = current_device(&dev))) return rc;
-    const Plan p = make_plan(N / TROWS, K, M, rows ? n_rows : 0, g_num_sms[dev]);
+    const Plan p = make_plan(N / TROWS, kernel_k(t, K), M, rows ? n_rows : 0, g_num_sms[dev], K);
     if (p.bytes > DLLM_NOALLOC_SCRATCH_BYTES) return DLLM_ERR_SCRATCH_LIMIT;
     uint8_t* scratch;
     if ((rc = noalloc_scratch(dev, &scratch))) return rc;
@@ -710,6 +727,7 @@ int dllm_debug_subblock_dots(const void* w, dllm_qtype t, int64_t N, int64_t K, 
                              int32_t* dots, dllm_stream_t stream) {
     int rc = check_shape(t, N, K);
     if (rc) return rc;
+    if (t == DLLM_Q5_K) return DLLM_ERR_ARG;
     if (!w || !q || !dots || M <= 0) return DLLM_ERR_ARG;
     int dev;
     if ((rc = current_device(&dev))) return rc;
@@ -743,6 +761,7 @@ int dllm_debug_bounded_wait(dllm_stream_t stream) {
     a.nseg = 1;
     a.n_tiles = 1;
     a.nsb = 1;
+    a.nsb_act = 1;
     a.kc = 1;
     a.n_units = 1;
     a.Mp = 16;
@@ -757,7 +776,7 @@ int dllm_debug_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int s
     if (n_tiles <= 0 || n_tiles > (1LL << 30) || K <= 0 || K % QK || K / QK > (1 << 20) || M <= 0 ||
         M > (1LL << 31) || n_rows < 0 || n_rows > 32 || sms <= 0 || sms > 4096 || !out)
         return DLLM_ERR_ARG;
-    const Plan p = make_plan(n_tiles, K, M, n_rows, sms);
+    const Plan p = make_plan(n_tiles, K, M, n_rows, sms, K);
     out[0] = p.kc;
     out[1] = p.full_tiles;
     out[2] = p.tail_k;

@@ -23,6 +23,7 @@ constexpr int QK = 256;             // weights per super-block
 constexpr int TROWS = 128;          // weight rows per tile (= tensor-memory lanes)
 constexpr int Q4K_BLOCK = 144;
 constexpr int Q6K_BLOCK = 210;
+constexpr int Q5K_BLOCK = 176;
 constexpr int Q4K_TILE = TROWS * Q4K_BLOCK;  // 18432
 constexpr int Q6K_TILE = TROWS * Q6K_BLOCK;  // 26880
 
@@ -67,6 +68,67 @@ __global__ void repack_q4k_kernel(const uint8_t* __restrict__ src, int64_t N, in
             for (int b = 0; b < 16; b++) {
                 const int r = (o + b) / 4, j = (o + b) % 4;
                 out[b] = src[((t * TROWS + r) * nsb + s) * Q4K_BLOCK + j];
+            }
+        }
+        uint4 v;
+        memcpy(&v, out, 16);
+        reinterpret_cast<uint4*>(dst)[g] = v;
+    }
+}
+
+// Q5_K (d, dmin, 12 scale bytes, 32 bytes of fifth bits qh, 128 bytes of low nibbles
+// qs; weight d*sc_j*q - dmin*m_j with q = low nibble + 16 * fifth bit) as two Q4_K-form
+// super-blocks of a matrix twice as wide: super-block s of a row becomes
+//   s            the low nibbles: d, dmin, the same scale bytes, qs unchanged
+//   nsb + s      the fifth bits as nibbles (0 or 1): d' = 16 d (exact: a power of two),
+//                dmin' = 0, the same scale bytes
+// so that d*sc*q - dmin*m = (d*sc*q4 - dmin*m) + (16 d)*sc*b exactly.  The result is in
+// the Q4_K tile layout for nsb2 = 2 nsb super-blocks per row.
+__global__ void repack_q5k_kernel(const uint8_t* __restrict__ src, int64_t N, int64_t nsb,
+                                  uint8_t* __restrict__ dst) {
+    const int64_t nsb2 = 2 * nsb;
+    const int64_t chunks_per_tile = Q4K_TILE / 16;  // 1152
+    const int64_t total = (N / TROWS) * nsb2 * chunks_per_tile;
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tile = g / chunks_per_tile;
+        const int c = (int)(g % chunks_per_tile);
+        const int64_t t = tile / nsb2, s2 = tile % nsb2;
+        const bool hi = s2 >= nsb;
+        const int64_t s = hi ? s2 - nsb : s2;
+        uint8_t out[16];
+        if (c < 1024) {  // quants: piece i (bytes 16i..16i+15 of the 128) of row r
+            const int i = c / TROWS, r = c % TROWS;
+            const uint8_t* blk = src + ((t * TROWS + r) * nsb + s) * Q5K_BLOCK;
+#pragma unroll
+            for (int b = 0; b < 16; b++) {
+                const int e = 16 * i + b, cc = e >> 5, l = e & 31;  // 32-byte chunk cc, element l
+                const uint8_t qh = blk[16 + l];
+                out[b] = hi ? (uint8_t)(((qh >> (2 * cc)) & 1) | (((qh >> (2 * cc + 1)) & 1) << 4)) : blk[48 + e];
+            }
+        } else if (c < 1024 + 96) {  // 12 scale bytes per row
+            const int o = (c - 1024) * 16;
+#pragma unroll
+            for (int b = 0; b < 16; b++) {
+                const int r = (o + b) / 12, j = (o + b) % 12;
+                out[b] = src[((t * TROWS + r) * nsb + s) * Q5K_BLOCK + 4 + j];
+            }
+        } else {  // d, dmin: 4 bytes per row
+            const int o = (c - 1120) * 16;
+#pragma unroll
+            for (int b = 0; b < 16; b++) {
+                const int r = (o + b) / 4, j = (o + b) % 4;
+                const uint8_t* blk = src + ((t * TROWS + r) * nsb + s) * Q5K_BLOCK;
+                if (!hi) {
+                    out[b] = blk[j];
+                } else if (j < 2) {
+                    const unsigned short dbits = (unsigned short)(blk[0] | (blk[1] << 8));
+                    const unsigned short d16 =
+                        __half_as_ushort(__float2half_rn(16.0f * __half2float(__ushort_as_half(dbits))));
+                    out[b] = (uint8_t)(j == 0 ? d16 & 255 : d16 >> 8);
+                } else {
+                    out[b] = 0;  // dmin' = +0
+                }
             }
         }
         uint4 v;

@@ -151,7 +151,8 @@ struct GemmArgs {
     Segment seg[3];
     int nseg;
     int32_t n_tiles;   // total 128-row tiles over all segments
-    int32_t nsb;       // K / 256
+    int32_t nsb;       // weight super-blocks per row (K / 256; 2K / 256 for Q5_K's split form)
+    int32_t nsb_act;   // activation super-blocks per row: weight super-block s reads s % nsb_act
     int32_t kc;        // K-chunks per tile (uniform split: tail_k == 0)
     // Tail split (tail_k > 0): tiles [0, full_tiles) run whole, one round of one tile per
     // CTA at a time; each remaining tile is cut into K-pieces so that the pieces fill
@@ -409,17 +410,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                         } else {
                             uint8_t* bs = b_stage + st * C::B_STAGE;
                             const int64_t t0 = un.m0;
+                            const int64_t sa = s % args.nsb_act;  // activation super-block
                             const uint32_t ntok = (uint32_t)un.len;
                             const uint32_t sums_bytes = C::B_SUMS ? ntok / 8 * SUMS_GROUP : 0;
                             if (part == 0) mbar_arrive_expect_tx(&full[st], ntok * 256 + sums_bytes + ntok * 4);
                             __syncwarp(smask);  // the stage's byte count is armed before any of its copies lands
                             if (part == 0)
-                                bulk_g2s_hint(bs, args.q + ((size_t)s * args.Mp + t0) * 256, ntok * 256, &full[st], pol);
+                                bulk_g2s_hint(bs, args.q + ((size_t)sa * args.Mp + t0) * 256, ntok * 256, &full[st], pol);
                             else if (part == 1)
-                                bulk_g2s_hint(bs + C::B_Q, args.sums + ((size_t)s * args.Mp + t0) / 8 * SUMS_GROUP,
+                                bulk_g2s_hint(bs + C::B_Q, args.sums + ((size_t)sa * args.Mp + t0) / 8 * SUMS_GROUP,
                                               sums_bytes, &full[st], pol);
                             else
-                                bulk_g2s_hint(bs + C::B_Q + C::B_SUMS, args.scale + (size_t)s * args.Mp + t0, ntok * 4,
+                                bulk_g2s_hint(bs + C::B_Q + C::B_SUMS, args.scale + (size_t)sa * args.Mp + t0, ntok * 4,
                                               &full[st], pol);
                         }
                         inflight = true;

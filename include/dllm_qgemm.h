@@ -16,7 +16,13 @@
  *   a = scale[m][k/256] * qa  (qa int8 in [-127, 127])
  *
  * Integer parts are exact (int32 tensor-core accumulation per super-block); the
- * per-super-block combine with d, dmin and the activation scale is f32.
+ * per-super-block combine with d and the activation scale is f32.  The Q4_K min term
+ * (dmin * m_j times the scaled activation sums) runs on the tf32 tensor cores: the
+ * hi + lo operand splits lose at most 2^-21 of each product's magnitude, and its f32
+ * accumulation over a work unit's K/32 sub-block steps adds at most (K/32) * 2^-24 of
+ * the running sum of magnitudes (2^-17 at K = 4096); both stay inside the tolerance
+ * max(1e-5 |ref|, 1e-6 * sum|terms|), and the tests run the worst case (every term of
+ * one sign, every m = 63, saturated activations) at K = 512, 3584 and 4096.
  *
  * Conventions for every call:
  *   - Device pointers unless stated otherwise; the caller allocates and owns every

@@ -835,27 +835,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     }
                     if (!epi_sync(sh, epi_ph)) goto epi_done;
                     if (sh.last_flag && live) {
-                        // sum the piece partials in piece order, four 16-byte loads in flight
-                        // at a time
-                        for (int c2 = 0; c2 < np; c2++) {
-                            const int64_t slot = TAIL ? un.slot0 + (int64_t)c2 * un.pstride : u - un.chunk + c2;
-                            const float* pp = args.partials + (size_t)slot * args.mu * TROWS + row * 4;
+                        // sum the piece partials in piece order.  Per 16-column group, up to
+                        // four pieces' loads (16 x 16 bytes) are in flight together: each
+                        // batch costs one L2 round trip.
 #pragma unroll
-                            for (int c4 = 0; c4 < EPI_COLS / 16; c4++) {
-                                float4 pv[4];
+                        for (int c4 = 0; c4 < EPI_COLS / 16; c4++) {
+#pragma unroll 1
+                            for (int c2b = 0; c2b < np; c2b += 4) {
+                                float4 pv[4][4];
 #pragma unroll
-                                for (int q4 = 0; q4 < 4; q4++) {
-                                    const int ml = (int)col0 + 16 * c4 + 4 * q4;
-                                    pv[q4] = ml < un.len
-                                                 ? __ldcg(reinterpret_cast<const float4*>(pp + (size_t)(ml / 4) * TROWS * 4))
-                                                 : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                                for (int k = 0; k < 4; k++) {
+                                    const int c2 = c2b + k;
+                                    const int64_t slot =
+                                        TAIL ? un.slot0 + (int64_t)c2 * un.pstride : u - un.chunk + c2;
+                                    const float* pp = args.partials + (size_t)slot * args.mu * TROWS + row * 4;
+#pragma unroll
+                                    for (int q4 = 0; q4 < 4; q4++) {
+                                        const int ml = (int)col0 + 16 * c4 + 4 * q4;
+                                        pv[k][q4] = c2 < np && ml < un.len
+                                                        ? __ldcg(reinterpret_cast<const float4*>(pp + (size_t)(ml / 4) * TROWS * 4))
+                                                        : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                                    }
                                 }
 #pragma unroll
-                                for (int q4 = 0; q4 < 4; q4++) {
-                                    const int a2 = 8 * c4 + 2 * q4;
-                                    const float2 lo = make_float2(pv[q4].x, pv[q4].y), hi = make_float2(pv[q4].z, pv[q4].w);
-                                    acc[a2] = c2 == 0 ? lo : __fadd2_rn(acc[a2], lo);
-                                    acc[a2 + 1] = c2 == 0 ? hi : __fadd2_rn(acc[a2 + 1], hi);
+                                for (int k = 0; k < 4; k++) {
+                                    const int c2 = c2b + k;
+                                    if (c2 < np) {
+#pragma unroll
+                                        for (int q4 = 0; q4 < 4; q4++) {
+                                            const int a2 = 8 * c4 + 2 * q4;
+                                            const float2 lo = make_float2(pv[k][q4].x, pv[k][q4].y);
+                                            const float2 hi = make_float2(pv[k][q4].z, pv[k][q4].w);
+                                            acc[a2] = c2 == 0 ? lo : __fadd2_rn(acc[a2], lo);
+                                            acc[a2 + 1] = c2 == 0 ? hi : __fadd2_rn(acc[a2 + 1], hi);
+                                        }
+                                    }
                                 }
                             }
                         }

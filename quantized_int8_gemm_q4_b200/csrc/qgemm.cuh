@@ -34,7 +34,7 @@
 // the running sum of magnitudes (about 2^-17 at K = 4096); both bounds are relative to
 // the min term's own sum of |terms|, a part of the 1e-6 * sum|terms| tolerance.
 //
-// Pipeline (20 warps, one CTA per SM, persistent over work units).  Per super-block
+// Pipeline (16 warps, one CTA per SM, persistent over work units).  Per super-block
 // the MMAs run plane-major: the 8 K-steps of plane 0 into accumulator P0, then the 8
 // of plane 1 into P1, then (Q4_K) the 3 min-term MMAs.  Every MMA covers all of the
 // unit's tokens (N <= 128; at N = 128 one int8 MMA takes ~64 cycles, the pipe's full
@@ -48,11 +48,13 @@
 //   warp 2      activation producer: bulk copies of activation tiles (int8 codes,
 //               scales, scaled sums), after the dependency wait
 //   warp 3      MMA issuer of plane 1 and of the min term (one thread)
-//   warps 4-11  unpack, two groups of four: thread = weight row; each group builds
-//               one quarter super-block (two K-steps, both weight planes) of every
-//               half super-block into a tensor-memory ring (the A operand); group 0
-//               also writes the min-term A operand (Q4_K) to shared memory and the f32 d
-//   warps 12-19 epilogue: two warps per tensor-memory lane quadrant, each on 64 of the
+//   warps 4-7   unpack, one group of four (UNPACK_GROUPS): thread = weight row; it
+//               builds both quarter super-blocks (two K-steps each, both weight planes)
+//               of every half super-block into a tensor-memory ring (the A operand), and
+//               writes the min-term A operand (Q4_K) to shared memory and the f32 d.
+//               A second group (20 warps, each group one quarter) measured slower: the
+//               512-thread CTA leaves the issuers and the epilogue more issue slots.
+//   warps 8-15  epilogue: two warps per tensor-memory lane quadrant, each on 64 of the
 //               token columns
 //
 // A work unit is (128 weight rows, up to 128 canvas rows, one K-chunk).  The number
@@ -66,7 +68,14 @@ namespace dllm {
 
 constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float MAGIC = 12582912.0f;
-constexpr int GEMM_THREADS = 640;
+// Unpack groups of four warps (one warp per tensor-memory lane quadrant).  With one
+// group the CTA has 512 threads, which leaves the epilogue enough registers to copy a
+// whole plane accumulator out and release it before its arithmetic.
+constexpr int UNPACK_GROUPS = 1;
+constexpr int UNPACK_THREADS = 128 * UNPACK_GROUPS;
+constexpr int EPI_WARP0 = 4 + 4 * UNPACK_GROUPS;  // first epilogue warp
+constexpr int GEMM_THREADS = 128 + UNPACK_THREADS + 256;
+constexpr bool EARLY_RELEASE = false;
 constexpr int UNIT_TOKENS = 128;
 constexpr int EPI_COLS = 64;                       // token columns per epilogue thread
 constexpr int MAX_KC = 16;                         // K-chunks per tile, at most
@@ -74,14 +83,15 @@ constexpr int S_SLOTS = 4;                         // d ring (unpack -> epilogue
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 // Registers per thread of each warpgroup after setmaxnreg: producers and issuers (one
 // warpgroup), unpack (two) and epilogue (two).  setmaxnreg.inc draws on the registers the
-// CTA was launched with (640 threads x the kernel's register count), so the split must
+// CTA was launched with (its threads x the kernel's register count), so the split must
 // not exceed them, or the increasing warps would wait for registers that never come
 // free.  REG_LAUNCH_MIN is the launch count the split assumes; the host checks the
 // compiled kernel's count against it before the first launch.
-constexpr int REG_CTRL = 48, REG_UNPACK = 64, REG_EPI = 152;
-constexpr int REG_SPLIT_TOTAL = 128 * REG_CTRL + 256 * REG_UNPACK + 256 * REG_EPI;
-constexpr int REG_LAUNCH_MIN = 96;
-static_assert(REG_SPLIT_TOTAL <= 640 * REG_LAUNCH_MIN && 640 * REG_LAUNCH_MIN <= 65536, "register split over the launch budget");
+constexpr int REG_CTRL = 48, REG_UNPACK = 64, REG_EPI = UNPACK_GROUPS == 1 ? 200 : 152;
+constexpr int REG_SPLIT_TOTAL = 128 * REG_CTRL + UNPACK_THREADS * REG_UNPACK + 256 * REG_EPI;
+constexpr int REG_LAUNCH_MIN = 65536 / GEMM_THREADS / 8 * 8;
+static_assert(REG_SPLIT_TOTAL <= GEMM_THREADS * REG_LAUNCH_MIN && GEMM_THREADS * REG_LAUNCH_MIN <= 65536,
+              "register split over the launch budget");
 static_assert(REG_CTRL % 8 == 0 && REG_UNPACK % 8 == 0 && REG_EPI % 8 == 0 && REG_CTRL >= 24, "setmaxnreg counts");
 
 // Activation "sums" operand of one super-block: per 8-row group 512 bytes =
@@ -342,11 +352,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
     const int64_t n_units = args.n_units;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], 256); }
+        for (int i = 0; i < C::W_STAGES; i++) { mbar_init(&sh.w_full[i], 1); mbar_init(&sh.w_empty[i], UNPACK_THREADS); }
         // an activation stage is released by a commit from each issuer (their MMAs are
         // done) and by the 256 epilogue threads (the scales are read)
         for (int i = 0; i < C::B_STAGES; i++) { mbar_init(&sh.b_full[i], 1); mbar_init(&sh.b_empty[i], 258); }
-        for (int i = 0; i < C::A_SLOTS; i++) { mbar_init(&sh.a_full[i], 256); mbar_init(&sh.a_empty[i], 2); }
+        for (int i = 0; i < C::A_SLOTS; i++) { mbar_init(&sh.a_full[i], UNPACK_THREADS); mbar_init(&sh.a_empty[i], 2); }
         for (int i = 0; i < 2; i++) { mbar_init(&sh.p_full[i], 1); mbar_init(&sh.p_empty[i], 256); }
         for (int i = 0; i < 2; i++) { mbar_init(&sh.m_full[i], 128); mbar_init(&sh.m_empty[i], 1); }
         mbar_init(&sh.min_full, 1);
@@ -510,7 +520,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
             (void)drain_bar(&sh.final_bar, 0);
             __syncwarp();
         }
-    } else if (warp < 12) {
+    } else if (warp < EPI_WARP0) {
         setmaxnreg_dec<REG_UNPACK>();
         // ============================================================ unpack
         // Two groups of four warps (one warp per lane quadrant each).  Per super-block
@@ -568,9 +578,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     }
 #pragma unroll 1
                     for (int hh = 0; hh < 2; hh++) {
-                        const int q = 2 * hh + grp;
                         const uint32_t hc = 2 * sbc + hh, sl = hc % C::A_SLOTS;
                         if (!wait_bar_warp(sh, &sh.a_empty[sl], ((hc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
+#pragma unroll 1
+                        for (int gq = grp; gq < 2; gq += UNPACK_GROUPS) {
+                        const int q = 2 * hh + gq;
                         // 32-byte quant chunk q: sub-block 2q in the low nibbles, 2q+1 in the high
                         const uint4 p0 = *reinterpret_cast<const uint4*>(tl + ((2 * q) * TROWS + row) * 16);
                         const uint4 p1 = *reinterpret_cast<const uint4*>(tl + ((2 * q + 1) * TROWS + row) * 16);
@@ -588,7 +600,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 v[i] = nib * lo3;
                                 v[8 + i] = nib * hi3;
                             }
-                            tmem_st16(tmem + lane_off + TM_A + 64 * sl + 32 * grp + 16 * kk, v);
+                            tmem_st16(tmem + lane_off + TM_A + 64 * sl + 32 * gq + 16 * kk, v);
+                        }
                         }
                         tmem_wait_st();
                         tc_fence_before();
@@ -607,9 +620,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     }
 #pragma unroll 1
                     for (int hh = 0; hh < 2; hh++) {
-                        const int q = 2 * hh + grp;
                         const uint32_t hc = 2 * sbc + hh, sl = hc % C::A_SLOTS;
                         if (!wait_bar_warp(sh, &sh.a_empty[sl], ((hc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
+#pragma unroll 1
+                        for (int gq = grp; gq < 2; gq += UNPACK_GROUPS) {
+                        const int q = 2 * hh + gq;
                         // K-steps 4h + g and 4h + g + 2 share their low-bit bytes (low and high
                         // nibbles) and the half's high-bit bytes
                         const int h = q >> 1, g = q & 1;
@@ -645,7 +660,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                                 v[i] = __byte_perm(pa, pb, 0x6420) ^ 0x80808080u;
                                 v[8 + i] = __byte_perm(pa, pb, 0x7531) ^ 0x80808080u;
                             }
-                            tmem_st16(tmem + lane_off + TM_A + 64 * sl + 32 * grp + 16 * kk, v);
+                            tmem_st16(tmem + lane_off + TM_A + 64 * sl + 32 * gq + 16 * kk, v);
+                        }
                         }
                         tmem_wait_st();
                         tc_fence_before();
@@ -661,9 +677,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
         setmaxnreg_inc<REG_EPI>();
         // ============================================================ epilogue
         const int quad = warp & 3;
-        const int half = (warp - 12) >> 2;
+        const int half = (warp - EPI_WARP0) >> 2;
         const int row = quad * 32 + lane;
-        const int etid = threadIdx.x - 384;  // 0..255
+        const int etid = threadIdx.x - (128 + UNPACK_THREADS);  // 0..255
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t col0 = (uint32_t)(half * EPI_COLS);
         // initial preset of both plane accumulators (this warp's lanes and columns)
@@ -747,6 +763,46 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     for (int pl = 0; pl < 2; pl++) {
                         if (!wait_bar_warp(sh, &sh.p_full[pl], sbc & 1)) goto epi_done;
                         tc_fence_after();
+                        if constexpr (EARLY_RELEASE) {
+                            // copy the plane's 64 columns out, preset and release it, then
+                            // do the arithmetic: the next super-block's MMAs on this plane
+                            // do not wait for it
+                            uint32_t x[EPI_COLS];
+                            if (live) {
+                                const uint32_t tp = tmem + lane_off + (pl ? C::TM_P1 : C::TM_P0) + col0;
+                                load_cols64(tp, x);
+                                tmem_wait_ld();
+                                preset_cols64(tp);
+                                tmem_wait_st();
+                            }
+                            tc_fence_before();
+                            mbar_arrive(&sh.p_empty[pl]);
+                            if (live) {
+                                // in chunks of 16 columns; the empty asm keeps the compiler from
+                                // loading every chunk's activation scales up front
+#pragma unroll
+                                for (int c = 0; c < EPI_COLS / 16; c++) {
+                                    asm volatile("" ::: "memory");
+                                    float4 dv4[4];
+#pragma unroll
+                                    for (int j = 0; j < 4; j++) dv4[j] = *reinterpret_cast<const float4*>(da + 16 * c + 4 * j);
+#pragma unroll
+                                    for (int j = 0; j < 4; j++) {
+#pragma unroll
+                                        for (int h2 = 0; h2 < 2; h2++) {
+                                            const int i = 8 * c + 2 * j + h2;
+                                            const float2 X =
+                                                make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
+                                            const float2 T = pl ? __ffma2_rn(X, kP, nkM) : __fadd2_rn(X, nM);
+                                            const float2 dd = __fmul2_rn(d2, h2 ? make_float2(dv4[j].z, dv4[j].w)
+                                                                                : make_float2(dv4[j].x, dv4[j].y));
+                                            acc[i] = __ffma2_rn(T, dd, acc[i]);
+                                        }
+                                    }
+                                }
+                            }
+                            continue;
+                        }
                         if (live) {
                             const uint32_t tp = tmem + lane_off + (pl ? C::TM_P1 : C::TM_P0) + col0;
 #pragma unroll

@@ -68,14 +68,12 @@ namespace dllm {
 
 constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23
 constexpr float MAGIC = 12582912.0f;
-// Unpack groups of four warps (one warp per tensor-memory lane quadrant).  With one
-// group the CTA has 512 threads, which leaves the epilogue enough registers to copy a
-// whole plane accumulator out and release it before its arithmetic.
+// Unpack groups of four warps (one warp per tensor-memory lane quadrant).  One group
+// (a 512-thread CTA) measured faster than two: fewer warps contend for issue slots.
 constexpr int UNPACK_GROUPS = 1;
 constexpr int UNPACK_THREADS = 128 * UNPACK_GROUPS;
 constexpr int EPI_WARP0 = 4 + 4 * UNPACK_GROUPS;  // first epilogue warp
 constexpr int GEMM_THREADS = 128 + UNPACK_THREADS + 256;
-constexpr bool EARLY_RELEASE = false;
 constexpr int UNIT_TOKENS = 128;
 constexpr int EPI_COLS = 64;                       // token columns per epilogue thread
 constexpr int MAX_KC = 16;                         // K-chunks per tile, at most
@@ -763,46 +761,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     for (int pl = 0; pl < 2; pl++) {
                         if (!wait_bar_warp(sh, &sh.p_full[pl], sbc & 1)) goto epi_done;
                         tc_fence_after();
-                        if constexpr (EARLY_RELEASE) {
-                            // copy the plane's 64 columns out, preset and release it, then
-                            // do the arithmetic: the next super-block's MMAs on this plane
-                            // do not wait for it
-                            uint32_t x[EPI_COLS];
-                            if (live) {
-                                const uint32_t tp = tmem + lane_off + (pl ? C::TM_P1 : C::TM_P0) + col0;
-                                load_cols64(tp, x);
-                                tmem_wait_ld();
-                                preset_cols64(tp);
-                                tmem_wait_st();
-                            }
-                            tc_fence_before();
-                            mbar_arrive(&sh.p_empty[pl]);
-                            if (live) {
-                                // in chunks of 16 columns; the empty asm keeps the compiler from
-                                // loading every chunk's activation scales up front
-#pragma unroll
-                                for (int c = 0; c < EPI_COLS / 16; c++) {
-                                    asm volatile("" ::: "memory");
-                                    float4 dv4[4];
-#pragma unroll
-                                    for (int j = 0; j < 4; j++) dv4[j] = *reinterpret_cast<const float4*>(da + 16 * c + 4 * j);
-#pragma unroll
-                                    for (int j = 0; j < 4; j++) {
-#pragma unroll
-                                        for (int h2 = 0; h2 < 2; h2++) {
-                                            const int i = 8 * c + 2 * j + h2;
-                                            const float2 X =
-                                                make_float2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
-                                            const float2 T = pl ? __ffma2_rn(X, kP, nkM) : __fadd2_rn(X, nM);
-                                            const float2 dd = __fmul2_rn(d2, h2 ? make_float2(dv4[j].z, dv4[j].w)
-                                                                                : make_float2(dv4[j].x, dv4[j].y));
-                                            acc[i] = __ffma2_rn(T, dd, acc[i]);
-                                        }
-                                    }
-                                }
-                            }
-                            continue;
-                        }
                         if (live) {
                             const uint32_t tp = tmem + lane_off + (pl ? C::TM_P1 : C::TM_P0) + col0;
 #pragma unroll

@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qgemm_kernel(const __grid_con
                     for (int hh = 0; hh < 2; hh++) {
                         const uint32_t hc = 2 * sbc + hh, sl = hc % C::A_SLOTS;
                         if (!wait_bar_warp(sh, &sh.a_empty[sl], ((hc / C::A_SLOTS) & 1) ^ 1)) goto unpack_done;
-#pragma unroll 1
+#pragma unroll
                         for (int gq = grp; gq < 2; gq += UNPACK_GROUPS) {
                         const int q = 2 * hh + gq;
                         // 32-byte quant chunk q: sub-block 2q in the low nibbles, 2q+1 in the high

@@ -978,6 +978,7 @@ def run_attn_config(args, dllm, torch, dev, model):
         assert dllm.dllm_get_device_status() == dllm.DLLM_OK
         us = e0.elapsed_time(e1) * 1e3 / reps
         del g
+        nt = dllm.dllm_debug_attention_tiles(L, H, torch.cuda.get_device_properties(dev).multi_processor_count)
         flops = 4.0 * L * L * dh * H
         t_tc = flops / (peak_tf * 1e12) * 1e6
         t_sfu = L * L * H / SFU_EX2_PER_S * 1e6
@@ -986,7 +987,8 @@ def run_attn_config(args, dllm, torch, dev, model):
             "workload": "attn", "model": model.name, "Lq": L, "Lk": L, "heads": H, "kv_heads": Hkv, "dh": dh},
             "us": round(us, 2), "tflops": round(flops / (us * 1e-6) / 1e12, 1), "t_star_us": round(tstar, 2),
             "bound": "tensor" if t_tc >= t_sfu else "sfu", "frac": round(tstar / us, 4),
-            "peak_tflops": peak_tf, "peak_source": peak_kind, "ctas": -(-L // 128) * H,
+            "peak_tflops": peak_tf, "peak_source": peak_kind, "query_tiles_per_cta": nt,
+            "ctas": -(-L // (128 * nt)) * H,
             "timing": f"CUDA events around one replay of a graph of {reps} launches, inputs rotated over "
                       f"{copies} copies beyond L2"})
         del ins, o

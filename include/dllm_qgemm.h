@@ -272,7 +272,10 @@ int dllm_qkv_qgemm(const void* wq, const void* wk, const void* wv, dllm_qtype t,
  * exceeds it by more than 2^8; the weights rounded to f16 for P V on the tensor
  * cores (f32 accumulation), the normaliser summed in f32 before that rounding, so each
  * normalised weight is off by at most about 2^-11 of itself plus the f32 effects.
- * One CTA per (128 queries, head), programmatic dependent launch like the GEMM.
+ * One CTA per (128 queries, head) while that grid fits one wave of CTAs on the
+ * device's SMs, else one CTA per (256 queries, head) with the two query tiles in
+ * ping-pong (dllm_debug_attention_tiles gives the choice); programmatic dependent
+ * launch like the GEMM.
  * Errors: DLLM_ERR_ARG (sizes, dh != 128, H % Hkv, null), DLLM_ERR_ALIGN,
  * DLLM_ERR_UNSUPPORTED, DLLM_ERR_CUDA; DLLM_ERR_TIMEOUT in the device error word.
  * ---------------------------------------------------------------------------- */
@@ -317,6 +320,11 @@ int dllm_debug_bounded_wait(dllm_stream_t stream);
  * super-tiles), mu (tokens per super-tile) and the workspace bytes.  The pages have no
  * counterpart; the split is this library's scheduling.  DLLM_ERR_ARG on bad sizes. */
 int dllm_debug_plan(int64_t n_tiles, int64_t K, int64_t M, int64_t n_rows, int sms, int64_t* out);
+
+/* Query tiles of 128 rows per CTA that dllm_attention uses for Lq queries and H heads
+ * on a device with `sms` SMs: 1 while ceil(Lq / 128) * H <= sms (one wave of one-tile
+ * CTAs), else 2.  Host only.  DLLM_ERR_ARG when an argument is below 1. */
+int dllm_debug_attention_tiles(int64_t Lq, int64_t H, int sms);
 
 /* int8 tensor-core throughput probe: on each of `ctas` CTAs, `issuers` warps (1..4)
  * each issue `iters` back-to-back tcgen05 kind::i8 MMAs of 128 x n x 32 into their own

@@ -103,6 +103,13 @@ __device__ __forceinline__ void att_tma_tile(uint8_t* tile, const CUtensorMap* t
     if (lane < 2) tma_load_3d(tile + lane * 16384, tmap, 64 * lane, head, r0, bar);
 }
 
+// max(a, b, c) in one instruction (PTX max.f32 with three sources; -inf is the identity).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // 2^x on the special-function unit (PTX ex2.approx.ftz: relative error below 2^-22,
 // 2^-inf = 0, results below the f32 normal range flush to 0).
 __device__ __forceinline__ float att_ex2(float x) {
@@ -400,6 +407,365 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == ATT_MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tm, ATT_TM_COLS);
+    }
+}
+
+
+// ------------------------------------------------------------------------------------
+// Two query tiles per CTA ("ping-pong"), for grids of more than one wave.
+//
+// One CTA per (two query tiles of 128 rows, head), 14 warps, key blocks of 64:
+//   warp 9      TMA producer of both Q tiles (once) and of K key blocks (four slots of
+//               64 keys); warp 10 the same for V
+//   warps 8, 11 one thread each issues S_t(kb) = Q_t K(kb)^T (128 x 64) for query tile
+//               0 / tile 1 into one of the tile's two S slots (warp 8 also owns tensor
+//               memory); so the tensor core computes the next block's scores while the
+//               softmax works on this one
+//   warps 12,13 one thread each issues O_t += P_t(kb) V(kb) for tile 0 / tile 1 once
+//               the softmax has written P_t(kb) over the first 32 columns of its S slot
+//               (which S_t(kb + 2) reuses only after that P V has completed).  One
+//               thread issues an MMA only every ~55 cycles, so the four streams have a
+//               thread each.
+//   warps 0-3   softmax of tile 0, warps 4-7 of tile 1; thread = query row = tensor-
+//               memory lane 32 (w % 4) + lane, all 64 key columns of the block in
+//               registers: block maximum, running maximum m (raised, with O_t and l
+//               rescaled once P V(kb - 1) is complete, only when a block maximum exceeds
+//               it by more than 8 binades), P = 2^(S c - m) rounded to f16, the running
+//               sum l; at the end O_t / l is stored.  Warps w and w + 4 share a sub-
+//               partition and its special-function unit; they take turns at the
+//               exponentials (tile 0 of block kb, tile 1 of block kb, tile 0 of block
+//               kb + 1, ...), so that each one's loads, maxima and stores run while the
+//               other's exponentials keep the unit busy.
+// K and V blocks are shared by the two tiles (each slot is released by the commits of
+// both issuers): each block crosses from L2 once per 256 queries.
+// Tensor memory: O_t at columns 256 t .. 256 t + 127, S slot s of tile t at
+// 256 t + 128 + 64 s (64 columns; P in the first 32 as f16 pairs).  A CTA whose
+// second tile lies past Lq runs the first one only.
+// Shared memory: Q_t as in the one-tile kernel (32 KB each); K and V slots of two TMA
+// boxes of 64 head-dim values x 64 keys (8 KB each, 128-byte swizzle): K-major for K
+// (second box at +8 KB), MN-major for V (the second 64 head-dim columns at +8 KB, 1024
+// bytes per 8 keys).
+constexpr int ATT_PP_S0_WARP = 8;  // issues tile 0's Q K^T; owns tensor memory
+constexpr int ATT_PP_K_WARP = 9;
+constexpr int ATT_PP_V_WARP = 10;
+constexpr int ATT_PP_S1_WARP = 11;   // issues tile 1's Q K^T
+constexpr int ATT_PP_PV0_WARP = 12;  // issues tile 0's P V
+constexpr int ATT_PP_PV1_WARP = 13;  // issues tile 1's P V
+constexpr int ATT_PP_THREADS = 32 * 14;
+constexpr int ATT_PP_BQ = 2 * ATT_BQ;  // queries per CTA
+constexpr int ATT_PP_BK = 64;          // keys per block
+constexpr int ATT_PP_SLOTS = 4;        // K and V slots
+constexpr int ATT_PP_KV = ATT_PP_BK * ATT_DH * 2;  // one K or V block, 16 KB
+// Q x2, K x4, V x4, barriers and tensor-memory address
+constexpr size_t ATT_PP_SMEM = 2 * (size_t)ATT_TILE + 2 * ATT_PP_SLOTS * (size_t)ATT_PP_KV + 512;
+
+// Query tiles per CTA for a grid over Lq queries and H heads on a device of `sms` SMs:
+// two when one tile per CTA would need more than one wave of CTAs, else one.
+__host__ __device__ constexpr int att_tiles_per_cta(int64_t Lq, int64_t H, int sms) {
+    return ((Lq + ATT_BQ - 1) / ATT_BQ) * H > sms ? 2 : 1;
+}
+
+// K step kk of a 64-key K block (second head-dim box at +8 KB), in 16-byte units.
+__host__ __device__ constexpr uint64_t att_k64_step(int kk) { return (uint64_t)((kk >> 2) * 512 + (kk & 3) * 2); }
+
+// Same arguments and grid rows (y = head) as attention_kernel, with K and V maps of
+// 64-row boxes; grid x = ceil(Lq / 256).
+// Barriers (tile t, S slot s = kb & 1, K/V slot v = kb & 3 for key block kb):
+//   q_full[t]                   TMA transaction count of Q_t
+//   k_full[v], v_full[v]        TMA transaction count of the 16 KB block
+//   k_empty[v], v_empty[v]      one commit per active tile, after Q_t K^T(kb) / P_t V(kb)
+//   s_full[t][s]                commit after Q_t K^T(kb)
+//   p_half[t][s], p_full[t][s]  the tile's four softmax warps (one arrival each), after
+//                               the first 32 keys of P_t(kb) / all of it
+//   o_done[t][s]                commit after P_t V(kb)
+//   ex[q][t]                    lane 0 of tile t's softmax warp of quadrant q, after its
+//                               exponentials of block kb (the turn passes to the other tile)
+// A barrier of slot kb % n completes once per use u = kb / n and a wait takes parity
+// u & 1: (kb >> 1) & 1 for the tile barriers, (kb >> 2) & 1 for the K/V slots.  No
+// barrier runs two uses ahead of a waiter, because its next use needs that waiter's own
+// progress.
+__global__ void __launch_bounds__(ATT_PP_THREADS, 1)
+    attention_pp_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                        const __grid_constant__ CUtensorMap tv, float* __restrict__ o, int Lq, int Lk, int H,
+                        int group) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* const sQ = smem;                                    // two tiles
+    uint8_t* const sK = smem + 2 * ATT_TILE;                     // four slots
+    uint8_t* const sV = sK + ATT_PP_SLOTS * ATT_PP_KV;           // four slots
+    uint64_t* const bars = reinterpret_cast<uint64_t*>(sV + ATT_PP_SLOTS * ATT_PP_KV);
+    uint64_t* const q_full = bars;       // [2]
+    uint64_t* const k_full = bars + 2;   // [4]
+    uint64_t* const v_full = bars + 6;   // [4]
+    uint64_t* const k_empty = bars + 10; // [4]
+    uint64_t* const v_empty = bars + 14; // [4]
+    uint64_t* const s_full = bars + 18;  // [2][2]
+    uint64_t* const p_full = bars + 22;  // [2][2]
+    uint64_t* const o_done = bars + 26;  // [2][2]
+    uint64_t* const fin = bars + 30;
+    uint64_t* const ex = bars + 31;      // [4][2]
+    uint64_t* const p_half = bars + 39;  // [2][2]
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bars + 43);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q0 = blockIdx.x * ATT_PP_BQ, h = blockIdx.y, hk = h / group;
+    const int ntiles = Lq - q0 > ATT_BQ ? 2 : 1;
+    const int nkb = (Lk + ATT_PP_BK - 1) / ATT_PP_BK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; i++) mbar_init(&q_full[i], 1);
+        for (int i = 0; i < ATT_PP_SLOTS; i++) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&k_empty[i], ntiles);
+            mbar_init(&v_empty[i], ntiles);
+        }
+        for (int i = 0; i < 4; i++) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&p_half[i], 4);
+            mbar_init(&o_done[i], 1);
+        }
+        mbar_init(fin, 4);
+        for (int i = 0; i < 8; i++) mbar_init(&ex[i], 1);
+        fence_mbar_init();
+    }
+    if (warp == ATT_PP_S0_WARP) {
+        tmem_alloc(tmem_slot, ATT_TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    pdl_wait();  // q, k, v may come from the previous kernel on the stream
+
+    if (warp == ATT_PP_K_WARP || warp == ATT_PP_V_WARP) {
+        // ---------------------------------------------------------------- TMA producers
+        const bool is_k = warp == ATT_PP_K_WARP;
+        if (is_k) {
+            for (int t = 0; t < ntiles; t++) {
+                if (lane == 0) mbar_arrive_expect_tx(&q_full[t], ATT_TILE);
+                __syncwarp();
+                if (lane < 2) tma_load_3d(sQ + t * ATT_TILE + lane * (ATT_TILE / 2), &tq, 64 * lane, h, q0 + t * ATT_BQ,
+                                          &q_full[t]);
+            }
+        }
+        uint64_t* const full = is_k ? k_full : v_full;
+        uint64_t* const empty = is_k ? k_empty : v_empty;
+        const CUtensorMap* const tmap = is_k ? &tk : &tv;
+        uint8_t* const dst = is_k ? sK : sV;
+        int issued = 0;
+        for (int kb = 0; kb < nkb; kb++) {
+            const int v = kb & 3;
+            if (kb >= ATT_PP_SLOTS && !__all_sync(~0u, att_wait(&empty[v], ((kb >> 2) - 1) & 1))) break;
+            if (lane == 0) mbar_arrive_expect_tx(&full[v], ATT_PP_KV);
+            __syncwarp();
+            if (lane < 2)
+                tma_load_3d(dst + v * ATT_PP_KV + lane * (ATT_PP_KV / 2), tmap, 64 * lane, hk, kb * ATT_PP_BK, &full[v]);
+            issued = kb + 1;
+        }
+        // No copy may still be landing in shared memory when the CTA exits, also when
+        // a wait ran out: wait for the last use of each slot (and for the Q tiles).
+        if (lane == 0) {
+            for (int kb = issued > ATT_PP_SLOTS ? issued - ATT_PP_SLOTS : 0; kb < issued; kb++)
+                drain_wait(&full[kb & 3], (kb >> 2) & 1);
+            if (is_k)
+                for (int t = 0; t < ntiles; t++) drain_wait(&q_full[t], 0);
+        }
+        __syncwarp();
+    } else if (warp == ATT_PP_S0_WARP || warp == ATT_PP_S1_WARP) {
+        // ---------------------------------------------------------------- Q K^T issue, tile t
+        const int t = warp == ATT_PP_S0_WARP ? 0 : 1;
+        if (lane == 0 && t < ntiles) {
+            constexpr uint32_t ID_S = idesc_f16(ATT_BQ, ATT_PP_BK);
+            const uint32_t tb = tm + 256 * t;  // O_t; S slots at +128 and +192
+            const uint64_t dq = att_qk_desc(sQ + t * ATT_TILE);
+            const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+            bool ok = att_wait(&q_full[t], 0);
+            for (int kb = 0; ok && kb < nkb; kb++) {
+                const int sl = kb & 1, v = kb & 3;
+                if (!att_wait(&k_full[v], (kb >> 2) & 1)) break;
+                // P V(kb - 2) has read P out of this S slot
+                if (kb >= 2 && !att_wait(&o_done[2 * t + sl], ((kb - 2) >> 1) & 1)) break;
+                tc_fence_after();
+                const uint32_t ds = tb + 128 + 64 * sl;
+                const uint64_t dk = dk0 + (uint64_t)(v * (ATT_PP_KV >> 4));
+                mma_f16_ss(ds, dq, dk, ID_S, 0);
+#pragma unroll
+                for (int kk = 1; kk < ATT_DH / 16; kk++)
+                    mma_f16_ss(ds, dq + att_qk_step(kk), dk + att_k64_step(kk), ID_S, 1);
+                tc_commit(&s_full[2 * t + sl]);
+                tc_commit(&k_empty[v]);
+            }
+        }
+        // Every MMA issued above completes before the tensor memory is released, also
+        // when a wait ran out (a thread that issued none arrives at once).
+        if (lane == 0) {
+            tc_commit(fin);
+            drain_wait(fin, 0);
+        }
+        __syncwarp();
+    } else if (warp == ATT_PP_PV0_WARP || warp == ATT_PP_PV1_WARP) {
+        // ---------------------------------------------------------------- P V issue, tile t
+        const int t = warp == ATT_PP_PV0_WARP ? 0 : 1;
+        if (lane == 0 && t < ntiles) {
+            constexpr uint32_t ID_O = idesc_f16(ATT_BQ, ATT_DH) | (1u << 16);  // B (V) MN-major
+            const uint32_t tb = tm + 256 * t;
+            const uint64_t dv0 = sdesc_sw128(smem_u32(sV), ATT_PP_KV / 2, 1024);
+            for (int kb = 0; kb < nkb; kb++) {
+                const int sl = kb & 1, v = kb & 3;
+                // O_t += P_t V: 4 steps of K = 16 keys (P from tensor memory, 8 columns a
+                // step), the first two as soon as the first half of P is in.
+                if (!att_wait(&p_half[2 * t + sl], (kb >> 1) & 1) || !att_wait(&v_full[v], (kb >> 2) & 1)) break;
+                tc_fence_after();
+                const uint32_t pa = tb + 128 + 64 * sl;
+                const uint64_t dv = dv0 + (uint64_t)(v * (ATT_PP_KV >> 4));
+                mma_f16_ts(tb, pa, dv, ID_O, kb > 0);
+                mma_f16_ts(tb, pa + 8, dv + att_v_step(1), ID_O, 1);
+                if (!att_wait(&p_full[2 * t + sl], (kb >> 1) & 1)) break;
+                tc_fence_after();
+                mma_f16_ts(tb, pa + 16, dv + att_v_step(2), ID_O, 1);
+                mma_f16_ts(tb, pa + 24, dv + att_v_step(3), ID_O, 1);
+                tc_commit(&o_done[2 * t + sl]);
+                tc_commit(&v_empty[v]);
+            }
+        }
+        if (lane == 0) {
+            tc_commit(fin);
+            drain_wait(fin, 0);
+        }
+        __syncwarp();
+    } else if ((warp >> 2) < ntiles) {
+        // ---------------------------------------------------------------- softmax, output
+        const int t = warp >> 2, qd = warp & 3;
+        const int row = 32 * qd + lane;  // query q0 + 128 t + row, tensor-memory lane row
+        const uint32_t tb = tm + ((uint32_t)(32 * qd) << 16) + 256 * t;  // this warp's lanes of O_t
+        float m = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; kb++) {
+            const int sl = kb & 1;
+            ok = __all_sync(~0u, att_wait(&s_full[2 * t + sl], (kb >> 1) & 1));  // warp-uniform
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t ts = tb + 128 + 64 * sl;
+            uint32_t sr[ATT_PP_BK];
+            // S in two halves: the maximum of the first runs while the second loads.
+            tmem_ld16(ts, sr);
+            tmem_ld16(ts + 16, sr + 16);
+            tmem_wait_ld();
+            tmem_ld16(ts + 32, sr + 32);
+            tmem_ld16(ts + 48, sr + 48);
+            // block maximum over the valid keys (eight independent chains of 3-input max)
+            const int kvalid = Lk - kb * ATT_PP_BK;
+            float mx[8];
+#pragma unroll
+            for (int e = 0; e < 8; e++) mx[e] = -INFINITY;
+            if (kvalid >= ATT_PP_BK) {  // uniform across the CTA: no masking
+#pragma unroll
+                for (int j = 0; j < ATT_PP_BK / 2; j += 2)
+                    mx[(j >> 1) & 7] = max3f(mx[(j >> 1) & 7], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = ATT_PP_BK / 2; j < ATT_PP_BK; j += 2)
+                    mx[(j >> 1) & 7] = max3f(mx[(j >> 1) & 7], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+            } else {
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < ATT_PP_BK; j++) {
+                    const float x = j < kvalid ? __uint_as_float(sr[j]) : -INFINITY;
+                    sr[j] = __float_as_uint(x);
+                    mx[j & 7] = fmaxf(mx[j & 7], x);
+                }
+            }
+            const float mc = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+                             ATT_C;  // finite: the block has a valid key
+            const bool raise = kb == 0 || mc > m + ATT_RESCALE_LOG2;
+            const float m_new = raise ? mc : m;
+            if (kb >= 1 && __any_sync(~0u, raise)) {
+                // O_t must hold blocks 0..kb-1 before it is rescaled to the new maximum
+                ok = __all_sync(~0u, att_wait(&o_done[2 * t + (sl ^ 1)], ((kb - 1) >> 1) & 1));
+                if (!ok) break;
+                tc_fence_after();
+                const float alpha = raise ? att_ex2(m - m_new) : 1.0f;
+                l *= alpha;
+#pragma unroll 1
+                for (int j = 0; j < ATT_DH / 16; j++) {
+                    uint32_t r[16];
+                    tmem_ld16(tb + 16 * j, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                    tmem_st16(tb + 16 * j, r);
+                }
+            }
+            m = m_new;
+            // this sub-partition's turn at the exponentials: tile 1 after tile 0 of the same
+            // block, tile 0 after tile 1 of the previous block
+            if (ntiles == 2 && (t == 1 || kb >= 1)) {
+                ok = __all_sync(~0u, att_wait(&ex[2 * qd + (t ^ 1)], (t == 1 ? kb : kb - 1) & 1));
+                if (!ok) break;
+            }
+            // P(kb) = 2^(s c - m) in f16 pairs over the slot's first 32 columns; l sums
+            // the unrounded weights.
+            float ps[8];
+#pragma unroll
+            for (int e = 0; e < 8; e++) ps[e] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < ATT_PP_BK / 32; c++) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; e++) {
+                    const float p0 = att_ex2(fmaf(__uint_as_float(sr[32 * c + 2 * e]), ATT_C, -m));
+                    const float p1 = att_ex2(fmaf(__uint_as_float(sr[32 * c + 2 * e + 1]), ATT_C, -m));
+                    ps[e & 7] += p0 + p1;
+                    const __half2 hp = __floats2half2_rn(p0, p1);
+                    pk[e] = *reinterpret_cast<const uint32_t*>(&hp);
+                }
+                tmem_st16(ts + 16 * c, pk);
+                if (c == 0) {
+                    // half way: P V may start on these keys, and the other tile may start
+                    // its exponentials
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&p_half[2 * t + sl]);
+                        mbar_arrive(&ex[2 * qd + t]);
+                    }
+                }
+            }
+            l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[2 * t + sl]);  // one arrival per warp
+        }
+        if (ok) ok = __all_sync(~0u, att_wait(&o_done[2 * t + ((nkb - 1) & 1)], ((nkb - 1) >> 1) & 1));
+        if (ok) {
+            tc_fence_after();
+            const int qi = q0 + ATT_BQ * t + row;
+            const float inv = 1.0f / l;
+            float* dst = o + ((int64_t)qi * H + h) * ATT_DH;
+#pragma unroll 1
+            for (int j = 0; j < ATT_DH / 16; j++) {
+                uint32_t r[16];
+                tmem_ld16(tb + 16 * j, r);
+                tmem_wait_ld();
+                if (qi < Lq) {
+#pragma unroll
+                    for (int e = 0; e < 4; e++)
+                        reinterpret_cast<float4*>(dst + 16 * j)[e] =
+                            make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                        __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == ATT_PP_S0_WARP) {
         tc_fence_after();
         tmem_dealloc(tm, ATT_TM_COLS);
     }

@@ -68,13 +68,13 @@ EncodeTiledFn encode_tiled() {
 }
 
 // A [rows][heads][128] f16 tensor as the 3-D tensor (head dim, head, row) with boxes of
-// 64 head-dim values x 1 head x 128 rows, 128-byte swizzled (half a tile).
-bool encode_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t heads) {
+// 64 head-dim values x 1 head x box_rows rows, 128-byte swizzled (half a tile).
+bool encode_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t heads, int box_rows) {
     const EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)ATT_DH, (cuuint64_t)heads, (cuuint64_t)rows};
     const cuuint64_t strides[2] = {(cuuint64_t)ATT_DH * 2, (cuuint64_t)(heads * ATT_DH * 2)};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)ATT_BK};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -83,22 +83,24 @@ bool encode_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t he
 
 // The last few encoded maps, per host thread (a layer's q, k and v, a few layers deep):
 // encoding costs about as much host time as the launch itself.
-bool cached_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t heads) {
+bool cached_head_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t heads, int box_rows) {
     struct Entry {
         const void* base;
         int64_t rows, heads;
+        int box_rows;
         CUtensorMap map;
     };
     constexpr int N = 12;
     thread_local Entry cache[N] = {};
     thread_local int next = 0;
     for (int i = 0; i < N; i++)
-        if (cache[i].base == base && cache[i].rows == rows && cache[i].heads == heads) {
+        if (cache[i].base == base && cache[i].rows == rows && cache[i].heads == heads &&
+            cache[i].box_rows == box_rows) {
             *m = cache[i].map;
             return true;
         }
-    if (!encode_head_rows(m, base, rows, heads)) return false;
-    cache[next] = {base, rows, heads, *m};
+    if (!encode_head_rows(m, base, rows, heads, box_rows)) return false;
+    cache[next] = {base, rows, heads, box_rows, *m};
     next = (next + 1) % N;
     return true;
 }
@@ -566,20 +568,40 @@ int dllm_attention(const void* q, const void* k, const void* v, int64_t Lq, int6
     if (rc) return rc;
     if (!g_att_attr_done[dev]) {
         if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATT_SMEM) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ATT_PP_SMEM) != cudaSuccess)
             return DLLM_ERR_CUDA;
         g_att_attr_done[dev] = true;
     }
+    // the two-tile kernel reads K and V in blocks of 64 keys
+    const bool pp = att_tiles_per_cta(Lq, H, g_num_sms[dev]) == 2;
+    const int kv_rows = pp ? ATT_PP_BK : ATT_BK;
     CUtensorMap tq, tk, tv;
-    if (!cached_head_rows(&tq, q, Lq, H) || !cached_head_rows(&tk, k, Lk, Hkv) || !cached_head_rows(&tv, v, Lk, Hkv))
+    if (!cached_head_rows(&tq, q, Lq, H, ATT_BQ) || !cached_head_rows(&tk, k, Lk, Hkv, kv_rows) ||
+        !cached_head_rows(&tv, v, Lk, Hkv, kv_rows))
         return DLLM_ERR_CUDA;
-    const dim3 grid((unsigned)((Lq + ATT_BQ - 1) / ATT_BQ), (unsigned)H);
-    if (launch_pdl(attention_kernel, grid, dim3(ATT_THREADS), ATT_SMEM, reinterpret_cast<cudaStream_t>(stream), tq,
-                   tk, tv, o, (int)Lq, (int)Lk, (int)H, (int)(H / Hkv)) != cudaSuccess) {
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (pp) {
+        const dim3 grid((unsigned)((Lq + ATT_PP_BQ - 1) / ATT_PP_BQ), (unsigned)H);
+        e = launch_pdl(attention_pp_kernel, grid, dim3(ATT_PP_THREADS), ATT_PP_SMEM, s, tq, tk, tv, o, (int)Lq,
+                       (int)Lk, (int)H, (int)(H / Hkv));
+    } else {
+        const dim3 grid((unsigned)((Lq + ATT_BQ - 1) / ATT_BQ), (unsigned)H);
+        e = launch_pdl(attention_kernel, grid, dim3(ATT_THREADS), ATT_SMEM, s, tq, tk, tv, o, (int)Lq, (int)Lk,
+                       (int)H, (int)(H / Hkv));
+    }
+    if (e != cudaSuccess) {
         (void)cudaGetLastError();
         return DLLM_ERR_CUDA;
     }
     return launch_status();
+}
+
+int dllm_debug_attention_tiles(int64_t Lq, int64_t H, int sms) {
+    if (Lq < 1 || H < 1 || sms < 1) return DLLM_ERR_ARG;
+    return att_tiles_per_cta(Lq, H, sms);
 }
 
 int dllm_get_device_status(dllm_stream_t stream) {

@@ -35,7 +35,7 @@ EXPORTS = (
     "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_attention",
     "dllm_get_device_status",
     "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_debug_bounded_wait",
-    "dllm_bench_mma_i8", "dllm_debug_plan",
+    "dllm_bench_mma_i8", "dllm_debug_plan", "dllm_debug_attention_tiles",
 )
 
 
@@ -81,6 +81,7 @@ def load() -> ctypes.CDLL:
         "dllm_debug_bounded_wait": [P],
         "dllm_bench_mma_i8": [I, I, I, I, I, I, P, P],
         "dllm_debug_plan": [I64, I64, I64, I64, I, ctypes.POINTER(ctypes.c_int64)],
+        "dllm_debug_attention_tiles": [I64, I64, I],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -255,3 +256,11 @@ def dllm_debug_plan(n_tiles: int, K: int, M: int, n_rows: int, sms: int) -> dict
     _check(load().dllm_debug_plan(n_tiles, K, M, n_rows, sms, out), "dllm_debug_plan")
     keys = ("kc", "full_tiles", "tail_k", "tail_big", "n_units", "n_st", "mu", "bytes")
     return dict(zip(keys, list(out)))
+
+
+def dllm_debug_attention_tiles(Lq: int, H: int, sms: int) -> int:
+    """Query tiles per CTA dllm_attention uses (host only): see include/dllm_qgemm.h."""
+    rc = load().dllm_debug_attention_tiles(Lq, H, sms)
+    if rc < 0:
+        _check(rc, "dllm_debug_attention_tiles")
+    return rc

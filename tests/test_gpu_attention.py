@@ -1,5 +1,7 @@
 """Tensor-core attention (dllm_attention) vs the oracle's fp64 attention, element by
-element, on the same f16 inputs.
+element, on the same f16 inputs.  Both kernels are covered: one query tile per CTA
+(grids of at most one wave) and two query tiles per CTA in ping-pong (larger grids);
+each case states which one its shape takes on the device.
 
 Tolerance, from the kernel's arithmetic (both sides see the same f16 q, k, v):
   * each weight p_j = 2^(s_j c - m) is rounded to f16 (relative 2^-11, or absolute
@@ -36,6 +38,10 @@ def _cuda():
     dllm.load()
     yield
     assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+
+def tiles(Lq, H):
+    return dllm.dllm_debug_attention_tiles(Lq, H, torch.cuda.get_device_properties(0).multi_processor_count)
 
 
 def run(q, k, v):
@@ -75,42 +81,52 @@ def check(q, k, v, rows=None):
     return float(np.max(err / tol))
 
 
-@pytest.mark.parametrize("Lq,Lk,H,Hkv", [
-    (1, 1, 1, 1),        # one query, one key: the output is v exactly up to rounding
-    (5, 3, 2, 1),        # far below one tile, grouped heads
-    (128, 128, 2, 2),    # one full tile and one full key block
-    (130, 200, 4, 2),    # ragged query tile and ragged key block
-    (257, 384, 2, 1),    # three query tiles, three key blocks, the last query tile of 1
-    (160, 160, 32, 32),  # LLaDA-8B heads at the 160-position canvas
-    (200, 200, 28, 4),   # Dream-7B heads (28 query heads over 4 key/value heads)
+@pytest.mark.parametrize("Lq,Lk,H,Hkv,nt", [
+    (1, 1, 1, 1, 1),        # one query, one key: the output is v exactly up to rounding
+    (5, 3, 2, 1, 1),        # far below one tile, grouped heads
+    (128, 128, 2, 2, 1),    # one full tile and one full key block
+    (130, 200, 4, 2, 1),    # ragged query tile and ragged key block
+    (257, 384, 2, 1, 1),    # three query tiles, three key blocks, the last query tile of 1
+    (160, 160, 32, 32, 1),  # LLaDA-8B heads at the 160-position canvas
+    (200, 200, 28, 4, 1),   # Dream-7B heads (28 query heads over 4 key/value heads)
+    (300, 333, 64, 8, 2),   # two tiles per CTA; the last CTA of each head has one tile
+    (400, 130, 48, 48, 2),  # two tiles per CTA, the second of the last CTA 16 rows long
+    (640, 1, 32, 4, 2),     # one key: every output row is that key's value
+    (512, 700, 40, 5, 2),   # two full tiles per CTA, ragged keys, 8 query heads per K/V head
 ])
-def test_attention_matches_oracle(Lq, Lk, H, Hkv):
+def test_attention_matches_oracle(Lq, Lk, H, Hkv, nt):
+    assert tiles(Lq, H) == nt
     q, k, v = synth.attention_inputs(Lq, Lk, H, Hkv, DH, 1, Lq, Lk, H)
     check(q, k, v)
 
 
 @pytest.mark.parametrize("spread", [2.0, 4.0])
-def test_attention_peaked_softmax(spread):
+@pytest.mark.parametrize("Lq,H,nt", [(192, 2, 1), (260, 64, 2)])
+def test_attention_peaked_softmax(spread, Lq, H, nt):
     """Logits of standard deviation spread^2: nearly one-hot rows."""
-    q, k, v = synth.attention_inputs(192, 640, 2, 1, DH, 2, int(spread))
+    assert tiles(Lq, H) == nt
+    q, k, v = synth.attention_inputs(Lq, 640, H, 1, DH, 2, int(spread))
     check(q, k, v)
 
 
-def test_attention_running_max_raised_across_blocks():
+@pytest.mark.parametrize("Lq,H,nt", [(130, 2, 1), (300, 64, 2)])
+def test_attention_running_max_raised_across_blocks(Lq, H, nt):
     """Key norms grow along the sequence: for queries leaning with the growth direction
     later 128-key blocks raise the running maximum by more than 2^8, so the output
     accumulator is rescaled in tensor memory; the other rows of the same warps keep
     theirs (the rescale factor is 1 for them)."""
-    q, k, v = synth.attention_inputs(130, 600, 2, 1, DH, 3, key_growth=0.02)
+    assert tiles(Lq, H) == nt
+    q, k, v = synth.attention_inputs(Lq, 600, H, 1, DH, 3, key_growth=0.02)
     s = np.einsum("qhd,kd->qhk", q.astype(np.float64), k[:, 0].astype(np.float64)) * C
     m = s[..., :128].max(-1)
     raised, mixed = 0, 0
+    n = Lq // 32 * 32
     for b in range(1, 5):
         bm = s[..., b * 128:(b + 1) * 128].max(-1)
         r = bm > m + 8
         m = np.where(r, bm, m)
         raised += int(r.sum())
-        w = r[:128].reshape(4, 32, -1)  # the four softmax warps of the first query tile
+        w = r[:n].reshape(n // 32, 32, -1)  # the softmax warps' 32-row groups
         mixed += int(np.sum(w.any(1) & ~w.all(1)))
     assert raised > 0, "inputs do not exercise the rescale"
     assert mixed > 0, "no warp mixes raised and kept maxima"
@@ -129,12 +145,13 @@ def test_attention_hard_attention_and_zero_query():
     check(q, k, v)
 
 
-def test_attention_full_canvas_sampled_rows():
-    """L = 1024 canvas, LLaDA-8B heads (the largest canvas of the workload): every
-    output row is computed by the kernel; 48 rows drawn across all eight query tiles
+@pytest.mark.parametrize("L,H,Hkv", [(1024, 32, 32), (1024, 28, 4), (4096, 32, 32)])
+def test_attention_full_canvas_sampled_rows(L, H, Hkv):
+    """Full canvases at LLaDA-8B (32/32) and Dream-7B (28/4) heads, two tiles per CTA:
+    every output row is computed by the kernel; 48 rows drawn across all query tiles
     are compared with the oracle run on those queries alone."""
-    L = 1024
-    q, k, v = synth.attention_inputs(L, L, 32, 32, DH, 5)
+    assert tiles(L, H) == 2
+    q, k, v = synth.attention_inputs(L, L, H, Hkv, DH, 5)
     rows = np.sort(np.random.default_rng(5).choice(L, 48, replace=False))
     check(q, k, v, rows=rows)
 

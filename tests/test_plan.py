@@ -129,3 +129,21 @@ def test_bad_arguments():
         plan(10, 300)
     with pytest.raises(dllm.DllmError):
         plan(10, 4096, n_rows=33)
+
+
+@pytest.mark.parametrize("Lq,H,sms,want", [
+    (1, 1, SMS, 1), (1024, 32, SMS, 2), (1024, 28, SMS, 2), (4096, 32, SMS, 2), (512, 32, SMS, 1),
+    (640, 28, SMS, 1), (160, 32, SMS, 1), (128, 148, SMS, 1), (128, 149, SMS, 2), (129, 74, SMS, 1),
+    (129, 75, SMS, 2), (1024, 32, 256, 1), (1024, 32, 255, 2),
+])
+def test_attention_takes_two_tiles_per_cta_beyond_one_wave(Lq, H, sms, want):
+    """dllm_attention runs one query tile per CTA while ceil(Lq / 128) * H CTAs fit one
+    wave on the SMs, two (ping-pong) beyond that."""
+    assert dllm.dllm_debug_attention_tiles(Lq, H, sms) == want
+
+
+@pytest.mark.parametrize("Lq,H,sms", [(0, 32, SMS), (1024, 0, SMS), (1024, 32, 0), (-5, 1, 1)])
+def test_attention_tiles_rejects_bad_arguments(Lq, H, sms):
+    with pytest.raises(dllm.DllmError) as e:
+        dllm.dllm_debug_attention_tiles(Lq, H, sms)
+    assert e.value.code == dllm.DLLM_ERR_ARG

@@ -194,12 +194,17 @@ def load_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+# The sources the GEMM kernel and its launch plan are built from (the attention and the
+# fused quantizers live in files of their own and do not move the GEMM's DRAM traffic).
+GEMM_SOURCES = ("dllm.cu", "layout.cuh", "ptx.cuh", "qgemm.cuh")
+
+
 def kernel_source_hash(texts=None):
-    """Hash of the CUDA sources with `//` comments and blank lines removed, so that a
-    comment edit does not mark stored ncu counters as stale."""
+    """Hash of the GEMM's CUDA sources with `//` comments and blank lines removed, so
+    that a comment edit does not mark stored ncu counters as stale."""
     import re
     if texts is None:
-        texts = [p.read_text() for p in sorted((ROOT / "quantized_int8_gemm_q4_b200" / "csrc").glob("*.cu*"))]
+        texts = [(ROOT / "quantized_int8_gemm_q4_b200" / "csrc" / f).read_text() for f in GEMM_SOURCES]
     h = hashlib.sha256()
     for t in texts:
         code = [re.sub(r"\s*//.*$", "", line).rstrip() for line in t.splitlines()]
@@ -943,10 +948,12 @@ def run_act_config(args, dllm, torch, dev, model):
 def run_attn_config(args, dllm, torch, dev, model):
     """Device time of dllm_attention per launch at the model's head layout, canvases
     128..1024 (the step sweep) and 4096, inputs rotated over copies beyond L2, against
-    t* = max(FLOPs / f16 tensor peak, exponentials / special-function-unit rate)."""
+    t* = max(FLOPs / f16 tensor peak, exponentials / special-function-unit rate), with
+    the SM clock sampled while the launches run."""
     from quantized_int8_gemm_q4_b200 import synth
     peak_tf, peak_kind = load_tensor_peak()
     H, Hkv, dh = model.heads, model.kv_heads, model.hidden // model.heads
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
     lines = []
     for L in (128, 256, 512, 1024, 4096):
         nbytes = 2 * (L * H * dh + 2 * L * Hkv * dh)
@@ -970,13 +977,22 @@ def run_attn_config(args, dllm, torch, dev, model):
                 run(i)
         g.replay()
         torch.cuda.synchronize()
+        # replays for about half a second, long enough for the clock sampler to see it
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         g.replay()
         e1.record()
         torch.cuda.synchronize()
+        n_rep = max(1, min(2000, int(0.5 / max(e0.elapsed_time(e1) * 1e-3, 1e-6))))
+        sampler.start()
+        e0.record()
+        for _ in range(n_rep):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
         assert dllm.dllm_get_device_status() == dllm.DLLM_OK
-        us = e0.elapsed_time(e1) * 1e3 / reps
+        us = e0.elapsed_time(e1) * 1e3 / (reps * n_rep)
         del g
         nt = dllm.dllm_debug_attention_tiles(L, H, torch.cuda.get_device_properties(dev).multi_processor_count)
         flops = 4.0 * L * L * dh * H
@@ -989,8 +1005,8 @@ def run_attn_config(args, dllm, torch, dev, model):
             "bound": "tensor" if t_tc >= t_sfu else "sfu", "frac": round(tstar / us, 4),
             "peak_tflops": peak_tf, "peak_source": peak_kind, "query_tiles_per_cta": nt,
             "ctas": -(-L // (128 * nt)) * H,
-            "timing": f"CUDA events around one replay of a graph of {reps} launches, inputs rotated over "
-                      f"{copies} copies beyond L2"})
+            "timing": f"CUDA events around {n_rep} replays of a graph of {reps} launches, inputs rotated over "
+                      f"{copies} copies beyond L2", "clocks": clocks})
         del ins, o
         torch.cuda.empty_cache()
     return lines

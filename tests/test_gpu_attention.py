@@ -171,3 +171,19 @@ def test_attention_rejects_misaligned_and_bad_shapes():
     with pytest.raises(dllm.DllmError) as e:
         dllm.dllm_attention(x, x, x, 4, 4, 3, 2, DH, o)
     assert e.value.code == dllm.DLLM_ERR_ARG
+
+
+def test_attention_on_requested_query_rows_only():
+    """The last layer needs attention outputs at the requested canvas rows only (keys and
+    values still span the whole canvas): the queries of those rows, gathered, give the
+    same rows as the full canvas's attention, within the bound, through either kernel."""
+    L, H, Hkv = 1024, 32, 32
+    q, k, v = synth.attention_inputs(L, L, H, Hkv, DH, 6)
+    rows = np.sort(synth.block_rows(L, 32, 6))
+    assert tiles(len(rows), H) == 1 and tiles(L, H) == 2
+    got_rows = run(np.ascontiguousarray(q[rows]), k, v)
+    got_full = run(q, k, v)[rows]
+    ref = oracle.attention(q[rows].astype(np.float32), k.astype(np.float32), v.astype(np.float32))
+    tol = tolerance(q[rows], k, v)
+    for got in (got_rows, got_full):
+        assert np.all(np.abs(got - ref) <= tol)

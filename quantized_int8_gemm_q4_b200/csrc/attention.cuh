@@ -425,7 +425,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 //               softmax works on this one
 //   warps 12,13 one thread each issues O_t += P_t(kb) V(kb) for tile 0 / tile 1 once
 //               the softmax has written P_t(kb) over the first 32 columns of its S slot
-//               (which S_t(kb + 2) reuses only after that P V has completed).  One
+//               (the first two K steps as soon as the first 32 keys are in; the slot is
+//               reused by S_t(kb + 2) only after that P V has completed).  One
 //               thread issues an MMA only every ~55 cycles, so the four streams have a
 //               thread each.
 //   warps 0-3   softmax of tile 0, warps 4-7 of tile 1; thread = query row = tensor-
@@ -436,8 +437,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 //               sum l; at the end O_t / l is stored.  Warps w and w + 4 share a sub-
 //               partition and its special-function unit; they take turns at the
 //               exponentials (tile 0 of block kb, tile 1 of block kb, tile 0 of block
-//               kb + 1, ...), so that each one's loads, maxima and stores run while the
-//               other's exponentials keep the unit busy.
+//               kb + 1, ...; each hands over half way through its block), so that each
+//               one's loads, maxima and stores run while the other's exponentials keep
+//               the unit busy.
 // K and V blocks are shared by the two tiles (each slot is released by the commits of
 // both issuers): each block crosses from L2 once per 256 queries.
 // Tensor memory: O_t at columns 256 t .. 256 t + 127, S slot s of tile t at
@@ -480,8 +482,9 @@ __host__ __device__ constexpr uint64_t att_k64_step(int kk) { return (uint64_t)(
 //   p_half[t][s], p_full[t][s]  the tile's four softmax warps (one arrival each), after
 //                               the first 32 keys of P_t(kb) / all of it
 //   o_done[t][s]                commit after P_t V(kb)
-//   ex[q][t]                    lane 0 of tile t's softmax warp of quadrant q, after its
-//                               exponentials of block kb (the turn passes to the other tile)
+//   ex[q][t]                    lane 0 of tile t's softmax warp of quadrant q, half way
+//                               through its exponentials of block kb (the turn passes to
+//                               the other tile)
 // A barrier of slot kb % n completes once per use u = kb / n and a wait takes parity
 // u & 1: (kb >> 1) & 1 for the tile barriers, (kb >> 2) & 1 for the K/V slots.  No
 // barrier runs two uses ahead of a waiter, because its next use needs that waiter's own

@@ -584,28 +584,56 @@ def run_ours(args, rank, world):
     tstar_meas = roofline_time(gemms, hbm_gbs, p_int8_meas) if p_int8_meas else None
     value = whole_job_rate(ops_step, world, ms_step) / 1e12
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers.  Every step copies its
+    # input canvas in from pinned host memory and its logits back out; as in a serving
+    # loop, those copies run on their own streams and overlap the neighbouring steps'
+    # compute (two device staging buffers each way, handed over with events).
     e2e = None
     if not args.no_e2e and rank == 0:
         x_host = torch.empty(xin.numel(), dtype=torch.float32, pin_memory=True)
-        x_host.copy_(xin.cpu())
-        out_host = torch.empty(logits.shape, dtype=torch.float32, pin_memory=True)
-        ke = max(1, min(args.steps, 100))
+        x_host.copy_(xin.reshape(-1).cpu())
+        out_host = [torch.empty(logits.shape, dtype=torch.float32, pin_memory=True) for _ in range(2)]
+        x_stage = [torch.empty_like(xin) for _ in range(2)]
+        o_stage = [torch.empty_like(logits) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev = lambda: torch.cuda.Event(enable_timing=False)
+        in_ready, in_free = [ev(), ev()], [ev(), ev()]
+        out_ready, out_free = [ev(), ev()], [ev(), ev()]
+        for b in range(2):
+            in_free[b].record(s)
+            out_free[b].record(s_out)
+        ke = max(2, min(args.steps, 100))
         torch.cuda.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(s):
-            for it in range(ke + 1):
-                if it == 1:
-                    a0.record(s)
-                xin.copy_(x_host, non_blocking=True)
+        a0.record(s_in)
+        for it in range(ke):
+            b = it & 1
+            with torch.cuda.stream(s_in):           # input of step it
+                s_in.wait_event(in_free[b])
+                x_stage[b].copy_(x_host.view_as(xin), non_blocking=True)
+                in_ready[b].record(s_in)
+            with torch.cuda.stream(s):              # step it
+                s.wait_event(in_ready[b])
+                xin.copy_(x_stage[b], non_blocking=True)
+                in_free[b].record(s)
                 g1.replay()
-                out_host.copy_(logits, non_blocking=True)
-            a1.record(s)
+                s.wait_event(out_free[b])
+                o_stage[b].copy_(logits, non_blocking=True)
+                out_ready[b].record(s)
+            with torch.cuda.stream(s_out):          # logits of step it
+                s_out.wait_event(out_ready[b])
+                out_host[b].copy_(o_stage[b], non_blocking=True)
+                out_free[b].record(s_out)
+        s_out.wait_stream(s)
+        a1.record(s_out)
         torch.cuda.synchronize()
         ms_e2e = a0.elapsed_time(a1) / ke
+        assert torch.equal(out_host[(ke - 1) & 1], logits.cpu())
         e2e = {"value": ops_step / (ms_e2e * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": int(xin.numel() * 4), "d2h_bytes_per_step": int(logits.numel() * 4)}
+               "h2d_bytes_per_step": int(xin.numel() * 4), "d2h_bytes_per_step": int(logits.numel() * 4),
+               "copies": "each step's input in and logits out through pinned host buffers, on their own "
+                         "streams, overlapping the neighbouring steps' compute"}
 
     traffic = None if args.gather_last else stored_traffic(f"{args.model}_L{L}")
     roof = None

@@ -311,6 +311,14 @@ int dllm_debug_sb_ints(const void* w, dllm_qtype t, int64_t N, int64_t K, const 
  * device status with dllm_get_device_status(). */
 int dllm_debug_bounded_wait(dllm_stream_t stream);
 
+/* The same check for the attention kernels: one CTA of the one-tile kernel (two_tiles ==
+ * 0) or of the two-tile kernel (two_tiles != 0) whose TMA producers issue no copy, so
+ * every other role's first wait runs out (after about 2 s).  The kernel records
+ * DLLM_ERR_TIMEOUT in the device error word, frees its tensor memory and returns without
+ * storing anything; its tensor maps cover the library's own scratch array.  Returns the
+ * launch status. */
+int dllm_debug_attention_stall(int two_tiles, dllm_stream_t stream);
+
 /* The work split the GEMM would use for a weight of n_tiles 128-row tiles, K inputs,
  * an M-row canvas (n_rows requested rows, 0 for all) on a device with `sms` SMs.
  * Host only: no device is touched.  out (host, 8 entries) receives kc (K-chunks per

@@ -129,8 +129,9 @@ __host__ __device__ constexpr uint64_t att_qk_step(int kk) { return (uint64_t)((
 __host__ __device__ constexpr uint64_t att_v_step(int kk) { return (uint64_t)(kk * 128); }
 
 // Tensor maps over q: f16 [Lq][H][128], k, v: f16 [Lk][Hkv][128] as 3-D tensors
-// (head dim, head, row) with boxes of 8 x 1 x 128; o: f32 [Lq][H][128]; group = H / Hkv.
-// Grid (ceil(Lq / 128), H).  Requires Lk >= 1.
+// (head dim, head, row) with boxes of 64 x 1 x 128; o: f32 [Lq][H][128]; group = H / Hkv.
+// Grid (ceil(Lq / 128), H).  Requires Lk >= 1.  stall != 0 (failure test only): the
+// producers issue no copy, so every other role's first wait runs out.
 //
 // Buffers with two slots (index b = kb & 1 for key block kb): K, V, S (tensor
 // memory), P.  Barriers, each completing once per use of its slot:
@@ -146,7 +147,7 @@ __host__ __device__ constexpr uint64_t att_v_step(int kk) { return (uint64_t)(kk
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, float* __restrict__ o, int Lq, int Lk, int H,
-                     int group) {
+                     int group, int stall) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* const sQ = smem;
     uint8_t* const sK = smem + ATT_TILE;      // two slots
@@ -195,7 +196,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (warp == ATT_K_WARP || warp == ATT_V_WARP) {
         // ---------------------------------------------------------------- TMA producers
         const bool is_k = warp == ATT_K_WARP;
-        if (is_k) {
+        const int n_prod = stall ? 0 : nkb;  // stall: no copy at all (failure test)
+        if (is_k && !stall) {
             if (lane == 0) mbar_arrive_expect_tx(q_full, ATT_TILE);
             __syncwarp();
             att_tma_tile(sQ, &tq, h, q0, q_full, lane);
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const CUtensorMap* const tmap = is_k ? &tk : &tv;
         uint8_t* const dst = is_k ? sK : sV;
         int issued = 0;
-        for (int kb = 0; kb < nkb; kb++) {
+        for (int kb = 0; kb < n_prod; kb++) {
             const int b = kb & 1;
             if (kb >= 2 && !__all_sync(~0u, att_wait(&empty[b], ((kb >> 1) - 1) & 1))) break;
             if (lane == 0) mbar_arrive_expect_tx(&full[b], ATT_TILE);
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         // a wait ran out: wait for the last use of each slot (and for Q).
         if (lane == 0) {
             for (int kb = issued > 2 ? issued - 2 : 0; kb < issued; kb++) drain_wait(&full[kb & 1], (kb >> 1) & 1);
-            if (is_k) drain_wait(q_full, 0);
+            if (is_k && !stall) drain_wait(q_full, 0);
         }
         __syncwarp();
     } else if (warp == ATT_MMA_WARP) {
@@ -492,7 +494,7 @@ __host__ __device__ constexpr uint64_t att_k64_step(int kk) { return (uint64_t)(
 __global__ void __launch_bounds__(ATT_PP_THREADS, 1)
     attention_pp_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                         const __grid_constant__ CUtensorMap tv, float* __restrict__ o, int Lq, int Lk, int H,
-                        int group) {
+                        int group, int stall) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* const sQ = smem;                                    // two tiles
     uint8_t* const sK = smem + 2 * ATT_TILE;                     // four slots
@@ -547,7 +549,8 @@ __global__ void __launch_bounds__(ATT_PP_THREADS, 1)
     if (warp == ATT_PP_K_WARP || warp == ATT_PP_V_WARP) {
         // ---------------------------------------------------------------- TMA producers
         const bool is_k = warp == ATT_PP_K_WARP;
-        if (is_k) {
+        const int n_prod = stall ? 0 : nkb;  // stall: no copy at all (failure test)
+        if (is_k && !stall) {
             for (int t = 0; t < ntiles; t++) {
                 if (lane == 0) mbar_arrive_expect_tx(&q_full[t], ATT_TILE);
                 __syncwarp();
@@ -560,7 +563,7 @@ __global__ void __launch_bounds__(ATT_PP_THREADS, 1)
         const CUtensorMap* const tmap = is_k ? &tk : &tv;
         uint8_t* const dst = is_k ? sK : sV;
         int issued = 0;
-        for (int kb = 0; kb < nkb; kb++) {
+        for (int kb = 0; kb < n_prod; kb++) {
             const int v = kb & 3;
             if (kb >= ATT_PP_SLOTS && !__all_sync(~0u, att_wait(&empty[v], ((kb >> 2) - 1) & 1))) break;
             if (lane == 0) mbar_arrive_expect_tx(&full[v], ATT_PP_KV);
@@ -574,7 +577,7 @@ __global__ void __launch_bounds__(ATT_PP_THREADS, 1)
         if (lane == 0) {
             for (int kb = issued > ATT_PP_SLOTS ? issued - ATT_PP_SLOTS : 0; kb < issued; kb++)
                 drain_wait(&full[kb & 3], (kb >> 2) & 1);
-            if (is_k)
+            if (is_k && !stall)
                 for (int t = 0; t < ntiles; t++) drain_wait(&q_full[t], 0);
         }
         __syncwarp();

@@ -517,6 +517,18 @@ __device__ __align__(256) uint8_t g_noalloc_scratch[DLLM_NOALLOC_SCRATCH_BYTES];
 
 uint8_t* g_noalloc_addr[MAX_DEV];  // device address of the array, per device, once known
 
+bool att_attributes(int dev) {
+    if (!g_att_attr_done[dev]) {
+        if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATT_SMEM) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ATT_PP_SMEM) != cudaSuccess)
+            return false;
+        g_att_attr_done[dev] = true;
+    }
+    return true;
+}
+
 int noalloc_scratch(int dev, uint8_t** ptr) {
     if (!g_noalloc_addr[dev]) {
         void* p = nullptr;
@@ -566,14 +578,7 @@ int dllm_attention(const void* q, const void* k, const void* v, int64_t Lq, int6
     int dev;
     int rc = current_device(&dev);
     if (rc) return rc;
-    if (!g_att_attr_done[dev]) {
-        if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ATT_SMEM) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(attention_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)ATT_PP_SMEM) != cudaSuccess)
-            return DLLM_ERR_CUDA;
-        g_att_attr_done[dev] = true;
-    }
+    if (!att_attributes(dev)) return DLLM_ERR_CUDA;
     // the two-tile kernel reads K and V in blocks of 64 keys
     const bool pp = att_tiles_per_cta(Lq, H, g_num_sms[dev]) == 2;
     const int kv_rows = pp ? ATT_PP_BK : ATT_BK;
@@ -586,12 +591,40 @@ int dllm_attention(const void* q, const void* k, const void* v, int64_t Lq, int6
     if (pp) {
         const dim3 grid((unsigned)((Lq + ATT_PP_BQ - 1) / ATT_PP_BQ), (unsigned)H);
         e = launch_pdl(attention_pp_kernel, grid, dim3(ATT_PP_THREADS), ATT_PP_SMEM, s, tq, tk, tv, o, (int)Lq,
-                       (int)Lk, (int)H, (int)(H / Hkv));
+                       (int)Lk, (int)H, (int)(H / Hkv), 0);
     } else {
         const dim3 grid((unsigned)((Lq + ATT_BQ - 1) / ATT_BQ), (unsigned)H);
         e = launch_pdl(attention_kernel, grid, dim3(ATT_THREADS), ATT_SMEM, s, tq, tk, tv, o, (int)Lq, (int)Lk,
-                       (int)H, (int)(H / Hkv));
+                       (int)H, (int)(H / Hkv), 0);
     }
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DLLM_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+int dllm_debug_attention_stall(int two_tiles, dllm_stream_t stream) {
+    // One CTA of either attention kernel whose producers issue no copy.  The tensor maps
+    // cover the library's own scratch array and are never read; nothing is stored.
+    int dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    uint8_t* base;
+    if ((rc = noalloc_scratch(dev, &base))) return rc;
+    if (!att_attributes(dev)) return DLLM_ERR_CUDA;
+    const int Lq = two_tiles ? 2 * ATT_BQ : ATT_BQ, Lk = ATT_BK;
+    CUtensorMap tq, tkv;
+    if (!encode_head_rows(&tq, base, Lq, 1, ATT_BQ) ||
+        !encode_head_rows(&tkv, base, Lk, 1, two_tiles ? ATT_PP_BK : ATT_BK))
+        return DLLM_ERR_CUDA;
+    float* o = reinterpret_cast<float*>(base + ((size_t)1 << 20));
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        two_tiles ? launch_pdl(attention_pp_kernel, dim3(1, 1), dim3(ATT_PP_THREADS), ATT_PP_SMEM, s, tq, tkv, tkv, o,
+                               Lq, Lk, 1, 1, 1)
+                  : launch_pdl(attention_kernel, dim3(1, 1), dim3(ATT_THREADS), ATT_SMEM, s, tq, tkv, tkv, o, Lq, Lk,
+                               1, 1, 1);
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
         return DLLM_ERR_CUDA;

@@ -36,6 +36,7 @@ EXPORTS = (
     "dllm_get_device_status",
     "dllm_status_string", "dllm_debug_subblock_dots", "dllm_debug_sb_ints", "dllm_debug_bounded_wait",
     "dllm_bench_mma_i8", "dllm_debug_plan", "dllm_debug_attention_tiles",
+    "dllm_debug_attention_stall",
 )
 
 
@@ -82,6 +83,7 @@ def load() -> ctypes.CDLL:
         "dllm_bench_mma_i8": [I, I, I, I, I, I, P, P],
         "dllm_debug_plan": [I64, I64, I64, I64, I, ctypes.POINTER(ctypes.c_int64)],
         "dllm_debug_attention_tiles": [I64, I64, I],
+        "dllm_debug_attention_stall": [I, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -211,6 +213,10 @@ def dllm_debug_sb_ints(w, qtype: int, N: int, K: int, q, scale, sums, M: int, S,
 
 def dllm_debug_bounded_wait(stream=None):
     _check(load().dllm_debug_bounded_wait(_stream(stream)), "dllm_debug_bounded_wait")
+
+
+def dllm_debug_attention_stall(two_tiles: bool, stream=None):
+    _check(load().dllm_debug_attention_stall(1 if two_tiles else 0, _stream(stream)), "dllm_debug_attention_stall")
 
 
 def dllm_bench_mma_i8(n: int, n_acc: int, a_from_tmem: int, issuers: int, iters: int, ctas: int, ns_out,

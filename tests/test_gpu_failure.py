@@ -48,3 +48,31 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     ok, worst = gu.tol_ok(out, ref, T)
     assert ok, worst
     assert np.isfinite(out).all()
+
+
+@pytest.mark.parametrize("two_tiles", [False, True])
+def test_attention_bounded_waits_report_timeout_and_context_survives(two_tiles):
+    """The attention kernels' waits are bounded too: with producers that issue no copy,
+    every role gives up after about 2 s, the status reads DLLM_ERR_TIMEOUT, and the same
+    context then computes attention correctly with that kernel."""
+    from quantized_int8_gemm_q4_b200 import synth
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    t0 = time.monotonic()
+    dllm.dllm_debug_attention_stall(two_tiles)
+    status = dllm.dllm_get_device_status()
+    elapsed = time.monotonic() - t0
+    assert status == dllm.DLLM_ERR_TIMEOUT, dllm.status_string(status)
+    assert 1.5 < elapsed < 60.0, elapsed
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+
+    Lq, Lk, H, Hkv = (300, 200, 64, 8) if two_tiles else (130, 200, 4, 2)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert dllm.dllm_debug_attention_tiles(Lq, H, sms) == (2 if two_tiles else 1)
+    q, k, v = synth.attention_inputs(Lq, Lk, H, Hkv, 128, 8)
+    o = torch.empty((Lq, H, 128), device="cuda")
+    dllm.dllm_attention(*(torch.from_numpy(a).cuda() for a in (q, k, v)), Lq, Lk, H, Hkv, 128, o)
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    f32 = [a.astype(np.float32) for a in (q, k, v)]
+    ref = oracle.attention(*f32)
+    A = oracle.attention(f32[0], f32[1], np.abs(f32[2]))
+    assert np.all(np.abs(o.cpu().numpy() - ref) <= 2.0 ** -9 * A + 2.0 ** -24 * Lk * np.abs(f32[2]).max())

@@ -59,8 +59,11 @@ typedef struct CUstream_st* dllm_stream_t; /* a cudaStream_t; NULL = legacy defa
  * as wide, the low nibbles (d, dmin, the same scales) and the fifth bits as 0/1 nibbles
  * (16*d, dmin 0, the same scales), since d*sc*q - dmin*m = (d*sc*q4 - dmin*m) +
  * (16d)*sc*b exactly.  It keeps 2 x 144 bytes per 256 weights resident (9 bits per
- * weight, 1.64 x the GGUF size) and streams them at the Q4_K kernel's rate. */
-typedef enum { DLLM_Q4_K = 12, DLLM_Q5_K = 13, DLLM_Q6_K = 14 } dllm_qtype;
+ * weight, 1.64 x the GGUF size) and streams them at the Q4_K kernel's rate.
+ * Q8_0 (the same row) has a kernel of its own: 32-weight blocks, each with an f16 scale d
+ * (w = d*q, q int8); every block's integer dot product is one int8 MMA K step into an
+ * accumulator of its own, combined in f32 as da * sum_b d_b * dot_b. */
+typedef enum { DLLM_Q8_0 = 8, DLLM_Q4_K = 12, DLLM_Q5_K = 13, DLLM_Q6_K = 14 } dllm_qtype;
 
 enum {
     DLLM_OK = 0,
@@ -98,6 +101,12 @@ int dllm_repack_q6k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dl
  * gives the size.  dllm_qgemm / dllm_qkv_qgemm / dllm_qgemm_noalloc take t = DLLM_Q5_K
  * with the ordinary K-wide activations. */
 int dllm_repack_q5k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
+/* Q8_0: gguf_blocks is [N][K/32] 34-byte blocks (f16 d, then 32 int8 q).  dst receives
+ * the codes as int8 [N][K] (row-major, read by TMA with the 128-byte swizzle) followed by
+ * the block scales as f16 [N/128][K/256][128 rows][8]: 272 bytes per 256 weights, the
+ * GGUF size.  dllm_qgemm / dllm_qkv_qgemm (one launch per projection) /
+ * dllm_qgemm_noalloc take t = DLLM_Q8_0; the workspace holds only gathered rows. */
+int dllm_repack_q80(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
 
 /* ------------------------------------------------------------------------------
  * Activations: int8 with one f32 scale per 256 elements, plus scaled per-32 sums

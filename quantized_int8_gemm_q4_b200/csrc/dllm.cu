@@ -5,6 +5,7 @@
 #include "../../include/dllm_qgemm.h"
 #include "actfuse.cuh"
 #include "attention.cuh"
+#include "q80.cuh"
 #include "layout.cuh"
 #include "qgemm.cuh"
 
@@ -244,12 +245,13 @@ int run_gemm(GemmArgs& a, cudaStream_t s) {
 // Q5_K runs on the Q4_K kernel in its exact two-super-block form (see repack_q5k_kernel):
 // weight width 2K, 2 x 144 repacked bytes per 256 weights.
 int64_t kernel_k(dllm_qtype t, int64_t K) { return t == DLLM_Q5_K ? 2 * K : K; }
+// Q8_0: the int8 codes (256 bytes) and eight f16 block scales per 256 weights of a row.
 size_t repacked_per_sb(dllm_qtype t) {
-    return t == DLLM_Q4_K ? Q4K_BLOCK : t == DLLM_Q5_K ? 2 * Q4K_BLOCK : Q6K_BLOCK;
+    return t == DLLM_Q4_K ? Q4K_BLOCK : t == DLLM_Q5_K ? 2 * Q4K_BLOCK : t == DLLM_Q8_0 ? 272 : Q6K_BLOCK;
 }
 
 int check_shape(dllm_qtype t, int64_t N, int64_t K) {
-    if (t != DLLM_Q4_K && t != DLLM_Q5_K && t != DLLM_Q6_K) return DLLM_ERR_ARG;
+    if (t != DLLM_Q4_K && t != DLLM_Q5_K && t != DLLM_Q6_K && t != DLLM_Q8_0) return DLLM_ERR_ARG;
     if (N <= 0 || K <= 0 || N % TROWS || K % QK) return DLLM_ERR_ARG;
     if (N / TROWS > (1LL << 30) || K / QK > (1 << 20)) return DLLM_ERR_ARG;
     return DLLM_OK;
@@ -259,6 +261,111 @@ int check_act(const int8_t* q, const float* scale, const uint8_t* sums, int64_t 
     if (!q || !scale || !sums || M <= 0) return DLLM_ERR_ARG;
     if (!aligned16(q) || !aligned16(scale) || !aligned16(sums)) return DLLM_ERR_ALIGN;
     return DLLM_OK;
+}
+
+// ---------------------------------------------------------------- Q8_0
+bool g_q80_attr_done[MAX_DEV];
+
+// Workspace of a Q8_0 GEMM: only the gathered requested rows (codes, scales, sums).
+size_t q80_workspace(int64_t K, int64_t n_rows) {
+    if (n_rows <= 0) return 0;
+    const int64_t Mp = round_up(n_rows, 16), nsb = K / QK;
+    return align256((size_t)Mp * K) + align256((size_t)nsb * Mp * 4) + align256((size_t)nsb * Mp * 64);
+}
+
+// The Q8_0 codes plane int8 [N][K] as a 2-D tensor with boxes of 128 bytes x 128 rows,
+// 128-byte swizzled; the last few maps are kept per host thread.
+bool q80_codes_map(CUtensorMap* m, const void* base, int64_t N, int64_t K) {
+    struct Entry {
+        const void* base;
+        int64_t N, K;
+        CUtensorMap map;
+    };
+    constexpr int NE = 8;
+    thread_local Entry cache[NE] = {};
+    thread_local int next = 0;
+    for (int i = 0; i < NE; i++)
+        if (cache[i].base == base && cache[i].N == N && cache[i].K == K) {
+            *m = cache[i].map;
+            return true;
+        }
+    const EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {128, (cuuint32_t)TROWS};
+    const cuuint32_t estr[2] = {1, 1};
+    if (fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    cache[next] = {base, N, K, *m};
+    next = (next + 1) % NE;
+    return true;
+}
+
+// One Q8_0 projection (rows: gathered into the workspace first, as for the K-quants).
+// stall != 0 is the failure test: the producer issues no copy.
+int q80_gemm(const void* w, int64_t N, int64_t K, const int8_t* q, const float* scale, const uint8_t* sums,
+             int64_t M, const int32_t* rows, int64_t n_rows, float* out, int64_t ldo, void* workspace,
+             size_t workspace_bytes, cudaStream_t s, int stall) {
+    int rc = check_shape(DLLM_Q8_0, N, K);
+    if (rc) return rc;
+    if ((rc = check_act(q, scale, sums, M))) return rc;
+    if (!w || !out || ldo < N) return DLLM_ERR_ARG;
+    if (!aligned16(w) || !aligned16(out) || ldo % 4) return DLLM_ERR_ALIGN;
+    if (rows && (n_rows < 1 || n_rows > 32)) return DLLM_ERR_ARG;
+    if (rows && !aligned16(rows)) return DLLM_ERR_ALIGN;
+    if (M > (1LL << 31)) return DLLM_ERR_ARG;
+    if (workspace && !aligned16(workspace)) return DLLM_ERR_ALIGN;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    const int64_t nsb = K / QK;
+    const int64_t Mp = round_up(rows ? n_rows : M, 16);
+    if (rows) {
+        const size_t need = q80_workspace(K, n_rows);
+        if (!workspace || workspace_bytes < need) return DLLM_ERR_WORKSPACE;
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        int8_t* gq = reinterpret_cast<int8_t*>(ws);
+        float* gs = reinterpret_cast<float*>(ws + align256((size_t)Mp * K));
+        uint8_t* gu = ws + align256((size_t)Mp * K) + align256((size_t)nsb * Mp * 4);
+        if (launch_pdl(gather_rows_kernel, dim3(grid_for(nsb * Mp * 21, 256)), dim3(256), 0, s, q, scale, sums, M,
+                       round_up(M, 16), rows, (int32_t)n_rows, Mp, (int32_t)nsb, gq, gs, gu) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return DLLM_ERR_CUDA;
+        }
+        if ((rc = launch_status())) return rc;
+        q = gq;
+        scale = gs;
+    }
+    if (!g_q80_attr_done[dev]) {
+        if (cudaFuncSetAttribute(q80_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Q80_SMEM) !=
+            cudaSuccess)
+            return DLLM_ERR_CUDA;
+        g_q80_attr_done[dev] = true;
+    }
+    CUtensorMap tw;
+    if (!q80_codes_map(&tw, w, N, K)) return DLLM_ERR_CUDA;
+    Q80Args a;
+    memset(&a, 0, sizeof(a));
+    a.w = static_cast<const uint8_t*>(w);
+    a.q = q;
+    a.scale = scale;
+    a.out = out;
+    a.ldo = ldo;
+    a.n_tiles = (int32_t)(N / TROWS);
+    a.nsb = (int32_t)nsb;
+    a.n_tok = (int32_t)((Mp + Q80_TOK - 1) / Q80_TOK);
+    a.n_units = (int64_t)a.n_tiles * a.n_tok;
+    a.Mp = (int32_t)Mp;
+    a.m_out = (int32_t)(rows ? n_rows : M);
+    a.stall = stall;
+    const int grid = (int)(a.n_units < g_num_sms[dev] ? a.n_units : g_num_sms[dev]);
+    if (launch_pdl(q80_gemm_kernel, dim3(stall ? 1 : grid), dim3(Q80_THREADS), Q80_SMEM, s, tw, a) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DLLM_ERR_CUDA;
+    }
+    return launch_status();
 }
 
 }  // namespace
@@ -279,7 +386,8 @@ static int repack(dllm_qtype t, const void* src, int64_t N, int64_t K, void* dst
     if (!src || !dst) return DLLM_ERR_ARG;
     if (!aligned16(dst)) return DLLM_ERR_ALIGN;
     const size_t bytes = (size_t)N * (K / QK) * repacked_per_sb(t);
-    const size_t src_bytes = (size_t)N * (K / QK) * (t == DLLM_Q4_K ? Q4K_BLOCK : t == DLLM_Q5_K ? Q5K_BLOCK : Q6K_BLOCK);
+    const size_t src_bytes = (size_t)N * (K / QK) *
+                             (t == DLLM_Q4_K ? Q4K_BLOCK : t == DLLM_Q5_K ? Q5K_BLOCK : t == DLLM_Q8_0 ? 272 : Q6K_BLOCK);
     const uint8_t* s8 = static_cast<const uint8_t*>(src);
     const uint8_t* d8 = static_cast<const uint8_t*>(dst);
     if (s8 < d8 + bytes && d8 < s8 + src_bytes) return DLLM_ERR_ARG;
@@ -291,6 +399,9 @@ static int repack(dllm_qtype t, const void* src, int64_t N, int64_t K, void* dst
         repack_q4k_kernel<<<grid_for(chunks, 256), 256, 0, s>>>(s8, N, K / QK, static_cast<uint8_t*>(dst));
     else if (t == DLLM_Q5_K)
         repack_q5k_kernel<<<grid_for(chunks, 256), 256, 0, s>>>(s8, N, K / QK, static_cast<uint8_t*>(dst));
+    else if (t == DLLM_Q8_0)
+        repack_q80_kernel<<<grid_for(N * K / 16 + N * (K / QK), 256), 256, 0, s>>>(s8, N, K,
+                                                                                  static_cast<uint8_t*>(dst));
     else
         repack_q6k_kernel<<<grid_for(chunks, 256), 256, 0, s>>>(s8, N, K / QK, static_cast<uint8_t*>(dst));
     return launch_status();
@@ -304,6 +415,9 @@ int dllm_repack_q6k(const void* g, int64_t N, int64_t K, void* dst, dllm_stream_
 }
 int dllm_repack_q5k(const void* g, int64_t N, int64_t K, void* dst, dllm_stream_t s) {
     return repack(DLLM_Q5_K, g, N, K, dst, s);
+}
+int dllm_repack_q80(const void* g, int64_t N, int64_t K, void* dst, dllm_stream_t s) {
+    return repack(DLLM_Q8_0, g, N, K, dst, s);
 }
 
 int dllm_act_bytes(int64_t M, int64_t K, size_t* q_bytes, size_t* scale_bytes, size_t* sums_bytes) {
@@ -383,7 +497,7 @@ int dllm_qgemm_workspace_bytes(dllm_qtype t, int64_t N, int64_t K, int64_t M, in
     if (M <= 0 || n_rows < 0 || n_rows > 32 || !bytes) return DLLM_ERR_ARG;
     int dev;
     if ((rc = current_device(&dev))) return rc;
-    *bytes = make_plan(N / TROWS, kernel_k(t, K), M, n_rows, g_num_sms[dev], K).bytes;
+    *bytes = t == DLLM_Q8_0 ? q80_workspace(K, n_rows) : make_plan(N / TROWS, kernel_k(t, K), M, n_rows, g_num_sms[dev], K).bytes;
     return DLLM_OK;
 }
 
@@ -401,7 +515,7 @@ static int gemm_common(GemmArgs& a, dllm_qtype t, int64_t N_total, int64_t K, co
     if (workspace && !aligned16(workspace)) return DLLM_ERR_ALIGN;
     int dev;
     if ((rc = current_device(&dev))) return rc;
-    if (dbg && t == DLLM_Q5_K) return DLLM_ERR_ARG;  // the integer debug view covers Q4_K and Q6_K
+    if (dbg && (t == DLLM_Q5_K || t == DLLM_Q8_0)) return DLLM_ERR_ARG;  // the integer view covers Q4_K and Q6_K
     Plan p = make_plan(N_total / TROWS, kernel_k(t, K), M, rows ? n_rows : 0, g_num_sms[dev], K);
     if (dbg) {  // integers per super-block: no chunk partials to combine
         p.kc = 1;
@@ -466,6 +580,8 @@ int dllm_qgemm(const void* w, dllm_qtype t, int64_t N, int64_t K, const int8_t* 
     if (!w || !out || ldo < N) return DLLM_ERR_ARG;
     if (!aligned16(w) || !aligned16(out) || ldo % 4) return DLLM_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (t == DLLM_Q8_0)
+        return q80_gemm(w, N, K, q, scale, sums, M, rows, n_rows, out, ldo, workspace, workspace_bytes, s, 0);
     GemmArgs a;
     int rc = gemm_common(a, t, N, K, q, scale, sums, M, rows, n_rows, workspace, workspace_bytes, false, s);
     if (rc) return rc;
@@ -488,6 +604,14 @@ int dllm_qkv_qgemm(const void* wq, const void* wk, const void* wv, dllm_qtype t,
         return DLLM_ERR_ALIGN;
     const int64_t N_total = Nq + (wv ? 2 : 1) * Nkv;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (t == DLLM_Q8_0) {  // one launch per projection, all on the same quantized activation
+        if ((rc = q80_gemm(wq, Nq, K, q, scale, sums, M, nullptr, 0, oq, ldo_q, workspace, workspace_bytes, s, 0)))
+            return rc;
+        if ((rc = q80_gemm(wk, Nkv, K, q, scale, sums, M, nullptr, 0, ok, ldo_kv, workspace, workspace_bytes, s, 0)))
+            return rc;
+        return wv ? q80_gemm(wv, Nkv, K, q, scale, sums, M, nullptr, 0, ov, ldo_kv, workspace, workspace_bytes, s, 0)
+                  : DLLM_OK;
+    }
     GemmArgs a;
     rc = gemm_common(a, t, N_total, K, q, scale, sums, M, nullptr, 0, workspace, workspace_bytes, false, s);
     if (rc) return rc;

@@ -14,6 +14,7 @@ LIB_PATH = Path(__file__).resolve().parent / "_build" / "libdllm_qgemm.so"
 DLLM_Q4_K = 12
 DLLM_Q6_K = 14
 DLLM_Q5_K = 13
+DLLM_Q8_0 = 8
 QK_K = 256
 BLOCK_BYTES = {DLLM_Q4_K: 144, DLLM_Q6_K: 210}
 
@@ -29,7 +30,8 @@ DLLM_ERR_SCRATCH_LIMIT = -8
 DLLM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 EXPORTS = (
-    "dllm_repacked_bytes", "dllm_repack_q4k", "dllm_repack_q6k", "dllm_repack_q5k", "dllm_act_bytes",
+    "dllm_repacked_bytes", "dllm_repack_q4k", "dllm_repack_q6k", "dllm_repack_q5k", "dllm_repack_q80",
+    "dllm_act_bytes",
     "dllm_quantize_act",
     "dllm_rmsnorm_quantize", "dllm_swiglu_quantize",
     "dllm_qgemm_workspace_bytes", "dllm_qgemm", "dllm_qgemm_noalloc", "dllm_qkv_qgemm", "dllm_attention",
@@ -66,6 +68,7 @@ def load() -> ctypes.CDLL:
         "dllm_repack_q4k": [P, I64, I64, P, P],
         "dllm_repack_q6k": [P, I64, I64, P, P],
         "dllm_repack_q5k": [P, I64, I64, P, P],
+        "dllm_repack_q80": [P, I64, I64, P, P],
         "dllm_act_bytes": [I64, I64, PSZ, PSZ, PSZ],
         "dllm_quantize_act": [P, I64, I64, I64, P, P, P, P],
         "dllm_rmsnorm_quantize": [P, I64, I64, I64, P, ctypes.c_float, P, I64, P, P, P, P],
@@ -134,6 +137,10 @@ def dllm_repack_q4k(gguf_blocks, N: int, K: int, dst, stream=None):
 
 def dllm_repack_q5k(gguf_blocks, N: int, K: int, dst, stream=None):
     _check(load().dllm_repack_q5k(_ptr(gguf_blocks), N, K, _ptr(dst), _stream(stream)), "dllm_repack_q5k")
+
+
+def dllm_repack_q80(gguf_blocks, N: int, K: int, dst, stream=None):
+    _check(load().dllm_repack_q80(_ptr(gguf_blocks), N, K, _ptr(dst), _stream(stream)), "dllm_repack_q80")
 
 
 def dllm_repack_q6k(gguf_blocks, N: int, K: int, dst, stream=None):
@@ -234,7 +241,8 @@ def repack(qtype: int, blocks, N: int, K: int, device="cuda", stream=None):
         blocks = torch.from_numpy(blocks.reshape(-1).copy())
     src = blocks.reshape(-1).to(device)
     dst = torch.empty(dllm_repacked_bytes(qtype, N, K), dtype=torch.uint8, device=device)
-    fn = {DLLM_Q4_K: dllm_repack_q4k, DLLM_Q5_K: dllm_repack_q5k, DLLM_Q6_K: dllm_repack_q6k}[qtype]
+    fn = {DLLM_Q4_K: dllm_repack_q4k, DLLM_Q5_K: dllm_repack_q5k, DLLM_Q6_K: dllm_repack_q6k,
+          DLLM_Q8_0: dllm_repack_q80}[qtype]
     fn(src, N, K, dst, stream)
     return dst
 

@@ -62,8 +62,8 @@ def test_bad_shapes_rejected(lib, N, K):
 
 def test_bad_qtype_rejected(lib):
     out = ctypes.c_size_t(0)
-    assert lib.dllm_repacked_bytes(8, 128, 256, ctypes.byref(out)) == dllm.DLLM_ERR_ARG   # Q8_0: no kernel
-    assert lib.dllm_repacked_bytes(15, 128, 256, ctypes.byref(out)) == dllm.DLLM_ERR_ARG
+    for t in (0, 2, 9, 10, 11, 15):
+        assert lib.dllm_repacked_bytes(t, 128, 256, ctypes.byref(out)) == dllm.DLLM_ERR_ARG
 
 
 def _fake(addr):
@@ -91,7 +91,8 @@ def test_gemm_argument_checks_before_launch(lib):
     assert call(ldo=258) == dllm.DLLM_ERR_ALIGN
     assert call(rows=_fake(A), n_rows=0) == dllm.DLLM_ERR_ARG
     assert call(rows=_fake(A), n_rows=33) == dllm.DLLM_ERR_ARG
-    assert call(t=8) == dllm.DLLM_ERR_ARG
+    assert call(t=9) == dllm.DLLM_ERR_ARG
+    assert call(t=dllm.DLLM_Q8_0, K=300) == dllm.DLLM_ERR_ARG
 
 
 def test_quantize_argument_checks(lib):
@@ -154,6 +155,14 @@ def test_qkv_argument_checks(lib):
     ok = f(_fake(A), _fake(A), None, dllm.DLLM_Q4_K, 256, 100, 512, _fake(A), _fake(A), _fake(A), 16,
            _fake(A), 256, _fake(A), None, 128, None, 0, None)
     assert ok == dllm.DLLM_ERR_ARG
+
+
+def test_q80_repacked_size_is_the_gguf_size(lib):
+    """Q8_0 keeps its 272 bytes per 256 weights (codes plane, then block scales)."""
+    out = ctypes.c_size_t(0)
+    assert lib.dllm_repacked_bytes(dllm.DLLM_Q8_0, 384, 4096, ctypes.byref(out)) == dllm.DLLM_OK
+    assert out.value == 384 * 16 * 272
+    assert lib.dllm_repacked_bytes(dllm.DLLM_Q8_0, 100, 4096, ctypes.byref(out)) == dllm.DLLM_ERR_ARG
 
 
 def test_q5k_repacked_size_is_the_split_form(lib):

@@ -45,7 +45,7 @@ P_INT8_NOMINAL = 4.5e15  # dense int8 tensor ops/s of a B200 (datasheet)
 FALLBACK_BF16_TFLOPS = 1590.0  # dense bf16 (= f16) tensor TFLOP/s measured earlier on this machine (burst)
 # special-function unit: 16 ex2 per clock per SM x 148 SMs x 1.965 GHz (max SM clock)
 SFU_EX2_PER_S = 16 * 148 * 1.965e9
-Q4, Q6 = 12, 14
+Q4, Q6, Q8 = 12, 14, 8
 
 
 def parse():
@@ -62,12 +62,12 @@ def parse():
                         "sampled on 1/64 of their output columns")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
-    p.add_argument("--config", choices=["c1", "c2", "c3", "act", "attn"], default=None,
+    p.add_argument("--config", choices=["c1", "c2", "c3", "act", "attn", "q80"], default=None,
                    help="time one of the single-GEMM workloads instead of the step: c1 attention projections "
                         "(QKV in one launch + O, 160 rows), c2 FFN (gate/up + down) over canvases 160..1024, "
                         "c3 output projection on 1..32 requested rows, act the fused quantizers at the step's "
-                        "canvas and at 2^24 elements, attn the bidirectional attention over canvases 128..4096; "
-                        "one JSON line per case")
+                        "canvas and at 2^24 elements, attn the bidirectional attention over canvases 128..4096, "
+                        "q80 Q8_0 projections of the model's shapes; one JSON line per case")
     p.add_argument("--parallel", choices=["replicas", "nsplit"], default="replicas",
                    help="with several ranks: replicas (each GPU runs the whole step, weak scaling) or nsplit "
                         "(each GPU owns 1/N of every projection's weight rows, outputs all-gathered over NCCL, "
@@ -89,11 +89,11 @@ class Gemm:
 
     @property
     def weight_bytes(self):
-        return self.N * (self.K // 256) * (144 if self.qtype == Q4 else 210)
+        return self.N * (self.K // 256) * {Q4: 144, Q6: 210, Q8: 272}[self.qtype]
 
     @property
     def bytes(self):
-        per = 1 + 4 / 256 + (16 / 256 if self.qtype == Q4 else 0)
+        per = 1 + 4 / 256 + (16 / 256 if self.qtype == Q4 else 0)  # codes, scales (and Q4_K's sums)
         return self.weight_bytes + self.M_act * self.K * per + self.M_out * self.N * 4
 
 
@@ -926,6 +926,9 @@ def config_cases(name, model):
     if name == "c2":
         return [(f"ffn M={M}", [Gemm("gate_up", Q4, 2 * f, h, M, M), Gemm("down", Q6, h, f, M, M)], M, None)
                 for M in (160, 256, 512, 1024)]
+    if name == "q80":
+        return ([(f"q80 o M={M}", [Gemm("q80_o", Q8, h, h, M, M)], M, None) for M in (32, 128, 160, 512)] +
+                [("q80 qkv-wide M=160", [Gemm("q80_qkv", Q8, model.q_out + 2 * model.kv_out, h, 160, 160)], 160, None)])
     return [(f"output rows={R}", [Gemm("output", Q6, model.vocab, h, R, R)], 160, R) for R in (1, 2, 4, 8, 16, 32)]
 
 
@@ -1072,7 +1075,7 @@ def run_config(args):
                 for n, pi in parts:
                     gg = synth.device_weights(g.qtype, n, g.K, 4, gi, pi, c, device=dev)
                     w = torch.empty(dllm.dllm_repacked_bytes(g.qtype, n, g.K), dtype=torch.uint8, device=dev)
-                    (dllm.dllm_repack_q4k if g.qtype == Q4 else dllm.dllm_repack_q6k)(gg, n, g.K, w)
+                    {Q4: dllm.dllm_repack_q4k, Q6: dllm.dllm_repack_q6k, Q8: dllm.dllm_repack_q80}[g.qtype](gg, n, g.K, w)
                     del gg
                     ws_.append(w)
                 cps.append(ws_)

@@ -198,6 +198,13 @@ def device_weights(qtype: int, N: int, K: int, seed, *sub, device="cuda"):
     g = _torch_gen(device, seed, qtype, *sub)
     bb = BLOCK_BYTES[qtype]
     blk = torch.empty((nb, bb), dtype=torch.uint8, device=device)
+    if qtype == Q8_0:  # eight 34-byte blocks per 256 weights: d in [1e-4, 1e-3), 32 int8 codes
+        b8 = blk.view(nb * 8, 34)
+        d8 = (torch.rand((nb * 8, 1), generator=g, device=device) * (1e-3 - 1e-4) + 1e-4).to(torch.float16)
+        b8[:, 0:2] = d8.contiguous().view(torch.uint8).reshape(nb * 8, 2)
+        b8[:, 2:] = torch.randint(-127, 128, (nb * 8, 32), generator=g, device=device,
+                                  dtype=torch.int8).view(torch.uint8)
+        return blk.reshape(-1)
     d = (torch.rand((nb, 2 if qtype == Q4_K else 1), generator=g, device=device) * (1e-2 - 1e-3) + 1e-3)
     d16 = d.to(torch.float16).contiguous().view(torch.uint8).reshape(nb, -1)
     if qtype == Q4_K:

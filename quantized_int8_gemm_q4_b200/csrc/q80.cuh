@@ -9,9 +9,10 @@
 // scale, so each block's dot product goes to an accumulator of its own: per super-block
 // eight accumulators of (128 weight rows x 32 tokens) in tensor memory, two sets of
 // them so the MMAs of the next super-block run while the epilogue reads this one.  The
-// epilogue makes each dot an f32 exactly (|dot| <= 32 * 128 * 127 < 2^22: the bits of
-// dot + bits(1.5 * 2^23) are the f32 1.5 * 2^23 + dot), and accumulates
-// da * sum_b d_b * dot_b in f32 registers.
+// accumulators are preset to the bits of 1.5 * 2^23 and the MMAs add to them, so each
+// holds the f32 1.5 * 2^23 + dot exactly (|dot| <= 32 * 128 * 127 < 2^22); the epilogue
+// subtracts 1.5 * 2^23 (exact), writes the preset back, and accumulates
+// da * sum_b d_b * dot_b in f32 registers with packed two-token operations.
 //
 // Repacked weights (dllm_repack_q80, same 272 bytes per 256 weights as GGUF):
 //   codes  int8 [N][K] row-major, read by TMA in boxes of 128 bytes x 128 rows with the
@@ -27,7 +28,8 @@
 //   warp 0      producer: per super-block one stage of 4 (codes by TMA, scales, the
 //               activation codes and scales by bulk copies), after the dependency wait
 //   warp 1      one thread issues the 8 MMAs of a super-block (kind::i8, A and B from
-//               shared memory, overwrite), and the warp owns tensor memory
+//               shared memory, accumulating onto the preset), and the warp owns tensor
+//               memory
 //   warps 2-9   epilogue: the warp's tensor-memory lane quadrant is warp % 4; warps 2-5
 //               take blocks 0-3 and warps 6-9 blocks 4-7 of each super-block, and the
 //               two halves' sums are added through shared memory at the end of a unit
@@ -105,7 +107,8 @@ __device__ __forceinline__ void q80_unit(const Q80Args& a, int64_t u, int& tile,
 //   empty[st]   the issuer's commit (MMAs read the codes) and the 8 epilogue warps (they
 //               read the scales)
 //   acc_full[c] the issuer's commit after the 8 MMAs
-//   acc_empty[c] the 8 epilogue warps, once the accumulators are in registers
+//   acc_empty[c] the 8 epilogue warps, once the accumulators are in registers and preset
+//               again (use 0: the first preset, before any MMA)
 //   epi         the 8 epilogue warps, twice per unit (halves added through shared memory)
 //   fin         the issuer's last commit, before tensor memory is freed
 // Each waits with parity (use & 1) where use counts the barrier's completions; no
@@ -190,8 +193,7 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
                 const uint32_t id = idesc_i8(TROWS, ntok, 1, 1);
                 for (int s = 0; s < a.nsb; s++, g++) {
                     const int st = (int)(g % Q80_STAGES), c = (int)(g & 1);
-                    if (!q80_wait(&full[st], (g / Q80_STAGES) & 1) ||
-                        (g >= 2 && !q80_wait(&acc_empty[c], ((g >> 1) - 1) & 1))) {
+                    if (!q80_wait(&full[st], (g / Q80_STAGES) & 1) || !q80_wait(&acc_empty[c], (g >> 1) & 1)) {
                         ok = false;
                         break;
                     }
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
 #pragma unroll
                     for (int b = 0; b < 8; b++)
                         mma_i8_ss(tm + 256 * c + 32 * b, da + (uint64_t)((b >> 2) * 1024 + (b & 3) * 2),
-                                  db + (uint64_t)(16 * b), id, 0u);
+                                  db + (uint64_t)(16 * b), id, 1u);
                     tc_commit(&acc_full[c]);
                     tc_commit(&empty[st]);
                 }
@@ -217,14 +219,34 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
         const int qd = warp & 3, hf = (warp - Q80_EPI_WARP0) >> 2;
         const int row = 32 * qd + lane;
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+        uint32_t magic[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) magic[i] = MAGIC_BITS;
+        // first preset of this warp's blocks in both accumulator sets
+#pragma unroll
+        for (int c = 0; c < 2; c++)
+#pragma unroll
+            for (int bb = 0; bb < 4; bb++) {
+                const uint32_t ta = tm + lane_off + 256 * c + 32 * (4 * hf + bb);
+                tmem_st16(ta, magic);
+                tmem_st16(ta + 16, magic);
+            }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&acc_empty[0]);
+            mbar_arrive(&acc_empty[1]);
+        }
+        const float2 nM = make_float2(-MAGIC, -MAGIC);
         uint32_t g = 0, eph = 0;
         bool ok = true;
         for (int64_t u = blockIdx.x; ok && u < a.n_units; u += gridDim.x) {
             int tile, m0, ntok;
             q80_unit(a, u, tile, m0, ntok);
-            float acc[Q80_TOK];
+            float2 acc[Q80_TOK / 2];
 #pragma unroll
-            for (int j = 0; j < Q80_TOK; j++) acc[j] = 0.0f;
+            for (int j = 0; j < Q80_TOK / 2; j++) acc[j] = make_float2(0.0f, 0.0f);
             for (int s = 0; s < a.nsb; s++, g++) {
                 const int st = (int)(g % Q80_STAGES), c = (int)(g & 1);
                 ok = __all_sync(~0u, q80_wait(&acc_full[c], (g >> 1) & 1) &&
@@ -235,9 +257,11 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
                 const uint2 dw = *reinterpret_cast<const uint2*>(sb + Q80_OFF_D + row * 16 + hf * 8);
                 const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dw.x));
                 const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dw.y));
-                const float* const das = reinterpret_cast<const float*>(sb + Q80_OFF_S);
-                // 16 token columns at a time; the accumulators are released once the last
-                // columns are in registers
+                const float2 dv[4] = {make_float2(d01.x, d01.x), make_float2(d01.y, d01.y),
+                                      make_float2(d23.x, d23.x), make_float2(d23.y, d23.y)};
+                const float2* const das = reinterpret_cast<const float2*>(sb + Q80_OFF_S);
+                // 16 token columns at a time: into registers, the preset written back; the
+                // accumulators are released once the last columns are preset again
 #pragma unroll
                 for (int cc = 0; cc < Q80_TOK / 16; cc++) {
                     if (16 * cc < ntok) {
@@ -246,19 +270,25 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
                         for (int bb = 0; bb < 4; bb++)
                             tmem_ld16(tm + lane_off + 256 * c + 32 * (4 * hf + bb) + 16 * cc, x[bb]);
                         tmem_wait_ld();
+#pragma unroll
+                        for (int bb = 0; bb < 4; bb++)
+                            tmem_st16(tm + lane_off + 256 * c + 32 * (4 * hf + bb) + 16 * cc, magic);
                         if (16 * (cc + 1) >= ntok) {
+                            tmem_wait_st();
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&acc_empty[c]);
                         }
 #pragma unroll
-                        for (int i = 0; i < 16; i++) {
-                            const int j = 16 * cc + i;
-                            float t = d01.x * (__uint_as_float(x[0][i] + MAGIC_BITS) - MAGIC);
-                            t = fmaf(d01.y, __uint_as_float(x[1][i] + MAGIC_BITS) - MAGIC, t);
-                            t = fmaf(d23.x, __uint_as_float(x[2][i] + MAGIC_BITS) - MAGIC, t);
-                            t = fmaf(d23.y, __uint_as_float(x[3][i] + MAGIC_BITS) - MAGIC, t);
-                            acc[j] = fmaf(das[j], t, acc[j]);
+                        for (int i = 0; i < 8; i++) {
+                            float2 t = make_float2(0.0f, 0.0f);
+#pragma unroll
+                            for (int bb = 0; bb < 4; bb++) {
+                                const float2 X = __fadd2_rn(
+                                    make_float2(__uint_as_float(x[bb][2 * i]), __uint_as_float(x[bb][2 * i + 1])), nM);
+                                t = __ffma2_rn(dv[bb], X, t);
+                            }
+                            acc[8 * cc + i] = __ffma2_rn(das[8 * cc + i], t, acc[8 * cc + i]);
                         }
                     }
                 }
@@ -269,8 +299,9 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
             float* const xr = xbuf + row * Q80_TOK;
             if (ok && hf == 1) {
 #pragma unroll
-                for (int j = 0; j < Q80_TOK; j += 4)
-                    *reinterpret_cast<float4*>(xr + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                for (int j = 0; j < Q80_TOK / 2; j += 2)
+                    *reinterpret_cast<float4*>(xr + 2 * j) =
+                        make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(epi);
@@ -281,7 +312,7 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
                 float* const dst = a.out + (int64_t)m0 * a.ldo + (int64_t)tile * TROWS + row;
 #pragma unroll
                 for (int j = 0; j < Q80_TOK; j++)
-                    if (j < cnt) dst[(int64_t)j * a.ldo] = acc[j] + xr[j];
+                    if (j < cnt) dst[(int64_t)j * a.ldo] = (j & 1 ? acc[j >> 1].y : acc[j >> 1].x) + xr[j];
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(epi);

@@ -14,6 +14,17 @@
 // subtracts 1.5 * 2^23 (exact), writes the preset back, and accumulates
 // da * sum_b d_b * dot_b in f32 registers with packed two-token operations.
 //
+// The period of a super-block is set by the tensor pipe and by tensor-memory latency,
+// not by HBM: an int8 MMA with A in shared memory takes ~110 cycles at N <= 128 whatever
+// the thread that issues it (two issuing threads give no more), so the eight MMAs of a
+// super-block take ~870 cycles; and each load -> wait -> preset -> wait round trip of
+// tensor memory takes ~150-350 cycles with 16 warps, against ~425 B per cycle per SM of
+// tensor-memory bandwidth that the epilogue uses only a third of.  Measured and kept
+// out: 64-token units (one accumulator set with a release per quarter, N = 64 halving
+// the MMAs per token) were slower because the epilogue round trips then sit on the
+// path of every quarter, and one round trip for all eight blocks leaves the epilogue's
+// arithmetic after the release, where it becomes the period.
+//
 // Repacked weights (dllm_repack_q80, same 272 bytes per 256 weights as GGUF):
 //   codes  int8 [N][K] row-major, read by TMA in boxes of 128 bytes x 128 rows with the
 //          128-byte swizzle (the K-major swizzled A operand: 1024 bytes between 8-row
@@ -24,15 +35,16 @@
 //
 // One CTA per SM, persistent over work units (128 weight rows, 32 tokens, all of K);
 // the units of one weight tile are consecutive, so the tile streams from HBM once and
-// from L2 for the other token groups.  10 warps:
-//   warp 0      producer: per super-block one stage of 4 (codes by TMA, scales, the
+// from L2 for the other token groups.  18 warps:
+//   warp 0      producer: per super-block one stage of 5 (codes by TMA, scales, the
 //               activation codes and scales by bulk copies), after the dependency wait
 //   warp 1      one thread issues the 8 MMAs of a super-block (kind::i8, A and B from
 //               shared memory, accumulating onto the preset), and the warp owns tensor
 //               memory
-//   warps 2-9   epilogue: the warp's tensor-memory lane quadrant is warp % 4; warps 2-5
-//               take blocks 0-3 and warps 6-9 blocks 4-7 of each super-block, and the
-//               two halves' sums are added through shared memory at the end of a unit
+//   warps 2-17  epilogue: the warp's tensor-memory lane quadrant is warp % 4 and its 8
+//               tokens (warp - 2) / 4; it takes all eight blocks of its rows and tokens,
+//               two blocks per tensor-memory round trip, so each output has one owner
+//               and is stored straight from registers
 #pragma once
 #include <cuda.h>
 
@@ -41,7 +53,7 @@
 namespace dllm {
 
 constexpr int Q80_TOK = 32;                    // tokens per unit (the MMA's N)
-constexpr int Q80_STAGES = 4;
+constexpr int Q80_STAGES = 5;
 constexpr int Q80_SQ = TROWS * QK;             // codes of a tile super-block, 32 KB
 constexpr int Q80_SA = Q80_TOK * QK;           // activation codes, 8 KB
 constexpr int Q80_SD = TROWS * 8 * 2;          // block scales, 2 KB
@@ -50,9 +62,10 @@ constexpr int Q80_OFF_A = Q80_SQ;
 constexpr int Q80_OFF_D = Q80_SQ + Q80_SA;
 constexpr int Q80_OFF_S = Q80_OFF_D + Q80_SD;
 constexpr int Q80_STAGE = (Q80_OFF_S + Q80_SS + 1023) / 1024 * 1024;
-constexpr int Q80_THREADS = 32 * 10;
 constexpr int Q80_EPI_WARP0 = 2;
-constexpr size_t Q80_SMEM = (size_t)Q80_STAGES * Q80_STAGE + (size_t)TROWS * Q80_TOK * 4 + 256;
+constexpr int Q80_EPI_WARPS = 16;
+constexpr int Q80_THREADS = 32 * (Q80_EPI_WARP0 + Q80_EPI_WARPS);
+constexpr size_t Q80_SMEM = (size_t)Q80_STAGES * Q80_STAGE + 256;
 constexpr uint64_t Q80_WAIT_NS = 2000000000ull;
 
 struct Q80Args {
@@ -102,41 +115,44 @@ __device__ __forceinline__ void q80_unit(const Q80Args& a, int64_t u, int& tile,
     ntok = min(Q80_TOK, a.Mp - m0);
 }
 
-// Barriers (stage st = g % 4, accumulator set c = g & 1 for the CTA's g-th super-block):
-//   full[st]    transaction bytes of the stage's copies
-//   empty[st]   the issuer's commit (MMAs read the codes) and the 8 epilogue warps (they
-//               read the scales)
-//   acc_full[c] the issuer's commit after the 8 MMAs
-//   acc_empty[c] the 8 epilogue warps, once the accumulators are in registers and preset
-//               again (use 0: the first preset, before any MMA)
-//   epi         the 8 epilogue warps, twice per unit (halves added through shared memory)
-//   fin         the issuer's last commit, before tensor memory is freed
+// 32 lanes x 8 consecutive 32-bit columns, all set to v.
+__device__ __forceinline__ void tmem_st8_same(uint32_t taddr, uint32_t v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
+                 : "memory");
+}
+
+// Barriers (stage st = g % Q80_STAGES, accumulator set c = g & 1 for the CTA's g-th
+// super-block):
+//   full[st]     transaction bytes of the stage's copies
+//   empty[st]    the issuer's commit (MMAs read the codes) and the 16 epilogue warps (they
+//                read the scales)
+//   acc_full[c]  the issuer's commit after the 8 MMAs
+//   acc_empty[c] the 16 epilogue warps, once their columns are in registers and preset
+//                again (use 0: the first preset, before any MMA)
+//   fin          the issuer's last commit, before tensor memory is freed
 // Each waits with parity (use & 1) where use counts the barrier's completions; no
 // barrier runs two uses ahead of a waiter, because its next use needs that waiter.
 __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_constant__ CUtensorMap tw,
                                                                  const __grid_constant__ Q80Args a) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    float* const xbuf = reinterpret_cast<float*>(smem + Q80_STAGES * Q80_STAGE);  // [128 rows][32]
-    uint64_t* const bars = reinterpret_cast<uint64_t*>(smem + Q80_STAGES * Q80_STAGE + TROWS * Q80_TOK * 4);
-    uint64_t* const full = bars;            // [4]
-    uint64_t* const empty = bars + 4;       // [4]
-    uint64_t* const acc_full = bars + 8;    // [2]
-    uint64_t* const acc_empty = bars + 10;  // [2]
-    uint64_t* const epi = bars + 12;
-    uint64_t* const fin = bars + 13;
-    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+    uint64_t* const bars = reinterpret_cast<uint64_t*>(smem + Q80_STAGES * Q80_STAGE);
+    uint64_t* const full = bars;                      // [Q80_STAGES]
+    uint64_t* const empty = bars + Q80_STAGES;        // [Q80_STAGES]
+    uint64_t* const acc_full = bars + 2 * Q80_STAGES; // [2]
+    uint64_t* const acc_empty = acc_full + 2;         // [2]
+    uint64_t* const fin = acc_full + 4;
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < Q80_STAGES; i++) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1 + 8);
+            mbar_init(&empty[i], 1 + Q80_EPI_WARPS);
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 8);
+            mbar_init(&acc_empty[i], Q80_EPI_WARPS);
         }
-        mbar_init(epi, 8);
         mbar_init(fin, 1);
         fence_mbar_init();
     }
@@ -215,22 +231,15 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue
+        // warp: lane quadrant warp % 4 (rows 32 qd + lane), tokens 8 tg .. 8 tg + 7 of the
+        // unit, all eight blocks of every super-block
         pdl_wait();  // the output may still be in use by the previous kernel
-        const int qd = warp & 3, hf = (warp - Q80_EPI_WARP0) >> 2;
+        const int qd = warp & 3, tg = (warp - Q80_EPI_WARP0) >> 2;
         const int row = 32 * qd + lane;
-        const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        uint32_t magic[16];
+        const uint32_t tcol = tm + ((uint32_t)(32 * qd) << 16) + 8 * tg;  // + 256 c + 32 b
+        // first preset of this warp's columns in both accumulator sets
 #pragma unroll
-        for (int i = 0; i < 16; i++) magic[i] = MAGIC_BITS;
-        // first preset of this warp's blocks in both accumulator sets
-#pragma unroll
-        for (int c = 0; c < 2; c++)
-#pragma unroll
-            for (int bb = 0; bb < 4; bb++) {
-                const uint32_t ta = tm + lane_off + 256 * c + 32 * (4 * hf + bb);
-                tmem_st16(ta, magic);
-                tmem_st16(ta + 16, magic);
-            }
+        for (int cb = 0; cb < 16; cb++) tmem_st8_same(tcol + 32 * cb, MAGIC_BITS);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -239,14 +248,17 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
             mbar_arrive(&acc_empty[1]);
         }
         const float2 nM = make_float2(-MAGIC, -MAGIC);
-        uint32_t g = 0, eph = 0;
+        uint32_t g = 0;
         bool ok = true;
         for (int64_t u = blockIdx.x; ok && u < a.n_units; u += gridDim.x) {
             int tile, m0, ntok;
             q80_unit(a, u, tile, m0, ntok);
-            float2 acc[Q80_TOK / 2];
+            // warp-uniform: a last group of 16 tokens leaves token groups 2 and 3 idle (the
+            // MMAs of N = 16 never write their columns, which keep the preset)
+            const bool act = 8 * tg < ntok;
+            float2 acc[4];
 #pragma unroll
-            for (int j = 0; j < Q80_TOK / 2; j++) acc[j] = make_float2(0.0f, 0.0f);
+            for (int j = 0; j < 4; j++) acc[j] = make_float2(0.0f, 0.0f);
             for (int s = 0; s < a.nsb; s++, g++) {
                 const int st = (int)(g % Q80_STAGES), c = (int)(g & 1);
                 ok = __all_sync(~0u, q80_wait(&acc_full[c], (g >> 1) & 1) &&
@@ -254,71 +266,63 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
                 if (!ok) break;
                 tc_fence_after();
                 const uint8_t* const sb = smem + st * Q80_STAGE;
-                const uint2 dw = *reinterpret_cast<const uint2*>(sb + Q80_OFF_D + row * 16 + hf * 8);
-                const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&dw.x));
-                const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&dw.y));
-                const float2 dv[4] = {make_float2(d01.x, d01.x), make_float2(d01.y, d01.y),
-                                      make_float2(d23.x, d23.x), make_float2(d23.y, d23.y)};
-                const float2* const das = reinterpret_cast<const float2*>(sb + Q80_OFF_S);
-                // 16 token columns at a time: into registers, the preset written back; the
-                // accumulators are released once the last columns are preset again
+                const uint4 dw = *reinterpret_cast<const uint4*>(sb + Q80_OFF_D + row * 16);
+                const uint32_t dh[4] = {dw.x, dw.y, dw.z, dw.w};
+                // two blocks at a time: into registers, preset again, folded into the
+                // weighted sums t; the accumulators are free for the MMAs of super-block
+                // g + 2 once the last two blocks are preset
+                float2 t[4];
 #pragma unroll
-                for (int cc = 0; cc < Q80_TOK / 16; cc++) {
-                    if (16 * cc < ntok) {
-                        uint32_t x[4][16];
+                for (int h = 0; h < 4; h++) {
+                    uint32_t x[2][8];
+                    if (act) {
 #pragma unroll
-                        for (int bb = 0; bb < 4; bb++)
-                            tmem_ld16(tm + lane_off + 256 * c + 32 * (4 * hf + bb) + 16 * cc, x[bb]);
+                        for (int b = 0; b < 2; b++) tmem_ld8(tcol + 256 * c + 32 * (2 * h + b), x[b]);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int bb = 0; bb < 4; bb++)
-                            tmem_st16(tm + lane_off + 256 * c + 32 * (4 * hf + bb) + 16 * cc, magic);
-                        if (16 * (cc + 1) >= ntok) {
-                            tmem_wait_st();
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&acc_empty[c]);
-                        }
+                        for (int b = 0; b < 2; b++) tmem_st8_same(tcol + 256 * c + 32 * (2 * h + b), MAGIC_BITS);
+                    }
+                    if (h == 3) {
+                        if (act) tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[c]);
+                    }
+                    if (act) {
 #pragma unroll
-                        for (int i = 0; i < 8; i++) {
-                            float2 t = make_float2(0.0f, 0.0f);
+                        for (int b = 0; b < 2; b++) {
+                            const float2 d2 = __half22float2(*reinterpret_cast<const __half2*>(&dh[h]));
+                            const float d = (b & 1) ? d2.y : d2.x;
+                            const float2 dd = make_float2(d, d);
 #pragma unroll
-                            for (int bb = 0; bb < 4; bb++) {
+                            for (int i = 0; i < 4; i++) {
                                 const float2 X = __fadd2_rn(
-                                    make_float2(__uint_as_float(x[bb][2 * i]), __uint_as_float(x[bb][2 * i + 1])), nM);
-                                t = __ffma2_rn(dv[bb], X, t);
+                                    make_float2(__uint_as_float(x[b][2 * i]), __uint_as_float(x[b][2 * i + 1])), nM);
+                                t[i] = (h == 0 && b == 0) ? __fmul2_rn(dd, X) : __ffma2_rn(dd, X, t[i]);
                             }
-                            acc[8 * cc + i] = __ffma2_rn(das[8 * cc + i], t, acc[8 * cc + i]);
                         }
                     }
                 }
+                const float4 s0 = *reinterpret_cast<const float4*>(sb + Q80_OFF_S + 32 * tg);
+                const float4 s1 = *reinterpret_cast<const float4*>(sb + Q80_OFF_S + 32 * tg + 16);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
+                if (act) {
+                    acc[0] = __ffma2_rn(make_float2(s0.x, s0.y), t[0], acc[0]);
+                    acc[1] = __ffma2_rn(make_float2(s0.z, s0.w), t[1], acc[1]);
+                    acc[2] = __ffma2_rn(make_float2(s1.x, s1.y), t[2], acc[2]);
+                    acc[3] = __ffma2_rn(make_float2(s1.z, s1.w), t[3], acc[3]);
+                }
             }
-            // the two halves of the blocks: half 1 hands its sums to half 0, which stores
-            float* const xr = xbuf + row * Q80_TOK;
-            if (ok && hf == 1) {
+            if (ok && act) {
+                const int cnt = min(ntok, a.m_out - m0) - 8 * tg;
+                float* const dst = a.out + (int64_t)(m0 + 8 * tg) * a.ldo + (int64_t)tile * TROWS + row;
 #pragma unroll
-                for (int j = 0; j < Q80_TOK / 2; j += 2)
-                    *reinterpret_cast<float4*>(xr + 2 * j) =
-                        make_float4(acc[j].x, acc[j].y, acc[j + 1].x, acc[j + 1].y);
+                for (int j = 0; j < 8; j++)
+                    if (j < cnt) dst[(int64_t)j * a.ldo] = (j & 1) ? acc[j >> 1].y : acc[j >> 1].x;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(epi);
-            ok = __all_sync(~0u, ok && q80_wait(epi, eph & 1));
-            eph++;
-            if (ok && hf == 0) {
-                const int cnt = min(ntok, a.m_out - m0);
-                float* const dst = a.out + (int64_t)m0 * a.ldo + (int64_t)tile * TROWS + row;
-#pragma unroll
-                for (int j = 0; j < Q80_TOK; j++)
-                    if (j < cnt) dst[(int64_t)j * a.ldo] = (j & 1 ? acc[j >> 1].y : acc[j >> 1].x) + xr[j];
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(epi);
-            ok = __all_sync(~0u, ok && q80_wait(epi, eph & 1));
-            eph++;
         }
+        tmem_wait_st();  // a wait that ran out may leave presets in flight
     }
     tc_fence_before();
     __syncthreads();

@@ -269,18 +269,26 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
                 const uint4 dw = *reinterpret_cast<const uint4*>(sb + Q80_OFF_D + row * 16);
                 const uint32_t dh[4] = {dw.x, dw.y, dw.z, dw.w};
                 // two blocks at a time: into registers, preset again, folded into the
-                // weighted sums t; the accumulators are free for the MMAs of super-block
-                // g + 2 once the last two blocks are preset
+                // weighted sums t, the next two blocks' load issued before this pair's
+                // arithmetic; the accumulators are free for the MMAs of super-block g + 2
+                // once the last two blocks are preset
                 float2 t[4];
+                uint32_t x[2][2][8];
+                if (act) {
+                    tmem_ld8(tcol + 256 * c, x[0][0]);
+                    tmem_ld8(tcol + 256 * c + 32, x[0][1]);
+                }
 #pragma unroll
                 for (int h = 0; h < 4; h++) {
-                    uint32_t x[2][8];
                     if (act) {
-#pragma unroll
-                        for (int b = 0; b < 2; b++) tmem_ld8(tcol + 256 * c + 32 * (2 * h + b), x[b]);
                         tmem_wait_ld();
 #pragma unroll
                         for (int b = 0; b < 2; b++) tmem_st8_same(tcol + 256 * c + 32 * (2 * h + b), MAGIC_BITS);
+                        if (h < 3) {
+#pragma unroll
+                            for (int b = 0; b < 2; b++)
+                                tmem_ld8(tcol + 256 * c + 32 * (2 * h + 2 + b), x[(h + 1) & 1][b]);
+                        }
                     }
                     if (h == 3) {
                         if (act) tmem_wait_st();
@@ -296,8 +304,9 @@ __global__ void __launch_bounds__(Q80_THREADS, 1) q80_gemm_kernel(const __grid_c
                             const float2 dd = make_float2(d, d);
 #pragma unroll
                             for (int i = 0; i < 4; i++) {
-                                const float2 X = __fadd2_rn(
-                                    make_float2(__uint_as_float(x[b][2 * i]), __uint_as_float(x[b][2 * i + 1])), nM);
+                                const float2 X = __fadd2_rn(make_float2(__uint_as_float(x[h & 1][b][2 * i]),
+                                                                        __uint_as_float(x[h & 1][b][2 * i + 1])),
+                                                            nM);
                                 t[i] = (h == 0 && b == 0) ? __fmul2_rn(dd, X) : __ffma2_rn(dd, X, t[i]);
                             }
                         }

@@ -79,6 +79,27 @@ def test_qgemm_q80_full_projection_sampled_columns():
         assert ok, (n0, worst)
 
 
+@pytest.mark.parametrize("M,cols", [
+    (512, (0, 2048, 3968)),   # 16 token groups x 32 tiles = 512 units: 3 or 4 per CTA
+    (176, (0, 3072, 3968)),   # 5 groups of 32 + one of 16 = 192 units: CTAs 0-43 take a
+                              # second unit, some of them a 16-token unit after a 32-token one
+])
+def test_qgemm_q80_several_units_per_cta(M, cols):
+    """More units than SMs: each CTA runs the persistent loop over several units (tensor
+    memory, the barrier phases and the stage ring carried from one unit to the next)."""
+    N, K = 4096, 4096
+    w = synth.weights(synth.Q8_0, N, K, 86, M)
+    x = synth.activations(M, K, 86, M)
+    wd = dllm.repack(Q8, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, Q8, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    for n0 in cols:
+        _, ref, T = oracle.qgemm(Q8, w, N, K, oq, os_, n0=n0, n1=n0 + 128)
+        ok, worst = gu.tol_ok(out[:, n0:n0 + 128], ref, T)
+        assert ok, (n0, worst)
+
+
 @pytest.mark.parametrize("n_rows", [1, 7, 32])
 def test_qgemm_q80_requested_rows_and_noalloc(n_rows):
     M, N, K = 160, 256, 2048

@@ -72,6 +72,9 @@ def parse():
                    help="with several ranks: replicas (each GPU runs the whole step, weak scaling) or nsplit "
                         "(each GPU owns 1/N of every projection's weight rows, outputs all-gathered over NCCL, "
                         "strong scaling)")
+    p.add_argument("--record-traffic", metavar="CSV", default=None,
+                   help="write the stored GEMM DRAM traffic (profiles/qgemm_dram_traffic.json) from the ncu CSV "
+                        "of a 1-layer step (its first five qgemm launches: QKV, O, gate/up, down, output) and exit")
     p.add_argument("--gather-last", action="store_true",
                    help="the last layer's O and FFN, and the final norm, on the requested rows only")
     return p.parse_args()
@@ -210,6 +213,55 @@ def kernel_source_hash(texts=None):
         code = [re.sub(r"\s*//.*$", "", line).rstrip() for line in t.splitlines()]
         h.update("\n".join(line for line in code if line).encode())
     return h.hexdigest()[:16]
+
+
+TRAFFIC_SHAPES = ("qkv", "o", "gate_up", "down", "output")
+TRAFFIC_COMMAND = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                   "--clock-control none -k regex:qgemm -s 0 -c 5 --csv --log-file {csv} "
+                   "python bench.py --layers 1 --steps 1 --warmup 3 --no-cpu --no-e2e")
+
+
+def record_traffic(args):
+    """Per-launch DRAM bytes of the GEMM from one ncu capture of the 1-layer step, whose
+    five GEMM launches have the full step's per-launch shapes, weighted by the full
+    step's launch mix and keyed to the current kernel source."""
+    import csv
+    per = {}
+    with open(args.record_traffic, newline="") as f:
+        for row in csv.DictReader(line for line in f if not line.startswith("==")):
+            if "qgemm" not in row.get("Kernel Name", ""):
+                continue
+            unit = row["Metric Unit"]
+            val = float(row["Metric Value"].replace(",", ""))
+            scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "ns": 1e-3, "us": 1.0, "usecond": 1.0,
+                     "nsecond": 1e-3, "msecond": 1e3}[unit]
+            per.setdefault(int(row["ID"]), {})[row["Metric Name"]] = val * scale
+    ids = sorted(per)[:len(TRAFFIC_SHAPES)]
+    if len(ids) != len(TRAFFIC_SHAPES):
+        sys.exit(f"expected {len(TRAFFIC_SHAPES)} qgemm launches in {args.record_traffic}, found {len(ids)}")
+    shapes = {name: {"dram_read": int(per[i]["dram__bytes_read.sum"]), "dram_write": int(per[i]["dram__bytes_write.sum"]),
+                     "us_cold": round(per[i]["gpu__time_duration.sum"], 2)} for name, i in zip(TRAFFIC_SHAPES, ids)}
+    from quantized_int8_gemm_q4_b200 import synth
+    model = synth.MODELS[args.model]()
+    n_layers = model.n_layers
+    step = step_gemms(model, args.canvas, n_layers)
+    counts = {"qkv": n_layers, "o": n_layers, "gate_up": n_layers, "down": n_layers, "output": 1}
+    total = sum(counts[k] * (v["dram_read"] + v["dram_write"]) for k, v in shapes.items())
+    key = f"{args.model}_L{args.canvas}"
+    out = {
+        "what": "DRAM bytes (read + write) per qgemm_kernel launch, mean over the step's launch mix "
+                f"({n_layers} x QKV, O, gate/up, down + the output projection), from one ncu capture of the "
+                "1-layer step whose five GEMM launches have the full step's per-launch shapes",
+        "command": TRAFFIC_COMMAND.format(csv=args.record_traffic),
+        "kernel_source_sha": kernel_source_hash(),
+        "per_launch_bytes": {key: round(total / len(step))},
+        "per_launch_shape": shapes,
+        f"algorithmic_bytes_per_launch_{key}": round(sum(g.bytes for g in step) / len(step)),
+        "note": "the f32 outputs and the quantized activations stay in L2 within a launch, so DRAM traffic is "
+                "the weight stream plus little else: no weight byte is read twice",
+    }
+    TRAFFIC_FILE.write_text(json.dumps(out, indent=1) + "\n")
+    return out
 
 
 def stored_traffic(workload_key):
@@ -1215,6 +1267,9 @@ def main():
     args = parse()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args)["per_launch_bytes"]), flush=True)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

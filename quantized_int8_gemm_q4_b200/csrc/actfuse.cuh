@@ -69,28 +69,33 @@ __device__ __forceinline__ void load8(const float* __restrict__ p, float (&v)[8]
 
 constexpr int FUSE_WARPS = 8;
 
-// RMSNorm + quantize.  One CTA per output row m in [0, Mp) with W = min(K/256, 32)
-// warps; warp w handles super-blocks w, w + W, ...  Output row m reads canvas row
-// rows[m] when a row list is given (M is then the list's length and M_src the canvas
-// height), else canvas row m.  Pass 1 loads the warp's first super-block of x and gamma
-// into registers and sums the squares in fp64 (each lane in element order, then a
-// fixed reduction tree); pass 2 normalises and quantizes from the registers,
-// re-reading only super-blocks beyond the first (K > 8192).  Rows M..Mp-1, and rows
-// whose list entry is outside [0, M_src), are written as zeros; the latter also set
-// ERR_ROW_RANGE.
+// RMSNorm + quantize.  One CTA per output row m in [0, Mp) with W <= MAXW warps (the
+// host picks the form: one super-block per warp while the rows fill at most two waves of
+// CTAs, else up to 4 per warp in CTAs of at most 4 warps, so that six rows are in
+// flight on each SM); warp w handles super-blocks w, w + W, ...  Output row m reads canvas row rows[m] when a row list is
+// given (M is then the list's length and M_src the canvas height), else canvas row m.
+// Pass 1 loads the warp's first SBR super-blocks of x into registers
+// and sums the squares in fp64 (each lane in element order, then a fixed reduction tree
+// over the lanes and, in warp 0, over the warps); pass 2 normalises and quantizes from
+// the registers (gamma, the same for every row, comes from L1), re-reading only
+// super-blocks beyond those (K > SBR * W * 256).
+// Rows M..Mp-1, and rows whose list entry is outside [0, M_src), are written as zeros;
+// the latter also set ERR_ROW_RANGE.
 constexpr int RMS_MAX_WARPS = 32;
 
-__global__ void __launch_bounds__(RMS_MAX_WARPS * 32) rmsnorm_quantize_kernel(
+template <int SBR, int MAXW>
+__global__ void __launch_bounds__(MAXW * 32, MAXW <= 4 ? 6 : 1) rmsnorm_quantize_kernel(
     const float* __restrict__ x, int64_t M, int64_t K, int64_t ldx, const float* __restrict__ gamma, float eps,
     const int32_t* __restrict__ rows, int64_t M_src, int64_t Mp, int8_t* __restrict__ q, float* __restrict__ scale,
     uint8_t* __restrict__ sums) {
-    __shared__ double red[RMS_MAX_WARPS];
+    __shared__ double red[MAXW];
+    __shared__ double rn_s;
     pdl_trigger();
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int W = blockDim.x >> 5;
     const int64_t m = blockIdx.x;
     const int64_t nsb = K / QK;
-    float xv[8], gv[8];
+    float xv[SBR][8];
     pdl_wait();  // x and rows may be outputs of the previous kernel on the stream
     int64_t src = m;
     if (rows != nullptr && m < M) {
@@ -102,15 +107,22 @@ __global__ void __launch_bounds__(RMS_MAX_WARPS * 32) rmsnorm_quantize_kernel(
     }
     const bool live = m < M && src >= 0;
     const float* xr = x + (live ? src : 0) * ldx;
-    load8(gamma + w * QK + 8 * lane, gv);
+#pragma unroll
+    for (int j = 0; j < SBR; j++) {
+        const int64_t sj = w + (int64_t)j * W;
+        if (sj < nsb && live) load8(xr + sj * QK + 8 * lane, xv[j]);
+    }
     double ss = 0.0;
     if (live) {
-        load8(xr + w * QK + 8 * lane, xv);
 #pragma unroll
-        for (int i = 0; i < 8; i++) ss = __dadd_rn(ss, __dmul_rn((double)xv[i], (double)xv[i]));
-        for (int64_t s = w + W; s < nsb; s += W) {
+        for (int j = 0; j < SBR; j++)
+            if (w + (int64_t)j * W < nsb) {
+#pragma unroll
+                for (int i = 0; i < 8; i++) ss = __dadd_rn(ss, __dmul_rn((double)xv[j][i], (double)xv[j][i]));
+            }
+        for (int64_t sj = w + (int64_t)SBR * W; sj < nsb; sj += W) {
             float v[8];
-            load8(xr + s * QK + 8 * lane, v);
+            load8(xr + sj * QK + 8 * lane, v);
 #pragma unroll
             for (int i = 0; i < 8; i++) ss = __dadd_rn(ss, __dmul_rn((double)v[i], (double)v[i]));
         }
@@ -119,20 +131,47 @@ __global__ void __launch_bounds__(RMS_MAX_WARPS * 32) rmsnorm_quantize_kernel(
     for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
     if (lane == 0) red[w] = ss;
     __syncthreads();
-    ss = red[0];
-    for (int i = 1; i < W; i++) ss = __dadd_rn(ss, red[i]);
-    const double rn = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)eps)));
-    for (int64_t s = w; s < nsb; s += W) {
-        if (s != w) {
-            load8(gamma + s * QK + 8 * lane, gv);
-            if (live) load8(xr + s * QK + 8 * lane, xv);
+    if (w == 0) {
+        double t = lane < W ? red[lane] : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, o));
+        if (lane == 0) rn_s = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(t, (double)K), (double)eps)));
+    }
+    __syncthreads();
+    const double rn = rn_s;
+#pragma unroll
+    for (int j = 0; j < SBR; j++) {
+        const int64_t sj = w + (int64_t)j * W;
+        if (sj < nsb) {
+            float g8[8], v[8];
+            load8(gamma + sj * QK + 8 * lane, g8);  // the same for every row: from L1
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                v[i] = live ? __double2float_rn(__dmul_rn(__dmul_rn((double)xv[j][i], rn), (double)g8[i])) : 0.0f;
+            quantize_store_lane(v, lane, m, sj, Mp, q, scale, sums);
         }
-        float v[8];
+    }
+    for (int64_t sj = w + (int64_t)SBR * W; sj < nsb; sj += W) {
+        float g8[8], x8[8], v[8];
+        load8(gamma + sj * QK + 8 * lane, g8);
+        if (live) load8(xr + sj * QK + 8 * lane, x8);
 #pragma unroll
         for (int i = 0; i < 8; i++)
-            v[i] = live ? __double2float_rn(__dmul_rn(__dmul_rn((double)xv[i], rn), (double)gv[i])) : 0.0f;
-        quantize_store_lane(v, lane, m, s, Mp, q, scale, sums);
+            v[i] = live ? __double2float_rn(__dmul_rn(__dmul_rn((double)x8[i], rn), (double)g8[i])) : 0.0f;
+        quantize_store_lane(v, lane, m, sj, Mp, q, scale, sums);
     }
+}
+
+// The form of rmsnorm_quantize_kernel for Mp output rows of K on `sms` SMs: few rows,
+// one super-block per warp and up to 32 warps (latency); many rows, up to 4 per warp
+// and at most 4 warps, six CTAs per SM (rows in flight).  Returns the warps per CTA; *wide tells which.
+constexpr int RMS_WIDE_SBR = 4, RMS_WIDE_WARPS = 4;
+inline int rms_warps(int64_t Mp, int64_t K, int sms, bool* wide) {
+    const int64_t nsb = K / QK;
+    *wide = Mp > 2 * (int64_t)sms;
+    if (!*wide) return (int)(nsb < RMS_MAX_WARPS ? nsb : RMS_MAX_WARPS);
+    const int64_t few = (nsb + RMS_WIDE_SBR - 1) / RMS_WIDE_SBR;
+    return (int)(few < RMS_WIDE_WARPS ? few : RMS_WIDE_WARPS);
 }
 
 // SwiGLU + quantize.  Grid (Mp, ceil(nsb / 8)); warp w of CTA (m, b) handles

@@ -462,8 +462,10 @@ int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, con
     int dev;
     if ((rc = current_device(&dev))) return rc;
     const int64_t Mp = round_up(M_out, 16);
-    const int64_t warps = K / QK < RMS_MAX_WARPS ? K / QK : RMS_MAX_WARPS;
-    if (launch_pdl(rmsnorm_quantize_kernel, dim3((unsigned)Mp), dim3((unsigned)(warps * 32)), 0,
+    bool wide = false;
+    const int warps = rms_warps(Mp, K, g_num_sms[dev], &wide);
+    if (launch_pdl(wide ? rmsnorm_quantize_kernel<RMS_WIDE_SBR, RMS_WIDE_WARPS> : rmsnorm_quantize_kernel<1, RMS_MAX_WARPS>,
+                   dim3((unsigned)Mp), dim3((unsigned)(warps * 32)), 0,
                    reinterpret_cast<cudaStream_t>(stream), x, M_out, K, ldx, gamma, eps, rows, M, Mp, q, scale,
                    sums) != cudaSuccess) {
         (void)cudaGetLastError();

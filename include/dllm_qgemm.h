@@ -150,12 +150,16 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  * operations and rounded to f32 once.  The f32 is then quantized exactly as in
  * dllm_quantize_act.
  *   RMSNorm: ss = sum over the row's K elements of x^2, r = 1 / sqrt(ss / K + eps),
- *            y = f32((x * r) * gamma[k]).  The order of the fp64 sum is unspecified.
- *            A different order can move y by one f32 rounding only when the fp64
- *            value lies within about K * 2^-53 (relative) of a rounding boundary.
+ *            y = f32((x * r) * gamma[k]).  The fp64 sum has one fixed order for
+ *            every row count and row list (per super-block: each lane's 8 squares
+ *            in element order, then a butterfly over 32 lanes; then slot l = the
+ *            super-blocks l, l + 32, ... in order, and a butterfly over 32 slots),
+ *            so a row list gives the full canvas's rows bit for bit.  Another order
+ *            (the oracle's) can move y by one f32 rounding only when the fp64 value
+ *            lies within about K * 2^-53 (relative) of a rounding boundary.
  *   SwiGLU:  h = f32((g / (1 + exp(-g))) * u).  exp is CUDA's fp64 exp.
  *
- * dllm_rmsnorm_quantize: x f32 [M][ldx] (ldx >= K, ldx % 4 == 0), gamma f32 [K],
+ * dllm_rmsnorm_quantize: x f32 [M][ldx] (ldx >= K, ldx % 4 == 0, K <= 65536), gamma f32 [K],
  *   eps > 0 and finite (else DLLM_ERR_ARG; eps = 0 would make an all-zero row 0/0).
  *   rows == NULL (n_rows = 0): all M canvas rows; the output has M rows.
  *   rows != NULL: device int32 list of n_rows >= 1 canvas rows (any order, duplicates
@@ -165,7 +169,9 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  *   input of the last layer, where only the requested positions continue past attention
  *   (step 3).  An entry outside [0, M) zero-fills its output row and sets
  *   DLLM_ERR_ROW_RANGE in the device error word.
- *   One CTA per output row (rounded up to 16 CTAs), min(K/256, 32) warps.
+ *   One CTA per output row (rounded up to 16 CTAs): min(K/256, 32) warps while the
+ *   rows fit in two waves of CTAs on the SMs, else min(ceil(K/1024), 4) warps that
+ *   hold up to four super-blocks each in registers.
  * dllm_swiglu_quantize: gate, up f32 [M][ld] each (ld >= K, ld % 4 == 0).  They may
  *   be two column ranges of one buffer, e.g. the out_q/out_k pair of dllm_qkv_qgemm
  *   run on the gate and up weights with ld = 2 * K and up = gate + K.

@@ -72,23 +72,39 @@ constexpr int FUSE_WARPS = 8;
 // RMSNorm + quantize.  One CTA per output row m in [0, Mp) with W <= MAXW warps (the
 // host picks the form: one super-block per warp while the rows fill at most two waves of
 // CTAs, else up to 4 per warp in CTAs of at most 4 warps, so that six rows are in
-// flight on each SM); warp w handles super-blocks w, w + W, ...  Output row m reads canvas row rows[m] when a row list is
-// given (M is then the list's length and M_src the canvas height), else canvas row m.
-// Pass 1 loads the warp's first SBR super-blocks of x into registers
-// and sums the squares in fp64 (each lane in element order, then a fixed reduction tree
-// over the lanes and, in warp 0, over the warps); pass 2 normalises and quantizes from
-// the registers (gamma, the same for every row, comes from L1), re-reading only
-// super-blocks beyond those (K > SBR * W * 256).
-// Rows M..Mp-1, and rows whose list entry is outside [0, M_src), are written as zeros;
-// the latter also set ERR_ROW_RANGE.
+// flight on each SM); warp w handles super-blocks w, w + W, ...  Output row m reads
+// canvas row rows[m] when a row list is given (M is then the list's length and M_src the
+// canvas height), else canvas row m.  The sum of squares is fp64 in one order whatever
+// the form (so a row list gives the full canvas's rows bit for bit): per super-block,
+// each lane's 8 squares in element order and then a butterfly over the 32 lanes; then,
+// over the super-blocks, slot l = sum of the super-blocks l, l + 32, ... in that order
+// (zero past the last) and a butterfly over the 32 slots.  Pass 1 keeps the warp's first
+// SBR super-blocks of x in registers; pass 2 normalises and quantizes from them (gamma,
+// the same for every row, comes from L1), re-reading only super-blocks beyond those
+// (K > SBR * W * 256).  Rows M..Mp-1, and rows whose list entry is outside [0, M_src),
+// are written as zeros; the latter also set ERR_ROW_RANGE.
 constexpr int RMS_MAX_WARPS = 32;
+constexpr int RMS_MAX_SB = 256;  // K <= 65536
+
+__device__ __forceinline__ double butterfly_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ double squares8(const float (&v)[8]) {
+    double ps = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) ps = __dadd_rn(ps, __dmul_rn((double)v[i], (double)v[i]));
+    return ps;
+}
 
 template <int SBR, int MAXW>
 __global__ void __launch_bounds__(MAXW * 32, MAXW <= 4 ? 6 : 1) rmsnorm_quantize_kernel(
     const float* __restrict__ x, int64_t M, int64_t K, int64_t ldx, const float* __restrict__ gamma, float eps,
     const int32_t* __restrict__ rows, int64_t M_src, int64_t Mp, int8_t* __restrict__ q, float* __restrict__ scale,
     uint8_t* __restrict__ sums) {
-    __shared__ double red[MAXW];
+    __shared__ double red[RMS_MAX_SB];
     __shared__ double rn_s;
     pdl_trigger();
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -112,29 +128,25 @@ __global__ void __launch_bounds__(MAXW * 32, MAXW <= 4 ? 6 : 1) rmsnorm_quantize
         const int64_t sj = w + (int64_t)j * W;
         if (sj < nsb && live) load8(xr + sj * QK + 8 * lane, xv[j]);
     }
-    double ss = 0.0;
-    if (live) {
 #pragma unroll
-        for (int j = 0; j < SBR; j++)
-            if (w + (int64_t)j * W < nsb) {
-#pragma unroll
-                for (int i = 0; i < 8; i++) ss = __dadd_rn(ss, __dmul_rn((double)xv[j][i], (double)xv[j][i]));
-            }
-        for (int64_t sj = w + (int64_t)SBR * W; sj < nsb; sj += W) {
-            float v[8];
-            load8(xr + sj * QK + 8 * lane, v);
-#pragma unroll
-            for (int i = 0; i < 8; i++) ss = __dadd_rn(ss, __dmul_rn((double)v[i], (double)v[i]));
+    for (int j = 0; j < SBR; j++) {
+        const int64_t sj = w + (int64_t)j * W;
+        if (sj < nsb) {
+            const double ps = butterfly_sum(live ? squares8(xv[j]) : 0.0);
+            if (lane == 0) red[sj] = ps;
         }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
-    if (lane == 0) red[w] = ss;
+    for (int64_t sj = w + (int64_t)SBR * W; sj < nsb; sj += W) {
+        float v[8];
+        if (live) load8(xr + sj * QK + 8 * lane, v);
+        const double ps = butterfly_sum(live ? squares8(v) : 0.0);
+        if (lane == 0) red[sj] = ps;
+    }
     __syncthreads();
     if (w == 0) {
-        double t = lane < W ? red[lane] : 0.0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) t = __dadd_rn(t, __shfl_xor_sync(0xffffffffu, t, o));
+        double t = lane < nsb ? red[lane] : 0.0;
+        for (int64_t l = lane + 32; l < nsb; l += 32) t = __dadd_rn(t, red[l]);
+        t = butterfly_sum(t);
         if (lane == 0) rn_s = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(t, (double)K), (double)eps)));
     }
     __syncthreads();

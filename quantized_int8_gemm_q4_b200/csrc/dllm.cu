@@ -451,7 +451,7 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
 int dllm_rmsnorm_quantize(const float* x, int64_t M, int64_t K, int64_t ldx, const float* gamma, float eps,
                           const int32_t* rows, int64_t n_rows, int8_t* q, float* scale, uint8_t* sums,
                           dllm_stream_t stream) {
-    if (!x || !gamma || M <= 0 || K <= 0 || K % QK || ldx < K) return DLLM_ERR_ARG;
+    if (!x || !gamma || M <= 0 || K <= 0 || K % QK || K > (int64_t)RMS_MAX_SB * QK || ldx < K) return DLLM_ERR_ARG;
     if (!(eps > 0.0f) || !(eps < INFINITY)) return DLLM_ERR_ARG;
     if (rows ? n_rows <= 0 : n_rows != 0) return DLLM_ERR_ARG;
     const int64_t M_out = rows ? n_rows : M;

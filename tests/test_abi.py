@@ -120,6 +120,7 @@ def test_fused_quantize_argument_checks(lib):
     assert rms(gamma=None) == dllm.DLLM_ERR_ARG
     assert rms(K=300, ldx=300) == dllm.DLLM_ERR_ARG
     assert rms(ldx=128) == dllm.DLLM_ERR_ARG
+    assert rms(K=65536 + 256, ldx=65536 + 256) == dllm.DLLM_ERR_ARG   # the documented K <= 65536
     assert rms(M=0) == dllm.DLLM_ERR_ARG
     assert rms(eps=0.0) == dllm.DLLM_ERR_ARG
     assert rms(eps=-1e-5) == dllm.DLLM_ERR_ARG

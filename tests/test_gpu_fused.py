@@ -130,7 +130,10 @@ def _rms_bracket(x, gamma, eps):
 
 
 @pytest.mark.parametrize("M,K", [(1, 256), (5, 512), (16, 256), (17, 768), (64, 3584), (128, 4096), (257, 1024),
-                                 (3, 8448), (2, 16384)])
+                                 (3, 8448), (2, 16384),
+                                 # more rows than two waves of CTAs: the form with up to four
+                                 # super-blocks per warp (uneven at 3584, re-read past 16 at 8448)
+                                 (300, 4096), (601, 3584), (297, 8448), (300, 256)])
 def test_rmsnorm_quantize(M, K):
     x = _rms_rows(M, K, 41)
     gamma = _gamma(K, K)
@@ -254,10 +257,12 @@ def _run_rms_rows(x, gamma, eps, rows):
     return q, s, u
 
 
-def test_rmsnorm_quantize_rows():
+@pytest.mark.parametrize("M", [160, 320])
+def test_rmsnorm_quantize_rows(M):
     """A row list: output row i is canvas row rows[i] (any order, duplicates), equal bit for
-    bit to that row of the full-canvas result."""
-    M, K = 160, 4096
+    bit to that row of the full-canvas result (at 320 rows the full canvas runs the form
+    with four super-blocks per warp, the 37-row list the one with one per warp)."""
+    K = 4096
     x = _rms_rows(M, K, 47)
     gamma = _gamma(K, 11)
     rows = np.concatenate([synth.block_rows(M, 32, 48), [0, M - 1, 5, 5, 37]]).astype(np.int32)

@@ -147,9 +147,11 @@ def test_rmsnorm_quantize(M, K):
         assert not s.cpu().numpy().reshape(K // 256, Mp)[:, M:].any()
 
 
-@pytest.mark.parametrize("eps", [1e-6, 1.0, 1e4])
-def test_rmsnorm_quantize_eps_and_stride(eps):
-    M, K, ldx = 24, 2048, 2304
+@pytest.mark.parametrize("eps,M", [(1e-6, 24), (1.0, 24), (1e4, 24), (1e-5, 300)])
+def test_rmsnorm_quantize_eps_and_stride(eps, M):
+    """eps across its range and a row stride ldx > K (at 300 rows, in the form with four
+    super-blocks per warp)."""
+    K, ldx = 2048, 2304
     x = _rms_rows(M, K, 42)
     gamma = _gamma(K, 7)
     q, s, u = _run_rms(x, gamma, eps, ldx=ldx)

@@ -100,6 +100,22 @@ def test_qgemm_q80_several_units_per_cta(M, cols):
         assert ok, (n0, worst)
 
 
+def test_qgemm_q80_wide_ldo_and_row_list_leave_other_columns():
+    """ldo > N: the columns past N keep what the caller put there, with and without a
+    row list."""
+    M, N, K, ldo = 40, 256, 512, 384
+    w = synth.weights(synth.Q8_0, N, K, 87)
+    x = synth.activations(M, K, 87)
+    wd = dllm.repack(Q8, w, N, K)
+    act = gu.Act(x)
+    oq, os_, _ = oracle.quantize_act(x)
+    for rows in (None, [39, 0, 17, 17, 5]):
+        out = gu.gemm(wd, Q8, N, K, act, rows=rows, ldo=ldo).cpu().numpy()
+        assert np.isnan(out[:, N:]).all()
+        _, ref, T = oracle.qgemm(Q8, w, N, K, oq, os_, rows=rows)
+        assert gu.tol_ok(out[:, :N], ref, T)[0]
+
+
 @pytest.mark.parametrize("n_rows", [1, 7, 32])
 def test_qgemm_q80_requested_rows_and_noalloc(n_rows):
     M, N, K = 160, 256, 2048

@@ -169,9 +169,9 @@ int dllm_quantize_act(const float* x, int64_t M, int64_t K, int64_t ldx, int8_t*
  *   input of the last layer, where only the requested positions continue past attention
  *   (step 3).  An entry outside [0, M) zero-fills its output row and sets
  *   DLLM_ERR_ROW_RANGE in the device error word.
- *   One CTA per output row (rounded up to 16 CTAs): min(K/256, 32) warps while the
- *   rows fit in two waves of CTAs on the SMs, else min(ceil(K/1024), 4) warps that
- *   hold up to four super-blocks each in registers.
+ *   One CTA per output row (rounded up to 16 CTAs): min(K/256, 32) warps up to 12
+ *   rows per SM, else min(ceil(K/1024), 4) warps that hold up to four super-blocks
+ *   each in registers.
  * dllm_swiglu_quantize: gate, up f32 [M][ld] each (ld >= K, ld % 4 == 0).  They may
  *   be two column ranges of one buffer, e.g. the out_q/out_k pair of dllm_qkv_qgemm
  *   run on the gate and up weights with ld = 2 * K and up = gate + K.

@@ -70,9 +70,9 @@ __device__ __forceinline__ void load8(const float* __restrict__ p, float (&v)[8]
 constexpr int FUSE_WARPS = 8;
 
 // RMSNorm + quantize.  One CTA per output row m in [0, Mp) with W <= MAXW warps (the
-// host picks the form: one super-block per warp while the rows fill at most two waves of
-// CTAs, else up to 4 per warp in CTAs of at most 4 warps, so that six rows are in
-// flight on each SM); warp w handles super-blocks w, w + W, ...  Output row m reads
+// host picks the form: one super-block per warp up to 12 rows per SM, else up to 4 per
+// warp in CTAs of at most 4 warps, so that six rows are in flight on each SM); warp w
+// handles super-blocks w, w + W, ...  Output row m reads
 // canvas row rows[m] when a row list is given (M is then the list's length and M_src the
 // canvas height), else canvas row m.  The sum of squares is fp64 in one order whatever
 // the form (so a row list gives the full canvas's rows bit for bit): per super-block,
@@ -174,13 +174,16 @@ __global__ void __launch_bounds__(MAXW * 32, MAXW <= 4 ? 6 : 1) rmsnorm_quantize
     }
 }
 
-// The form of rmsnorm_quantize_kernel for Mp output rows of K on `sms` SMs: few rows,
-// one super-block per warp and up to 32 warps (latency); many rows, up to 4 per warp
-// and at most 4 warps, six CTAs per SM (rows in flight).  Returns the warps per CTA; *wide tells which.
+// The form of rmsnorm_quantize_kernel for Mp output rows of K on `sms` SMs: up to 12
+// rows per SM, one super-block per warp and up to 32 warps (the shortest chain per row;
+// with a partial wave, or behind the previous kernel's tail, the chain sets the time:
+// at 512 and 1024 rows the wide form cost 3-5 us more per launch inside the step);
+// beyond, up to 4 per warp and at most 4 warps, six CTAs per SM (rows in flight: 4096
+// rows 46 -> 35 us).  Returns the warps per CTA; *wide tells which.
 constexpr int RMS_WIDE_SBR = 4, RMS_WIDE_WARPS = 4;
 inline int rms_warps(int64_t Mp, int64_t K, int sms, bool* wide) {
     const int64_t nsb = K / QK;
-    *wide = Mp > 2 * (int64_t)sms;
+    *wide = Mp > 12 * (int64_t)sms;
     if (!*wide) return (int)(nsb < RMS_MAX_WARPS ? nsb : RMS_MAX_WARPS);
     const int64_t few = (nsb + RMS_WIDE_SBR - 1) / RMS_WIDE_SBR;
     return (int)(few < RMS_WIDE_WARPS ? few : RMS_WIDE_WARPS);

@@ -131,9 +131,9 @@ def _rms_bracket(x, gamma, eps):
 
 @pytest.mark.parametrize("M,K", [(1, 256), (5, 512), (16, 256), (17, 768), (64, 3584), (128, 4096), (257, 1024),
                                  (3, 8448), (2, 16384),
-                                 # more rows than two waves of CTAs: the form with up to four
+                                 # more than 12 rows per SM (148 SMs): the form with up to four
                                  # super-blocks per warp (uneven at 3584, re-read past 16 at 8448)
-                                 (300, 4096), (601, 3584), (297, 8448), (300, 256)])
+                                 (1800, 4096), (1790, 3584), (1781, 8448), (1800, 256)])
 def test_rmsnorm_quantize(M, K):
     x = _rms_rows(M, K, 41)
     gamma = _gamma(K, K)
@@ -147,9 +147,9 @@ def test_rmsnorm_quantize(M, K):
         assert not s.cpu().numpy().reshape(K // 256, Mp)[:, M:].any()
 
 
-@pytest.mark.parametrize("eps,M", [(1e-6, 24), (1.0, 24), (1e4, 24), (1e-5, 300)])
+@pytest.mark.parametrize("eps,M", [(1e-6, 24), (1.0, 24), (1e4, 24), (1e-5, 1800)])
 def test_rmsnorm_quantize_eps_and_stride(eps, M):
-    """eps across its range and a row stride ldx > K (at 300 rows, in the form with four
+    """eps across its range and a row stride ldx > K (at 1800 rows, in the form with four
     super-blocks per warp)."""
     K, ldx = 2048, 2304
     x = _rms_rows(M, K, 42)
@@ -259,10 +259,10 @@ def _run_rms_rows(x, gamma, eps, rows):
     return q, s, u
 
 
-@pytest.mark.parametrize("M", [160, 320])
+@pytest.mark.parametrize("M", [160, 1800])
 def test_rmsnorm_quantize_rows(M):
     """A row list: output row i is canvas row rows[i] (any order, duplicates), equal bit for
-    bit to that row of the full-canvas result (at 320 rows the full canvas runs the form
+    bit to that row of the full-canvas result (at 1800 rows the full canvas runs the form
     with four super-blocks per warp, the 37-row list the one with one per warp)."""
     K = 4096
     x = _rms_rows(M, K, 47)

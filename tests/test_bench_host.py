@@ -149,3 +149,45 @@ def test_parity_ratio_is_the_tolerance():
     got = ref + np.array([[1e-3, 0.5, 5e-6]])
     # 1e-3 / (1e-5*100) = 1, 0.5 / (1e-6*1e6) = 0.5, 5e-6 / (1e-6*10) = 0.5
     assert abs(bench.parity_ratio(got.astype(np.float32), ref, T) - 1.0) < 1e-3
+
+
+def test_record_traffic_weights_the_step_launch_mix(tmp_path, monkeypatch):
+    """--record-traffic: the five qgemm launches of a 1-layer step's ncu CSV (values with
+    thousands separators, other kernels and ncu's own lines mixed in) become per-shape
+    DRAM bytes and their mean over the full step's 129 launches, keyed to the current
+    kernel source."""
+    import csv
+    import io
+    import json
+    import types
+    hdr = ["ID", "Process ID", "Process Name", "Host Name", "Kernel Name", "Context", "Stream", "Block Size",
+           "Grid Size", "Device", "CC", "Section Name", "Metric Name", "Metric Unit", "Metric Value"]
+    shapes = [(1000, 0, 10000), (2000, 16, 20000), (3000, 32, 30000), (4000, 0, 40000), (50000, 64, 50000)]
+    buf = io.StringIO()
+    wr = csv.writer(buf, quoting=csv.QUOTE_ALL)
+    wr.writerow(hdr)
+    i = 0
+    for rd, wt, ns in shapes:
+        if i == 1:  # a quantizer launch between two GEMMs is ignored
+            wr.writerow([str(i), "1", "python", "h", "void dllm::quantize_act_kernel(...)", "1", "7", "(256, 1, 1)",
+                         "(16, 16, 1)", "0", "10.0", "", "dram__bytes_read.sum", "byte", "999"])
+            i += 1
+        for name, unit, val in (("dram__bytes_read.sum", "byte", rd), ("dram__bytes_write.sum", "byte", wt),
+                                ("gpu__time_duration.sum", "nsecond", ns)):
+            wr.writerow([str(i), "1", "python", "h", "void dllm::qgemm_kernel<12, false, false>(dllm::GemmArgs)",
+                         "1", "7", "(512, 1, 1)", "(148, 1, 1)", "0", "10.0", "", name, unit, f"{val:,}"])
+        i += 1
+    path = tmp_path / "launches.csv"
+    path.write_text("==PROF== Connected to process 1\n" + buf.getvalue())
+    out_file = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", out_file)
+    args = types.SimpleNamespace(record_traffic=str(path), model="llada-8b", canvas=128)
+    bench.record_traffic(args)
+    d = json.loads(out_file.read_text())
+    assert d["kernel_source_sha"] == bench.kernel_source_hash()
+    assert d["per_launch_shape"]["o"] == {"dram_read": 2000, "dram_write": 16, "us_cold": 20.0}
+    expect = (32 * (1000 + 2016 + 3032 + 4000) + 50064) / 129
+    assert d["per_launch_bytes"]["llada-8b_L128"] == round(expect)
+    step = bench.step_gemms(synth.MODELS["llada-8b"](), 128, 32)
+    assert len(step) == 129
+    assert d["algorithmic_bytes_per_launch_llada-8b_L128"] == round(sum(g.bytes for g in step) / 129)

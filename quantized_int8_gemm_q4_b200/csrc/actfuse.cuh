@@ -79,8 +79,9 @@ constexpr int FUSE_WARPS = 8;
 // each lane's 8 squares in element order and then a butterfly over the 32 lanes; then,
 // over the super-blocks, slot l = sum of the super-blocks l, l + 32, ... in that order
 // (zero past the last) and a butterfly over the 32 slots.  Pass 1 keeps the warp's first
-// SBR super-blocks of x in registers; pass 2 normalises and quantizes from them (gamma,
-// the same for every row, comes from L1), re-reading only super-blocks beyond those
+// SBR super-blocks of x in registers (and, with SBR = 1, the gamma of its super-block);
+// pass 2 normalises and quantizes from them (the wide form reads gamma, the same for
+// every row, from L1 there), re-reading only super-blocks beyond those
 // (K > SBR * W * 256).  Rows M..Mp-1, and rows whose list entry is outside [0, M_src),
 // are written as zeros; the latter also set ERR_ROW_RANGE.
 constexpr int RMS_MAX_WARPS = 32;
@@ -128,6 +129,11 @@ __global__ void __launch_bounds__(MAXW * 32, MAXW <= 4 ? 6 : 1) rmsnorm_quantize
         const int64_t sj = w + (int64_t)j * W;
         if (sj < nsb && live) load8(xr + sj * QK + 8 * lane, xv[j]);
     }
+    // one super-block per warp: its gamma too, so that pass 2 waits on no load
+    float g1[8];
+    if constexpr (SBR == 1) {
+        if (w < nsb) load8(gamma + w * QK + 8 * lane, g1);
+    }
 #pragma unroll
     for (int j = 0; j < SBR; j++) {
         const int64_t sj = w + (int64_t)j * W;
@@ -156,7 +162,12 @@ __global__ void __launch_bounds__(MAXW * 32, MAXW <= 4 ? 6 : 1) rmsnorm_quantize
         const int64_t sj = w + (int64_t)j * W;
         if (sj < nsb) {
             float g8[8], v[8];
-            load8(gamma + sj * QK + 8 * lane, g8);  // the same for every row: from L1
+            if constexpr (SBR == 1) {
+#pragma unroll
+                for (int i = 0; i < 8; i++) g8[i] = g1[i];
+            } else {
+                load8(gamma + sj * QK + 8 * lane, g8);  // the same for every row: from L1
+            }
 #pragma unroll
             for (int i = 0; i < 8; i++)
                 v[i] = live ? __double2float_rn(__dmul_rn(__dmul_rn((double)xv[j][i], rn), (double)g8[i])) : 0.0f;

@@ -153,6 +153,55 @@ def test_qkv_q80_three_segments():
         assert gu.tol_ok(o.cpu().numpy(), ref, T)[0]
 
 
+def test_q80_extreme_codes_and_scales():
+    """The exact conversion at its limits: every code -128 (the int8 minimum) against
+    activations that quantize to +-127, the largest block dot (32 * 128 * 127 = 520,192,
+    inside the 2^22 the preset trick allows); every code 127 under the largest f16 scale
+    (65504); blocks whose scale is 0; all-zero activation rows."""
+    M, N, K = 48, 256, 1024
+    w = synth.weights(synth.Q8_0, N, K, 88).copy()
+    b = w.reshape(N, K // 32, 34)
+    b[:64, :, 2:] = 0x80                                  # q = -128
+    b[:64, :, 0:2] = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+    b[64:128, :, 2:] = 127
+    b[64:128, :, 0:2] = np.frombuffer(np.float16(65504.0).tobytes(), np.uint8)
+    b[128:192, :, 0:2] = 0                                # d = 0: no contribution
+    x = synth.activations(M, K, 88)
+    x[0] = 3.0                                            # quantizes to +127 everywhere
+    x[1] = -3.0                                           # -127
+    x[2] = 0.0                                            # all-zero row: scale 0
+    x[3, ::2] = 5.0
+    x[3, 1::2] = -5.0
+    wd = dllm.repack(Q8, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, Q8, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    assert (oq[0] == 127).all() and (oq[1] == -127).all()
+    _, ref, T = oracle.qgemm(Q8, w, N, K, oq, os_)
+    ok, worst = gu.tol_ok(out, ref, T)
+    assert ok, worst
+    assert not out[2].any() and not out[:, 128:192].any()
+    # the extreme rows in closed form: 32 blocks of 32 codes, d = 1, da = 3/127
+    np.testing.assert_allclose(out[0, :64], -128 * 127 * K * (3.0 / 127), rtol=1e-6)
+
+
+def test_q80_vocabulary_width_sampled():
+    """The 126464-row output projection in Q8_0 on 32 requested rows: 988 weight tiles,
+    several per CTA, sampled column ranges against the oracle."""
+    M, N, K = 160, 126464, 4096
+    w = synth.weights(synth.Q8_0, N, K, 89)
+    x = synth.activations(M, K, 89)
+    wd = dllm.repack(Q8, w, N, K)
+    act = gu.Act(x)
+    rows = synth.block_rows(M, 32, 89)
+    out = gu.gemm(wd, Q8, N, K, act, rows=rows).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    for n0 in (0, 63232, N - 128):
+        _, ref, T = oracle.qgemm(Q8, w, N, K, oq, os_, rows=rows, n0=n0, n1=n0 + 128)
+        ok, worst = gu.tol_ok(out[:, n0:n0 + 128], ref, T)
+        assert ok, (n0, worst)
+
+
 def test_q80_deterministic_and_integer_views_rejected():
     M, N, K = 48, 128, 512
     w = synth.weights(synth.Q8_0, N, K, 85)

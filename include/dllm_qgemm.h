@@ -58,7 +58,8 @@ typedef struct CUstream_st* dllm_stream_t; /* a cudaStream_t; NULL = legacy defa
  * turns each 176-byte Q5_K super-block into two Q4_K-form super-blocks of a matrix twice
  * as wide, the low nibbles (d, dmin, the same scales) and the fifth bits as 0/1 nibbles
  * (16*d, dmin 0, the same scales), since d*sc*q - dmin*m = (d*sc*q4 - dmin*m) +
- * (16d)*sc*b exactly.  It keeps 2 x 144 bytes per 256 weights resident (9 bits per
+ * (16d)*sc*b exactly, provided 16 d is a finite f16 (|d| < 4096; GGUF scales are many
+ * orders of magnitude smaller).  It keeps 2 x 144 bytes per 256 weights resident (9 bits per
  * weight, 1.64 x the GGUF size) and streams them at the Q4_K kernel's rate.
  * Q8_0 (the same row) has a kernel of its own: 32-weight blocks, each with an f16 scale d
  * (w = d*q, q int8); every block's integer dot product is one int8 MMA K step into an
@@ -74,8 +75,11 @@ enum {
     DLLM_ERR_ROW_RANGE = -5,   /* device-detected: a rows[] entry outside [0, M)               */
     DLLM_ERR_TIMEOUT = -6,     /* device-detected: a bounded wait inside a kernel ran out      */
     DLLM_ERR_WORKSPACE = -7,   /* workspace smaller than dllm_qgemm_workspace_bytes() asks     */
-    DLLM_ERR_SCRATCH_LIMIT = -8 /* dllm_qgemm_noalloc: the call needs more scratch than the
-                                   library's fixed array holds                               */
+    DLLM_ERR_SCRATCH_LIMIT = -8, /* dllm_qgemm_noalloc: the call needs more scratch than the
+                                    library's fixed array holds                              */
+    DLLM_ERR_SCALE_RANGE = -9   /* device-detected: dllm_repack_q5k met a block scale d with
+                                   |d| >= 4096, which the split form cannot hold (16 d is not a
+                                   finite f16); those blocks' fifth-bit part is not usable      */
 };
 
 /* ------------------------------------------------------------------------------
@@ -99,7 +103,8 @@ int dllm_repack_q6k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dl
  * the split form, [N/128][2K/256] tiles of 18432 bytes (super-block s of a row at tile
  * column s for its low nibbles and K/256 + s for its fifth bits).  dllm_repacked_bytes
  * gives the size.  dllm_qgemm / dllm_qkv_qgemm / dllm_qgemm_noalloc take t = DLLM_Q5_K
- * with the ordinary K-wide activations. */
+ * with the ordinary K-wide activations.  A block scale with |d| >= 4096 (or not finite)
+ * sets DLLM_ERR_SCALE_RANGE in the device error word (dllm_get_device_status). */
 int dllm_repack_q5k(const void* gguf_blocks, int64_t N, int64_t K, void* dst, dllm_stream_t stream);
 /* Q8_0: gguf_blocks is [N][K/32] 34-byte blocks (f16 d, then 32 int8 q).  dst receives
  * the codes as int8 [N][K] (row-major, read by TMA with the 128-byte swizzle) followed by

@@ -782,6 +782,7 @@ const char* dllm_status_string(int code) {
         case DLLM_ERR_TIMEOUT: return "bounded device wait ran out";
         case DLLM_ERR_WORKSPACE: return "workspace too small";
         case DLLM_ERR_SCRATCH_LIMIT: return "call needs more scratch than the fixed no-allocation array holds";
+        case DLLM_ERR_SCALE_RANGE: return "a Q5_K block scale d with |d| >= 4096: 16 d is not a finite f16";
         default: return "unknown status";
     }
 }

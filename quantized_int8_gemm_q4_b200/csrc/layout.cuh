@@ -17,6 +17,7 @@ __device__ __forceinline__ void set_err(int code) { atomicCAS(&g_err, 0, code); 
 
 constexpr int ERR_ROW_RANGE = -5;
 constexpr int ERR_TIMEOUT = -6;
+constexpr int ERR_SCALE_RANGE = -9;
 
 // ---------------------------------------------------------------- sizes
 constexpr int QK = 256;             // weights per super-block
@@ -122,9 +123,11 @@ __global__ void repack_q5k_kernel(const uint8_t* __restrict__ src, int64_t N, in
                 if (!hi) {
                     out[b] = blk[j];
                 } else if (j < 2) {
+                    // 16 d is exact in f16 unless it overflows: |d| >= 4096 cannot be split
                     const unsigned short dbits = (unsigned short)(blk[0] | (blk[1] << 8));
-                    const unsigned short d16 =
-                        __half_as_ushort(__float2half_rn(16.0f * __half2float(__ushort_as_half(dbits))));
+                    const float d16f = 16.0f * __half2float(__ushort_as_half(dbits));
+                    if (j == 0 && !(fabsf(d16f) <= 65504.0f)) set_err(ERR_SCALE_RANGE);
+                    const unsigned short d16 = __half_as_ushort(__float2half_rn(d16f));
                     out[b] = (uint8_t)(j == 0 ? d16 & 255 : d16 >> 8);
                 } else {
                     out[b] = 0;  // dmin' = +0

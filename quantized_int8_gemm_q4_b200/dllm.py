@@ -27,6 +27,7 @@ DLLM_ERR_ROW_RANGE = -5
 DLLM_ERR_TIMEOUT = -6
 DLLM_ERR_WORKSPACE = -7
 DLLM_ERR_SCRATCH_LIMIT = -8
+DLLM_ERR_SCALE_RANGE = -9
 DLLM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 EXPORTS = (

@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9):
         assert dllm.status_string(code) not in ("", "unknown status")
     assert dllm.status_string(-99) == "unknown status"
 

@@ -48,6 +48,58 @@ def test_qgemm_q5k_matches_oracle(M, N, K):
     assert ok, worst
 
 
+def test_qgemm_q5k_extreme_blocks():
+    """The split at its limits (block [d, dmin, 12 scale bytes, 32 qh, 128 qs]): every
+    5-bit code 31 (all low nibbles 15, every fifth bit set) with sc = m = 63; the same
+    under the largest d the split can hold (4094: 16 d = 65504, the f16 maximum) and the
+    largest dmin; all codes 0, so only -dmin * m is left; against activations that
+    quantize to +-127 and an all-zero row."""
+    M, N, K = 48, 256, 1024
+    w = synth.q5k_weights(N, K, 73).copy()
+    b = w.reshape(N, K // 256, 176)
+    one = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+    big_d = np.frombuffer(np.float16(4094.0).tobytes(), np.uint8)
+    big = np.frombuffer(np.float16(65504.0).tobytes(), np.uint8)
+    b[:128, :, 4:16] = 0xFF                               # sc_j = m_j = 63 for every j
+    b[:128, :, 16:176] = 0xFF                             # qh and qs: every q = 31
+    b[:64, :, 0:2] = one
+    b[:64, :, 2:4] = one
+    b[64:128, :, 0:2] = big_d
+    b[64:128, :, 2:4] = big
+    b[128:192, :, 16:176] = 0                             # q = 0: the min term alone
+    x = synth.activations(M, K, 73)
+    x[0] = 3.0
+    x[1] = -3.0
+    x[2] = 0.0
+    wd = dllm.repack(Q5, w, N, K)
+    act = gu.Act(x)
+    out = gu.gemm(wd, Q5, N, K, act).cpu().numpy()
+    oq, os_, _ = oracle.quantize_act(x)
+    assert (oq[0] == 127).all() and (oq[1] == -127).all()
+    _, ref, T = oracle.qgemm(Q5, w, N, K, oq, os_)
+    ok, worst = gu.tol_ok(out, ref, T)
+    assert ok, worst
+    assert not out[2].any()
+    # closed form of row 0 on the first rows: (63 * 31 - 63) per weight, K weights, da = 3/127
+    np.testing.assert_allclose(out[0, :64], (63 * 31 - 63) * 127 * K * (3.0 / 127), rtol=1e-6)
+
+
+def test_repack_q5k_scale_out_of_range_is_reported():
+    """|d| >= 4096 cannot be split (16 d overflows f16): the repack reports
+    DLLM_ERR_SCALE_RANGE in the device error word and nothing faults; the largest
+    splittable d (4094) is accepted."""
+    N, K = 128, 512
+    w = synth.q5k_weights(N, K, 74).copy()
+    b = w.reshape(N, K // 256, 176)
+    b[5, 1, 0:2] = np.frombuffer(np.float16(4094.0).tobytes(), np.uint8)
+    dllm.repack(Q5, w, N, K)
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK
+    b[7, 0, 0:2] = np.frombuffer(np.float16(4096.0).tobytes(), np.uint8)
+    dllm.repack(Q5, w, N, K)
+    assert dllm.dllm_get_device_status() == dllm.DLLM_ERR_SCALE_RANGE
+    assert dllm.dllm_get_device_status() == dllm.DLLM_OK  # read and cleared
+
+
 def test_qgemm_q5k_requested_rows_and_noalloc():
     M, N, K = 160, 256, 2048
     w = synth.q5k_weights(N, K, 72)
